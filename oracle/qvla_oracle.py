@@ -1,0 +1,305 @@
+"""CPU oracle for the Omega-QVLA rotated W4A4 linear layer.
+
+    y = s_x * s_w * ( q(R^T P^T x) . q(W P R)^T ) + b
+
+TEST INFRASTRUCTURE ONLY.  This module is a plain, slow, double-precision
+statement of what the layer computes, used by the test suite, by the package's
+smoke check and by the benchmark's CPU-baseline leg.  The library's CUDA path
+never imports, calls or links it, and it imports nothing from that path.
+
+Sources (web pages on the method; page title, then section):
+  [PT]  "{Omega}-QVLA: Robust Quantization for Vision-Language-Action Models via
+        Composite Rotation and Per-step Scaling" (gist.science, Portuguese
+        technical summary), Metodologia 1 "Rotacao Composta SVD.Hadamard"
+        (bullets "Rotacao SVD", "Rotacao Hadamard", "Implementacao em Blocos")
+        and 2 "Escalonamento de Ativacao DiT por Passo".
+  [FR]  the same paper's French technical summary (gist.science), Methodologie
+        1 "Rotation Composite SVD.Hadamard" and 2 "Mise a l'Echelle ... par Etape".
+  [VN]  "Omega-QVLA: Nen VLA W4A4 tren Edge" (vnrobo.com), sections "Y tuong
+        paper: xoay truoc, scale theo step sau" and "Build DiT action head pack"
+        (flags --use-rtn, --w-bits 4, --a-bits 4, --act-percentile 99.9,
+        --duquant-block-size 64).
+  [ES]  "Omega-QVLA Reduce el Modelo de Vision de Robot por 71% Sin
+        Reentrenamiento" (aiexpert.news): step-count mismatch / truncated table
+        as a failure mode.
+  [FQ]  "FoldQuantVLA: Native Low-Bit Quantization of Vision-Language-Action
+        Models via Consistent Folding" (radar.vhtltd.com): dynamic per-token
+        activation quantisation.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+  * Layouts follow PyTorch Linear: W is [N, K] (out x in), x is [M, K].
+  * R_SVD of a block is the matrix of right singular vectors of that block of
+    W (eigenvectors of its Gram matrix), columns ordered by descending singular
+    value, each column's largest-magnitude entry (first on ties) made positive.
+  * H is the Sylvester Hadamard matrix of order b scaled by 1/sqrt(b).
+  * The zigzag permutation sorts input channels by the L2 norm of their weight
+    column, descending (ties: lower index first), and deals them to the blocks
+    in a snake order, one channel per block per round.
+  * Weights: symmetric per-output-channel RTN, s_w = max|W'|/7, codes in [-7, 7].
+    Activations: s_x = max|x'|/7 per token (dynamic) or s = table[t][l]
+    (per-step table), codes clamped to [-8, 7].  Rounding is to nearest, ties to
+    even; the divisions that decide a code are IEEE fp32 divisions of fp32
+    operands.  A scale of 0 gives all-zero codes.
+  * Nibble packing: byte j holds code 2j in its low nibble and code 2j+1 in its
+    high nibble, both as 4-bit two's complement.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+WEIGHT_QMAX = 7
+ACT_QMIN, ACT_QMAX = -8, 7
+
+
+# --------------------------------------------------------------------------
+# Zigzag channel permutation  ([PT] "Implementacao em Blocos"; [FR] "par Blocs")
+# --------------------------------------------------------------------------
+
+def column_norms(W: np.ndarray) -> np.ndarray:
+    """c_k = ||W[:, k]||_2 in double."""
+    W = np.asarray(W, dtype=np.float64)
+    return np.sqrt(np.sum(W * W, axis=0))
+
+
+def zigzag_permutation(W: np.ndarray, block: int) -> np.ndarray:
+    """perm[j] = original input channel placed at permuted position j.
+
+    Channels are ranked by weight-column norm (descending, ties to the lower
+    index).  Rank r belongs to round r // nb and is dealt to block
+    (r % nb) on even rounds and nb-1-(r % nb) on odd rounds, landing at
+    position `round` inside that block.  Every block therefore receives one
+    channel from each stratum of nb consecutive ranks, which spreads high- and
+    low-norm channels evenly over the blocks."""
+    K = W.shape[1]
+    if K % block:
+        raise ValueError("K must be a multiple of the block size")
+    nb = K // block
+    c = column_norms(W)
+    order = sorted(range(K), key=lambda k: (-c[k], k))
+    perm = np.empty(K, dtype=np.int64)
+    for r, ch in enumerate(order):
+        rnd, pos = divmod(r, nb)
+        blk = pos if rnd % 2 == 0 else nb - 1 - pos
+        perm[blk * block + rnd] = ch
+    return perm
+
+
+# --------------------------------------------------------------------------
+# Composite rotation R = R_SVD . H  ([PT]/[FR] "Rotacao SVD", "Rotacao Hadamard")
+# --------------------------------------------------------------------------
+
+def hadamard(b: int) -> np.ndarray:
+    """Normalised Sylvester Hadamard matrix: H[i, j] = (-1)^popcount(i & j) / sqrt(b)."""
+    if b < 1 or b & (b - 1):
+        raise ValueError("Hadamard order must be a power of two")
+    H = np.empty((b, b), dtype=np.float64)
+    for i in range(b):
+        for j in range(b):
+            H[i, j] = -1.0 if bin(i & j).count("1") % 2 else 1.0
+    return H / np.sqrt(b)
+
+
+def _canonical_signs(V: np.ndarray) -> np.ndarray:
+    V = V.copy()
+    for j in range(V.shape[1]):
+        i = int(np.argmax(np.abs(V[:, j])))      # first index on ties
+        if V[i, j] < 0:
+            V[:, j] = -V[:, j]
+    return V
+
+
+def svd_rotation_blocks(W: np.ndarray, perm: np.ndarray, block: int) -> np.ndarray:
+    """R_SVD for every block, [nb, b, b] double.
+
+    For block B, A_B = (W P)[:, B] is N x b.  Its SVD A_B = U S V^T gives the
+    rotation whose columns are the right singular vectors: the columns of
+    A_B V are U S, so each rotated weight channel carries exactly one singular
+    value's energy.  V is obtained here as the eigenvectors of the Gram matrix
+    A_B^T A_B (eigenvalues S^2), sorted by descending eigenvalue."""
+    W = np.asarray(W, dtype=np.float64)
+    K = W.shape[1]
+    nb = K // block
+    out = np.empty((nb, block, block), dtype=np.float64)
+    for B in range(nb):
+        A = W[:, perm[B * block:(B + 1) * block]]
+        G = A.T @ A
+        lam, V = np.linalg.eigh(G)               # ascending
+        idx = sorted(range(block), key=lambda i: (-lam[i], i))
+        out[B] = _canonical_signs(V[:, idx])
+    return out
+
+
+def composite_blocks(rsvd: np.ndarray) -> np.ndarray:
+    """R_B = R_SVD,B . H_b for every block."""
+    b = rsvd.shape[1]
+    H = hadamard(b)
+    return np.stack([r @ H for r in rsvd])
+
+
+def rotate_weights(W: np.ndarray, perm: np.ndarray, R: np.ndarray) -> np.ndarray:
+    """W' = W P R (block diagonal R), double [N, K]."""
+    W = np.asarray(W, dtype=np.float64)
+    nb, b, _ = R.shape
+    out = np.empty_like(W)
+    for B in range(nb):
+        out[:, B * b:(B + 1) * b] = W[:, perm[B * b:(B + 1) * b]] @ R[B]
+    return out
+
+
+def rotate_activations(x: np.ndarray, perm: np.ndarray, R: np.ndarray) -> np.ndarray:
+    """Row form of x' = R^T P^T x: x'[m, B] = x[m, perm[B]] . R_B, double [M, K]."""
+    x = np.asarray(x, dtype=np.float64)
+    nb, b, _ = R.shape
+    out = np.empty_like(x)
+    for B in range(nb):
+        out[:, B * b:(B + 1) * b] = x[:, perm[B * b:(B + 1) * b]] @ R[B]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Round-to-nearest quantisation  ([VN] "Build DiT action head pack": --use-rtn,
+# --w-bits 4, --a-bits 4; [FQ] dynamic per-token activation quantisation;
+# [PT]/[FR] 2, per-step activation scale table)
+# --------------------------------------------------------------------------
+
+def _rtn_codes(v32: np.ndarray, s32: np.ndarray, qmin: int, qmax: int) -> np.ndarray:
+    """clamp(rint(v / s), qmin, qmax) with an IEEE fp32 division; s == 0 gives 0."""
+    v32 = np.asarray(v32, dtype=np.float32)
+    s32 = np.asarray(s32, dtype=np.float32)
+    safe = np.where(s32 == 0, np.float32(1), s32).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        r = np.rint(np.divide(v32, safe, dtype=np.float32))
+    q = np.clip(r, qmin, qmax)
+    q = np.where(s32 == 0, 0, q)
+    return q.astype(np.int8)
+
+
+def quantize_weights_fp32(Wr32: np.ndarray):
+    """Symmetric per-output-channel RTN of fp32 rotated weights [N, K].
+    s_w[n] = fp32(max_k |W'[n,k]| / 7), codes in [-7, 7]."""
+    Wr32 = np.asarray(Wr32, dtype=np.float32)
+    amax = np.max(np.abs(Wr32), axis=1)
+    s = np.divide(amax, np.float32(WEIGHT_QMAX), dtype=np.float32)
+    q = _rtn_codes(Wr32, s[:, None], -WEIGHT_QMAX, WEIGHT_QMAX)
+    return q, s
+
+
+def quantize_acts_dynamic_fp32(xr32: np.ndarray):
+    """Per-token dynamic RTN of fp32 rotated activations [M, K].
+    s_x[m] = fp32(max_k |x'[m,k]| / 7), codes clamped to [-8, 7]."""
+    xr32 = np.asarray(xr32, dtype=np.float32)
+    amax = np.max(np.abs(xr32), axis=1) if xr32.shape[1] else np.zeros(xr32.shape[0], np.float32)
+    s = np.divide(amax, np.float32(ACT_QMAX), dtype=np.float32)
+    q = _rtn_codes(xr32, s[:, None], ACT_QMIN, ACT_QMAX)
+    return q, s
+
+
+def table_scale(table: np.ndarray, step: int, layer: int) -> np.float32:
+    """Per-step static activation scale: table[step][layer].  A step or layer
+    outside the table is an error, never a clamp ([ES]: a step-count mismatch or
+    a truncated table is a failure mode)."""
+    T, L = table.shape
+    if not (0 <= step < T) or not (0 <= layer < L):
+        raise IndexError("step/layer outside the activation scale table")
+    return np.float32(table[step, layer])
+
+
+def quantize_acts_table_fp32(xr32: np.ndarray, s: np.float32):
+    xr32 = np.asarray(xr32, dtype=np.float32)
+    sv = np.full(xr32.shape[0], s, dtype=np.float32)
+    q = _rtn_codes(xr32, sv[:, None], ACT_QMIN, ACT_QMAX)
+    return q, sv
+
+
+# --------------------------------------------------------------------------
+# Nibble packing, integer GEMM, dequantisation
+# --------------------------------------------------------------------------
+
+def pack_nibbles(q: np.ndarray) -> np.ndarray:
+    """[R, K] int codes in [-8, 7] -> [R, K/2] uint8; code 2j in the low nibble."""
+    q = np.asarray(q, dtype=np.int64)
+    if q.shape[-1] % 2:
+        raise ValueError("K must be even")
+    lo = q[..., 0::2] & 0xF
+    hi = q[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(p: np.ndarray) -> np.ndarray:
+    p = np.asarray(p, dtype=np.int64)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def int_gemm(qx: np.ndarray, qw: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k qx[m, k] * qw[n, k] in int64."""
+    return np.asarray(qx, dtype=np.int64) @ np.asarray(qw, dtype=np.int64).T
+
+
+def dequantize(acc: np.ndarray, s_x: np.ndarray, s_w: np.ndarray, bias=None) -> np.ndarray:
+    """y[m, n] = s_x[m] * s_w[n] * acc[m, n] + b[n] in double."""
+    y = (np.asarray(s_x, np.float64)[:, None] * np.asarray(s_w, np.float64)[None, :]
+         * np.asarray(acc, np.float64))
+    if bias is not None:
+        y = y + np.asarray(bias, np.float64)[None, :]
+    return y
+
+
+# --------------------------------------------------------------------------
+# Whole-layer compositions
+# --------------------------------------------------------------------------
+
+class PackedLinear:
+    """What the offline pack step produces for one linear (all on the host)."""
+
+    def __init__(self, perm, rsvd, R, Wr, qw, s_w, bias):
+        self.perm, self.rsvd, self.R, self.Wr = perm, rsvd, R, Wr
+        self.qw, self.s_w, self.bias = qw, s_w, bias
+
+    @property
+    def wq(self):
+        return pack_nibbles(self.qw)
+
+
+def pack_linear(W: np.ndarray, block: int, bias=None, perm=None, rsvd=None) -> PackedLinear:
+    """Offline pack: zigzag P, per-block R_SVD, R = R_SVD.H, W' = W P R, then RTN
+    of fp32(W').  `perm` / `rsvd` may be given to pin the non-unique parts."""
+    if perm is None:
+        perm = zigzag_permutation(W, block)
+    if rsvd is None:
+        rsvd = svd_rotation_blocks(W, perm, block)
+    R = composite_blocks(rsvd)
+    Wr = rotate_weights(W, perm, R)
+    qw, s_w = quantize_weights_fp32(Wr.astype(np.float32))
+    return PackedLinear(perm, rsvd, R, Wr, qw, s_w, bias)
+
+
+def rotate_quant_act(x: np.ndarray, pk: PackedLinear, mode: str = "dynamic",
+                     table=None, step: int = 0, layer: int = 0):
+    """Activation side in double, quantised like the fp32 path but from the
+    double x' (the end-to-end reference).  Returns (x' double, codes, s_x double)."""
+    xr = rotate_activations(x, pk.perm, pk.R)
+    if mode == "dynamic":
+        s = np.max(np.abs(xr), axis=1) / ACT_QMAX
+    elif mode == "table":
+        s = np.full(xr.shape[0], float(table_scale(table, step, layer)))
+    else:
+        raise ValueError(mode)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.rint(xr / np.where(s == 0, 1.0, s)[:, None])
+    q = np.where((s == 0)[:, None], 0, np.clip(r, ACT_QMIN, ACT_QMAX)).astype(np.int8)
+    return xr, q, s
+
+
+def linear_forward(x, pk: PackedLinear, mode="dynamic", table=None, step=0, layer=0):
+    """End-to-end layer output (double) and the intermediates it used."""
+    xr, qx, s_x = rotate_quant_act(x, pk, mode, table, step, layer)
+    acc = int_gemm(qx, pk.qw)
+    y = dequantize(acc, s_x, pk.s_w, pk.bias)
+    return dict(xr=xr, qx=qx, s_x=s_x, acc=acc, y=y)

@@ -1,0 +1,337 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+Each check compares the oracle with something other than itself: hand-worked
+fixtures under tests/golden/, closed forms, invariants, a different LAPACK
+routine (SVD instead of the oracle's symmetric eigensolver), and brute force
+with dense K x K matrices and scalar loops on tiny shapes.  The planted-mistake
+test at the end shows that a plausible bug in each oracle stage trips a pin.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import qvla_oracle as O
+from w4a4_post_quantization_zigzag_b200 import inputs as I
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- Hadamard
+
+def test_hadamard_golden_order4():
+    g = gold("hadamard4.json")
+    np.testing.assert_array_equal(O.hadamard(4) * 2.0, np.array(g["H_times_sqrt_b"], float))
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8, 32, 64, 128, 256])
+def test_hadamard_orthonormal_symmetric(b):
+    H = O.hadamard(b)
+    assert np.abs(H @ H.T - np.eye(b)).max() <= 1e-14
+    assert np.array_equal(H, H.T)
+    assert np.allclose(np.abs(H), 1 / np.sqrt(b), rtol=0, atol=1e-16)
+    # Sylvester recursion H_2b = [[H_b, H_b], [H_b, -H_b]] / sqrt(2)
+    if b >= 2:
+        h = O.hadamard(b // 2)
+        rec = np.block([[h, h], [h, -h]]) / np.sqrt(2)
+        assert np.abs(rec - H).max() <= 1e-15
+
+
+def test_hadamard_rejects_non_power_of_two():
+    with pytest.raises(ValueError):
+        O.hadamard(24)
+
+
+# ------------------------------------------------------------------- zigzag
+
+@pytest.mark.parametrize("case", gold("zigzag_cases.json")["cases"])
+def test_zigzag_golden(case):
+    W = np.array(case["W"], float)
+    perm = O.zigzag_permutation(W, case["block"])
+    assert perm.tolist() == case["perm"]
+    c = O.column_norms(W)
+    b = case["block"]
+    sums = [float(c[perm[B * b:(B + 1) * b]].sum()) for B in range(W.shape[1] // b)]
+    assert np.allclose(sums, case["block_norm_sums"])
+
+
+def _ranks(W):
+    c = O.column_norms(W)
+    order = sorted(range(W.shape[1]), key=lambda k: (-c[k], k))
+    rank = np.empty(W.shape[1], int)
+    rank[order] = np.arange(W.shape[1])
+    return c, rank
+
+
+@pytest.mark.parametrize("K,b", [(256, 64), (1024, 64), (2048, 128), (512, 32), (512, 256)])
+def test_zigzag_structure(K, b):
+    W = I.weights(7 + K + b, 64, K, col_spread=30.0)
+    perm = O.zigzag_permutation(W, b)
+    assert sorted(perm.tolist()) == list(range(K))           # a permutation
+    c, rank = _ranks(W)
+    nb = K // b
+    for B in range(nb):
+        for pos in range(b):
+            r = rank[perm[B * b + pos]]
+            # position `pos` of every block holds a channel of stratum `pos`
+            assert r // nb == pos
+            # snake: even strata run left to right, odd strata right to left
+            want = B if pos % 2 == 0 else nb - 1 - B
+            assert r % nb == want
+    sums = np.array([c[perm[B * b:(B + 1) * b]].sum() for B in range(nb)])
+    # balance: the spread of block norm sums never exceeds c_max - c_min
+    assert sums.max() - sums.min() <= c.max() - c.min() + 1e-12
+
+
+# ------------------------------------------------------------------ R_SVD
+
+@pytest.mark.parametrize("N,K,b", [(256, 256, 64), (96, 128, 32), (300, 256, 128), (512, 256, 256)])
+def test_rsvd_against_library_svd(N, K, b):
+    W = I.weights(11 + N + K, N, K, n_outlier_rows=3, col_spread=10.0).astype(np.float64)
+    perm = O.zigzag_permutation(W, b)
+    rs = O.svd_rotation_blocks(W, perm, b)
+    for B in range(K // b):
+        V = rs[B]
+        assert np.abs(V.T @ V - np.eye(b)).max() <= 1e-12      # R_SVD^T R_SVD = I
+        A = W[:, perm[B * b:(B + 1) * b]]
+        AV = A @ V
+        sv = np.linalg.svd(A, compute_uv=False)                 # a different LAPACK routine
+        norms = np.linalg.norm(AV, axis=0)
+        # each rotated channel carries one singular value's energy, descending
+        assert np.allclose(norms, sv, rtol=1e-10, atol=1e-12 * sv[0])
+        gram = AV.T @ AV
+        off = gram - np.diag(np.diag(gram))
+        assert np.abs(off).max() <= 1e-10 * sv[0] ** 2          # columns orthogonal
+        # canonical sign: largest-magnitude entry of every column is positive
+        idx = np.argmax(np.abs(V), axis=0)
+        assert np.all(V[idx, np.arange(b)] > 0)
+
+
+@pytest.mark.parametrize("N,K,b", [(256, 256, 64), (128, 256, 128), (64, 64, 32)])
+def test_composite_equalises_channel_energy(N, K, b):
+    """Columns of A_B R_SVD H all have squared norm ||A_B||_F^2 / b (closed form:
+    A_B R_SVD = U S with orthonormal U, and every H entry squared is 1/b)."""
+    W = I.weights(23 + K, N, K, n_outlier_rows=3, row_scale=15.0, col_spread=30.0).astype(np.float64)
+    perm = O.zigzag_permutation(W, b)
+    R = O.composite_blocks(O.svd_rotation_blocks(W, perm, b))
+    for B in range(K // b):
+        A = W[:, perm[B * b:(B + 1) * b]]
+        assert np.abs(R[B].T @ R[B] - np.eye(b)).max() <= 1e-12
+        n2 = np.sum((A @ R[B]) ** 2, axis=0)
+        target = np.sum(A * A) / b
+        assert np.allclose(n2, target, rtol=1e-10)
+
+
+def test_rotation_preserves_the_product():
+    """(W P R)(R^T P^T x) = W x before quantisation, within 1e-9 relative."""
+    wl = I.single_linear()
+    lin = wl.linears[0]
+    W, x = lin.make_w().astype(np.float64), lin.make_x().astype(np.float64)
+    pk = O.pack_linear(W, lin.block)
+    xr = O.rotate_activations(x, pk.perm, pk.R)
+    ref = x @ W.T
+    got = xr @ pk.Wr.T
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-9
+
+
+# ------------------------------------------------ dense brute force (tiny)
+
+def _dense_P(perm):
+    K = len(perm)
+    P = np.zeros((K, K))
+    P[perm, np.arange(K)] = 1.0          # (W P)[:, j] = W[:, perm[j]]
+    return P
+
+
+def _dense_R(Rb):
+    nb, b, _ = Rb.shape
+    R = np.zeros((nb * b, nb * b))
+    for B in range(nb):
+        R[B * b:(B + 1) * b, B * b:(B + 1) * b] = Rb[B]
+    return R
+
+
+@pytest.mark.parametrize("M,N,K,b,seed", [(1, 4, 8, 4, 0), (3, 4, 16, 4, 1), (2, 3, 16, 8, 2),
+                                          (3, 4, 16, 8, 3)])
+def test_tiny_pipeline_against_dense_matrices(M, N, K, b, seed):
+    W = I.weights(seed, N, K, std=1.0).astype(np.float64)
+    x = I.activations(seed + 50, M, K, dtype="f32").astype(np.float64)
+    pk = O.pack_linear(W, b)
+    P, R = _dense_P(pk.perm), _dense_R(pk.R)
+    assert np.abs(P @ P.T - np.eye(K)).max() == 0
+    assert np.abs(R.T @ R - np.eye(K)).max() <= 1e-12
+    np.testing.assert_allclose(pk.Wr, W @ P @ R, rtol=0, atol=1e-12)
+    xr = O.rotate_activations(x, pk.perm, pk.R)
+    np.testing.assert_allclose(xr, (R.T @ P.T @ x.T).T, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------- RTN
+
+def test_rtn_golden_scalars():
+    g = gold("rtn_cases.json")
+    for c in g["activation_cases"]:
+        q, _ = O.quantize_acts_table_fp32(np.array([[c["v"]]], np.float32), np.float32(c["s"]))
+        assert int(q[0, 0]) == c["q"], c
+    for c in g["weight_cases"]:
+        q = O._rtn_codes(np.float32(c["v"]), np.float32(c["s"]), -7, 7)
+        assert int(q) == c["q"], c
+
+
+def test_rtn_golden_rows():
+    g = gold("rtn_cases.json")
+    for c in g["dynamic_rows"]:
+        q, s = O.quantize_acts_dynamic_fp32(np.array([c["x"]], np.float32))
+        assert float(s[0]) == c["s"] and q[0].tolist() == c["q"]
+    for c in g["weight_rows"]:
+        q, s = O.quantize_weights_fp32(np.array([c["w"]], np.float32))
+        assert int(s.view(np.uint32)[0]) == int(c["s_f32_hex"], 16)
+        assert q[0].tolist() == c["q"]
+
+
+def _brute_rtn(v, s, lo, hi):
+    """Scalar loop: fp32 quotient, then ties-to-even by hand."""
+    if s == 0:
+        return 0
+    t = float(np.float32(v) / np.float32(s))
+    f = np.floor(t)
+    d = t - f
+    r = f + 1 if d > 0.5 else f if d < 0.5 else (f if f % 2 == 0 else f + 1)
+    return int(min(max(r, lo), hi))
+
+
+def test_rtn_brute_force_and_ranges():
+    x = I.activations(5, 6, 64, n_outlier_cols=2, dtype="f32")
+    q, s = O.quantize_acts_dynamic_fp32(x)
+    for m in range(x.shape[0]):
+        assert s[m] == np.float32(np.float32(np.abs(x[m]).max()) / np.float32(7))
+        for k in range(x.shape[1]):
+            assert q[m, k] == _brute_rtn(x[m, k], s[m], -8, 7)
+    assert q.min() >= -8 and q.max() <= 7
+    W = I.weights(6, 8, 64, n_outlier_rows=2)
+    W[3] = 0.0
+    qw, sw = O.quantize_weights_fp32(W)
+    assert qw.min() >= -7 and qw.max() <= 7
+    for n in range(W.shape[0]):
+        if sw[n] == 0:
+            assert not qw[n].any()
+        else:
+            assert np.abs(qw[n]).max() == 7          # the row max always lands on +-7
+        for k in range(W.shape[1]):
+            assert qw[n, k] == _brute_rtn(W[n, k], sw[n], -7, 7)
+
+
+def test_table_lookup_rejects_out_of_range():
+    tab = np.ones((8, 3), np.float32)
+    assert O.table_scale(tab, 7, 2) == 1.0
+    for t, l in [(8, 0), (-1, 0), (0, 3)]:
+        with pytest.raises(IndexError):
+            O.table_scale(tab, t, l)
+
+
+# -------------------------------------------------------- pack / GEMM / dequant
+
+@pytest.mark.parametrize("case", gold("pack_cases.json")["cases"])
+def test_pack_golden(case):
+    assert O.pack_nibbles(np.array([case["q"]])).tolist() == [case["bytes"]]
+
+
+def test_pack_roundtrip_all_bytes():
+    b = np.arange(256, dtype=np.uint8)[None, :]
+    q = O.unpack_nibbles(b)
+    assert q.min() == -8 and q.max() == 7
+    assert np.array_equal(O.pack_nibbles(q), b)
+
+
+def test_int_gemm_brute_force():
+    qx = I.int_codes(1, 3, 24, -8, 7)
+    qw = I.int_codes(2, 5, 24, -7, 7)
+    acc = O.int_gemm(qx, qw)
+    for m in range(3):
+        for n in range(5):
+            assert acc[m, n] == sum(int(qx[m, k]) * int(qw[n, k]) for k in range(24))
+    # extreme magnitudes stay far inside int32 at the largest K in use
+    K = 16384
+    assert 8 * 7 * K < 2 ** 31
+
+
+def test_dequant_brute_force():
+    acc = np.array([[3, -2], [0, 7]])
+    sx, sw, b = np.array([0.5, 2.0]), np.array([0.25, 1.0]), np.array([0.1, -0.1])
+    y = O.dequantize(acc, sx, sw, b)
+    want = [[0.5 * 0.25 * 3 + 0.1, 0.5 * 1.0 * -2 - 0.1], [0.1, 2.0 * 7 - 0.1]]
+    np.testing.assert_allclose(y, want, rtol=0, atol=1e-15)
+
+
+def test_end_to_end_quantised_layer_is_close_to_fp_layer():
+    """Sanity: the rotated W4A4 layer approximates the fp layer (what the method
+    is for); rotation must beat no rotation on outlier-heavy inputs."""
+    wl = I.single_linear()
+    lin = wl.linears[0]
+    W, x, bb = lin.make_w(), lin.make_x(), lin.make_bias()
+    pk = O.pack_linear(W, lin.block, bias=bb)
+    out = O.linear_forward(x, pk)
+    ref = x.astype(np.float64) @ W.T.astype(np.float64) + bb
+    err_rot = np.linalg.norm(out["y"] - ref) / np.linalg.norm(ref)
+    # the same RTN without any rotation
+    qw, sw = O.quantize_weights_fp32(W)
+    qx, sx = O.quantize_acts_dynamic_fp32(x)
+    y0 = O.dequantize(O.int_gemm(qx, qw), sx, sw, bb)
+    err_plain = np.linalg.norm(y0 - ref) / np.linalg.norm(ref)
+    assert err_rot < err_plain
+
+
+# ------------------------------------------------------ planted mistakes
+
+def test_pins_catch_planted_mistakes():
+    """Plant a plausible bug in each oracle stage and show a pin fails."""
+    W = I.weights(3, 128, 256, n_outlier_rows=3, col_spread=30.0).astype(np.float64)
+    b = 64
+
+    def composite_equal_norms(Rfun):
+        perm = O.zigzag_permutation(W, b)
+        R = Rfun(O.svd_rotation_blocks(W, perm, b))
+        A = W[:, perm[:b]]
+        n2 = np.sum((A @ R[0]) ** 2, axis=0)
+        return np.allclose(n2, np.sum(A * A) / b, rtol=1e-10)
+
+    assert composite_equal_norms(O.composite_blocks)
+    # H applied on the wrong side (H . R_SVD instead of R_SVD . H)
+    assert not composite_equal_norms(lambda rs: np.stack([O.hadamard(b) @ r for r in rs]))
+    # R_SVD transposed
+    assert not composite_equal_norms(lambda rs: np.stack([r.T @ O.hadamard(b) for r in rs]))
+
+    # zigzag without the snake (plain round robin) breaks the golden case
+    case = gold("zigzag_cases.json")["cases"][0]
+    orig = O.zigzag_permutation
+
+    def round_robin(Wm, block):
+        K = Wm.shape[1]
+        nb = K // block
+        c = O.column_norms(Wm)
+        order = sorted(range(K), key=lambda k: (-c[k], k))
+        perm = np.empty(K, int)
+        for r, ch in enumerate(order):
+            perm[(r % nb) * block + r // nb] = ch
+        return perm
+    assert round_robin(np.array(case["W"], float), case["block"]).tolist() != case["perm"]
+    assert orig(np.array(case["W"], float), case["block"]).tolist() == case["perm"]
+
+    # Hadamard without its 1/sqrt(b) normalisation fails orthonormality
+    Hn = O.hadamard(8) * np.sqrt(8)
+    assert np.abs(Hn @ Hn.T - np.eye(8)).max() > 1e-3
+
+    # double instead of fp32 division changes a golden RTN code
+    v, s = np.float32(-3.0), np.float32(0.4)
+    assert int(np.clip(np.rint(float(v) / float(s)), -8, 7)) != -8
+    assert int(O._rtn_codes(v, s, -8, 7)) == -8
+
+    # swapped nibble order fails the 0x78 pin
+    q = np.array([[-8, 7]])
+    swapped = ((q[:, 1::2] & 0xF) | ((q[:, 0::2] & 0xF) << 4)).astype(np.uint8)
+    assert swapped.tolist() != [[0x78]] and O.pack_nibbles(q).tolist() == [[0x78]]
