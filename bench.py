@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated W4A4 linear layer on B200.
+
+Default workload: the DiT action-head MLP stack (50 action tokens x batch 1,
+hidden 1024, gate/up 1024->4096 and down 4096->1024, 4 layers, bf16 input,
+10 denoising steps, per-step scale table [10][12], rotation block 64).
+One timed step = one denoising step = 12 rotated W4A4 linears, each a fused
+rotate-quantise launch plus a W4A4 GEMM launch, replayed from a CUDA graph.
+The activation step index is a device scalar read by the rotate-quantise
+kernel.  L2 is flushed (512 MB write) before every timed step, so every step
+streams its packed weights from HBM.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on the
+same workload instead (the reference arm).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from w4a4_post_quantization_zigzag_b200 import inputs as I  # noqa: E402
+
+METRIC = "µs per DiT denoise step"
+UNIT = "us/step"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="dit_mlp_stack",
+                   choices=["dit_mlp_stack", "dit_denoise_loop", "backbone_prefill",
+                            "single_linear"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-steps", type=int, default=0,
+                   help="oracle steps for the CPU baseline (0: sized to ~15 s)")
+    p.add_argument("--quick", action="store_true",
+                   help="skip clocks, e2e and the CPU baseline (for profiler runs)")
+    return p.parse_args()
+
+
+def make_workload(name):
+    return {"dit_mlp_stack": I.dit_mlp_stack, "dit_denoise_loop": I.dit_denoise_loop,
+            "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.strip()]
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ traffic record
+def recorded_traffic(kernel, workload):
+    """dram bytes per launch from a committed ncu summary, only while the kernel
+    source is unchanged since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(f"{kernel}:{workload}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "w4a4_post_quantization_zigzag_b200", "csrc", rec["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+            return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_step(wl, packs, xs, t):
+    from oracle import qvla_oracle as O
+    out = []
+    for lin, pk, x in zip(wl.linears, packs, xs[t]):
+        if wl.mode == "table":
+            r = O.linear_forward(x, pk, "table", wl.table, t, lin.layer)
+        else:
+            r = O.linear_forward(x, pk)
+        out.append(r["y"])
+    return out
+
+
+def oracle_setup(wl, steps):
+    from oracle import qvla_oracle as O
+    packs = [O.pack_linear(l.make_w(), l.block, bias=l.make_bias()) for l in wl.linears]
+    xs = [[l.make_x(seed_offset=t, std=(float(wl.sigmas[t]) if wl.sigmas is not None else None))
+           for l in wl.linears] for t in range(steps)]
+    return packs, xs
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl, sample_steps):
+    T = max(1, wl.steps)
+    packs, xs = oracle_setup(wl, min(T, max(1, sample_steps)))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(wl, packs, xs, n % len(xs))
+        n += 1
+        el = time.perf_counter() - t0
+        if (sample_steps and n >= sample_steps) or (not sample_steps and (el > 12.0 or n >= 50)):
+            break
+    us = el / n * 1e6
+    return {"value": us, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full denoise step(s) of {wl.name} ({len(wl.linears)} linears each); "
+                      f"numpy fp64 rotation, fp32 RTN, int64 GEMM, fp64 dequant"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = make_workload(args.workload)
+    packs, xs = oracle_setup(wl, min(max(1, wl.steps), 2))
+    for i in range(args.warmup):
+        oracle_step(wl, packs, xs, i % len(xs))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(wl, packs, xs, i % len(xs))
+    el = time.perf_counter() - t0
+    us = el / args.steps * 1e6
+    line = {"impl": "reference", "metric": METRIC, "value": us, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name},
+            "cpu_baseline": {"value": us, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: one full denoise step of {wl.name}"},
+            "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from w4a4_post_quantization_zigzag_b200 import build as B
+    B.build()
+    from w4a4_post_quantization_zigzag_b200 import qvla as Q
+
+    wl = make_workload(args.workload)
+    T = max(1, wl.steps)
+    table = torch.from_numpy(wl.table).to(dev) if wl.table is not None else None
+    steps_dev = torch.arange(T, dtype=torch.int32, device=dev)
+    mode = Q.QVLA_SCALE_TABLE if wl.mode == "table" else Q.QVLA_SCALE_DYNAMIC
+
+    # pack (offline step, timed for information)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    packs = []
+    for lin in wl.linears:
+        W = torch.from_numpy(lin.make_w()).to(dev)
+        packs.append(Q.qvla_pack_weights(W, lin.block, bias=torch.from_numpy(lin.make_bias()).to(dev)))
+        del W
+    torch.cuda.synchronize()
+    pack_s = time.perf_counter() - t0
+
+    # per-step inputs (device resident) and outputs
+    xdt = torch.bfloat16 if wl.linears[0].x_dtype == "bf16" else torch.float32
+    xs_host = [[torch.from_numpy(l.make_x(seed_offset=t, std=(float(wl.sigmas[t])
+                                                              if wl.sigmas is not None else None)))
+                .to(xdt).pin_memory() for l in wl.linears] for t in range(T)]
+    xs = [[x.to(dev) for x in row] for row in xs_host]
+    xq = [torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev) for l in wl.linears]
+    sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
+    ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
+
+    def step(t, rec=None):
+        for i, (lin, L) in enumerate(zip(wl.linears, packs)):
+            if rec is not None:
+                rec[i][0].record()
+            Q.qvla_rotate_quant_act(xs[t][i], L, mode, table=table, step=steps_dev[t:t + 1],
+                                    layer=lin.layer, xq=xq[i], s_x=sx[i])
+            if rec is not None:
+                rec[i][1].record()
+            Q.qvla_w4a4_gemm(xq[i], sx[i], L, y=ys[i])
+            if rec is not None:
+                rec[i][2].record()
+
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        step(0)                       # first call resolves attributes outside capture
+        torch.cuda.synchronize()
+        graphs = []
+        for t in range(T):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(t)
+            graphs.append(g)
+    torch.cuda.synchronize()
+    assert Q.qvla_read_error_word(clear=True) == 0
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    # ---- warm-up
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            flush.zero_()
+            graphs[i % T].replay()
+    # ---- timed steps: graph replay, L2 flushed before each
+    starts = [ev() for _ in range(args.steps)]
+    ends = [ev() for _ in range(args.steps)]
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_uuid) if not args.quick else None
+    barrier()
+    if sampler:
+        sampler.__enter__()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record()
+            graphs[i % T].replay()
+            ends[i].record()
+    barrier()
+    if sampler:
+        sampler.__exit__()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    tot_ms = sum(per_step_ms)
+    if world > 1:
+        tt = torch.tensor([tot_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        tot_ms = float(tt.item())
+    ms_per_step = tot_ms / args.steps
+    us_job = tot_ms * 1e3 / (args.steps * world)
+
+    # ---- per-kernel breakdown (eager launches, events on the launching stream)
+    nl = len(wl.linears)
+    krot, kgemm = [], []
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            rec = [[ev(), ev(), ev()] for _ in range(nl)]
+            flush.zero_()
+            step(i % T, rec)
+            stream.synchronize()
+            for j in range(nl):
+                krot.append((j, rec[j][0].elapsed_time(rec[j][1])))
+                kgemm.append((j, rec[j][1].elapsed_time(rec[j][2])))
+    assert Q.qvla_read_error_word(clear=True) == 0
+
+    # ---- end to end: pinned-host inputs in, outputs back, every step
+    e2e = None
+    if not args.quick:
+        y_host = [torch.empty(l.M, l.N, dtype=torch.bfloat16).pin_memory() for l in wl.linears]
+        h2d = sum(x.numel() * x.element_size() for x in xs_host[0])
+        d2h = sum(y.numel() * y.element_size() for y in y_host)
+        e0, e1 = ev(), ev()
+        barrier()
+        with torch.cuda.stream(stream):
+            e0.record()
+            for i in range(args.steps):
+                t = i % T
+                for x_d, x_h in zip(xs[t], xs_host[t]):
+                    x_d.copy_(x_h, non_blocking=True)
+                graphs[t].replay()
+                for y_d, y_h in zip(ys, y_host):
+                    y_h.copy_(y_d, non_blocking=True)
+            e1.record()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": e2e_ms * 1e3 / (args.steps * world), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- roofline of the dominant kernel
+    hbm, bf16_tf, peak_src = load_peaks()
+    gemm_bytes = sum(l.N * l.K // 2 + l.M * l.K // 2 + 2 * l.M * l.N + 4 * l.M + 8 * l.N
+                     for l in wl.linears)
+    rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + l.M * l.K // 2 + 4 * l.M
+                    + 4 * l.K * l.block + 4 * l.K for l in wl.linears)
+    t_gemm = sum(t for _, t in kgemm) / args.steps          # ms per step
+    t_rot = sum(t for _, t in krot) / args.steps
+    dom = "w4a4_gemm" if t_gemm >= t_rot else "rotate_quant"
+    if dom == "w4a4_gemm":
+        per_launch_bytes, per_launch_ms = gemm_bytes / nl, t_gemm / nl
+    else:
+        per_launch_bytes, per_launch_ms = rot_bytes / nl, t_rot / nl
+    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "peak_source": f"hbm_gbs ({peak_src})",
+            "traffic": recorded_traffic(dom, wl.name),
+            "algorithmic_bytes_per_launch": per_launch_bytes,
+            "avg_launch_us": per_launch_ms * 1e3}
+
+    ops = wl.ops_per_step()
+    line = {
+        "metric": METRIC, "value": us_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens_M": wl.linears[0].M,
+                   "linears_per_step": nl, "denoise_steps_T": T,
+                   "block": wl.linears[0].block, "scale": wl.mode,
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single"},
+        "roofline": roof,
+        "tops": ops / (ms_per_step * 1e-3) / 1e12,
+        "weight_gbs": wl.packed_weight_bytes() / (ms_per_step * 1e-3) / 1e9,
+        "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3,
+                                "eager_sum": (t_rot + t_gemm) * 1e3},
+        "pack_s": pack_s,
+        "gpu_launches": 2 * nl * args.steps,
+        "e2e": e2e,
+    }
+    if sampler:
+        line["clocks"] = sampler.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_steps)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+/*
+ * qvla.h -- C ABI of the B200 (sm_100a) rotated W4A4 linear layer.
+ *
+ *     y = s_x * s_w * ( q(R^T P^T x) . q(W P R)^T ) + b
+ *
+ * The method is Omega-QVLA's composite SVD.Hadamard rotation with a zigzag
+ * channel permutation and per-step activation scaling.  Sources cited below:
+ *  [PT]/[FR] "{Omega}-QVLA: Robust Quantization for Vision-Language-Action
+ *           Models via Composite Rotation and Per-step Scaling", Portuguese
+ *           and French technical summaries (gist.science), Methodology 1
+ *           (composite SVD.Hadamard rotation, block implementation with the
+ *           zigzag permutation) and 2 (per-step DiT activation scaling).
+ *  [VN]     "Omega-QVLA: Nen VLA W4A4 tren Edge" (vnrobo.com), sections
+ *           "Y tuong paper" (act_scale_table looked up per denoising step)
+ *           and "Build DiT action head pack" (--use-rtn, --w-bits 4,
+ *           --a-bits 4, --duquant-block-size 64).
+ *  [ES]     "Omega-QVLA Reduce el Modelo ..." (aiexpert.news): a step-count
+ *           mismatch or truncated table is a failure mode.
+ *  [FQ]     "FoldQuantVLA: Native Low-Bit Quantization of VLA Models via
+ *           Consistent Folding" (radar.vhtltd.com): dynamic per-token
+ *           activation quantisation, native integer W4A4 execution.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layouts follow PyTorch Linear: W is [N][K] (out x in) row-major fp32;
+ *    x is [M][ldx] row-major (bf16 or fp32); y is [M][ldy] row-major bf16.
+ *  - `block` (b) is the rotation block: 32, 64, 128 or 256; K % b == 0;
+ *    nb = K / b.  K <= QVLA_MAX_K.
+ *  - perm[j] is the ORIGINAL input channel placed at permuted position j,
+ *    so (P^T x)[j] = x[perm[j]].
+ *  - rot holds the R_SVD blocks, fp32 [nb][b][b]: rot[B][i][j] is row i,
+ *    column j of R_SVD of block B.  The composite block rotation is
+ *    R_B = R_SVD,B . H_b with H_b the Sylvester Hadamard matrix of order b
+ *    scaled by 1/sqrt(b); H is never stored.
+ *  - Packed 4-bit codes: byte j of a row holds code 2j in its low nibble and
+ *    code 2j+1 in its high nibble, 4-bit two's complement.  Weight codes lie
+ *    in [-7, 7], activation codes in [-8, 7].
+ *  - Rounding: the division that decides a code is an IEEE fp32 division of
+ *    fp32 operands, rounded to nearest with ties to even; a zero scale gives
+ *    all-zero codes.
+ *  - Memory: the caller allocates every buffer.  Pointers documented as
+ *    "device" must be device memory of the current CUDA device; "host"
+ *    pointers are ordinary host memory.  No entry point keeps a pointer
+ *    after it returns (kernels still in flight read them).
+ *  - Streams: work is enqueued on `stream` (0 = legacy default stream) and
+ *    runs asynchronously unless an entry point says otherwise.  The return
+ *    status covers argument validation and launch errors only; errors found
+ *    by a kernel while it runs set bits of the device error word, read with
+ *    qvla_read_error_word().
+ *  - Alignment: every device pointer must be 16-byte aligned and every row
+ *    pitch a multiple of 16 bytes, or QVLA_ERR_ALIGN is returned.
+ *  - Nothing is done and QVLA_OK is returned when M == 0.
+ */
+#ifndef QVLA_H_
+#define QVLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QVLA_ABI_VERSION 1
+#define QVLA_MAX_K 32768
+
+typedef enum {
+  QVLA_OK = 0,
+  QVLA_ERR_ARG = 1,          /* null pointer or invalid enum value            */
+  QVLA_ERR_SHAPE = 2,        /* sizes outside the supported set               */
+  QVLA_ERR_ALIGN = 3,        /* pointer or pitch not 16-byte aligned          */
+  QVLA_ERR_STEP_RANGE = 4,   /* denoising step or layer outside the table     */
+  QVLA_ERR_UNSUPPORTED = 5,  /* device is not sm_100 or feature unavailable   */
+  QVLA_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed          */
+  QVLA_ERR_DEVICE_FLAG = 7,  /* the device error word was non-zero            */
+  QVLA_ERR_WORKSPACE = 8     /* workspace missing or too small                */
+} qvla_status;
+
+typedef enum { QVLA_DTYPE_F32 = 0, QVLA_DTYPE_BF16 = 1 } qvla_dtype;
+
+/* Activation scale selection ([PT]/[FR] Methodology 2; [FQ]):
+ *   DYNAMIC: s_x[m] = fp32(max_k |x'[m,k]| / 7), per token.
+ *   TABLE:   s_x[m] = table[step][layer] for every token (the per-step
+ *            activation scale table of the DiT action head).            */
+typedef enum { QVLA_SCALE_DYNAMIC = 0, QVLA_SCALE_TABLE = 1 } qvla_scale_mode;
+
+/* Bits of the device error word. */
+#define QVLA_DEVERR_STEP_RANGE 0x1u   /* device step index outside [0, T)    */
+#define QVLA_DEVERR_TIMEOUT 0x2u      /* a bounded wait in a kernel expired  */
+#define QVLA_DEVERR_TMEM 0x4u         /* tensor-memory allocation failed     */
+
+/* One packed linear: what qvla_pack_weights() produces.  All pointers are
+ * device pointers owned by the caller.                                     */
+typedef struct {
+  int32_t N, K, block;
+  const int32_t* perm;      /* [K]  zigzag permutation                      */
+  const float* rot;         /* [nb][b][b] R_SVD blocks                      */
+  const uint8_t* wq;        /* [N][K/2] packed weight codes                 */
+  const float* w_scale;     /* [N]  s_w                                      */
+  const float* bias;        /* [N]  or NULL                                  */
+} qvla_packed_linear;
+
+const char* qvla_status_str(qvla_status s);
+int qvla_abi_version(void);
+
+/* Reads the current device's error word into *out and, if clear != 0, resets
+ * it to 0.  Synchronises the device.  Returns QVLA_ERR_CUDA on a CUDA error. */
+qvla_status qvla_read_error_word(uint32_t* out, int clear);
+
+/* Byte sizes of the buffers a packed linear needs:
+ *   *wq_bytes   = N * K / 2
+ *   *rot_bytes  = 4 * K * block
+ *   *ws_bytes   = workspace of qvla_pack_weights().                         */
+qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t* rot_bytes,
+                              size_t* ws_bytes);
+
+/* ---------------------------------------------------------------------------
+ * Offline pack ([PT]/[FR] Methodology 1: zigzag permutation by weight-column
+ * norm, per-block R_SVD, normalised Hadamard, R = R_SVD . H; [VN] "Build DiT
+ * action head pack": RTN, 4-bit weights, block 64).
+ *
+ * W        device fp32 [N][K].
+ * perm_in  host int32 [K] or NULL.  NULL: the zigzag permutation is computed
+ *          (column L2 norms in fp64 on the device, sorted descending with
+ *          ties to the lower index, dealt to blocks in snake order).
+ * rsvd_in  host fp64 [nb][b][b] or NULL.  NULL: each
+ *          block's Gram matrix A_B^T A_B is formed in fp64 on the device, its
+ *          eigenvectors are found on the host (cyclic Jacobi, fp64), ordered
+ *          by descending eigenvalue with the largest-magnitude entry of each
+ *          made positive.
+ * Outputs (device): perm_out [K], rot_out [nb][b][b] fp32, wq_out [N][K/2],
+ *          w_scale_out [N].  W' = W P R is formed in fp64 and
+ *          rounded once to fp32 before RTN.
+ * workspace device, >= ws_bytes from qvla_packed_sizes().
+ * Blocks the calling thread: the stream is synchronised twice (after the
+ * norms and after the Gram matrices) for the host-side sort and eigensolve.
+ * ------------------------------------------------------------------------- */
+qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
+                              const double* rsvd_in, int32_t* perm_out, float* rot_out,
+                              uint8_t* wq_out, float* w_scale_out, void* workspace,
+                              size_t ws_bytes, cudaStream_t stream);
+
+/* Device step of the pack: W'_f32 = fp32(W P R), computed in fp64 from fp64
+ * R_SVD blocks.  W device fp32 [N][K]; perm device [K]; rsvd64 device fp64
+ * [nb][b][b]; Wr_out device fp32 [N][K].  Asynchronous.                    */
+qvla_status qvla_rotate_weights_f32(const float* W, int N, int K, int block, const int32_t* perm,
+                                    const double* rsvd64, float* Wr_out, cudaStream_t stream);
+
+/* Device step of the pack: RTN + nibble packing of fp32 rotated weights.
+ * s_w[n] = fp32(max_k |W'[n,k]| / 7); q = clamp(rint(W'/s_w), -7, 7).
+ * Asynchronous.                                                            */
+qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* wq_out,
+                                        float* w_scale_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Run-time activation rotate + quantise: one fused kernel per token tile.
+ * For each token row m: gather x[m, perm[j]], apply R_SVD,B^T per block,
+ * then the fast Walsh-Hadamard transform (scaled by 1/sqrt(b)), select the
+ * scale (DYNAMIC or TABLE), round to 4-bit codes and nibble-pack them.
+ *
+ * x       device, [M][ldx] of `xdt` (ldx >= K, in elements).
+ * L       host pointer to a packed linear (device pointers inside); only
+ *         perm, rot, K and block are read.
+ * table   device fp32 [T][Lcount], required for TABLE mode.
+ * step_dev device int32 or NULL.  If non-NULL the step is read on the device
+ *         (so one captured graph serves every denoising step); a step outside
+ *         [0, T) sets QVLA_DEVERR_STEP_RANGE and the kernel writes all-zero
+ *         codes and s_x = 0 (y becomes the bias) rather than reading outside
+ *         the table ([ES]).  If NULL, `step_host` is used and checked on the
+ *         host (QVLA_ERR_STEP_RANGE).
+ * layer   column of the table; 0 <= layer < Lcount (checked on the host).
+ * Outputs (device): xq [M][K/2] packed codes, s_x [M] fp32.
+ * ------------------------------------------------------------------------- */
+qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
+                                  const qvla_packed_linear* L, qvla_scale_mode mode,
+                                  const float* table, int T, int Lcount, const int32_t* step_dev,
+                                  int step_host, int layer, uint8_t* xq, float* s_x,
+                                  cudaStream_t stream);
+
+/* The rotation alone, for parity checks: xr_out device fp32 [M][K] = the
+ * same fp32 x' the fused kernel quantises.                                  */
+qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
+                                const qvla_packed_linear* L, float* xr_out, cudaStream_t stream);
+
+/* The quantiser alone, from fp32 rotated activations xr [M][K] (device):
+ * identical scale selection, rounding and packing as the fused kernel.     */
+qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mode,
+                               const float* table, int T, int Lcount, const int32_t* step_dev,
+                               int step_host, int layer, uint8_t* xq, float* s_x,
+                               cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * W4A4 GEMM with fused dequantisation:
+ *   acc[m,n] = sum_k q_x[m,k] q_w[n,k]            (exact, int32)
+ *   y[m,n]   = bf16( fp32(s_x[m] * s_w[n]) * fp32(acc) + b[n] )
+ * int4 codes are unpacked to 8-bit in shared memory and multiplied on the
+ * tcgen05 tensor cores (kind::i8, int32 accumulators in tensor memory).
+ * Each code q is unpacked as the int8 value 16*q (a nibble moved into the
+ * high half of its byte), so the tensor cores accumulate 256*acc exactly
+ * (|256*acc| <= 256*64*K < 2^31 for K <= QVLA_MAX_K) and the epilogue
+ * shifts it back.
+ * Small M uses split-K over a thread-block cluster with the partial sums
+ * reduced through distributed shared memory (no workspace).
+ * xq device [M][K/2]; s_x device [M]; y device bf16 [M][ldy].
+ * split_k: 0 = automatic, else 1, 2, 4, 8 or 16, at most ceil(K / 256)
+ * (K is consumed in 256-wide tiles; split s takes a contiguous run of them).
+ * N may be any positive size; ragged M, N and K tails are zero-filled.      */
+qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
+                           const qvla_packed_linear* L, void* y, int ldy, int split_k,
+                           cudaStream_t stream);
+
+/* Same GEMM, writing the raw int32 accumulators acc [M][N] (device) instead
+ * of y, for bit-exact parity checks.                                        */
+qvla_status qvla_w4a4_gemm_s32(const uint8_t* xq, int M, const qvla_packed_linear* L,
+                               int32_t* acc, int split_k, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QVLA_H_ */

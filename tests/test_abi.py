@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/qvla.h declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib_mod():
+    from w4a4_post_quantization_zigzag_b200 import build
+    build.build()
+    from w4a4_post_quantization_zigzag_b200 import qvla
+    return qvla
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "qvla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qvla_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("qvla_pack_weights", "qvla_rotate_quant_act", "qvla_w4a4_gemm"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol():
+    q = _lib_mod()
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+    assert set(declared_symbols()) == set(q.EXPORTED)
+
+
+def test_status_strings_and_version():
+    q = _lib_mod()
+    assert q.qvla_abi_version() == 1
+    for code in range(9):
+        assert q.qvla_status_str(code)
+    assert q.qvla_status_str(q.QVLA_ERR_STEP_RANGE).startswith("denoising step")
+
+
+def test_packed_sizes_and_shape_errors():
+    q = _lib_mod()
+    wq, rot, ws = q.qvla_packed_sizes(4096, 1024, 64)
+    assert wq == 4096 * 1024 // 2 and rot == 1024 * 64 * 4 and ws > 4096 * 1024 * 4
+    for args in ((4096, 1000, 64), (4096, 1024, 48), (0, 1024, 64), (16, 65536, 64),
+                 (16, 1024, 512)):
+        with pytest.raises(q.QvlaError) as e:
+            q.qvla_packed_sizes(*args)
+        assert e.value.code == q.QVLA_ERR_SHAPE
+
+
+def test_argument_errors_before_any_cuda_call():
+    q = _lib_mod()
+    lib = q._lib
+    # null packed linear
+    assert lib.qvla_rotate_quant_act(None, 1, 4, 64, None, 0, None, 0, 0, None, 0, 0, None,
+                                     None, None) == q.QVLA_ERR_ARG
+    L = q.qvla_packed_linear(128, 256, 64, 0, 0, 0, 0, None)
+    assert lib.qvla_w4a4_gemm(None, None, 4, ctypes.byref(L), None, 128, 0, None) == q.QVLA_ERR_ARG
+    # bad shape inside the struct
+    Lbad = q.qvla_packed_linear(128, 250, 64, 16, 16, 16, 16, None)
+    assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lbad),
+                                   ctypes.c_void_p(16), None) == q.QVLA_ERR_SHAPE
+    # misaligned pointers
+    Lmis = q.qvla_packed_linear(128, 256, 64, 16, 24, 16, 16, None)
+    assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lmis),
+                                   ctypes.c_void_p(16), None) == q.QVLA_ERR_ALIGN
+    # table mode: layer or host step outside the table -> STEP_RANGE, never a clamp
+    Lok = q.qvla_packed_linear(128, 256, 64, 16, 16, 16, 16, None)
+    args = lambda step, layer: (ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lok),
+                                q.QVLA_SCALE_TABLE, ctypes.c_void_p(16), 10, 12, None, step,
+                                layer, ctypes.c_void_p(16), ctypes.c_void_p(16), None)
+    assert lib.qvla_rotate_quant_act(*args(10, 0)) == q.QVLA_ERR_STEP_RANGE
+    assert lib.qvla_rotate_quant_act(*args(-1, 0)) == q.QVLA_ERR_STEP_RANGE
+    assert lib.qvla_rotate_quant_act(*args(0, 12)) == q.QVLA_ERR_STEP_RANGE
+    # table mode without a table
+    assert lib.qvla_quant_act_f32(ctypes.c_void_p(16), 4, 256, q.QVLA_SCALE_TABLE, None, 10, 12,
+                                  None, 0, 0, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                  None) == q.QVLA_ERR_ARG
+    # empty input is a no-op
+    assert lib.qvla_rotate_quant_act(None, 1, 0, 256, ctypes.byref(Lok), 0, None, 0, 0, None, 0,
+                                     0, None, None, None) == q.QVLA_OK
+    assert lib.qvla_w4a4_gemm_s32(None, 0, ctypes.byref(Lok), None, 0, None) == q.QVLA_OK
+    # split-K factor must be a power of two <= 16 and <= the number of 256-wide K tiles
+    Lw = q.qvla_packed_linear(128, 256, 64, 16, 16, 16, 16, None)
+    assert lib.qvla_w4a4_gemm_s32(ctypes.c_void_p(16), 4, ctypes.byref(Lw), ctypes.c_void_p(16),
+                                  3, None) == q.QVLA_ERR_ARG
+    assert lib.qvla_w4a4_gemm_s32(ctypes.c_void_p(16), 4, ctypes.byref(Lw), ctypes.c_void_p(16),
+                                  2, None) == q.QVLA_ERR_SHAPE
+
+
+def test_pack_workspace_check():
+    q = _lib_mod()
+    lib = q._lib
+    assert lib.qvla_pack_weights(ctypes.c_void_p(16), 64, 256, 64, None, None,
+                                 ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                 ctypes.c_void_p(16), None, 0, None) == q.QVLA_ERR_WORKSPACE

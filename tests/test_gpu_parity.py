@@ -1,0 +1,256 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact: packed weights and scales, activation codes and scales when both
+sides quantise the same fp32 rotated inputs, and int32 accumulators for the
+same codes.  Within tolerance: the fp32 rotation (vs fp64), end-to-end
+activation codes (+-1 only at a rounding boundary), bf16 outputs
+(2e-2 absolute + 1e-2 relative).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import qvla_oracle as O
+from w4a4_post_quantization_zigzag_b200 import inputs as I
+from _parity import check_codes_near_boundary, check_y, unpack
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    from w4a4_post_quantization_zigzag_b200 import build
+    build.build()
+    from w4a4_post_quantization_zigzag_b200 import qvla
+    assert torch.cuda.is_available()
+    qvla.qvla_read_error_word(clear=True)
+    return qvla
+
+
+def cu(a, dt=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dt is not None:
+        t = t.to(dt)
+    return t.cuda()
+
+
+def x_dev(x32, dtype):
+    return cu(x32).to(torch.bfloat16) if dtype == "bf16" else cu(x32)
+
+
+def no_device_error(q):
+    assert q.qvla_read_error_word(clear=True) == 0
+
+
+# ------------------------------------------------------ quantisers (bit-exact)
+
+@pytest.mark.parametrize("M,K", [(1, 32), (7, 256), (50, 1024), (33, 4096)])
+def test_act_quant_from_fp32_is_bit_exact(q, M, K):
+    xr = I.activations(100 + M, M, K, std=1.7, n_outlier_cols=2, dtype="f32")
+    xr[0, :] = 0.0                                   # an all-zero row: s = 0, codes 0
+    qx_ref, s_ref = O.quantize_acts_dynamic_fp32(xr)
+    xq, s = q.qvla_quant_act_f32(cu(xr), q.QVLA_SCALE_DYNAMIC)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), O.pack_nibbles(qx_ref))
+    # table mode with a small scale: saturation at -8 / 7
+    tab = I.scale_table(3, 4, 5, I.step_sigmas(4)) * 0.25
+    qx_t, _ = O.quantize_acts_table_fp32(xr, O.table_scale(tab, 2, 3))
+    xq_t, s_t = q.qvla_quant_act_f32(cu(xr), q.QVLA_SCALE_TABLE, table=cu(tab), step=2, layer=3)
+    assert np.array_equal(xq_t.cpu().numpy(), O.pack_nibbles(qx_t))
+    assert (s_t.cpu().numpy() == tab[2, 3]).all()
+    assert unpack(xq_t.cpu().numpy()).min() == -8
+    no_device_error(q)
+
+
+@pytest.mark.parametrize("N,K", [(3, 64), (256, 256), (1000, 1024)])
+def test_weight_quant_from_fp32_is_bit_exact(q, N, K):
+    Wr = I.weights(200 + N, N, K, n_outlier_rows=2)
+    Wr[1] = 0.0
+    qw_ref, s_ref = O.quantize_weights_fp32(Wr)
+    wq, s = q.qvla_quant_pack_weights_f32(cu(Wr))
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(wq.cpu().numpy(), O.pack_nibbles(qw_ref))
+    no_device_error(q)
+
+
+# ----------------------------------------------------------------- pack
+
+@pytest.mark.parametrize("N,K,b", [(256, 256, 64), (130, 512, 32), (256, 1024, 128),
+                                   (96, 512, 256)])
+def test_pack_parity(q, N, K, b):
+    W = I.weights(300 + K + b, N, K, n_outlier_rows=3, col_spread=10.0)
+    ref = O.pack_linear(W, b)
+    # the GPU's own permutation and R_SVD
+    pk = q.qvla_pack_weights(cu(W), b)
+    assert np.array_equal(pk.perm.cpu().numpy(), ref.perm)
+    rot = pk.rot.cpu().numpy().astype(np.float64)
+    assert np.abs(rot - ref.rsvd).max() <= 1e-6          # fp32-rounded R_SVD
+    # with the oracle's perm and R_SVD both sides quantise the same rotation
+    pk2 = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    assert np.array_equal(pk2.w_scale.cpu().numpy().view(np.uint32), ref.s_w.view(np.uint32))
+    flips = check_codes_near_boundary(unpack(pk2.wq.cpu().numpy()), ref.qw, ref.Wr,
+                                      ref.s_w.astype(np.float64), "packed weights")
+    assert flips == 0
+    # the weight rotation alone: fp32(W P R) computed in fp64
+    Wr = q.qvla_rotate_weights_f32(cu(W), b, pk2.perm, cu(ref.rsvd))
+    assert np.array_equal(Wr.cpu().numpy(), ref.Wr.astype(np.float32))
+    no_device_error(q)
+
+
+# ----------------------------------------------------- activation rotation
+
+@pytest.mark.parametrize("M,K,b,dt", [(16, 256, 64, "f32"), (50, 1024, 64, "bf16"),
+                                      (5, 2048, 128, "bf16"), (3, 512, 32, "bf16"),
+                                      (9, 1024, 256, "bf16"), (2, 16384, 128, "bf16")])
+def test_rotation_fp32_vs_fp64(q, M, K, b, dt):
+    W = I.weights(400 + K, 64, K)
+    ref = O.pack_linear(W, b)
+    L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    x = I.activations(401 + M, M, K, n_outlier_cols=3, dtype=dt)
+    xr = q.qvla_rotate_act_f32(x_dev(x, dt), L).cpu().numpy().astype(np.float64)
+    xr_ref = O.rotate_activations(x, ref.perm, ref.R)
+    scale = np.abs(xr_ref).max(axis=1, keepdims=True)
+    assert (np.abs(xr - xr_ref) <= 2e-6 * scale).all()
+
+
+@pytest.mark.parametrize("M,K,b,dt,mode", [
+    (16, 256, 64, "f32", "dynamic"), (50, 1024, 64, "bf16", "table"),
+    (50, 4096, 64, "bf16", "table"), (37, 2048, 128, "bf16", "dynamic"),
+    (8, 1024, 32, "bf16", "dynamic"), (8, 1024, 256, "bf16", "table"),
+    (3, 16384, 128, "bf16", "dynamic")])
+def test_rotate_quant_end_to_end(q, M, K, b, dt, mode):
+    W = I.weights(500 + K + b, 96, K)
+    ref = O.pack_linear(W, b)
+    L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    x = I.activations(501 + M, M, K, std=1.3, n_outlier_cols=4, dtype=dt)
+    tab = I.scale_table(7, 10, 12, I.step_sigmas(10) * 1.3)
+    if mode == "dynamic":
+        xq, s = q.qvla_rotate_quant_act(x_dev(x, dt), L, q.QVLA_SCALE_DYNAMIC)
+        xr_ref, qx_ref, s_ref = O.rotate_quant_act(x, ref, "dynamic")
+        np.testing.assert_allclose(s.cpu().numpy(), s_ref, rtol=2e-6)
+    else:
+        step = torch.tensor([4], dtype=torch.int32, device="cuda")
+        xq, s = q.qvla_rotate_quant_act(x_dev(x, dt), L, q.QVLA_SCALE_TABLE, table=cu(tab),
+                                        step=step, layer=7)
+        xr_ref, qx_ref, s_ref = O.rotate_quant_act(x, ref, "table", tab, 4, 7)
+        assert (s.cpu().numpy() == tab[4, 7]).all()
+    check_codes_near_boundary(unpack(xq.cpu().numpy()), qx_ref, xr_ref, s_ref, "activations")
+    no_device_error(q)
+
+
+def test_rotate_quant_ragged_pitch_and_empty(q):
+    M, K, b = 5, 512, 64
+    W = I.weights(600, 64, K)
+    ref = O.pack_linear(W, b)
+    L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    x = I.activations(601, M, K + 64, dtype="bf16")
+    xd = x_dev(x, "bf16")[:, :K]                     # row pitch K + 64
+    xq, s = q.qvla_rotate_quant_act(xd, L, q.QVLA_SCALE_DYNAMIC)
+    xr_ref, qx_ref, s_ref = O.rotate_quant_act(x[:, :K], ref, "dynamic")
+    check_codes_near_boundary(unpack(xq.cpu().numpy()), qx_ref, xr_ref, s_ref)
+    e = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    xq0, s0 = q.qvla_rotate_quant_act(e, L, q.QVLA_SCALE_DYNAMIC)
+    assert xq0.shape == (0, K // 2)
+
+
+def test_device_step_out_of_range_sets_flag_and_zeroes(q):
+    M, K, b = 4, 256, 64
+    W = I.weights(700, 64, K)
+    ref = O.pack_linear(W, b)
+    L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    x = x_dev(I.activations(701, M, K), "bf16")
+    tab = cu(I.scale_table(1, 8, 3, I.step_sigmas(8)))
+    q.qvla_read_error_word(clear=True)
+    bad = torch.tensor([8], dtype=torch.int32, device="cuda")
+    xq, s = q.qvla_rotate_quant_act(x, L, q.QVLA_SCALE_TABLE, table=tab, step=bad, layer=1)
+    word = q.qvla_read_error_word(clear=True)
+    assert word & q.QVLA_DEVERR_STEP_RANGE
+    assert not xq.cpu().numpy().any() and not s.cpu().numpy().any()
+    ok = torch.tensor([7], dtype=torch.int32, device="cuda")
+    q.qvla_rotate_quant_act(x, L, q.QVLA_SCALE_TABLE, table=tab, step=ok, layer=1)
+    assert q.qvla_read_error_word(clear=True) == 0
+
+
+# ------------------------------------------------------------------ GEMM
+
+GEMM_CASES = [
+    # M, N, K, split_k
+    (1, 256, 256, 0), (16, 256, 256, 1), (50, 4096, 1024, 0), (50, 1024, 4096, 0),
+    (64, 384, 1024, 4), (64, 200, 512, 2), (100, 256, 2048, 8), (128, 512, 768, 1),
+    (200, 384, 1024, 1), (256, 256, 512, 0), (300, 1000, 1056, 1), (520, 256, 2048, 0),
+    (33, 640, 4096, 16),
+]
+
+
+@pytest.mark.parametrize("M,N,K,split", GEMM_CASES)
+def test_gemm_int32_accumulators_bit_exact(q, M, N, K, split):
+    qx = I.int_codes(800 + M, M, K, -8, 7)
+    qw = I.int_codes(801 + N, N, K, -7, 7)
+    qx[0, :] = -8                                   # extreme magnitudes
+    qw[0, :] = -7
+    acc_ref = O.int_gemm(qx, qw)
+    L = q.from_host_packed(O.pack_nibbles(qw), np.ones(N, np.float32),
+                           np.arange(K, dtype=np.int32), np.zeros((K // 32, 32, 32)))
+    acc = q.qvla_w4a4_gemm_s32(cu(O.pack_nibbles(qx)), L, split_k=split)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), acc_ref)
+    no_device_error(q)
+
+
+@pytest.mark.parametrize("M,N,K,split", [(50, 4096, 1024, 0), (16, 256, 256, 0),
+                                         (300, 1000, 1056, 1), (64, 384, 1024, 4)])
+def test_gemm_bf16_epilogue(q, M, N, K, split):
+    qx = I.int_codes(900 + M, M, K, -8, 7)
+    qw = I.int_codes(901 + N, N, K, -7, 7)
+    s_x = I.positive_scales(902, M, 0.05, 0.6)
+    s_w = I.positive_scales(903, N, 1e-3, 2e-2)
+    b = I.bias(904, N)
+    L = q.from_host_packed(O.pack_nibbles(qw), s_w, np.arange(K, dtype=np.int32),
+                           np.zeros((K // 32, 32, 32)), bias=b)
+    y = q.qvla_w4a4_gemm(cu(O.pack_nibbles(qx)), cu(s_x), L, split_k=split)
+    y_ref = O.dequantize(O.int_gemm(qx, qw), s_x, s_w, b)
+    check_y(y.float().cpu().numpy(), y_ref)
+    # output row pitch larger than N
+    yp = torch.zeros(M, N + 8, dtype=torch.bfloat16, device="cuda")
+    q.qvla_w4a4_gemm(cu(O.pack_nibbles(qx)), cu(s_x), L, split_k=split, y=yp[:, :N])
+    check_y(yp[:, :N].float().cpu().numpy(), y_ref)
+    assert not yp[:, N:].float().abs().sum().item()
+    no_device_error(q)
+
+
+# ----------------------------------------------------- whole layer
+
+def _layer(q, lin, mode="dynamic", tab=None, step=0, x_std=None):
+    W, x, bb = lin.make_w(), lin.make_x(std=x_std), lin.make_bias()
+    ref = O.pack_linear(W, lin.block, bias=bb)
+    L = q.qvla_pack_weights(cu(W), lin.block, bias=cu(bb), perm_in=ref.perm.astype(np.int32),
+                            rsvd_in=ref.rsvd)
+    xd = x_dev(x, lin.x_dtype)
+    if mode == "dynamic":
+        xq, s = q.qvla_rotate_quant_act(xd, L, q.QVLA_SCALE_DYNAMIC)
+        out = O.linear_forward(x, ref)
+    else:
+        xq, s = q.qvla_rotate_quant_act(xd, L, q.QVLA_SCALE_TABLE, table=cu(tab), step=step,
+                                        layer=lin.layer)
+        out = O.linear_forward(x, ref, "table", tab, step, lin.layer)
+    y = q.qvla_w4a4_gemm(xq, s, L)
+    qx_gpu = unpack(xq.cpu().numpy())
+    check_codes_near_boundary(qx_gpu, out["qx"], out["xr"], out["s_x"])
+    # several roundings are valid at a boundary: score y against the oracle's
+    # dequantisation of the codes the GPU chose
+    y_ref = O.dequantize(O.int_gemm(qx_gpu, ref.qw), out["s_x"], ref.s_w, bb)
+    check_y(y.float().cpu().numpy(), y_ref)
+    return y, out
+
+
+def test_single_linear_layer(q):
+    wl = I.single_linear()
+    _layer(q, wl.linears[0])
+    no_device_error(q)
+
+
+def test_dit_mlp_layer_each_kind(q):
+    wl = I.dit_mlp_stack()
+    for lin in wl.linears[:3]:                       # gate, up, down of layer 0
+        for step in (0, 9):
+            _layer(q, lin, "table", wl.table, step, x_std=float(wl.sigmas[step]))
+    no_device_error(q)

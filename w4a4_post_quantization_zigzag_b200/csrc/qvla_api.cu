@@ -1,0 +1,495 @@
+// C ABI of the rotated W4A4 linear layer: argument validation, status codes,
+// the per-device error word, and the offline pack orchestration (zigzag
+// permutation and R_SVD eigensolve on the host, everything else on the GPU).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <thread>
+#include <vector>
+
+#include "qvla_common.cuh"
+#include "qvla_internal.h"
+
+// Device error word: kernels OR QVLA_DEVERR_* bits into it.
+__device__ unsigned int g_qvla_error_word = 0u;
+
+namespace qvla {
+
+unsigned int* device_error_word() {
+  static std::mutex mu;
+  static unsigned int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_qvla_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_block(int b) { return b == 32 || b == 64 || b == 128 || b == 256; }
+
+qvla_status check_shape(int N, int K, int block) {
+  if (N <= 0 || K <= 0 || !valid_block(block)) return QVLA_ERR_SHAPE;
+  if (K % block != 0 || K > QVLA_MAX_K) return QVLA_ERR_SHAPE;
+  return QVLA_OK;
+}
+
+qvla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVLA_OK : QVLA_ERR_CUDA; }
+
+qvla_status check_linear(const qvla_packed_linear* L, bool need_weights) {
+  if (!L) return QVLA_ERR_ARG;
+  qvla_status st = check_shape(L->N, L->K, L->block);
+  if (st != QVLA_OK) return st;
+  if (!L->perm || !L->rot) return QVLA_ERR_ARG;
+  if (need_weights && (!L->wq || !L->w_scale)) return QVLA_ERR_ARG;
+  if (!aligned16(L->perm) || !aligned16(L->rot)) return QVLA_ERR_ALIGN;
+  if (need_weights && (!aligned16(L->wq) || !aligned16(L->w_scale))) return QVLA_ERR_ALIGN;
+  if (L->bias && !aligned16(L->bias)) return QVLA_ERR_ALIGN;
+  return QVLA_OK;
+}
+
+qvla_status check_scale(qvla_scale_mode mode, const float* table, int T, int Lcount,
+                        const int32_t* step_dev, int step_host, int layer) {
+  if (mode == QVLA_SCALE_DYNAMIC) return QVLA_OK;
+  if (mode != QVLA_SCALE_TABLE) return QVLA_ERR_ARG;
+  if (!table || T <= 0 || Lcount <= 0) return QVLA_ERR_ARG;
+  if (layer < 0 || layer >= Lcount) return QVLA_ERR_STEP_RANGE;
+  if (!step_dev && (step_host < 0 || step_host >= T)) return QVLA_ERR_STEP_RANGE;
+  return QVLA_OK;
+}
+
+// ------------------------------------------------------------ host eigensolve
+// Cyclic Jacobi eigen-decomposition of a symmetric n x n matrix (fp64).
+// Each rotation in the (p, q) plane zeroes A[p][q]:
+//   theta = (A[q][q] - A[p][p]) / (2 A[p][q]),
+//   t = sign(theta) / (|theta| + sqrt(theta^2 + 1)),  c = 1/sqrt(1+t^2), s = t c,
+//   A[p][p] -= t A[p][q],  A[q][q] += t A[p][q],
+//   rows/columns p, q and the accumulated eigenvector columns rotate by (c, s).
+// Sweeps stop when the off-diagonal Frobenius norm is below 1e-15 ||A||_F.
+void jacobi_eig(std::vector<double>& A, int n, std::vector<double>& V) {
+  V.assign(static_cast<size_t>(n) * n, 0.0);
+  for (int i = 0; i < n; ++i) V[static_cast<size_t>(i) * n + i] = 1.0;
+  double frob = 0.0;
+  for (double a : A) frob += a * a;
+  frob = std::sqrt(frob);
+  if (frob == 0.0) return;
+  for (int sweep = 0; sweep < 100; ++sweep) {
+    double off = 0.0;
+    for (int p = 0; p < n; ++p)
+      for (int q = p + 1; q < n; ++q) off += 2.0 * A[static_cast<size_t>(p) * n + q] * A[static_cast<size_t>(p) * n + q];
+    if (std::sqrt(off) <= 1e-15 * frob) break;
+    for (int p = 0; p < n - 1; ++p) {
+      for (int q = p + 1; q < n; ++q) {
+        const double apq = A[static_cast<size_t>(p) * n + q];
+        if (apq == 0.0) continue;
+        const double app = A[static_cast<size_t>(p) * n + p];
+        const double aqq = A[static_cast<size_t>(q) * n + q];
+        const double theta = (aqq - app) / (2.0 * apq);
+        const double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
+        const double c = 1.0 / std::sqrt(t * t + 1.0);
+        const double s = t * c;
+        for (int k = 0; k < n; ++k) {
+          if (k == p || k == q) continue;
+          const double akp = A[static_cast<size_t>(k) * n + p];
+          const double akq = A[static_cast<size_t>(k) * n + q];
+          const double nkp = c * akp - s * akq;
+          const double nkq = s * akp + c * akq;
+          A[static_cast<size_t>(k) * n + p] = nkp;
+          A[static_cast<size_t>(p) * n + k] = nkp;
+          A[static_cast<size_t>(k) * n + q] = nkq;
+          A[static_cast<size_t>(q) * n + k] = nkq;
+        }
+        A[static_cast<size_t>(p) * n + p] = app - t * apq;
+        A[static_cast<size_t>(q) * n + q] = aqq + t * apq;
+        A[static_cast<size_t>(p) * n + q] = 0.0;
+        A[static_cast<size_t>(q) * n + p] = 0.0;
+        for (int k = 0; k < n; ++k) {
+          const double vkp = V[static_cast<size_t>(k) * n + p];
+          const double vkq = V[static_cast<size_t>(k) * n + q];
+          V[static_cast<size_t>(k) * n + p] = c * vkp - s * vkq;
+          V[static_cast<size_t>(k) * n + q] = s * vkp + c * vkq;
+        }
+      }
+    }
+  }
+}
+
+// R_SVD of one block from its Gram matrix: eigenvectors by descending
+// eigenvalue (ties to the lower index), largest-magnitude entry of each
+// column made positive (first index on ties).  out is row-major [i][j].
+void rsvd_from_gram(const double* G, int b, double* out) {
+  std::vector<double> A(G, G + static_cast<size_t>(b) * b), V;
+  jacobi_eig(A, b, V);
+  std::vector<int> idx(b);
+  for (int i = 0; i < b; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
+    return A[static_cast<size_t>(x) * b + x] > A[static_cast<size_t>(y) * b + y];
+  });
+  for (int j = 0; j < b; ++j) {
+    const int src = idx[j];
+    int imax = 0;
+    double vmax = -1.0;
+    for (int i = 0; i < b; ++i) {
+      const double v = std::fabs(V[static_cast<size_t>(i) * b + src]);
+      if (v > vmax) {
+        vmax = v;
+        imax = i;
+      }
+    }
+    const double sg = V[static_cast<size_t>(imax) * b + src] < 0 ? -1.0 : 1.0;
+    for (int i = 0; i < b; ++i) out[static_cast<size_t>(i) * b + j] = sg * V[static_cast<size_t>(i) * b + src];
+  }
+}
+
+// Zigzag permutation from column norms (see qvla_pack_weights).
+void zigzag_from_norms(const std::vector<double>& c, int block, std::vector<int32_t>& perm) {
+  const int K = static_cast<int>(c.size());
+  const int nb = K / block;
+  std::vector<int> order(K);
+  for (int k = 0; k < K; ++k) order[k] = k;
+  std::sort(order.begin(), order.end(), [&](int a, int b) {
+    return c[a] > c[b] || (c[a] == c[b] && a < b);
+  });
+  perm.assign(K, 0);
+  for (int r = 0; r < K; ++r) {
+    const int rnd = r / nb, pos = r % nb;
+    const int blk = (rnd % 2 == 0) ? pos : nb - 1 - pos;
+    perm[static_cast<size_t>(blk) * block + rnd] = order[r];
+  }
+}
+
+size_t pack_ws_bytes(int N, int K, int block) {
+  const size_t nb = K / block;
+  size_t b = 0;
+  b += static_cast<size_t>(K) * 8;                               // norms
+  b += nb * block * block * 8;                                   // Gram
+  b += nb * block * block * 8;                                   // R_SVD fp64
+  b = (b + 255) & ~static_cast<size_t>(255);
+  b += static_cast<size_t>(N) * K * 4;                           // W' fp32
+  return b;
+}
+
+}  // namespace
+}  // namespace qvla
+
+using namespace qvla;
+
+extern "C" {
+
+const char* qvla_status_str(qvla_status s) {
+  switch (s) {
+    case QVLA_OK: return "ok";
+    case QVLA_ERR_ARG: return "invalid argument (null pointer or enum)";
+    case QVLA_ERR_SHAPE: return "unsupported shape";
+    case QVLA_ERR_ALIGN: return "pointer or pitch not 16-byte aligned";
+    case QVLA_ERR_STEP_RANGE: return "denoising step or layer outside the scale table";
+    case QVLA_ERR_UNSUPPORTED: return "unsupported device or feature";
+    case QVLA_ERR_CUDA: return "CUDA error";
+    case QVLA_ERR_DEVICE_FLAG: return "device error word set";
+    case QVLA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int qvla_abi_version(void) { return QVLA_ABI_VERSION; }
+
+qvla_status qvla_read_error_word(uint32_t* out, int clear) {
+  if (!out) return QVLA_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QVLA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_qvla_error_word, sizeof(v)) != cudaSuccess) return QVLA_ERR_CUDA;
+  *out = v;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_qvla_error_word, &z, sizeof(z)) != cudaSuccess) return QVLA_ERR_CUDA;
+  }
+  return QVLA_OK;
+}
+
+qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t* rot_bytes,
+                              size_t* ws_bytes) {
+  qvla_status st = check_shape(N, K, block);
+  if (st != QVLA_OK) return st;
+  if (K % 32) return QVLA_ERR_SHAPE;
+  if (wq_bytes) *wq_bytes = static_cast<size_t>(N) * K / 2;
+  if (rot_bytes) *rot_bytes = static_cast<size_t>(K) * block * 4;
+  if (ws_bytes) *ws_bytes = pack_ws_bytes(N, K, block);
+  return QVLA_OK;
+}
+
+qvla_status qvla_rotate_weights_f32(const float* W, int N, int K, int block, const int32_t* perm,
+                                    const double* rsvd64, float* Wr_out, cudaStream_t stream) {
+  qvla_status st = check_shape(N, K, block);
+  if (st != QVLA_OK) return st;
+  if (!W || !perm || !rsvd64 || !Wr_out) return QVLA_ERR_ARG;
+  if (!aligned16(W) || !aligned16(Wr_out) || !aligned16(perm) || !aligned16(rsvd64))
+    return QVLA_ERR_ALIGN;
+  return cuda_status(launch_rotate_weights(W, N, K, block, perm, rsvd64, Wr_out, stream));
+}
+
+qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* wq_out,
+                                        float* w_scale_out, cudaStream_t stream) {
+  if (N <= 0 || K <= 0 || K % 32 || K > QVLA_MAX_K) return QVLA_ERR_SHAPE;
+  if (!Wr || !wq_out || !w_scale_out) return QVLA_ERR_ARG;
+  if (!aligned16(Wr) || !aligned16(wq_out) || !aligned16(w_scale_out)) return QVLA_ERR_ALIGN;
+  QuantArgs a = {};
+  a.xr = Wr;
+  a.rows = N;
+  a.K = K;
+  a.qmin = -7;
+  a.qmax = 7;
+  a.dynamic = 1;
+  a.q_out = wq_out;
+  a.s_out = w_scale_out;
+  return cuda_status(launch_quant_rows(a, stream));
+}
+
+qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
+                              const double* rsvd_in, int32_t* perm_out, float* rot_out,
+                              uint8_t* wq_out, float* w_scale_out, void* workspace,
+                              size_t ws_bytes, cudaStream_t stream) {
+  qvla_status st = check_shape(N, K, block);
+  if (st != QVLA_OK) return st;
+  if (K % 32) return QVLA_ERR_SHAPE;
+  if (!W || !perm_out || !rot_out || !wq_out || !w_scale_out) return QVLA_ERR_ARG;
+  if (!workspace || ws_bytes < pack_ws_bytes(N, K, block)) return QVLA_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(perm_out) || !aligned16(rot_out) || !aligned16(wq_out) ||
+      !aligned16(w_scale_out) || !aligned16(workspace))
+    return QVLA_ERR_ALIGN;
+  const int nb = K / block;
+  const size_t bb = static_cast<size_t>(block) * block;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* norms = reinterpret_cast<double*>(ws);
+  double* gram = norms + K;
+  double* rsvd_dev = gram + nb * bb;
+  size_t off = (static_cast<size_t>(K) * 8 + 2 * nb * bb * 8 + 255) & ~static_cast<size_t>(255);
+  float* Wr = reinterpret_cast<float*>(ws + off);
+
+  // 1. zigzag permutation
+  std::vector<int32_t> perm(K);
+  if (perm_in) {
+    std::vector<char> seen(K, 0);
+    for (int k = 0; k < K; ++k) {
+      const int p = perm_in[k];
+      if (p < 0 || p >= K || seen[p]) return QVLA_ERR_ARG;
+      seen[p] = 1;
+      perm[k] = p;
+    }
+  } else {
+    if (launch_column_norms(W, N, K, norms, stream) != cudaSuccess) return QVLA_ERR_CUDA;
+    std::vector<double> c(K);
+    if (cudaMemcpyAsync(c.data(), norms, K * sizeof(double), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return QVLA_ERR_CUDA;
+    zigzag_from_norms(c, block, perm);
+  }
+  if (cudaMemcpyAsync(perm_out, perm.data(), K * sizeof(int32_t), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+
+  // 2. R_SVD per block
+  std::vector<double> rs(nb * bb);
+  if (rsvd_in) {
+    std::memcpy(rs.data(), rsvd_in, rs.size() * sizeof(double));
+  } else {
+    if (launch_block_gram(W, N, K, block, perm_out, gram, stream) != cudaSuccess)
+      return QVLA_ERR_CUDA;
+    std::vector<double> G(nb * bb);
+    if (cudaMemcpyAsync(G.data(), gram, G.size() * sizeof(double), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return QVLA_ERR_CUDA;
+    unsigned nthreads = std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+    nthreads = std::min<unsigned>(nthreads, static_cast<unsigned>(nb));
+    std::vector<std::thread> pool;
+    for (unsigned t = 0; t < nthreads; ++t)
+      pool.emplace_back([&, t]() {
+        for (int B = static_cast<int>(t); B < nb; B += static_cast<int>(nthreads))
+          rsvd_from_gram(G.data() + B * bb, block, rs.data() + B * bb);
+      });
+    for (auto& th : pool) th.join();
+  }
+  std::vector<float> rs32(rs.size());
+  for (size_t i = 0; i < rs.size(); ++i) rs32[i] = static_cast<float>(rs[i]);
+  if (cudaMemcpyAsync(rsvd_dev, rs.data(), rs.size() * sizeof(double), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess ||
+      cudaMemcpyAsync(rot_out, rs32.data(), rs32.size() * sizeof(float), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+
+  // 3. W' = fp32(W P R) in fp64, then RTN + packing
+  if (launch_rotate_weights(W, N, K, block, perm_out, rsvd_dev, Wr, stream) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+  QuantArgs q = {};
+  q.xr = Wr;
+  q.rows = N;
+  q.K = K;
+  q.qmin = -7;
+  q.qmax = 7;
+  q.dynamic = 1;
+  q.q_out = wq_out;
+  q.s_out = w_scale_out;
+  if (launch_quant_rows(q, stream) != cudaSuccess) return QVLA_ERR_CUDA;
+  // host staging vectors must outlive the copies
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return QVLA_ERR_CUDA;
+  return QVLA_OK;
+}
+
+qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
+                                  const qvla_packed_linear* L, qvla_scale_mode mode,
+                                  const float* table, int T, int Lcount, const int32_t* step_dev,
+                                  int step_host, int layer, uint8_t* xq, float* s_x,
+                                  cudaStream_t stream) {
+  qvla_status st = check_linear(L, false);
+  if (st != QVLA_OK) return st;
+  if (M < 0) return QVLA_ERR_SHAPE;
+  if (xdt != QVLA_DTYPE_F32 && xdt != QVLA_DTYPE_BF16) return QVLA_ERR_ARG;
+  if ((st = check_scale(mode, table, T, Lcount, step_dev, step_host, layer)) != QVLA_OK) return st;
+  if (M == 0) return QVLA_OK;
+  if (!x || !xq || !s_x) return QVLA_ERR_ARG;
+  if (ldx < L->K) return QVLA_ERR_SHAPE;
+  const size_t esz = xdt == QVLA_DTYPE_F32 ? 4 : 2;
+  if (!aligned16(x) || (ldx * esz) % 16 || !aligned16(xq) || !aligned16(s_x)) return QVLA_ERR_ALIGN;
+  if (static_cast<size_t>(L->K) * 4 > 200 * 1024) return QVLA_ERR_SHAPE;
+  ActArgs a = {};
+  a.x = x;
+  a.xdt = xdt;
+  a.M = M;
+  a.ldx = ldx;
+  a.K = L->K;
+  a.block = L->block;
+  a.perm = L->perm;
+  a.rot = L->rot;
+  a.dynamic = mode == QVLA_SCALE_DYNAMIC;
+  a.table = table;
+  a.T = T;
+  a.Lcount = Lcount;
+  a.step_dev = step_dev;
+  a.step_host = step_host;
+  a.layer = layer;
+  a.xq = xq;
+  a.s_x = s_x;
+  return cuda_status(launch_rotate_quant(a, stream));
+}
+
+qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
+                                const qvla_packed_linear* L, float* xr_out, cudaStream_t stream) {
+  qvla_status st = check_linear(L, false);
+  if (st != QVLA_OK) return st;
+  if (M < 0) return QVLA_ERR_SHAPE;
+  if (xdt != QVLA_DTYPE_F32 && xdt != QVLA_DTYPE_BF16) return QVLA_ERR_ARG;
+  if (M == 0) return QVLA_OK;
+  if (!x || !xr_out) return QVLA_ERR_ARG;
+  if (ldx < L->K) return QVLA_ERR_SHAPE;
+  const size_t esz = xdt == QVLA_DTYPE_F32 ? 4 : 2;
+  if (!aligned16(x) || (ldx * esz) % 16 || !aligned16(xr_out)) return QVLA_ERR_ALIGN;
+  if (static_cast<size_t>(L->K) * 4 > 200 * 1024) return QVLA_ERR_SHAPE;
+  ActArgs a = {};
+  a.x = x;
+  a.xdt = xdt;
+  a.M = M;
+  a.ldx = ldx;
+  a.K = L->K;
+  a.block = L->block;
+  a.perm = L->perm;
+  a.rot = L->rot;
+  a.dynamic = 1;
+  a.xr_out = xr_out;
+  return cuda_status(launch_rotate_quant(a, stream));
+}
+
+qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mode,
+                               const float* table, int T, int Lcount, const int32_t* step_dev,
+                               int step_host, int layer, uint8_t* xq, float* s_x,
+                               cudaStream_t stream) {
+  if (M < 0 || K <= 0 || K % 32 || K > QVLA_MAX_K) return QVLA_ERR_SHAPE;
+  qvla_status st = check_scale(mode, table, T, Lcount, step_dev, step_host, layer);
+  if (st != QVLA_OK) return st;
+  if (M == 0) return QVLA_OK;
+  if (!xr || !xq || !s_x) return QVLA_ERR_ARG;
+  if (!aligned16(xr) || !aligned16(xq) || !aligned16(s_x)) return QVLA_ERR_ALIGN;
+  QuantArgs a = {};
+  a.xr = xr;
+  a.rows = M;
+  a.K = K;
+  a.qmin = -8;
+  a.qmax = 7;
+  a.dynamic = mode == QVLA_SCALE_DYNAMIC;
+  a.table = table;
+  a.T = T;
+  a.Lcount = Lcount;
+  a.step_dev = step_dev;
+  a.step_host = step_host;
+  a.layer = layer;
+  a.q_out = xq;
+  a.s_out = s_x;
+  return cuda_status(launch_quant_rows(a, stream));
+}
+
+static qvla_status gemm_common(const uint8_t* xq, const float* s_x, int M,
+                               const qvla_packed_linear* L, void* y, int ldy, int32_t* acc,
+                               int split_k, cudaStream_t stream) {
+  qvla_status st = check_linear(L, true);
+  if (st != QVLA_OK) return st;
+  if (M < 0) return QVLA_ERR_SHAPE;
+  if (L->K % 32) return QVLA_ERR_SHAPE;
+  if (M == 0) return QVLA_OK;
+  if (!xq) return QVLA_ERR_ARG;
+  if (!aligned16(xq)) return QVLA_ERR_ALIGN;
+  const int nkt = (L->K + 255) / 256;
+  if (split_k != 0 && split_k != 1 && split_k != 2 && split_k != 4 && split_k != 8 &&
+      split_k != 16)
+    return QVLA_ERR_ARG;
+  if (split_k > nkt) return QVLA_ERR_SHAPE;
+  GemmArgs g = {};
+  g.xq = xq;
+  g.s_x = s_x;
+  g.M = M;
+  g.N = L->N;
+  g.K = L->K;
+  g.wq = L->wq;
+  g.w_scale = L->w_scale;
+  g.bias = L->bias;
+  g.y = y;
+  g.ldy = ldy;
+  g.acc = acc;
+  g.split_k = split_k;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+  if (major != 10) return QVLA_ERR_UNSUPPORTED;
+  return cuda_status(launch_w4a4_gemm(g, stream));
+}
+
+qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
+                           const qvla_packed_linear* L, void* y, int ldy, int split_k,
+                           cudaStream_t stream) {
+  if (M > 0) {
+    if (!s_x || !y || !L) return QVLA_ERR_ARG;
+    if (ldy < L->N) return QVLA_ERR_SHAPE;
+    if (!aligned16(s_x) || !aligned16(y) || (static_cast<size_t>(ldy) * 2) % 16)
+      return QVLA_ERR_ALIGN;
+  }
+  return gemm_common(xq, s_x, M, L, y, ldy, nullptr, split_k, stream);
+}
+
+qvla_status qvla_w4a4_gemm_s32(const uint8_t* xq, int M, const qvla_packed_linear* L,
+                               int32_t* acc, int split_k, cudaStream_t stream) {
+  if (M > 0) {
+    if (!acc) return QVLA_ERR_ARG;
+    if (!aligned16(acc)) return QVLA_ERR_ALIGN;
+  }
+  return gemm_common(xq, nullptr, M, L, nullptr, 0, acc, split_k, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// Internal (C++) launch interfaces shared by the C-ABI layer and the kernels'
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qvla.h"
+
+namespace qvla {
+
+// Device error word of the current device (lazily resolved symbol address).
+unsigned int* device_error_word();
+
+// ---- activation rotate + quantise (rotate_quant.cu)
+struct ActArgs {
+  const void* x;
+  qvla_dtype xdt;
+  int M, ldx, K, block;
+  const int32_t* perm;
+  const float* rot;
+  int dynamic;            // 1: per-token absmax, 0: table
+  const float* table;
+  int T, Lcount;
+  const int32_t* step_dev;
+  int step_host, layer;
+  uint8_t* xq;
+  float* s_x;
+  float* xr_out;          // rotate-only mode when non-null and xq == nullptr
+};
+cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream);
+
+// quantise already-rotated fp32 rows: activations (qmin -8) or weights (qmin -7)
+struct QuantArgs {
+  const float* xr;
+  int rows, K;
+  int qmin, qmax;
+  int dynamic;
+  const float* table;
+  int T, Lcount;
+  const int32_t* step_dev;
+  int step_host, layer;
+  uint8_t* q_out;
+  float* s_out;
+};
+cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream);
+
+// ---- pack helpers (pack_kernels.cu)
+cudaError_t launch_column_norms(const float* W, int N, int K, double* norms, cudaStream_t s);
+cudaError_t launch_block_gram(const float* W, int N, int K, int block, const int32_t* perm,
+                              double* gram, cudaStream_t s);
+cudaError_t launch_rotate_weights(const float* W, int N, int K, int block, const int32_t* perm,
+                                  const double* rsvd64, float* Wr, cudaStream_t s);
+
+// ---- GEMM (gemm_w4a4.cu)
+struct GemmArgs {
+  const uint8_t* xq;
+  const float* s_x;
+  int M, N, K;
+  const uint8_t* wq;
+  const float* w_scale;
+  const float* bias;
+  void* y;                // bf16 [M][ldy] or nullptr
+  int ldy;
+  int32_t* acc;           // int32 [M][N] when y == nullptr
+  int split_k;
+};
+cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream);
+int gemm_choose_split(int M, int N, int K);
+
+}  // namespace qvla

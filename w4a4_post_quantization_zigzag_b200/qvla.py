@@ -1,0 +1,284 @@
+"""ctypes binding of ``libqvla.so`` (the C ABI declared in ``include/qvla.h``).
+
+Argument marshalling only: every function here validates Python-side types,
+allocates output tensors with PyTorch (device memory is PyTorch's job) and calls
+the C entry point of the same name.  No step of the layer's arithmetic runs in
+Python.  Importing this module loads the library and raises ImportError when it
+has not been built (``python -m w4a4_post_quantization_zigzag_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_double, c_int, c_int32, c_size_t, c_uint32, c_void_p
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqvla.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m w4a4_post_quantization_zigzag_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+QVLA_OK = 0
+QVLA_ERR_ARG = 1
+QVLA_ERR_SHAPE = 2
+QVLA_ERR_ALIGN = 3
+QVLA_ERR_STEP_RANGE = 4
+QVLA_ERR_UNSUPPORTED = 5
+QVLA_ERR_CUDA = 6
+QVLA_ERR_DEVICE_FLAG = 7
+QVLA_ERR_WORKSPACE = 8
+
+QVLA_DTYPE_F32 = 0
+QVLA_DTYPE_BF16 = 1
+QVLA_SCALE_DYNAMIC = 0
+QVLA_SCALE_TABLE = 1
+
+QVLA_DEVERR_STEP_RANGE = 0x1
+QVLA_DEVERR_TIMEOUT = 0x2
+QVLA_DEVERR_TMEM = 0x4
+
+# Every symbol include/qvla.h declares.
+EXPORTED = (
+    "qvla_status_str", "qvla_abi_version", "qvla_read_error_word", "qvla_packed_sizes",
+    "qvla_pack_weights", "qvla_rotate_weights_f32", "qvla_quant_pack_weights_f32",
+    "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
+    "qvla_w4a4_gemm_s32",
+)
+
+
+class qvla_packed_linear(ctypes.Structure):
+    _fields_ = [("N", c_int32), ("K", c_int32), ("block", c_int32),
+                ("perm", c_void_p), ("rot", c_void_p), ("wq", c_void_p),
+                ("w_scale", c_void_p), ("bias", c_void_p)]
+
+
+_P = POINTER(qvla_packed_linear)
+_sig = {
+    "qvla_status_str": (ctypes.c_char_p, [c_int]),
+    "qvla_abi_version": (c_int, []),
+    "qvla_read_error_word": (c_int, [POINTER(c_uint32), c_int]),
+    "qvla_packed_sizes": (c_int, [c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t),
+                                  POINTER(c_size_t)]),
+    "qvla_pack_weights": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qvla_rotate_weights_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p]),
+    "qvla_quant_pack_weights_f32": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                            c_void_p]),
+    "qvla_rotate_quant_act": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_int, c_void_p, c_int,
+                                      c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                      c_void_p]),
+    "qvla_rotate_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_void_p, c_void_p]),
+    "qvla_quant_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_int,
+                                   c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "qvla_w4a4_gemm": (c_int, [c_void_p, c_void_p, c_int, _P, c_void_p, c_int, c_int, c_void_p]),
+    "qvla_w4a4_gemm_s32": (c_int, [c_void_p, c_int, _P, c_void_p, c_int, c_void_p]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class QvlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {qvla_status_str(code)} (status {code})")
+
+
+def qvla_status_str(code: int) -> str:
+    return _lib.qvla_status_str(code).decode()
+
+
+def qvla_abi_version() -> int:
+    return _lib.qvla_abi_version()
+
+
+def _check(rc: int, where: str):
+    if rc != QVLA_OK:
+        raise QvlaError(rc, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return c_void_p(stream.cuda_stream)
+    return c_void_p(int(stream))
+
+
+def qvla_read_error_word(clear: bool = True) -> int:
+    v = c_uint32(0)
+    _check(_lib.qvla_read_error_word(ctypes.byref(v), int(clear)), "qvla_read_error_word")
+    return int(v.value)
+
+
+def qvla_packed_sizes(N: int, K: int, block: int) -> Tuple[int, int, int]:
+    a, b, c = c_size_t(), c_size_t(), c_size_t()
+    _check(_lib.qvla_packed_sizes(N, K, block, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "qvla_packed_sizes")
+    return a.value, b.value, c.value
+
+
+class PackedLinear:
+    """Device buffers of one packed linear plus the C struct that points at them."""
+
+    def __init__(self, N, K, block, perm, rot, wq, w_scale, bias=None):
+        self.N, self.K, self.block = int(N), int(K), int(block)
+        self.perm, self.rot, self.wq, self.w_scale, self.bias = perm, rot, wq, w_scale, bias
+        self._s = qvla_packed_linear(self.N, self.K, self.block, perm.data_ptr(), rot.data_ptr(),
+                                     wq.data_ptr(), w_scale.data_ptr(),
+                                     bias.data_ptr() if bias is not None else None)
+
+    @property
+    def struct(self):
+        return ctypes.byref(self._s)
+
+    def device_bytes(self) -> int:
+        n = sum(t.numel() * t.element_size() for t in (self.perm, self.rot, self.wq, self.w_scale))
+        return n + (self.bias.numel() * 4 if self.bias is not None else 0)
+
+
+def qvla_pack_weights(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
+                      perm_in: Optional[np.ndarray] = None, rsvd_in: Optional[np.ndarray] = None,
+                      stream=None) -> PackedLinear:
+    """W: cuda fp32 [N, K].  perm_in: host int32 [K]; rsvd_in: host float64 [nb, b, b]."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    wq_b, rot_b, ws_b = qvla_packed_sizes(N, K, block)
+    dev = W.device
+    perm = torch.empty(K, dtype=torch.int32, device=dev)
+    rot = torch.empty(rot_b // 4, dtype=torch.float32, device=dev)
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    p_in = r_in = None
+    if perm_in is not None:
+        perm_in = np.ascontiguousarray(perm_in, dtype=np.int32)
+        assert perm_in.shape == (K,)
+        p_in = perm_in.ctypes.data_as(c_void_p)
+    if rsvd_in is not None:
+        rsvd_in = np.ascontiguousarray(rsvd_in, dtype=np.float64)
+        assert rsvd_in.shape == (K // block, block, block)
+        r_in = rsvd_in.ctypes.data_as(c_void_p)
+    _check(_lib.qvla_pack_weights(_ptr(W), N, K, block, p_in, r_in, _ptr(perm), _ptr(rot),
+                                  _ptr(wq), _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
+           "qvla_pack_weights")
+    if bias is not None:
+        assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
+        bias = bias.contiguous()
+    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias)
+
+
+def qvla_rotate_weights_f32(W: torch.Tensor, block: int, perm: torch.Tensor,
+                            rsvd64: torch.Tensor, stream=None) -> torch.Tensor:
+    N, K = W.shape
+    Wr = torch.empty(N, K, dtype=torch.float32, device=W.device)
+    _check(_lib.qvla_rotate_weights_f32(_ptr(W), N, K, block, _ptr(perm), _ptr(rsvd64), _ptr(Wr),
+                                        _stream(stream)), "qvla_rotate_weights_f32")
+    return Wr
+
+
+def qvla_quant_pack_weights_f32(Wr: torch.Tensor, stream=None):
+    N, K = Wr.shape
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=Wr.device)
+    s_w = torch.empty(N, dtype=torch.float32, device=Wr.device)
+    _check(_lib.qvla_quant_pack_weights_f32(_ptr(Wr), N, K, _ptr(wq), _ptr(s_w), _stream(stream)),
+           "qvla_quant_pack_weights_f32")
+    return wq, s_w
+
+
+def _dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return QVLA_DTYPE_BF16
+    if x.dtype == torch.float32:
+        return QVLA_DTYPE_F32
+    raise TypeError(f"unsupported activation dtype {x.dtype}")
+
+
+def _step_args(step):
+    """int -> checked on the host; cuda int32 tensor -> read on the device."""
+    if step is None:
+        return None, 0
+    if isinstance(step, torch.Tensor):
+        assert step.is_cuda and step.dtype == torch.int32
+        return _ptr(step), 0
+    return None, int(step)
+
+
+def qvla_rotate_quant_act(x: torch.Tensor, L: PackedLinear, mode: int = QVLA_SCALE_DYNAMIC,
+                          table: Optional[torch.Tensor] = None, step=None, layer: int = 0,
+                          xq: Optional[torch.Tensor] = None, s_x: Optional[torch.Tensor] = None,
+                          stream=None):
+    M = x.shape[0]
+    if xq is None:
+        xq = torch.empty(M, L.K // 2, dtype=torch.uint8, device=x.device)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    T, Lc = (table.shape if table is not None else (0, 0))
+    sd, sh = _step_args(step)
+    _check(_lib.qvla_rotate_quant_act(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct, mode,
+                                      _ptr(table), T, Lc, sd, sh, layer, _ptr(xq), _ptr(s_x),
+                                      _stream(stream)), "qvla_rotate_quant_act")
+    return xq, s_x
+
+
+def qvla_rotate_act_f32(x: torch.Tensor, L: PackedLinear, stream=None) -> torch.Tensor:
+    M = x.shape[0]
+    xr = torch.empty(M, L.K, dtype=torch.float32, device=x.device)
+    _check(_lib.qvla_rotate_act_f32(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct, _ptr(xr),
+                                    _stream(stream)), "qvla_rotate_act_f32")
+    return xr
+
+
+def qvla_quant_act_f32(xr: torch.Tensor, mode: int = QVLA_SCALE_DYNAMIC,
+                       table: Optional[torch.Tensor] = None, step=None, layer: int = 0,
+                       stream=None):
+    M, K = xr.shape
+    xq = torch.empty(M, K // 2, dtype=torch.uint8, device=xr.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=xr.device)
+    T, Lc = (table.shape if table is not None else (0, 0))
+    sd, sh = _step_args(step)
+    _check(_lib.qvla_quant_act_f32(_ptr(xr), M, K, mode, _ptr(table), T, Lc, sd, sh, layer,
+                                   _ptr(xq), _ptr(s_x), _stream(stream)), "qvla_quant_act_f32")
+    return xq, s_x
+
+
+def qvla_w4a4_gemm(xq: torch.Tensor, s_x: torch.Tensor, L: PackedLinear, split_k: int = 0,
+                   y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M = xq.shape[0]
+    if y is None:
+        y = torch.empty(M, L.N, dtype=torch.bfloat16, device=xq.device)
+    _check(_lib.qvla_w4a4_gemm(_ptr(xq), _ptr(s_x), M, L.struct, _ptr(y), y.stride(0), split_k,
+                               _stream(stream)), "qvla_w4a4_gemm")
+    return y
+
+
+def qvla_w4a4_gemm_s32(xq: torch.Tensor, L: PackedLinear, split_k: int = 0,
+                       stream=None) -> torch.Tensor:
+    M = xq.shape[0]
+    acc = torch.empty(M, L.N, dtype=torch.int32, device=xq.device)
+    _check(_lib.qvla_w4a4_gemm_s32(_ptr(xq), M, L.struct, _ptr(acc), split_k, _stream(stream)),
+           "qvla_w4a4_gemm_s32")
+    return acc
+
+
+def from_host_packed(wq: np.ndarray, s_w: np.ndarray, perm: np.ndarray, rsvd: np.ndarray,
+                     bias: Optional[np.ndarray] = None, device="cuda") -> PackedLinear:
+    """Uploads host arrays into a PackedLinear (e.g. to run the GEMM on given codes)."""
+    N, Kh = wq.shape
+    K = 2 * Kh
+    block = rsvd.shape[-1]
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(device)
+    return PackedLinear(N, K, block, t(perm, np.int32), t(rsvd, np.float32), t(wq, np.uint8),
+                        t(s_w, np.float32), None if bias is None else t(bias, np.float32))
