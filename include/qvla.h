@@ -205,6 +205,8 @@ qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mo
  * xq device [M][K/2]; s_x device [M]; y device bf16 [M][ldy].
  * split_k: 0 = automatic, else 1, 2, 4, 8 or 16, at most ceil(K / 256)
  * (K is consumed in 256-wide tiles; split s takes a contiguous run of them).
+ * Split-K applies for M <= 128; larger M always runs unsplit (its token
+ * tiles supply the parallelism), whatever split_k says.
  * N may be any positive size; ragged M, N and K tails are zero-filled.      */
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
                            const qvla_packed_linear* L, void* y, int ldy, int split_k,

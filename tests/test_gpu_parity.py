@@ -47,7 +47,8 @@ def no_device_error(q):
 @pytest.mark.parametrize("M,K", [(1, 32), (7, 256), (50, 1024), (33, 4096)])
 def test_act_quant_from_fp32_is_bit_exact(q, M, K):
     xr = I.activations(100 + M, M, K, std=1.7, n_outlier_cols=2, dtype="f32")
-    xr[0, :] = 0.0                                   # an all-zero row: s = 0, codes 0
+    if M > 1:
+        xr[M - 1, :] = 0.0                           # an all-zero row: s = 0, codes 0
     qx_ref, s_ref = O.quantize_acts_dynamic_fp32(xr)
     xq, s = q.qvla_quant_act_f32(cu(xr), q.QVLA_SCALE_DYNAMIC)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
@@ -84,7 +85,19 @@ def test_pack_parity(q, N, K, b):
     pk = q.qvla_pack_weights(cu(W), b)
     assert np.array_equal(pk.perm.cpu().numpy(), ref.perm)
     rot = pk.rot.cpu().numpy().astype(np.float64)
-    assert np.abs(rot - ref.rsvd).max() <= 1e-6          # fp32-rounded R_SVD
+    for B in range(K // b):
+        A = W.astype(np.float64)[:, ref.perm[B * b:(B + 1) * b]]
+        lam = np.linalg.eigvalsh(A.T @ A)[::-1]
+        # columns with a simple, non-zero eigenvalue are unique up to the sign
+        # rule and must match; with N < b the null space has no unique basis,
+        # so there only orthonormality and A v = 0 are checked
+        gap = np.minimum(np.r_[np.inf, lam[:-1] - lam[1:]], np.r_[lam[:-1] - lam[1:], np.inf])
+        uniq = (lam > 1e-9 * lam[0]) & (gap > 1e-6 * lam[0])
+        assert np.abs(rot[B][:, uniq] - ref.rsvd[B][:, uniq]).max() <= 1e-6
+        assert np.abs(rot[B].T @ rot[B] - np.eye(b)).max() <= 1e-5
+        null = lam <= 1e-9 * lam[0]
+        if null.any():
+            assert np.abs(A @ rot[B][:, null]).max() <= 1e-5 * np.sqrt(lam[0])
     # with the oracle's perm and R_SVD both sides quantise the same rotation
     pk2 = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
     assert np.array_equal(pk2.w_scale.cpu().numpy().view(np.uint32), ref.s_w.view(np.uint32))
@@ -178,7 +191,7 @@ GEMM_CASES = [
     (1, 256, 256, 0), (16, 256, 256, 1), (50, 4096, 1024, 0), (50, 1024, 4096, 0),
     (64, 384, 1024, 4), (64, 200, 512, 2), (100, 256, 2048, 8), (128, 512, 768, 1),
     (200, 384, 1024, 1), (256, 256, 512, 0), (300, 1000, 1056, 1), (520, 256, 2048, 0),
-    (33, 640, 4096, 16),
+    (33, 640, 4096, 16), (120, 512, 1024, 2), (260, 384, 1024, 4),
 ]
 
 

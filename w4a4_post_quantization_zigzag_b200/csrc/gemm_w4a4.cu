@@ -50,13 +50,14 @@ struct Cfg {
   static constexpr int kRows = kBM + NT;
   static constexpr int kPStageBytes = kRows * kRowP;   // packed: A rows then B rows
   static constexpr int kUStageBytes = kRows * kKU;     // unpacked int8
-  static constexpr int kPS = NT <= 64 ? 2 : (NT == 128 ? 3 : 2);
-  static constexpr int kUS = NT <= 64 ? 2 : (NT == 128 ? 3 : 2);
+  static constexpr int kPS = 2;
+  static constexpr int kUS = 2;
   static constexpr int kTmemCols = NT < 32 ? 32 : NT;
   static constexpr int kRedPitch = NT + 4;             // int32 per row of the split-K buffer
-  static constexpr int kSmemBytes = kPS * kPStageBytes + kUS * kUStageBytes + 1024;
-  static_assert(kBM * kRedPitch * 4 <= kPS * kPStageBytes + kUS * kUStageBytes,
-                "split-K buffer must fit in the stage memory");
+  static constexpr int kStageBytes = kPS * kPStageBytes + kUS * kUStageBytes;
+  static constexpr int kRecvBytes = kBM * kRedPitch * 4;   // split-K receive buffer
+  static constexpr int kSmemBytes = kStageBytes + 1024;    // + kRecvBytes when split
+  static constexpr bool kCanSplit = kSmemBytes + kRecvBytes <= 227 * 1024;
 };
 
 struct Barriers {
@@ -112,13 +113,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = bars.tmem_base;
+  // split-K: announce that this CTA runs; remote shared-memory stores wait for
+  // every CTA of the cluster to have done so
+  if (S > 1) cluster_arrive_relaxed();
+  bool cluster_waited = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
       int issued = 0;
-      for (int i = 0; i < nk && ok; ++i) {
+      // Weights do not depend on the previous kernel in the stream: the first
+      // stages' weight tiles are requested before waiting for it (programmatic
+      // dependent launch), the activation tiles after.
+      const int pre = nk < C::kPS ? nk : C::kPS;
+      // the whole weight range of this CTA is requested into L2 at once, so
+      // HBM streaming is not limited by the depth of the stage ring
+      for (int i = pre; i < nk; ++i) tma_prefetch_l2_2d(&tmap_w, (kt0 + i) * kRowP, n0);
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&bars.full_p[i], C::kPStageBytes);
+        tma_load_2d(pstage + i * C::kPStageBytes, &tmap_w, &bars.full_p[i], (kt0 + i) * kRowP, n0);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) {
+        tma_load_2d(pstage + i * C::kPStageBytes + kBM * kRowP, &tmap_x, &bars.full_p[i],
+                    (kt0 + i) * kRowP, m0);
+        ++issued;
+      }
+      for (int i = pre; i < nk && ok; ++i) {
         const int s = i % C::kPS;
         const uint32_t ph = (i / C::kPS) & 1;
         ok = mbar_wait(&bars.empty_p[s], ph ^ 1u, err);
@@ -210,21 +232,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = n0 + nl;
     const bool have = ok && mbar_wait(&bars.acc_full, 0, err);
     tc_fence_after();
+    pdl_launch_dependents();
+    pdl_wait();                       // s_x comes from the previous kernel
     if (have) {
       const float sw = (n < N) ? __ldg(s_w + n) : 0.f;
       const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
-      int32_t* red = reinterpret_cast<int32_t*>(base);
+      // split-K: this CTA's partial rows go to the receive buffer of the CTA
+      // that owns them (rows [r*128/S, (r+1)*128/S) belong to cluster rank r),
+      // slot `split`, as fire-and-forget distributed-shared-memory stores
+      const int rpr = kBM / S;
+      const uint32_t owner = static_cast<uint32_t>(nl / rpr);
+      const uint32_t recv_row =
+          smem_u32(base + C::kStageBytes) +
+          static_cast<uint32_t>(((split * rpr + nl % rpr) * C::kRedPitch) * 4);
+      const uint32_t remote_row = S > 1 ? map_shared_rank(recv_row, owner) : 0u;
+      if (S > 1) {
+        cluster_wait();
+        cluster_waited = true;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < NT; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
         tmem_ld_wait();
         if (S > 1) {
-          int4* dst = reinterpret_cast<int4*>(red + nl * C::kRedPitch + c0);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            dst[q] = make_int4(static_cast<int>(r[4 * q]), static_cast<int>(r[4 * q + 1]),
-                               static_cast<int>(r[4 * q + 2]), static_cast<int>(r[4 * q + 3]));
+            st_shared_cluster_v4(remote_row + (c0 + 4 * q) * 4,
+                                 make_int4(static_cast<int>(r[4 * q]), static_cast<int>(r[4 * q + 1]),
+                                           static_cast<int>(r[4 * q + 2]),
+                                           static_cast<int>(r[4 * q + 3])));
         } else if (n < N) {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -250,25 +287,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (S > 1) {
     // ------------------------------------------- cluster split-K reduction
-    cluster_sync();
+    if (!cluster_waited) cluster_wait();
+    cluster_sync();                  // every partial tile has landed
     if (warp >= 2) {
       const int wt = tid - 64;
       const uint32_t rank = cluster_ctarank();
       const int rpr = kBM / S;                     // channel rows reduced by this CTA
-      const uint32_t red_u32 = smem_u32(base);
+      const int32_t* recv = reinterpret_cast<const int32_t*>(base + C::kStageBytes);
       for (int e = wt; e < rpr * NT; e += kWorkers) {
-        const int nl = rank * rpr + e % rpr;
+        const int lr = e % rpr;
         const int col = e / rpr;
-        const uint32_t off = static_cast<uint32_t>((nl * C::kRedPitch + col) * 4);
         int32_t sum = 0;
-        for (int src = 0; src < S; ++src) {
-          uint32_t v;
-          asm volatile("ld.shared::cluster.u32 %0, [%1];"
-                       : "=r"(v)
-                       : "r"(map_shared_rank(red_u32 + off, src))
-                       : "memory");
-          sum += static_cast<int32_t>(v);
-        }
+        for (int src = 0; src < S; ++src) sum += recv[(src * rpr + lr) * C::kRedPitch + col];
+        const int nl = rank * rpr + lr;
         const int n = n0 + nl, m = m0 + col;
         if (n < N && m < M) {
           const int32_t a = sum >> 8;
@@ -283,7 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    cluster_sync();
   }
 
   if (warp == 1) {
@@ -330,6 +360,7 @@ bool make_packed_map(CUtensorMap* map, const uint8_t* ptr, int rows, int K, int 
 template <int NT>
 cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
   using C = Cfg<NT>;
+  if (!C::kCanSplit) S = 1;   // large token tiles supply the parallelism themselves
   CUtensorMap mw, mx;
   if (!make_packed_map(&mw, g.wq, g.N, g.K, kBM) || !make_packed_map(&mx, g.xq, g.M, g.K, NT))
     return cudaErrorInvalidValue;
@@ -337,7 +368,8 @@ cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kCanSplit ? C::kSmemBytes + C::kRecvBytes : C::kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
@@ -346,15 +378,24 @@ cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((g.N + kBM - 1) / kBM, (g.M + NT - 1) / NT, S);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmemBytes + (S > 1 ? C::kRecvBytes : 0);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = S;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (S > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = S;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = S > 1 ? 1 : 0;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, mw, mx, g.M, g.N, g.K, g.s_x, g.w_scale, g.bias,
                          static_cast<__nv_bfloat16*>(g.y), g.ldy, g.acc, device_error_word());
   if (e != cudaSuccess) return e;
@@ -365,6 +406,7 @@ cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
 
 int gemm_choose_split(int M, int N, int K) {
   const int nt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  if (nt == 256) return 1;
   const int tiles = ((N + kBM - 1) / kBM) * ((M + nt - 1) / nt);
   const int nkt = (K + kKP - 1) / kKP;
   int S = 1;

@@ -3,6 +3,7 @@
 // permutation and R_SVD eigensolve on the host, everything else on the GPU).
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <thread>
@@ -28,6 +29,14 @@ unsigned int* device_error_word() {
     addr[dev] = static_cast<unsigned int*>(p);
   }
   return addr[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QVLA_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 namespace {

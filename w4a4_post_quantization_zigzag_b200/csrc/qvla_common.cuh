@@ -98,6 +98,15 @@ QVLA_DEVICE void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, uint64_t* 
       : "memory");
 }
 
+// Prefetch a 2-D tile of a tensor-mapped global array into L2 (no shared
+// memory, no completion tracking).
+QVLA_DEVICE void tma_prefetch_l2_2d(const CUtensorMap* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 QVLA_DEVICE void tma_prefetch_desc(const CUtensorMap* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
@@ -206,6 +215,12 @@ QVLA_DEVICE uint32_t cluster_ctarank() {
   return r;
 }
 
+QVLA_DEVICE void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
+QVLA_DEVICE void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
+
 QVLA_DEVICE void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
@@ -223,6 +238,27 @@ QVLA_DEVICE int4 ld_shared_cluster_v4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
+}
+
+// ---------------------------------------------- programmatic dependent launch
+// Blocks until every grid this launch depends on has completed and its memory
+// is visible (no-op when launched without the programmatic attribute).
+QVLA_DEVICE void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the dependent grid in the stream start launching once every CTA of this
+// grid has issued this (or exited).
+QVLA_DEVICE void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+QVLA_DEVICE void st_shared_cluster_v4(uint32_t addr, int4 v) {
+  asm volatile("st.shared::cluster.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+QVLA_DEVICE void st_shared_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 }  // namespace qvla

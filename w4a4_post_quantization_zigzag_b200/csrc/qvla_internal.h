@@ -12,6 +12,9 @@ namespace qvla {
 // Device error word of the current device (lazily resolved symbol address).
 unsigned int* device_error_word();
 
+// Programmatic dependent launch on/off (environment QVLA_PDL=0 turns it off).
+bool pdl_enabled();
+
 // ---- activation rotate + quantise (rotate_quant.cu)
 struct ActArgs {
   const void* x;

@@ -1,15 +1,10 @@
-// Run-time activation rotate + quantise (CUDA-core path).
+// Run-time activation rotate + quantise.
 //
 // For every token row m and rotation block B:
 //     x'_B = H_b . (R_SVD,B^T . x[m, perm[B*b .. B*b+b)])        (fp32)
 // i.e. the row form of x' = R^T P^T x with R = blockdiag(R_SVD,B . H_b)
 // ("{Omega}-QVLA: Robust Quantization ...", Methodology 1: composite
 // SVD.Hadamard rotation applied in blocks after the zigzag permutation).
-// The dense b x b product runs as fp32 FMAs in input order; the Hadamard
-// factor is a fast Walsh-Hadamard transform: butterflies with distance < 32
-// through warp shuffles, larger distances inside each lane's registers, then
-// one multiply by 1/sqrt(b).
-//
 // Scale selection ("Methodology 2", per-step DiT activation scale table;
 // "FoldQuantVLA", dynamic per-token quantisation):
 //     DYNAMIC  s = fp32(max_k |x'[m,k]| / 7) over the whole rotated row
@@ -17,11 +12,24 @@
 // Codes q = clamp(rint(x'/s), -8, 7) (IEEE fp32 division, ties to even),
 // nibble-packed two per byte, even index in the low nibble.
 //
-// Work split: a CTA stages `tpc` token rows in shared memory (fp32) and its
-// warps walk (token, block) items.  DYNAMIC mode keeps whole rows in one CTA
-// and recomputes the rotation in a second pass once the row maximum is known
-// (no scratch memory, one launch); TABLE mode splits the blocks of a row over
-// several CTAs.
+// One CTA owns a tile of TT tokens and a contiguous run of rotation blocks.
+// Per block it
+//   1. gathers x[m, perm[B*b + i]] for its tokens into shared memory (fp32,
+//      token-contiguous), while R_SVD,B streams in through cp.async in
+//      double-buffered chunks of rows;
+//   2. forms R_SVD,B^T x_B with fp32 FMAs in input order, each thread holding a
+//      2-channel x TPT-token register tile;
+//   3. applies the Walsh-Hadamard factor per token in one warp (butterflies with
+//      distance < 32 through shuffles, larger ones in registers) and the
+//      1/sqrt(b) scale.
+// TABLE mode quantises each block at once.  DYNAMIC mode keeps the CTA's
+// rotated slice in shared memory, takes the row maximum across the CTAs of a
+// thread-block cluster (the blocks of a row are split over up to 16 CTAs)
+// through distributed shared memory, then quantises the kept slice: one pass,
+// no scratch memory.
+//
+// Programmatic dependent launch: the permutation slice and the first R_SVD
+// chunk are staged before waiting on the previous kernel in the stream.
 #include <cuda_bf16.h>
 
 #include "qvla_common.cuh"
@@ -32,8 +40,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr size_t kRowSmemBudget = 96 * 1024;
-constexpr size_t kRowSmemCeiling = QVLA_MAX_K * sizeof(float);   // 128 KB: one row at K max
+constexpr int kSmemCap = 220 * 1024;
+
+enum Mode { kTable = 0, kDynamic = 1, kRotateOnly = 2 };
 
 template <int BS>
 struct InvSqrtB;
@@ -54,47 +63,36 @@ struct InvSqrtB<256> {
   static constexpr float v = 0.0625f;
 };
 
-// One warp rotates one block of one token.  On return lane l holds
-// v[c] = x'[B*BS + l + 32c].
 template <int BS>
-QVLA_DEVICE void rotate_block_warp(const float* __restrict__ xs, int K,
-                                   const int32_t* __restrict__ permB,
-                                   const float* __restrict__ RB, int lane, float (&v)[BS / 32]) {
-  constexpr int C = BS / 32;
-  float acc[C];
-#pragma unroll
-  for (int c = 0; c < C; ++c) acc[c] = 0.f;
-  // (R_SVD,B^T x_B)_j = sum_i R_SVD,B[i][j] * x_B[i]
-#pragma unroll 4
-  for (int i = 0; i < BS; ++i) {
-    const int p = __ldg(permB + i);
-    const float xi = xs[static_cast<unsigned>(p) < static_cast<unsigned>(K) ? p : 0];
-    const float* Rrow = RB + i * BS + lane;
-#pragma unroll
-    for (int c = 0; c < C; ++c) acc[c] = fmaf(__ldg(Rrow + 32 * c), xi, acc[c]);
+struct Geo {
+  static constexpr int RCH = BS * BS * 4 <= 32768 ? BS : 8192 / BS;   // R rows per chunk
+  static constexpr int NCH = BS / RCH;                                  // chunks per block
+  static constexpr int kChunkFloats = RCH * BS;
+  static constexpr int NJP = BS / 2;                                    // channel pairs
+  static constexpr int NTG = kThreads / NJP;                            // token groups
+};
+
+template <int BS, int TT>
+struct Smem {
+  // [perm slice][R chunk x2][xg / ys][keep]
+  static size_t bytes(int nbc, bool keep) {
+    size_t b = static_cast<size_t>(nbc) * BS * 4;
+    b = (b + 15) & ~static_cast<size_t>(15);
+    b += 2 * static_cast<size_t>(Geo<BS>::kChunkFloats) * 4;
+    b += static_cast<size_t>(BS) * TT * 4;
+    if (keep) b += static_cast<size_t>(TT) * (nbc * BS + 4) * 4;
+    return b;
   }
-  // Walsh-Hadamard butterflies; element j = lane + 32c.
-#pragma unroll
-  for (int h = 1; h < 32 && h < BS; h <<= 1) {
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-      const float o = __shfl_xor_sync(0xffffffffu, acc[c], h);
-      acc[c] = (lane & h) ? (o - acc[c]) : (acc[c] + o);
-    }
-  }
-#pragma unroll
-  for (int hc = 1; hc < C; hc <<= 1) {
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-      if ((c & hc) == 0) {
-        const float a = acc[c], b = acc[c | hc];
-        acc[c] = a + b;
-        acc[c | hc] = a - b;
-      }
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < C; ++c) v[c] = acc[c] * InvSqrtB<BS>::v;
+};
+
+QVLA_DEVICE void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+QVLA_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+QVLA_DEVICE void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 QVLA_DEVICE int quant_code(float v, float s, int qmin, int qmax) {
@@ -104,132 +102,236 @@ QVLA_DEVICE int quant_code(float v, float s, int qmin, int qmax) {
   return static_cast<int>(r);
 }
 
-template <typename Tin>
-QVLA_DEVICE void stage_row(const Tin* __restrict__ src, float* __restrict__ dst, int K, int tid);
-
-template <>
-QVLA_DEVICE void stage_row<float>(const float* __restrict__ src, float* __restrict__ dst, int K,
-                                  int tid) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-  float4* d4 = reinterpret_cast<float4*>(dst);
-  for (int i = tid; i < K / 4; i += kThreads) d4[i] = __ldg(s4 + i);
+QVLA_DEVICE float load_x(const float* p) { return __ldg(p); }
+QVLA_DEVICE float load_x(const __nv_bfloat16* p) {
+  return __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p)))
+                         << 16);
 }
 
-template <>
-QVLA_DEVICE void stage_row<__nv_bfloat16>(const __nv_bfloat16* __restrict__ src,
-                                          float* __restrict__ dst, int K, int tid) {
-  const uint4* s8 = reinterpret_cast<const uint4*>(src);
-  for (int i = tid; i < K / 8; i += kThreads) {
-    const uint4 u = __ldg(s8 + i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    float4 lo, hi;
-    lo.x = __uint_as_float(w[0] << 16);
-    lo.y = __uint_as_float(w[0] & 0xFFFF0000u);
-    lo.z = __uint_as_float(w[1] << 16);
-    lo.w = __uint_as_float(w[1] & 0xFFFF0000u);
-    hi.x = __uint_as_float(w[2] << 16);
-    hi.y = __uint_as_float(w[2] & 0xFFFF0000u);
-    hi.z = __uint_as_float(w[3] << 16);
-    hi.w = __uint_as_float(w[3] & 0xFFFF0000u);
-    reinterpret_cast<float4*>(dst)[2 * i] = lo;
-    reinterpret_cast<float4*>(dst)[2 * i + 1] = hi;
-  }
-}
-
-// Resolves the table scale; returns false (and flags the error word) when the
-// device step index lies outside the table.
-QVLA_DEVICE bool table_scale(const float* table, int T, int Lcount, const int32_t* step_dev,
-                             int step_host, int layer, float* s, unsigned int* err) {
+// Resolves the table scale; flags the error word and returns 0 when the step
+// or layer lies outside the table (never reads outside it).
+QVLA_DEVICE float table_scale(const float* table, int T, int Lcount, const int32_t* step_dev,
+                              int step_host, int layer, unsigned int* err) {
   const int step = step_dev ? *step_dev : step_host;
   if (step < 0 || step >= T || layer < 0 || layer >= Lcount) {
-    if (threadIdx.x == 0) report(err, QVLA_DEVERR_STEP_RANGE);
-    *s = 0.f;
-    return false;
+    report(err, QVLA_DEVERR_STEP_RANGE);
+    return 0.f;
   }
-  *s = __ldg(table + static_cast<size_t>(step) * Lcount + layer);
-  return true;
+  return __ldg(table + static_cast<size_t>(step) * Lcount + layer);
 }
 
-template <int BS, typename Tin, bool kRotateOnly>
-__global__ void __launch_bounds__(kThreads)
-    rotate_quant_kernel(const Tin* __restrict__ x, int M, int ldx, int K,
-                        const int32_t* __restrict__ perm, const float* __restrict__ rot,
-                        int dynamic, const float* __restrict__ table, int T, int Lcount,
-                        const int32_t* __restrict__ step_dev, int step_host, int layer,
-                        uint8_t* __restrict__ xq, float* __restrict__ s_x,
-                        float* __restrict__ xr_out, unsigned int* err, int tpc, int bpc) {
+template <int BS>
+QVLA_DEVICE void fwht_lanes(float (&v)[BS / 32], int lane) {
   constexpr int C = BS / 32;
-  extern __shared__ __align__(16) float smem_rows[];
-  __shared__ unsigned int amax_bits[8];
-  __shared__ float s_table;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int m0 = blockIdx.x * tpc;
-  const int ntok = min(tpc, M - m0);
-  const int nb = K / BS;
-  const int b0 = blockIdx.y * bpc;
-  const int nblk = min(bpc, nb - b0);
-  if (ntok <= 0 || nblk <= 0) return;
-
-  for (int t = 0; t < ntok; ++t)
-    stage_row<Tin>(x + static_cast<size_t>(m0 + t) * ldx, smem_rows + static_cast<size_t>(t) * K,
-                   K, tid);
-  if (tid < 8) amax_bits[tid] = 0u;
-  if (tid == 0) {
-    float s = 0.f;
-    if (!kRotateOnly && !dynamic) table_scale(table, T, Lcount, step_dev, step_host, layer, &s, err);
-    s_table = s;
-  }
-  __syncthreads();
-
-  const int nitems = ntok * nblk;
-  float v[C];
-
-  if (kRotateOnly) {
-    for (int it = warp; it < nitems; it += kWarps) {
-      const int t = it / nblk, B = b0 + it % nblk;
-      rotate_block_warp<BS>(smem_rows + static_cast<size_t>(t) * K, K, perm + B * BS,
-                            rot + static_cast<size_t>(B) * BS * BS, lane, v);
-      float* dst = xr_out + static_cast<size_t>(m0 + t) * K + B * BS + lane;
 #pragma unroll
-      for (int c = 0; c < C; ++c) dst[32 * c] = v[c];
-    }
-    return;
-  }
-
-  if (dynamic) {
-    // pass 1: row maxima of |x'|
-    for (int it = warp; it < nitems; it += kWarps) {
-      const int t = it / nblk, B = b0 + it % nblk;
-      rotate_block_warp<BS>(smem_rows + static_cast<size_t>(t) * K, K, perm + B * BS,
-                            rot + static_cast<size_t>(B) * BS * BS, lane, v);
-      float mx = 0.f;
-#pragma unroll
-      for (int c = 0; c < C; ++c) mx = fmaxf(mx, fabsf(v[c]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) atomicMax(&amax_bits[t], __float_as_uint(mx));
-    }
-    __syncthreads();
-  }
-
-  // pass 2: quantise and pack
-  for (int it = warp; it < nitems; it += kWarps) {
-    const int t = it / nblk, B = b0 + it % nblk;
-    rotate_block_warp<BS>(smem_rows + static_cast<size_t>(t) * K, K, perm + B * BS,
-                          rot + static_cast<size_t>(B) * BS * BS, lane, v);
-    const float s = dynamic ? __fdiv_rn(__uint_as_float(amax_bits[t]), 7.0f) : s_table;
-    uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS) / 2;
+  for (int h = 1; h < 32 && h < BS; h <<= 1) {
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-      const int q = quant_code(v[c], s, -8, 7);
-      const int qn = __shfl_down_sync(0xffffffffu, q, 1);
-      if ((lane & 1) == 0) dst[(lane + 32 * c) >> 1] = static_cast<uint8_t>((q & 15) | ((qn & 15) << 4));
+      const float o = __shfl_xor_sync(0xffffffffu, v[c], h);
+      v[c] = (lane & h) ? (o - v[c]) : (v[c] + o);
     }
   }
+#pragma unroll
+  for (int hc = 1; hc < C; hc <<= 1) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      if ((c & hc) == 0) {
+        const float a = v[c], b = v[c | hc];
+        v[c] = a + b;
+        v[c | hc] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < C; ++c) v[c] *= InvSqrtB<BS>::v;
+}
 
-  if (blockIdx.y == 0 && tid < ntok)
-    s_x[m0 + tid] = dynamic ? __fdiv_rn(__uint_as_float(amax_bits[tid]), 7.0f) : s_table;
+// Packs the codes of 32 consecutive channels (lane l holds channel l) into 16
+// bytes and stores them as four 32-bit words from lanes 0, 8, 16, 24.
+QVLA_DEVICE void store_codes32(uint8_t* dst, int q, int lane) {
+  const int qn = __shfl_down_sync(0xffffffffu, q, 1);
+  const uint32_t byte = static_cast<uint32_t>((q & 15) | ((qn & 15) << 4));   // even lanes
+  const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 2);
+  const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 4);
+  const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 6);
+  if ((lane & 7) == 0)
+    *reinterpret_cast<uint32_t*>(dst + (lane >> 1)) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+template <int BS, int TT, typename Tin, int MODE>
+__global__ void __launch_bounds__(kThreads)
+    rotq_kernel(const Tin* __restrict__ x, int M, int ldx, int K,
+                const int32_t* __restrict__ perm, const float* __restrict__ rot,
+                const float* __restrict__ table, int T, int Lcount,
+                const int32_t* __restrict__ step_dev, int step_host, int layer,
+                uint8_t* __restrict__ xq, float* __restrict__ s_x, float* __restrict__ xr_out,
+                unsigned int* err, int blocks_per_cta) {
+  using G = Geo<BS>;
+  constexpr int C = BS / 32;
+  constexpr int TPT = TT / G::NTG;          // tokens per thread in the product
+  static_assert(TPT >= 1, "token tile too small for this block size");
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ unsigned int amax_s[TT];
+  __shared__ float scale_s[TT];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int m0 = blockIdx.x * TT;
+  const int ntok = min(TT, M - m0);
+  const int nb = K / BS;
+  const int B0 = blockIdx.y * blocks_per_cta;
+  const int nbc = max(0, min(blocks_per_cta, nb - B0));
+
+  int32_t* perm_s = reinterpret_cast<int32_t*>(smem);
+  float* rbuf = reinterpret_cast<float*>(
+      smem + ((static_cast<size_t>(blocks_per_cta) * BS * 4 + 15) & ~static_cast<size_t>(15)));
+  float* xg = rbuf + 2 * G::kChunkFloats;     // [BS][TT], later ys [TT][BS]
+  float* keep = xg + BS * TT;                  // [TT][blocks_per_cta*BS + 4]  (DYNAMIC only)
+  const int kpitch = blocks_per_cta * BS + 4;
+
+  // ---- prologue: weight-side data, independent of the previous kernel
+  for (int e = tid; e < nbc * BS; e += kThreads) perm_s[e] = __ldg(perm + B0 * BS + e);
+  if (tid < TT) amax_s[tid] = 0u;
+  const int nchunks = nbc * G::NCH;
+  auto issue_chunk = [&](int g) {
+    const int bl = g / G::NCH, ch = g % G::NCH;
+    const float* src = rot + (static_cast<size_t>(B0 + bl) * BS + ch * G::RCH) * BS;
+    float* dst = rbuf + (g & 1) * G::kChunkFloats;
+    for (int e = tid * 4; e < G::kChunkFloats; e += kThreads * 4) cp_async16(dst + e, src + e);
+    cp_async_commit();
+  };
+  if (nchunks > 0) issue_chunk(0);
+
+  pdl_wait();
+  pdl_launch_dependents();
+  float s_tab = 0.f;
+  if (MODE == kTable) s_tab = table_scale(table, T, Lcount, step_dev, step_host, layer, err);
+  __syncthreads();   // perm_s visible
+
+  const int jp = tid % G::NJP, tg = tid / G::NJP;
+  for (int bl = 0; bl < nbc; ++bl) {
+    const int B = B0 + bl;
+    // 1. gather the block's inputs, token-contiguous
+    for (int e = tid; e < BS * TT; e += kThreads) {
+      const int i = e / TT, t = e % TT;
+      const int p = perm_s[bl * BS + i];
+      float v = 0.f;
+      if (t < ntok && static_cast<unsigned>(p) < static_cast<unsigned>(K))
+        v = load_x(x + static_cast<size_t>(m0 + t) * ldx + p);
+      xg[e] = v;
+    }
+    // 2. dense product over R chunks
+    float acc[TPT][2];
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) acc[u][0] = acc[u][1] = 0.f;
+    for (int ch = 0; ch < G::NCH; ++ch) {
+      const int g = bl * G::NCH + ch;
+      if (g + 1 < nchunks) {
+        issue_chunk(g + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const float* Rc = rbuf + (g & 1) * G::kChunkFloats;
+#pragma unroll 4
+      for (int ii = 0; ii < G::RCH; ++ii) {
+        const float2 r = *reinterpret_cast<const float2*>(Rc + ii * BS + 2 * jp);
+        const float* xrow = xg + (ch * G::RCH + ii) * TT + tg * TPT;
+#pragma unroll
+        for (int u = 0; u < TPT; ++u) {
+          const float xv = xrow[u];
+          acc[u][0] = fmaf(r.x, xv, acc[u][0]);
+          acc[u][1] = fmaf(r.y, xv, acc[u][1]);
+        }
+      }
+      __syncthreads();   // chunk buffer (g & 1) may be refilled next
+    }
+    // 3. stage the products token-major (over the gather buffer)
+#pragma unroll
+    for (int u = 0; u < TPT; ++u)
+      *reinterpret_cast<float2*>(xg + (tg * TPT + u) * BS + 2 * jp) =
+          make_float2(acc[u][0], acc[u][1]);
+    __syncthreads();
+    // 4. Hadamard factor per token, then quantise / keep / store
+    for (int t = warp; t < ntok; t += kWarps) {
+      float v[C];
+#pragma unroll
+      for (int c = 0; c < C; ++c) v[c] = xg[t * BS + lane + 32 * c];
+      fwht_lanes<BS>(v, lane);
+      if (MODE == kRotateOnly) {
+        float* dst = xr_out + static_cast<size_t>(m0 + t) * K + B * BS + lane;
+#pragma unroll
+        for (int c = 0; c < C; ++c) dst[32 * c] = v[c];
+      } else if (MODE == kTable) {
+        uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS) / 2;
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+          store_codes32(dst + 16 * c, quant_code(v[c], s_tab, -8, 7), lane);
+      } else {
+        float mx = 0.f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+          keep[t * kpitch + bl * BS + lane + 32 * c] = v[c];
+          mx = fmaxf(mx, fabsf(v[c]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(&amax_s[t], __float_as_uint(mx));
+      }
+    }
+    __syncthreads();   // gather buffer reused by the next block
+  }
+
+  if (MODE == kTable) {
+    if (blockIdx.y == 0 && tid < ntok) s_x[m0 + tid] = s_tab;
+    return;
+  }
+  if (MODE == kRotateOnly) return;
+
+  // ---- DYNAMIC: row maximum over the cluster, then quantise the kept slice
+  const int cs = gridDim.y;                    // the cluster spans grid y
+  if (cs > 1) {
+    cluster_sync();                            // partial maxima published
+    if (tid < TT) {
+      unsigned int mx = 0u;
+      const uint32_t a = smem_u32(&amax_s[tid]);
+      for (int r = 0; r < cs; ++r) {
+        uint32_t v;
+        asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                     : "=r"(v)
+                     : "r"(map_shared_rank(a, static_cast<uint32_t>(r)))
+                     : "memory");
+        mx = max(mx, v);
+      }
+      scale_s[tid] = __fdiv_rn(__uint_as_float(mx), 7.0f);
+    }
+    cluster_arrive_relaxed();                  // done reading peers' maxima
+  } else if (tid < TT) {
+    scale_s[tid] = __fdiv_rn(__uint_as_float(amax_s[tid]), 7.0f);
+  }
+  __syncthreads();
+  if (blockIdx.y == 0 && tid < ntok) s_x[m0 + tid] = scale_s[tid];
+  const int nch = nbc * BS;                    // channels held by this CTA (multiple of 32)
+  for (int t = warp; t < ntok; t += kWarps) {
+    const float s = scale_s[t];
+    uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B0 * BS) / 2;
+    for (int c0 = 0; c0 < nch; c0 += 256) {
+      const int k = c0 + 8 * lane;            // 8 channels -> 4 bytes per lane
+      if (k < nch) {
+        const float4 a = *reinterpret_cast<const float4*>(keep + t * kpitch + k);
+        const float4 b = *reinterpret_cast<const float4*>(keep + t * kpitch + k + 4);
+        const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t w = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int lo = quant_code(f[2 * q], s, -8, 7), hi = quant_code(f[2 * q + 1], s, -8, 7);
+          w |= static_cast<uint32_t>((lo & 15) | ((hi & 15) << 4)) << (8 * q);
+        }
+        *reinterpret_cast<uint32_t*>(dst + k / 2) = w;
+      }
+    }
+  }
+  if (cs > 1) cluster_wait();                  // peers finished reading our maxima
 }
 
 // Quantise fp32 rows (already rotated): one CTA per row.
@@ -256,9 +358,7 @@ __global__ void __launch_bounds__(kThreads)
       s_sh = __fdiv_rn(m, static_cast<float>(qmax));
     }
   } else if (tid == 0) {
-    float s;
-    table_scale(table, T, Lcount, step_dev, step_host, layer, &s, err);
-    s_sh = s;
+    s_sh = table_scale(table, T, Lcount, step_dev, step_host, layer, err);
   }
   __syncthreads();
   const float s = s_sh;
@@ -271,59 +371,101 @@ __global__ void __launch_bounds__(kThreads)
   if (tid == 0) s_out[row] = s;
 }
 
-template <int BS, typename Tin, bool kRotateOnly>
-cudaError_t launch_bs(const ActArgs& a, cudaStream_t stream) {
+template <int BS, int TT, typename Tin, int MODE>
+cudaError_t launch_cfg(const ActArgs& a, cudaStream_t stream) {
   const int K = a.K, nb = K / BS;
-  int tpc = static_cast<int>(kRowSmemBudget / (static_cast<size_t>(K) * sizeof(float)));
-  tpc = tpc < 1 ? 1 : (tpc > 8 ? 8 : tpc);
-  const int gx = (a.M + tpc - 1) / tpc;
-  int gy = 1;
-  if (!a.dynamic || kRotateOnly) {
+  const int gx = (a.M + TT - 1) / TT;
+  int bpc, gy, cs = 1;
+  if (MODE == kDynamic) {
+    // split the row's blocks over a cluster of cs CTAs: enough CTAs to fill the
+    // GPU and a kept slice that fits in shared memory
+    while (cs < 16 && cs < nb &&
+           (gx * cs < 148 || Smem<BS, TT>::bytes((nb + cs - 1) / cs, true) > kSmemCap))
+      cs *= 2;
+    bpc = (nb + cs - 1) / cs;
+    gy = cs;
+    if (Smem<BS, TT>::bytes(bpc, true) > kSmemCap) return cudaErrorInvalidConfiguration;
+  } else {
     const int target = 2 * 148;
-    gy = (target + gx - 1) / gx;
-    if (gy > nb) gy = nb;
-    if (gy < 1) gy = 1;
+    int g = (target + gx - 1) / gx;
+    g = g < 1 ? 1 : (g > nb ? nb : g);
+    bpc = (nb + g - 1) / g;
+    gy = (nb + bpc - 1) / bpc;
   }
-  const int bpc = (nb + gy - 1) / gy;
-  gy = (nb + bpc - 1) / bpc;
-  const size_t smem = static_cast<size_t>(tpc) * K * sizeof(float);
-  auto kern = rotate_quant_kernel<BS, Tin, kRotateOnly>;
-  // one fixed ceiling per kernel (the largest row stage any K can ask for), so
-  // launches captured in a graph never see the attribute shrink afterwards
+  const size_t smem = Smem<BS, TT>::bytes(bpc, MODE == kDynamic);
+  auto kern = rotq_kernel<BS, TT, Tin, MODE>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kRowSmemCeiling));
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
     if (e != cudaSuccess) return e;
+    if (MODE == kDynamic) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
-  if (smem > kRowSmemCeiling) return cudaErrorInvalidValue;
-  kern<<<dim3(gx, gy), kThreads, smem, stream>>>(
-      static_cast<const Tin*>(a.x), a.M, a.ldx, K, a.perm, a.rot, a.dynamic, a.table, a.T,
-      a.Lcount, a.step_dev, a.step_host, a.layer, a.xq, a.s_x, a.xr_out, device_error_word(),
-      tpc, bpc);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, gy, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cs > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = cs;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(a.x), a.M, a.ldx, K,
+                                     a.perm, a.rot, a.table, a.T, a.Lcount, a.step_dev,
+                                     a.step_host, a.layer, a.xq, a.s_x, a.xr_out,
+                                     device_error_word(), bpc);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <typename Tin, bool kRotateOnly>
-cudaError_t launch_t(const ActArgs& a, cudaStream_t stream) {
+template <int BS, typename Tin, int MODE>
+cudaError_t launch_tt(const ActArgs& a, cudaStream_t stream) {
+  // token tile: 16 for small M, block 32 or very long dynamic rows (keeps the
+  // dynamic slice in shared memory), else 32
+  if (a.M <= 16 || BS == 32 || (MODE == kDynamic && a.K > 8192))
+    return launch_cfg<BS, 16, Tin, MODE>(a, stream);
+  return launch_cfg<BS, 32, Tin, MODE>(a, stream);
+}
+
+template <typename Tin, int MODE>
+cudaError_t launch_bs(const ActArgs& a, cudaStream_t stream) {
   switch (a.block) {
-    case 32: return launch_bs<32, Tin, kRotateOnly>(a, stream);
-    case 64: return launch_bs<64, Tin, kRotateOnly>(a, stream);
-    case 128: return launch_bs<128, Tin, kRotateOnly>(a, stream);
-    case 256: return launch_bs<256, Tin, kRotateOnly>(a, stream);
+    case 32: return launch_tt<32, Tin, MODE>(a, stream);
+    case 64: return launch_tt<64, Tin, MODE>(a, stream);
+    case 128: return launch_tt<128, Tin, MODE>(a, stream);
+    case 256: return launch_tt<256, Tin, MODE>(a, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <typename Tin>
+cudaError_t launch_mode(const ActArgs& a, cudaStream_t stream) {
+  if (a.xq == nullptr) return launch_bs<Tin, kRotateOnly>(a, stream);
+  if (a.dynamic) return launch_bs<Tin, kDynamic>(a, stream);
+  return launch_bs<Tin, kTable>(a, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream) {
-  const bool rot_only = a.xq == nullptr;
-  if (a.xdt == QVLA_DTYPE_BF16)
-    return rot_only ? launch_t<__nv_bfloat16, true>(a, stream)
-                    : launch_t<__nv_bfloat16, false>(a, stream);
-  return rot_only ? launch_t<float, true>(a, stream) : launch_t<float, false>(a, stream);
+  if (a.xdt == QVLA_DTYPE_BF16) return launch_mode<__nv_bfloat16>(a, stream);
+  return launch_mode<float>(a, stream);
 }
 
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream) {
