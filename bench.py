@@ -4,8 +4,11 @@
 Default workload: the DiT action-head MLP stack (50 action tokens x batch 1,
 hidden 1024, gate/up 1024->4096 and down 4096->1024, 4 layers, bf16 input,
 10 denoising steps, per-step scale table [10][12], rotation block 64).
-One timed step = one denoising step = 12 rotated W4A4 linears, each a fused
-rotate-quantise launch plus a W4A4 GEMM launch, replayed from a CUDA graph.
+One timed step = one denoising step = 12 rotated W4A4 linears: one batched
+rotate-quantise launch for all 12, then one batched W4A4 GEMM launch for all 12
+(the step's linears are independent: each draws its own input), replayed from a
+CUDA graph.  The same step with one launch per kernel and linear is reported
+beside it.
 The activation step index is a device scalar read by the rotate-quantise
 kernel.  L2 is flushed (512 MB write) before every timed step, so every step
 streams its packed weights from HBM.
@@ -133,6 +136,27 @@ def recorded_traffic(kernel, workload):
     return float(rec["dram_bytes_per_launch"])
 
 
+# --------------------------------------------------------- replica timing
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank timing over all ranks (identity without a process
+    group).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_time_per_unit(total_ms: float, steps: int, world: int) -> float:
+    """Job-level microseconds per unit of work: N replicas each run `steps`
+    units in (max over ranks) total_ms."""
+    return total_ms * 1e3 / (steps * world)
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_step(wl, packs, xs, t):
     from oracle import qvla_oracle as O
@@ -250,30 +274,47 @@ def run_ours(args):
     xq = [torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev) for l in wl.linears]
     sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
     ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
+    nl = len(wl.linears)
+    # one problem set per denoising step: same packed weights and buffers, the
+    # step's own inputs and device step index
+    probs = [[Q.LinearProblem(L, xs[t][i], mode, table=table, step=steps_dev[t:t + 1],
+                              layer=lin.layer, xq=xq[i], s_x=sx[i], y=ys[i])
+              for i, (lin, L) in enumerate(zip(wl.linears, packs))] for t in range(T)]
 
-    def step(t, rec=None):
+    def step_batched(t, rec=None):
+        if rec is not None:
+            rec[0].record()
+        Q.qvla_rotate_quant_act_batched(probs[t])
+        if rec is not None:
+            rec[1].record()
+        Q.qvla_w4a4_gemm_batched(probs[t])
+        if rec is not None:
+            rec[2].record()
+
+    def step_per_linear(t):
         for i, (lin, L) in enumerate(zip(wl.linears, packs)):
-            if rec is not None:
-                rec[i][0].record()
             Q.qvla_rotate_quant_act(xs[t][i], L, mode, table=table, step=steps_dev[t:t + 1],
                                     layer=lin.layer, xq=xq[i], s_x=sx[i])
-            if rec is not None:
-                rec[i][1].record()
             Q.qvla_w4a4_gemm(xq[i], sx[i], L, y=ys[i])
-            if rec is not None:
-                rec[i][2].record()
 
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    with torch.cuda.stream(stream):
-        step(0)                       # first call resolves attributes outside capture
-        torch.cuda.synchronize()
-        graphs = []
+
+    def capture(fn):
+        gs = []
         for t in range(T):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                step(t)
-            graphs.append(g)
+                fn(t)
+            gs.append(g)
+        return gs
+
+    with torch.cuda.stream(stream):
+        step_batched(0)               # first calls resolve attributes outside capture
+        step_per_linear(0)
+        torch.cuda.synchronize()
+        graphs = capture(step_batched)
+        graphs_pl = capture(step_per_linear)
     torch.cuda.synchronize()
     assert Q.qvla_read_error_word(clear=True) == 0
 
@@ -283,49 +324,57 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed_replays(gs, n):
+        starts = [ev() for _ in range(n)]
+        ends = [ev() for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                flush.zero_()
+                starts[i].record()
+                gs[i % T].replay()
+                ends[i].record()
+        return starts, ends
+
     # ---- warm-up
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             flush.zero_()
             graphs[i % T].replay()
-    # ---- timed steps: graph replay, L2 flushed before each
-    starts = [ev() for _ in range(args.steps)]
-    ends = [ev() for _ in range(args.steps)]
+            flush.zero_()
+            graphs_pl[i % T].replay()
+    # ---- timed steps: graph replay of the batched step, L2 flushed before each
     gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_uuid) if not args.quick else None
     barrier()
     if sampler:
         sampler.__enter__()
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record()
-            graphs[i % T].replay()
-            ends[i].record()
+    starts, ends = timed_replays(graphs, args.steps)
     barrier()
     if sampler:
         sampler.__exit__()
-    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    tot_ms = sum(per_step_ms)
-    if world > 1:
-        tt = torch.tensor([tot_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        tot_ms = float(tt.item())
+    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    tot_ms = max_over_ranks(sum(per_step_ms), dev)
     ms_per_step = tot_ms / args.steps
-    us_job = tot_ms * 1e3 / (args.steps * world)
+    us_job = job_time_per_unit(tot_ms, args.steps, world)
 
-    # ---- per-kernel breakdown (eager launches, events on the launching stream)
-    nl = len(wl.linears)
+    # ---- the same steps, one launch per kernel and linear (informational)
+    s2, e2 = timed_replays(graphs_pl, args.steps)
+    torch.cuda.synchronize()
+    per_linear_us = sum(a.elapsed_time(b) for a, b in zip(s2, e2)) * 1e3 / args.steps
+
+    # ---- per-kernel breakdown: eager launches with events on the launching
+    # stream; a GPU sleep ahead of the events keeps host enqueue time out
     krot, kgemm = [], []
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            rec = [[ev(), ev(), ev()] for _ in range(nl)]
+            rec = [ev(), ev(), ev()]
             flush.zero_()
-            step(i % T, rec)
+            torch.cuda._sleep(2_000_000)
+            step_batched(i % T, rec)
             stream.synchronize()
-            for j in range(nl):
-                krot.append((j, rec[j][0].elapsed_time(rec[j][1])))
-                kgemm.append((j, rec[j][1].elapsed_time(rec[j][2])))
+            krot.append(rec[0].elapsed_time(rec[1]))
+            kgemm.append(rec[1].elapsed_time(rec[2]))
     assert Q.qvla_read_error_word(clear=True) == 0
 
     # ---- end to end: pinned-host inputs in, outputs back, every step
@@ -347,12 +396,8 @@ def run_ours(args):
                     y_h.copy_(y_d, non_blocking=True)
             e1.record()
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": e2e_ms * 1e3 / (args.steps * world), "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": job_time_per_unit(e2e_ms, args.steps, world), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- roofline of the dominant kernel
@@ -361,13 +406,13 @@ def run_ours(args):
                      for l in wl.linears)
     rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + l.M * l.K // 2 + 4 * l.M
                     + 4 * l.K * l.block + 4 * l.K for l in wl.linears)
-    t_gemm = sum(t for _, t in kgemm) / args.steps          # ms per step
-    t_rot = sum(t for _, t in krot) / args.steps
+    t_gemm = sum(kgemm) / args.steps          # ms per step (one batched launch)
+    t_rot = sum(krot) / args.steps
     dom = "w4a4_gemm" if t_gemm >= t_rot else "rotate_quant"
     if dom == "w4a4_gemm":
-        per_launch_bytes, per_launch_ms = gemm_bytes / nl, t_gemm / nl
+        per_launch_bytes, per_launch_ms = gemm_bytes, t_gemm
     else:
-        per_launch_bytes, per_launch_ms = rot_bytes / nl, t_rot / nl
+        per_launch_bytes, per_launch_ms = rot_bytes, t_rot
     achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
     roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "peak_source": f"hbm_gbs ({peak_src})",
@@ -388,10 +433,10 @@ def run_ours(args):
         "roofline": roof,
         "tops": ops / (ms_per_step * 1e-3) / 1e12,
         "weight_gbs": wl.packed_weight_bytes() / (ms_per_step * 1e-3) / 1e9,
-        "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3,
-                                "eager_sum": (t_rot + t_gemm) * 1e3},
+        "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3},
+        "per_linear_launches_us_per_step": per_linear_us,
         "pack_s": pack_s,
-        "gpu_launches": 2 * nl * args.steps,
+        "gpu_launches": 2 * args.steps,
         "e2e": e2e,
     }
     if sampler:
@@ -400,7 +445,7 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_steps)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
+    del graphs, graphs_pl
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -217,6 +217,41 @@ qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
 qvla_status qvla_w4a4_gemm_s32(const uint8_t* xq, int M, const qvla_packed_linear* L,
                                int32_t* acc, int split_k, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Batched calls: several INDEPENDENT linears (each with its own packed
+ * weights, input, codes and output; e.g. the gate and up projections of an
+ * MLP, q/k/v, or the linears of a denoising step whose inputs are already
+ * known) run in as few launches as possible instead of one launch each.
+ * Linears are grouped by kernel configuration (rotation block, token tile,
+ * input type, scale mode); each launch takes up to 16 of them.  Results are
+ * identical to calling the single-linear entry points one by one.  No two
+ * problems may share an output buffer.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const qvla_packed_linear* L;   /* host pointer to the packed linear          */
+  const void* x;                 /* device [M][ldx] activations (rotate-quant) */
+  int32_t xdt;                   /* qvla_dtype                                  */
+  int32_t M, ldx;
+  int32_t mode;                  /* qvla_scale_mode                             */
+  const float* table;            /* device [T][Lcount] for TABLE mode           */
+  int32_t T, Lcount;
+  const int32_t* step_dev;       /* device step index or NULL (use step_host)   */
+  int32_t step_host, layer;
+  uint8_t* xq;                   /* device [M][K/2] codes: output, then input   */
+  float* s_x;                    /* device [M] scales: output, then input       */
+  void* y;                       /* device bf16 [M][ldy] GEMM output            */
+  int32_t ldy;
+} qvla_linear_problem;
+
+/* qvla_rotate_quant_act for every problem (reads x, writes xq and s_x). */
+qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int n,
+                                          cudaStream_t stream);
+
+/* qvla_w4a4_gemm for every problem (reads xq and s_x, writes y); split_k as
+ * for qvla_w4a4_gemm, one factor shared by all problems of a launch.        */
+qvla_status qvla_w4a4_gemm_batched(const qvla_linear_problem* probs, int n, int split_k,
+                                   cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

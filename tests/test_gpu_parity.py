@@ -267,3 +267,40 @@ def test_dit_mlp_layer_each_kind(q):
         for step in (0, 9):
             _layer(q, lin, "table", wl.table, step, x_std=float(wl.sigmas[step]))
     no_device_error(q)
+
+
+# ------------------------------------------------------------ batched calls
+
+def test_batched_calls_match_single_calls(q):
+    """Independent linears in one batched call give the same bytes and outputs
+    as one call each (mixed block sizes, modes, dtypes, token tiles, M = 0)."""
+    specs = [  # M, K, N, b, mode, dtype
+        (50, 1024, 4096, 64, "table", "bf16"), (50, 4096, 1024, 64, "table", "bf16"),
+        (50, 1024, 512, 64, "table", "bf16"), (16, 256, 256, 64, "dynamic", "f32"),
+        (37, 2048, 384, 128, "dynamic", "bf16"), (200, 512, 256, 32, "table", "bf16"),
+        (0, 256, 128, 64, "table", "bf16"), (3, 1024, 256, 256, "dynamic", "bf16"),
+    ]
+    tab = cu(I.scale_table(11, 6, 8, I.step_sigmas(6)))
+    step = torch.tensor([5], dtype=torch.int32, device="cuda")
+    probs, singles = [], []
+    for i, (M, K, N, b, mode, dt) in enumerate(specs):
+        W = I.weights(1100 + i, N, K)
+        L = q.qvla_pack_weights(cu(W), b, bias=cu(I.bias(1150 + i, N)))
+        x = x_dev(I.activations(1200 + i, max(M, 1), K, n_outlier_cols=2, dtype=dt), dt)[:M]
+        md = q.QVLA_SCALE_TABLE if mode == "table" else q.QVLA_SCALE_DYNAMIC
+        kw = dict(table=tab, step=step, layer=i) if mode == "table" else {}
+        probs.append(q.LinearProblem(L, x, md, **kw))
+        if M:
+            xq, s = q.qvla_rotate_quant_act(x, L, md, **kw)
+            singles.append((xq, s, q.qvla_w4a4_gemm(xq, s, L)))
+        else:
+            singles.append(None)
+    q.qvla_rotate_quant_act_batched(probs)
+    q.qvla_w4a4_gemm_batched(probs)
+    torch.cuda.synchronize()
+    for p, ref in zip(probs, singles):
+        if ref is None:
+            continue
+        assert torch.equal(p.xq, ref[0]) and torch.equal(p.s_x, ref[1])
+        assert torch.equal(p.y, ref[2])
+    no_device_error(q)

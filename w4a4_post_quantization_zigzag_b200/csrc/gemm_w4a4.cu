@@ -11,8 +11,8 @@
 //   1. TMA-loads packed int4 tiles (128 bytes of K per row, 128B swizzle) of
 //      the weights [128 rows] and the activations [NT rows] into a ring of
 //      shared-memory stages (one elected producer thread);
-//   2. unpacks them with four warps into the UMMA K-major "interleaved"
-//      layout: every code q becomes the int8 value 16*q (its nibble moved into
+//   2. unpacks them with four warps into 128-byte-swizzled K-major UMMA
+//      operand rows: every code q becomes the int8 value 16*q (its nibble moved into
 //      the high half of the byte: `w & 0xF0F0F0F0` for odd codes,
 //      `(w << 4) & 0xF0F0F0F0` for even codes).  Even codes of a 32-code
 //      group fill the first 16-byte K chunk and odd codes the second; both
@@ -21,7 +21,8 @@
 //      from one thread into an int32 accumulator in tensor memory, which
 //      therefore holds 256*acc exactly;
 //   4. reads the accumulator back with tcgen05.ld (one output channel per
-//      thread, tokens along registers) and applies the epilogue.
+//      thread, tokens along registers), applies the epilogue into a bf16
+//      shared-memory tile and writes it back with one TMA tensor store.
 // Weights take the UMMA M slot and tokens the N slot for every M, so the small
 // token counts of a DiT action chunk (16-64) still fill a 128-row MMA.
 // Small M adds split-K over a thread-block cluster along grid z: every CTA of
@@ -31,6 +32,10 @@
 // All waits are bounded (2 s) and flag QVLA_DEVERR_TIMEOUT instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstring>
+#include <vector>
 
 #include "qvla_common.cuh"
 #include "qvla_internal.h"
@@ -65,22 +70,61 @@ struct Barriers {
   uint32_t tmem_base;
 };
 
+// One linear of a batched launch.  Independent linears (different weights,
+// inputs and outputs) share one launch; CTAs are numbered problem by problem.
+constexpr int kMaxBatch = 16;
+struct GemmProblem {
+  CUtensorMap tw;                 // packed weights  [N][K/2]
+  CUtensorMap tx;                 // packed codes    [M][K/2]
+  CUtensorMap ty;                 // bf16 output [M][ldy], box = (128/S channels) x NT tokens
+  const float* s_x;
+  const float* s_w;
+  const float* bias;
+  __nv_bfloat16* y;
+  int32_t* acc;
+  int M, N, K, ldy;
+  int tiles_n;                    // ceil(N / 128)
+  int tiles;                      // tiles_n * ceil(M / NT)
+  int S;                          // split-K factor: 1 or the launch's cluster size
+};
+struct GemmBatch {
+  int n;
+  int tile_start[kMaxBatch + 1];  // prefix sums of tiles_n * tiles_m
+  GemmProblem p[kMaxBatch];
+};
+
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                     const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K,
-                     const float* __restrict__ s_x, const float* __restrict__ s_w,
-                     const float* __restrict__ bias, __nv_bfloat16* __restrict__ y, int ldy,
-                     int32_t* __restrict__ acc_out, unsigned int* err) {
+    w4a4_gemm_kernel(const __grid_constant__ GemmBatch batch, unsigned int* err) {
   using C = Cfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
+  __shared__ __align__(16) float bars_sx[NT];   // s_x of this token tile
+
+  int pi = 0;
+  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.tile_start[pi + 1]) ++pi;
+  const GemmProblem& P = batch.p[pi];
+  const CUtensorMap* tmap_w = &P.tw;
+  const CUtensorMap* tmap_x = &P.tx;
+  const int M = P.M, N = P.N, K = P.K, ldy = P.ldy;
+  const float* __restrict__ s_x = P.s_x;
+  const float* __restrict__ s_w = P.s_w;
+  const float* __restrict__ bias = P.bias;
+  __nv_bfloat16* __restrict__ y = P.y;
+  int32_t* __restrict__ acc_out = P.acc;
+  const int local = static_cast<int>(blockIdx.x) - batch.tile_start[pi];
+  // A problem with S > 1 spans whole clusters (S consecutive CTAs share a
+  // tile, one K range each); a problem with S == 1 is padded to whole
+  // clusters, and the padding CTAs leave at once (they take part in no
+  // cluster barrier: only split problems use them).
+  const int S = P.S;
+  if (local >= P.tiles * S) return;
+  const int tile = local / S;
+  const int split = local % S;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * kBM;
-  const int m0 = blockIdx.y * NT;
-  const int S = gridDim.z;
-  const int split = blockIdx.z;
+  const int n0 = (tile % P.tiles_n) * kBM;
+  const int m0 = (tile / P.tiles_n) * NT;
   const int nkt = (K + kKP - 1) / kKP;
   const int kt0 = split * nkt / S, kt1 = (split + 1) * nkt / S;
   const int nk = kt1 - kt0;
@@ -102,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars.acc_full, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&tmap_w);
-    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(tmap_w);
+    tma_prefetch_desc(tmap_x);
   }
   if (warp == 1) {
     tmem_alloc(&bars.tmem_base, C::kTmemCols);
@@ -129,14 +173,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pre = nk < C::kPS ? nk : C::kPS;
       // the whole weight range of this CTA is requested into L2 at once, so
       // HBM streaming is not limited by the depth of the stage ring
-      for (int i = pre; i < nk; ++i) tma_prefetch_l2_2d(&tmap_w, (kt0 + i) * kRowP, n0);
+      for (int i = pre; i < nk; ++i) tma_prefetch_l2_2d(tmap_w, (kt0 + i) * kRowP, n0);
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&bars.full_p[i], C::kPStageBytes);
-        tma_load_2d(pstage + i * C::kPStageBytes, &tmap_w, &bars.full_p[i], (kt0 + i) * kRowP, n0);
+        tma_load_2d(pstage + i * C::kPStageBytes, tmap_w, &bars.full_p[i], (kt0 + i) * kRowP, n0);
       }
       pdl_wait();
       for (int i = 0; i < pre; ++i) {
-        tma_load_2d(pstage + i * C::kPStageBytes + kBM * kRowP, &tmap_x, &bars.full_p[i],
+        tma_load_2d(pstage + i * C::kPStageBytes + kBM * kRowP, tmap_x, &bars.full_p[i],
                     (kt0 + i) * kRowP, m0);
         ++issued;
       }
@@ -148,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = pstage + s * C::kPStageBytes;
         mbar_arrive_expect_tx(&bars.full_p[s], C::kPStageBytes);
         const int xbyte = (kt0 + i) * kRowP;
-        tma_load_2d(dst, &tmap_w, &bars.full_p[s], xbyte, n0);
-        tma_load_2d(dst + kBM * kRowP, &tmap_x, &bars.full_p[s], xbyte, m0);
+        tma_load_2d(dst, tmap_w, &bars.full_p[s], xbyte, n0);
+        tma_load_2d(dst + kBM * kRowP, tmap_x, &bars.full_p[s], xbyte, m0);
         ++issued;
       }
       // never leave with copies in flight: wait for the last load of each stage
@@ -171,9 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b0 = a0 + kBM * kKU;
 #pragma unroll
         for (int q = 0; q < kKU / 32; ++q) {
-          // chunks 2q (even codes) and 2q+1 (odd codes) of this stage
-          const uint64_t ad = smem_desc_kmajor_noswizzle(a0 + 2 * q * (kBM * 16), kBM * 16, 128);
-          const uint64_t bd = smem_desc_kmajor_noswizzle(b0 + 2 * q * (NT * 16), NT * 16, 128);
+          // bytes [32q, 32q+32) of every 128-byte row: the even and the odd
+          // codes of packed chunk q of this half stage
+          const uint64_t ad = smem_desc_kmajor_sw128(a0 + 32 * q);
+          const uint64_t bd = smem_desc_kmajor_sw128(b0 + 32 * q);
           umma_i8(tmem_d, ad, bd, idesc, (j > 0 || q > 0) ? 1u : 0u);
         }
         umma_commit(&bars.empty_u[u]);
@@ -184,6 +229,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // --------------------------------------------------- unpack (4 warps)
     const int wt = tid - 64;   // 0..127
+    // epilogue operands, loaded early so their latency hides under the main
+    // loop (s_x comes from the previous kernel in the stream)
+    pdl_wait();
+    float* sx_s = reinterpret_cast<float*>(bars_sx);
+    if (acc_out == nullptr)
+      for (int c = wt; c < NT; c += kWorkers) sx_s[c] = (m0 + c < M) ? __ldg(s_x + m0 + c) : 0.f;
+    const int quarter = warp & 3;
+    const int nl = quarter * 32 + lane;          // local output channel (TMEM lane)
+    const int n = n0 + nl;
+    const float sw = (acc_out == nullptr && n < N) ? __ldg(s_w + n) : 0.f;
+    const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
+    constexpr int kItems = (C::kRows * 4 + kWorkers - 1) / kWorkers;
     bool ok = true;
     for (int i = 0; i < nk && ok; ++i) {
       const int s = i % C::kPS;
@@ -194,31 +251,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < 2; ++h) {
         const int j = 2 * i + h;
         const int u = j % C::kUS;
+        // all packed loads of this half stage first (independent), then the
+        // nibble moves and the swizzled 16-byte stores
+        uint4 w[kItems];
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+          const int it = wt + k * kWorkers;
+          if (it < C::kRows * 4) {
+            const int row = ((it >> 5) << 3) + (it & 7);   // A rows, then B rows
+            const int cl = (it >> 3) & 3;                  // packed 16-byte chunk of the half
+            w[k] = *reinterpret_cast<const uint4*>(ps + row * kRowP +
+                                                   (((4 * h + cl) ^ (row & 7)) << 4));
+          }
+        }
         ok = mbar_wait(&bars.empty_u[u], ((j / C::kUS) & 1) ^ 1u, err);
         if (!ok) break;
         uint8_t* us = ustage + u * C::kUStageBytes;
-        for (int it = wt; it < C::kRows * 4; it += kWorkers) {
-          const bool isA = it < kBM * 4;
-          const int e = isA ? it : it - kBM * 4;
-          const int r = (e >> 5) * 8 + (e & 7);        // 8 consecutive threads: 8 rows
-          const int cl = (e >> 3) & 3;                 // packed 16-byte chunk in this half
-          const int rows = isA ? kBM : NT;
-          const uint8_t* src = ps + (isA ? 0 : kBM * kRowP) + r * kRowP +
-                               ((((4 * h + cl) ^ (r & 7))) << 4);
-          const uint4 w = *reinterpret_cast<const uint4*>(src);
-          uint4 ev, od;
-          ev.x = (w.x << 4) & 0xF0F0F0F0u;
-          ev.y = (w.y << 4) & 0xF0F0F0F0u;
-          ev.z = (w.z << 4) & 0xF0F0F0F0u;
-          ev.w = (w.w << 4) & 0xF0F0F0F0u;
-          od.x = w.x & 0xF0F0F0F0u;
-          od.y = w.y & 0xF0F0F0F0u;
-          od.z = w.z & 0xF0F0F0F0u;
-          od.w = w.w & 0xF0F0F0F0u;
-          uint8_t* dreg = us + (isA ? 0 : kBM * kKU);
-          const int core = (r >> 3) * 128 + (r & 7) * 16;
-          *reinterpret_cast<uint4*>(dreg + (2 * cl) * (rows * 16) + core) = ev;
-          *reinterpret_cast<uint4*>(dreg + (2 * cl + 1) * (rows * 16) + core) = od;
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+          const int it = wt + k * kWorkers;
+          if (it < C::kRows * 4) {
+            const int row = ((it >> 5) << 3) + (it & 7);
+            const int cl = (it >> 3) & 3;
+            uint4 ev, od;
+            ev.x = (w[k].x << 4) & 0xF0F0F0F0u;
+            ev.y = (w[k].y << 4) & 0xF0F0F0F0u;
+            ev.z = (w[k].z << 4) & 0xF0F0F0F0u;
+            ev.w = (w[k].w << 4) & 0xF0F0F0F0u;
+            od.x = w[k].x & 0xF0F0F0F0u;
+            od.y = w[k].y & 0xF0F0F0F0u;
+            od.z = w[k].z & 0xF0F0F0F0u;
+            od.w = w[k].w & 0xF0F0F0F0u;
+            // 128-byte swizzled K-major rows (A rows 0..127, then B rows):
+            // chunk 2cl holds the even codes, 2cl+1 the odd codes
+            uint8_t* rowp = us + row * kKU;
+            *reinterpret_cast<uint4*>(rowp + (((2 * cl) ^ (row & 7)) << 4)) = ev;
+            *reinterpret_cast<uint4*>(rowp + (((2 * cl + 1) ^ (row & 7)) << 4)) = od;
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars.full_u[u]);
@@ -227,16 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------- epilogue
-    const int quarter = warp & 3;
-    const int nl = quarter * 32 + lane;          // local output channel (TMEM lane)
-    const int n = n0 + nl;
     const bool have = ok && mbar_wait(&bars.acc_full, 0, err);
     tc_fence_after();
     pdl_launch_dependents();
-    pdl_wait();                       // s_x comes from the previous kernel
     if (have) {
-      const float sw = (n < N) ? __ldg(s_w + n) : 0.f;
-      const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
       // split-K: this CTA's partial rows go to the receive buffer of the CTA
       // that owns them (rows [r*128/S, (r+1)*128/S) belong to cluster rank r),
       // slot `split`, as fire-and-forget distributed-shared-memory stores
@@ -250,6 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         cluster_wait();
         cluster_waited = true;
       }
+      // bf16 output tile [NT tokens][128 channels] in the (now idle) stage
+      // memory, written back by one TMA tensor store
+      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base);
 #pragma unroll 1
       for (int c0 = 0; c0 < NT; c0 += 16) {
         uint32_t r[16];
@@ -262,22 +328,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  make_int4(static_cast<int>(r[4 * q]), static_cast<int>(r[4 * q + 1]),
                                            static_cast<int>(r[4 * q + 2]),
                                            static_cast<int>(r[4 * q + 3])));
-        } else if (n < N) {
+        } else if (acc_out) {
+          if (n < N) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int m = m0 + c0 + c;
-            if (m < M) {
-              const int32_t a = static_cast<int32_t>(r[c]) >> 8;
-              if (acc_out) {
-                acc_out[static_cast<size_t>(m) * N + n] = a;
-              } else {
-                const float sc = __ldg(s_x + m) * sw;
-                y[static_cast<size_t>(m) * ldy + n] =
-                    __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
-              }
+            for (int c = 0; c < 16; ++c) {
+              const int m = m0 + c0 + c;
+              if (m < M) acc_out[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(r[c]) >> 8;
             }
           }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float sc = sx_s[c0 + c] * sw;
+            const int32_t a = static_cast<int32_t>(r[c]) >> 8;
+            otile[(c0 + c) * kBM + nl] = __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
+          }
         }
+      }
+      if (S == 1 && acc_out == nullptr) {
+        fence_proxy_async_smem();
+        named_barrier(1, kWorkers);
+        if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0, m0);
       }
     }
     tc_fence_before();
@@ -294,6 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t rank = cluster_ctarank();
       const int rpr = kBM / S;                     // channel rows reduced by this CTA
       const int32_t* recv = reinterpret_cast<const int32_t*>(base + C::kStageBytes);
+      // output tile [NT tokens][rpr channels] for one TMA store of this CTA's rows
+      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base);
       for (int e = wt; e < rpr * NT; e += kWorkers) {
         const int lr = e % rpr;
         const int col = e / rpr;
@@ -301,17 +374,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int src = 0; src < S; ++src) sum += recv[(src * rpr + lr) * C::kRedPitch + col];
         const int nl = rank * rpr + lr;
         const int n = n0 + nl, m = m0 + col;
-        if (n < N && m < M) {
-          const int32_t a = sum >> 8;
-          if (acc_out) {
-            acc_out[static_cast<size_t>(m) * N + n] = a;
-          } else {
-            const float sc = __ldg(s_x + m) * __ldg(s_w + n);
-            const float bn = bias != nullptr ? __ldg(bias + n) : 0.f;
-            y[static_cast<size_t>(m) * ldy + n] =
-                __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
-          }
+        const int32_t a = sum >> 8;
+        if (acc_out) {
+          if (n < N && m < M) acc_out[static_cast<size_t>(m) * N + n] = a;
+        } else {
+          const float sc = n < N ? bars_sx[col] * __ldg(s_w + n) : 0.f;
+          const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
+          otile[col * rpr + lr] = __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
         }
+      }
+      if (acc_out == nullptr) {
+        fence_proxy_async_smem();
+        named_barrier(1, kWorkers);
+        if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0 + static_cast<int>(rank) * rpr, m0);
       }
     }
   }
@@ -357,28 +432,66 @@ bool make_packed_map(CUtensorMap* map, const uint8_t* ptr, int rows, int K, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [M][ldy] output; box = box_n channels x box_m tokens, no swizzle.
+bool make_output_map(CUtensorMap* map, void* ptr, int M, int N, int ldy, int box_n, int box_m) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldy) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_n), static_cast<cuuint32_t>(box_m)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NT>
-cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
-  using C = Cfg<NT>;
-  if (!C::kCanSplit) S = 1;   // large token tiles supply the parallelism themselves
-  CUtensorMap mw, mx;
-  if (!make_packed_map(&mw, g.wq, g.N, g.K, kBM) || !make_packed_map(&mx, g.xq, g.M, g.K, NT))
-    return cudaErrorInvalidValue;
+cudaError_t launch_group(const GemmArgs* const* gs, const int* splits, int n, int C,
+                         cudaStream_t stream) {
+  using C_ = Cfg<NT>;
+  GemmBatch batch;
+  std::memset(&batch, 0, sizeof(batch));
+  batch.n = n;
+  int ctas = 0;
+  for (int i = 0; i < n; ++i) {
+    const GemmArgs& g = *gs[i];
+    GemmProblem& P = batch.p[i];
+    const int S = splits[i];
+    if (!make_packed_map(&P.tw, g.wq, g.N, g.K, kBM) || !make_packed_map(&P.tx, g.xq, g.M, g.K, NT))
+      return cudaErrorInvalidValue;
+    if (g.y != nullptr && !make_output_map(&P.ty, g.y, g.M, g.N, g.ldy, kBM / S, NT))
+      return cudaErrorInvalidValue;
+    P.s_x = g.s_x;
+    P.s_w = g.w_scale;
+    P.bias = g.bias;
+    P.y = static_cast<__nv_bfloat16*>(g.y);
+    P.acc = g.acc;
+    P.M = g.M;
+    P.N = g.N;
+    P.K = g.K;
+    P.ldy = g.ldy;
+    P.tiles_n = (g.N + kBM - 1) / kBM;
+    P.tiles = P.tiles_n * ((g.M + NT - 1) / NT);
+    P.S = S;
+    batch.tile_start[i] = ctas;
+    ctas += (P.tiles * S + C - 1) / C * C;     // whole clusters
+  }
+  batch.tile_start[n] = ctas;
   auto kern = w4a4_gemm_kernel<NT>;
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kCanSplit ? C::kSmemBytes + C::kRecvBytes : C::kSmemBytes);
+                             C_::kCanSplit ? C_::kSmemBytes + C_::kRecvBytes : C_::kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((g.N + kBM - 1) / kBM, (g.M + NT - 1) / NT, S);
+  cfg.gridDim = dim3(ctas, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes + (S > 1 ? C::kRecvBytes : 0);
+  cfg.dynamicSmemBytes = C_::kSmemBytes + (C > 1 ? C_::kRecvBytes : 0);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -387,25 +500,74 @@ cudaError_t launch_nt(const GemmArgs& g, int S, cudaStream_t stream) {
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
-  if (S > 1) {
+  if (C > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.x = C;
     attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = S;
+    attr[na].val.clusterDim.z = 1;
     ++na;
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  e = cudaLaunchKernelEx(&cfg, kern, mw, mx, g.M, g.N, g.K, g.s_x, g.w_scale, g.bias,
-                         static_cast<__nv_bfloat16*>(g.y), g.ldy, g.acc, device_error_word());
+  e = cudaLaunchKernelEx(&cfg, kern, batch, device_error_word());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+int token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+// Split-K factors of a launch (1 or the launch's cluster size C per problem).
+// Requested: the same factor everywhere.  Automatic: one factor for all,
+// raised while the launch has fewer CTAs than SMs.
+template <int NT>
+int choose_splits(const GemmArgs* const* gs, int n, int split_k, int* splits) {
+  if (!Cfg<NT>::kCanSplit) {
+    for (int i = 0; i < n; ++i) splits[i] = 1;
+    return 1;
+  }
+  if (split_k > 0) {
+    for (int i = 0; i < n; ++i) splits[i] = split_k;
+    return split_k;
+  }
+  // (Splitting only the long-K problems of a batch balances the K walk, but
+  // the split-K receive buffer then halves the CTAs per SM for the whole
+  // launch, which costs more than it gains; so the automatic factor is
+  // uniform.)
+  int min_nkt = 1 << 30;
+  for (int i = 0; i < n; ++i) min_nkt = std::min(min_nkt, (gs[i]->K + kKP - 1) / kKP);
+  int C = 1;
+  for (int i = 0; i < n; ++i) splits[i] = 1;
+  auto total = [&]() {
+    int t = 0;
+    for (int i = 0; i < n; ++i)
+      t += ((gs[i]->N + kBM - 1) / kBM) * ((gs[i]->M + NT - 1) / NT) * splits[i];
+    return t;
+  };
+  bool uniform = true;
+  for (int i = 0; i < n; ++i) uniform = uniform && splits[i] == C;
+  while (uniform && C < 8 && total() < 148 && 2 * C <= min_nkt) {
+    C *= 2;
+    for (int i = 0; i < n; ++i) splits[i] = C;
+  }
+  return C;
+}
+
+template <int NT>
+cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cudaStream_t stream) {
+  for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+    const int m = std::min(kMaxBatch, n - i0);
+    int splits[kMaxBatch];
+    const int C = choose_splits<NT>(gs + i0, m, split_k, splits);
+    cudaError_t e = launch_group<NT>(gs + i0, splits, m, C, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
 
 int gemm_choose_split(int M, int N, int K) {
-  const int nt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  const int nt = token_tile(M);
   if (nt == 256) return 1;
   const int tiles = ((N + kBM - 1) / kBM) * ((M + nt - 1) / nt);
   const int nkt = (K + kKP - 1) / kKP;
@@ -414,13 +576,29 @@ int gemm_choose_split(int M, int N, int K) {
   return S;
 }
 
+cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream) {
+  // group by token tile (a template parameter of the kernel)
+  static const int kTiles[5] = {16, 32, 64, 128, 256};
+  for (int t : kTiles) {
+    std::vector<const GemmArgs*> grp;
+    for (int i = 0; i < n; ++i)
+      if (gs[i].M > 0 && token_tile(gs[i].M) == t) grp.push_back(&gs[i]);
+    if (grp.empty()) continue;
+    cudaError_t e;
+    switch (t) {
+      case 16: e = launch_nt_batches<16>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
+      case 32: e = launch_nt_batches<32>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
+      case 64: e = launch_nt_batches<64>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
+      case 128: e = launch_nt_batches<128>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
+      default: e = launch_nt_batches<256>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream) {
-  int S = g.split_k > 0 ? g.split_k : gemm_choose_split(g.M, g.N, g.K);
-  if (g.M <= 16) return launch_nt<16>(g, S, stream);
-  if (g.M <= 32) return launch_nt<32>(g, S, stream);
-  if (g.M <= 64) return launch_nt<64>(g, S, stream);
-  if (g.M <= 128) return launch_nt<128>(g, S, stream);
-  return launch_nt<256>(g, S, stream);
+  return launch_w4a4_gemm_batch(&g, 1, g.split_k, stream);
 }
 
 }  // namespace qvla

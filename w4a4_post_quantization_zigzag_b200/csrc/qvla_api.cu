@@ -353,23 +353,25 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
   return QVLA_OK;
 }
 
-qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
-                                  const qvla_packed_linear* L, qvla_scale_mode mode,
-                                  const float* table, int T, int Lcount, const int32_t* step_dev,
-                                  int step_host, int layer, uint8_t* xq, float* s_x,
-                                  cudaStream_t stream) {
+// Validates one rotate-quantise call and fills its launch arguments.
+static qvla_status prepare_act(const void* x, qvla_dtype xdt, int M, int ldx,
+                               const qvla_packed_linear* L, qvla_scale_mode mode,
+                               const float* table, int T, int Lcount, const int32_t* step_dev,
+                               int step_host, int layer, uint8_t* xq, float* s_x,
+                               ActArgs* out) {
   qvla_status st = check_linear(L, false);
   if (st != QVLA_OK) return st;
   if (M < 0) return QVLA_ERR_SHAPE;
   if (xdt != QVLA_DTYPE_F32 && xdt != QVLA_DTYPE_BF16) return QVLA_ERR_ARG;
   if ((st = check_scale(mode, table, T, Lcount, step_dev, step_host, layer)) != QVLA_OK) return st;
+  *out = ActArgs{};
+  out->M = M;
   if (M == 0) return QVLA_OK;
   if (!x || !xq || !s_x) return QVLA_ERR_ARG;
   if (ldx < L->K) return QVLA_ERR_SHAPE;
   const size_t esz = xdt == QVLA_DTYPE_F32 ? 4 : 2;
   if (!aligned16(x) || (ldx * esz) % 16 || !aligned16(xq) || !aligned16(s_x)) return QVLA_ERR_ALIGN;
-  if (static_cast<size_t>(L->K) * 4 > 200 * 1024) return QVLA_ERR_SHAPE;
-  ActArgs a = {};
+  ActArgs& a = *out;
   a.x = x;
   a.xdt = xdt;
   a.M = M;
@@ -387,7 +389,33 @@ qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
   a.layer = layer;
   a.xq = xq;
   a.s_x = s_x;
+  return QVLA_OK;
+}
+
+qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
+                                  const qvla_packed_linear* L, qvla_scale_mode mode,
+                                  const float* table, int T, int Lcount, const int32_t* step_dev,
+                                  int step_host, int layer, uint8_t* xq, float* s_x,
+                                  cudaStream_t stream) {
+  ActArgs a;
+  qvla_status st = prepare_act(x, xdt, M, ldx, L, mode, table, T, Lcount, step_dev, step_host,
+                               layer, xq, s_x, &a);
+  if (st != QVLA_OK || M == 0) return st;
   return cuda_status(launch_rotate_quant(a, stream));
+}
+
+qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int n,
+                                          cudaStream_t stream) {
+  if (n < 0 || (n > 0 && !probs)) return QVLA_ERR_ARG;
+  std::vector<ActArgs> v(n);
+  for (int i = 0; i < n; ++i) {
+    const qvla_linear_problem& p = probs[i];
+    qvla_status st = prepare_act(p.x, static_cast<qvla_dtype>(p.xdt), p.M, p.ldx, p.L,
+                                 static_cast<qvla_scale_mode>(p.mode), p.table, p.T, p.Lcount,
+                                 p.step_dev, p.step_host, p.layer, p.xq, p.s_x, &v[i]);
+    if (st != QVLA_OK) return st;
+  }
+  return cuda_status(launch_rotate_quant_batch(v.data(), n, stream));
 }
 
 qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
@@ -401,7 +429,6 @@ qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
   if (ldx < L->K) return QVLA_ERR_SHAPE;
   const size_t esz = xdt == QVLA_DTYPE_F32 ? 4 : 2;
   if (!aligned16(x) || (ldx * esz) % 16 || !aligned16(xr_out)) return QVLA_ERR_ALIGN;
-  if (static_cast<size_t>(L->K) * 4 > 200 * 1024) return QVLA_ERR_SHAPE;
   ActArgs a = {};
   a.x = x;
   a.xdt = xdt;
@@ -444,25 +471,36 @@ qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mo
   return cuda_status(launch_quant_rows(a, stream));
 }
 
-static qvla_status gemm_common(const uint8_t* xq, const float* s_x, int M,
-                               const qvla_packed_linear* L, void* y, int ldy, int32_t* acc,
-                               int split_k, cudaStream_t stream) {
+// Validates one GEMM call and fills its launch arguments.
+static qvla_status prepare_gemm(const uint8_t* xq, const float* s_x, int M,
+                                const qvla_packed_linear* L, void* y, int ldy, int32_t* acc,
+                                int split_k, GemmArgs* out) {
   qvla_status st = check_linear(L, true);
   if (st != QVLA_OK) return st;
   if (M < 0) return QVLA_ERR_SHAPE;
   if (L->K % 32) return QVLA_ERR_SHAPE;
+  *out = GemmArgs{};
+  out->M = M;
   if (M == 0) return QVLA_OK;
   if (!xq) return QVLA_ERR_ARG;
   if (!aligned16(xq)) return QVLA_ERR_ALIGN;
+  if (y) {
+    if (!s_x) return QVLA_ERR_ARG;
+    if (ldy < L->N) return QVLA_ERR_SHAPE;
+    if (!aligned16(s_x) || !aligned16(y) || (static_cast<size_t>(ldy) * 2) % 16)
+      return QVLA_ERR_ALIGN;
+  } else {
+    if (!acc) return QVLA_ERR_ARG;
+    if (!aligned16(acc)) return QVLA_ERR_ALIGN;
+  }
   const int nkt = (L->K + 255) / 256;
   if (split_k != 0 && split_k != 1 && split_k != 2 && split_k != 4 && split_k != 8 &&
       split_k != 16)
     return QVLA_ERR_ARG;
   if (split_k > nkt) return QVLA_ERR_SHAPE;
-  GemmArgs g = {};
+  GemmArgs& g = *out;
   g.xq = xq;
   g.s_x = s_x;
-  g.M = M;
   g.N = L->N;
   g.K = L->K;
   g.wq = L->wq;
@@ -472,32 +510,52 @@ static qvla_status gemm_common(const uint8_t* xq, const float* s_x, int M,
   g.ldy = ldy;
   g.acc = acc;
   g.split_k = split_k;
+  return QVLA_OK;
+}
+
+static qvla_status check_sm100() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
     return QVLA_ERR_CUDA;
-  if (major != 10) return QVLA_ERR_UNSUPPORTED;
+  return major == 10 ? QVLA_OK : QVLA_ERR_UNSUPPORTED;
+}
+
+static qvla_status gemm_common(const uint8_t* xq, const float* s_x, int M,
+                               const qvla_packed_linear* L, void* y, int ldy, int32_t* acc,
+                               int split_k, cudaStream_t stream) {
+  GemmArgs g;
+  qvla_status st = prepare_gemm(xq, s_x, M, L, y, ldy, acc, split_k, &g);
+  if (st != QVLA_OK || M == 0) return st;
+  if ((st = check_sm100()) != QVLA_OK) return st;
   return cuda_status(launch_w4a4_gemm(g, stream));
+}
+
+qvla_status qvla_w4a4_gemm_batched(const qvla_linear_problem* probs, int n, int split_k,
+                                   cudaStream_t stream) {
+  if (n < 0 || (n > 0 && !probs)) return QVLA_ERR_ARG;
+  std::vector<GemmArgs> v(n);
+  for (int i = 0; i < n; ++i) {
+    const qvla_linear_problem& p = probs[i];
+    if (p.M > 0 && !p.y) return QVLA_ERR_ARG;
+    qvla_status st = prepare_gemm(p.xq, p.s_x, p.M, p.L, p.y, p.ldy, nullptr, split_k, &v[i]);
+    if (st != QVLA_OK) return st;
+  }
+  if (n == 0) return QVLA_OK;
+  qvla_status st = check_sm100();
+  if (st != QVLA_OK) return st;
+  return cuda_status(launch_w4a4_gemm_batch(v.data(), n, split_k, stream));
 }
 
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
                            const qvla_packed_linear* L, void* y, int ldy, int split_k,
                            cudaStream_t stream) {
-  if (M > 0) {
-    if (!s_x || !y || !L) return QVLA_ERR_ARG;
-    if (ldy < L->N) return QVLA_ERR_SHAPE;
-    if (!aligned16(s_x) || !aligned16(y) || (static_cast<size_t>(ldy) * 2) % 16)
-      return QVLA_ERR_ALIGN;
-  }
+  if (M > 0 && !y) return QVLA_ERR_ARG;
   return gemm_common(xq, s_x, M, L, y, ldy, nullptr, split_k, stream);
 }
 
 qvla_status qvla_w4a4_gemm_s32(const uint8_t* xq, int M, const qvla_packed_linear* L,
                                int32_t* acc, int split_k, cudaStream_t stream) {
-  if (M > 0) {
-    if (!acc) return QVLA_ERR_ARG;
-    if (!aligned16(acc)) return QVLA_ERR_ALIGN;
-  }
   return gemm_common(xq, nullptr, M, L, nullptr, 0, acc, split_k, stream);
 }
 

@@ -107,6 +107,23 @@ QVLA_DEVICE void tma_prefetch_l2_2d(const CUtensorMap* tmap, int x, int y) {
                : "memory");
 }
 
+// 2-D tiled bulk tensor store from this CTA's shared memory (out-of-range
+// rows and columns of the box are not written), then wait until it is done.
+QVLA_DEVICE void tma_store_2d_and_wait(const CUtensorMap* tmap, const void* smem_src, int x,
+                                       int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n\t"
+      "cp.async.bulk.commit_group;\n\t"
+      "cp.async.bulk.wait_group 0;" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Barrier over `count` threads (a multiple of 32) on hardware barrier `id`.
+QVLA_DEVICE void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 QVLA_DEVICE void tma_prefetch_desc(const CUtensorMap* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
@@ -189,6 +206,21 @@ QVLA_DEVICE uint64_t smem_desc_kmajor_noswizzle(uint32_t saddr, uint32_t lbo, ui
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;  // version
   // base offset 0, lbo mode 0, layout type 0 (no swizzle)
+  return d;
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: each row holds
+// 128 bytes of K with its 16-byte chunks XOR-permuted by (row & 7); 8-row
+// groups are 1024 bytes apart (SBO).  The tile base must be 1024-byte aligned;
+// successive K slices inside the 128-byte row are addressed by advancing the
+// start address.
+QVLA_DEVICE uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;                   // LBO (unused when swizzled)
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;           // SBO
+  d |= 1ull << 46;                                        // version
+  d |= 2ull << 61;                                        // layout: SWIZZLE_128B
   return d;
 }
 

@@ -32,6 +32,8 @@ struct ActArgs {
   float* xr_out;          // rotate-only mode when non-null and xq == nullptr
 };
 cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream);
+// independent linears in as few launches as possible (grouped by kernel config)
+cudaError_t launch_rotate_quant_batch(const ActArgs* as, int n, cudaStream_t stream);
 
 // quantise already-rotated fp32 rows: activations (qmin -8) or weights (qmin -7)
 struct QuantArgs {
@@ -69,6 +71,8 @@ struct GemmArgs {
   int split_k;
 };
 cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream);
+// independent linears in as few launches as possible (grouped by token tile)
+cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream);
 int gemm_choose_split(int M, int N, int K);
 
 }  // namespace qvla

@@ -32,6 +32,10 @@
 // chunk are staged before waiting on the previous kernel in the stream.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
 #include "qvla_common.cuh"
 #include "qvla_internal.h"
 
@@ -158,14 +162,32 @@ QVLA_DEVICE void store_codes32(uint8_t* dst, int q, int lane) {
     *reinterpret_cast<uint32_t*>(dst + (lane >> 1)) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
+// One linear of a batched launch; CTAs are numbered problem by problem along
+// grid x (token tile fastest, then block group); DYNAMIC mode splits each row
+// over the cluster along grid y instead.
+constexpr int kMaxBatch = 16;
+struct ActProblem {
+  const void* x;
+  const int32_t* perm;
+  const float* rot;
+  const float* table;
+  const int32_t* step_dev;
+  uint8_t* xq;
+  float* s_x;
+  float* xr_out;
+  int M, ldx, K, T, Lcount, step_host, layer;
+  int gx;                     // token tiles
+  int bpc;                    // rotation blocks per CTA
+};
+struct ActBatch {
+  int n;
+  int cta_start[kMaxBatch + 1];
+  ActProblem p[kMaxBatch];
+};
+
 template <int BS, int TT, typename Tin, int MODE>
 __global__ void __launch_bounds__(kThreads)
-    rotq_kernel(const Tin* __restrict__ x, int M, int ldx, int K,
-                const int32_t* __restrict__ perm, const float* __restrict__ rot,
-                const float* __restrict__ table, int T, int Lcount,
-                const int32_t* __restrict__ step_dev, int step_host, int layer,
-                uint8_t* __restrict__ xq, float* __restrict__ s_x, float* __restrict__ xr_out,
-                unsigned int* err, int blocks_per_cta) {
+    rotq_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
   using G = Geo<BS>;
   constexpr int C = BS / 32;
   constexpr int TPT = TT / G::NTG;          // tokens per thread in the product
@@ -174,11 +196,26 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ unsigned int amax_s[TT];
   __shared__ float scale_s[TT];
 
+  int pi = 0;
+  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[pi + 1]) ++pi;
+  const ActProblem& P = batch.p[pi];
+  const Tin* __restrict__ x = static_cast<const Tin*>(P.x);
+  const int M = P.M, ldx = P.ldx, K = P.K;
+  const int32_t* __restrict__ perm = P.perm;
+  const float* __restrict__ rot = P.rot;
+  uint8_t* __restrict__ xq = P.xq;
+  float* __restrict__ s_x = P.s_x;
+  float* __restrict__ xr_out = P.xr_out;
+  const int blocks_per_cta = P.bpc;
+  const int local = static_cast<int>(blockIdx.x) - batch.cta_start[pi];
+  const int tile = local % P.gx;
+  const int group = MODE == kDynamic ? static_cast<int>(blockIdx.y) : local / P.gx;
+
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int m0 = blockIdx.x * TT;
+  const int m0 = tile * TT;
   const int ntok = min(TT, M - m0);
   const int nb = K / BS;
-  const int B0 = blockIdx.y * blocks_per_cta;
+  const int B0 = group * blocks_per_cta;
   const int nbc = max(0, min(blocks_per_cta, nb - B0));
 
   int32_t* perm_s = reinterpret_cast<int32_t*>(smem);
@@ -204,7 +241,8 @@ __global__ void __launch_bounds__(kThreads)
   pdl_wait();
   pdl_launch_dependents();
   float s_tab = 0.f;
-  if (MODE == kTable) s_tab = table_scale(table, T, Lcount, step_dev, step_host, layer, err);
+  if (MODE == kTable)
+    s_tab = table_scale(P.table, P.T, P.Lcount, P.step_dev, P.step_host, P.layer, err);
   __syncthreads();   // perm_s visible
 
   const int jp = tid % G::NJP, tg = tid / G::NJP;
@@ -283,7 +321,7 @@ __global__ void __launch_bounds__(kThreads)
   }
 
   if (MODE == kTable) {
-    if (blockIdx.y == 0 && tid < ntok) s_x[m0 + tid] = s_tab;
+    if (group == 0 && tid < ntok) s_x[m0 + tid] = s_tab;
     return;
   }
   if (MODE == kRotateOnly) return;
@@ -371,28 +409,70 @@ __global__ void __launch_bounds__(kThreads)
   if (tid == 0) s_out[row] = s;
 }
 
-template <int BS, int TT, typename Tin, int MODE>
-cudaError_t launch_cfg(const ActArgs& a, cudaStream_t stream) {
-  const int K = a.K, nb = K / BS;
-  const int gx = (a.M + TT - 1) / TT;
-  int bpc, gy, cs = 1;
+// Grid of one problem: token tiles gx, CTAs per token tile (block groups, or
+// the cluster size in DYNAMIC mode) and rotation blocks per CTA.
+template <int BS, int TT, int MODE>
+void problem_grid(int M, int K, int* gx, int* per_tile, int* bpc) {
+  const int nb = K / BS;
+  *gx = (M + TT - 1) / TT;
   if (MODE == kDynamic) {
-    // split the row's blocks over a cluster of cs CTAs: enough CTAs to fill the
-    // GPU and a kept slice that fits in shared memory
+    int cs = 1;
     while (cs < 16 && cs < nb &&
-           (gx * cs < 148 || Smem<BS, TT>::bytes((nb + cs - 1) / cs, true) > kSmemCap))
+           (*gx * cs < 148 || Smem<BS, TT>::bytes((nb + cs - 1) / cs, true) > kSmemCap))
       cs *= 2;
-    bpc = (nb + cs - 1) / cs;
-    gy = cs;
-    if (Smem<BS, TT>::bytes(bpc, true) > kSmemCap) return cudaErrorInvalidConfiguration;
+    *bpc = (nb + cs - 1) / cs;
+    *per_tile = cs;
   } else {
     const int target = 2 * 148;
-    int g = (target + gx - 1) / gx;
+    int g = (target + *gx - 1) / *gx;
     g = g < 1 ? 1 : (g > nb ? nb : g);
-    bpc = (nb + g - 1) / g;
-    gy = (nb + bpc - 1) / bpc;
+    *bpc = (nb + g - 1) / g;
+    *per_tile = (nb + *bpc - 1) / *bpc;
   }
-  const size_t smem = Smem<BS, TT>::bytes(bpc, MODE == kDynamic);
+}
+
+// Launches up to kMaxBatch problems that share (BS, TT, Tin, MODE) and, in
+// DYNAMIC mode, the cluster size.
+template <int BS, int TT, typename Tin, int MODE>
+cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream) {
+  ActBatch batch;
+  std::memset(&batch, 0, sizeof(batch));
+  batch.n = n;
+  int ctas = 0, cs = 1, bpc_max = 1;
+  for (int i = 0; i < n; ++i) {
+    const ActArgs& a = *as[i];
+    int gx, per_tile, bpc;
+    problem_grid<BS, TT, MODE>(a.M, a.K, &gx, &per_tile, &bpc);
+    ActProblem& P = batch.p[i];
+    P.x = a.x;
+    P.perm = a.perm;
+    P.rot = a.rot;
+    P.table = a.table;
+    P.step_dev = a.step_dev;
+    P.xq = a.xq;
+    P.s_x = a.s_x;
+    P.xr_out = a.xr_out;
+    P.M = a.M;
+    P.ldx = a.ldx;
+    P.K = a.K;
+    P.T = a.T;
+    P.Lcount = a.Lcount;
+    P.step_host = a.step_host;
+    P.layer = a.layer;
+    P.gx = gx;
+    P.bpc = bpc;
+    batch.cta_start[i] = ctas;
+    if (MODE == kDynamic) {
+      ctas += gx;
+      cs = per_tile;                 // equal within a group (the caller groups by it)
+    } else {
+      ctas += gx * per_tile;
+    }
+    bpc_max = std::max(bpc_max, bpc);
+  }
+  batch.cta_start[n] = ctas;
+  const size_t smem = Smem<BS, TT>::bytes(bpc_max, MODE == kDynamic);
+  if (smem > static_cast<size_t>(kSmemCap)) return cudaErrorInvalidConfiguration;
   auto kern = rotq_kernel<BS, TT, Tin, MODE>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -406,7 +486,7 @@ cudaError_t launch_cfg(const ActArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(gx, gy, 1);
+  cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -417,7 +497,7 @@ cudaError_t launch_cfg(const ActArgs& a, cudaStream_t stream) {
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
-  if (cs > 1) {
+  if (MODE == kDynamic && cs > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = 1;
     attr[na].val.clusterDim.y = cs;
@@ -426,46 +506,99 @@ cudaError_t launch_cfg(const ActArgs& a, cudaStream_t stream) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(a.x), a.M, a.ldx, K,
-                                     a.perm, a.rot, a.table, a.T, a.Lcount, a.step_dev,
-                                     a.step_host, a.layer, a.xq, a.s_x, a.xr_out,
-                                     device_error_word(), bpc);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, batch, device_error_word());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+template <int BS, int TT, typename Tin, int MODE>
+cudaError_t launch_cfg_batches(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  if (MODE != kDynamic) {
+    for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
+      const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+      cudaError_t e = launch_group<BS, TT, Tin, MODE>(v.data() + i0, n, stream);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  // DYNAMIC: one launch per cluster size
+  for (int cs = 1; cs <= 16; cs *= 2) {
+    std::vector<const ActArgs*> g;
+    for (const ActArgs* a : v) {
+      int gx, per_tile, bpc;
+      problem_grid<BS, TT, MODE>(a->M, a->K, &gx, &per_tile, &bpc);
+      if (per_tile == cs) g.push_back(a);
+    }
+    for (size_t i0 = 0; i0 < g.size(); i0 += kMaxBatch) {
+      const int n = static_cast<int>(std::min<size_t>(kMaxBatch, g.size() - i0));
+      cudaError_t e = launch_group<BS, TT, Tin, MODE>(g.data() + i0, n, stream);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
+}
+
+int token_tile_for(int M, int K, int BS, int mode) {
+  // 16 for small M, block 32 or very long dynamic rows (keeps the dynamic
+  // slice in shared memory), else 32
+  return (M <= 16 || BS == 32 || (mode == kDynamic && K > 8192)) ? 16 : 32;
+}
+
 template <int BS, typename Tin, int MODE>
-cudaError_t launch_tt(const ActArgs& a, cudaStream_t stream) {
-  // token tile: 16 for small M, block 32 or very long dynamic rows (keeps the
-  // dynamic slice in shared memory), else 32
-  if (a.M <= 16 || BS == 32 || (MODE == kDynamic && a.K > 8192))
-    return launch_cfg<BS, 16, Tin, MODE>(a, stream);
-  return launch_cfg<BS, 32, Tin, MODE>(a, stream);
+cudaError_t launch_bs(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  std::vector<const ActArgs*> t16, t32;
+  for (const ActArgs* a : v) (token_tile_for(a->M, a->K, BS, MODE) == 16 ? t16 : t32).push_back(a);
+  cudaError_t e = cudaSuccess;
+  if (!t16.empty()) e = launch_cfg_batches<BS, 16, Tin, MODE>(t16, stream);
+  if (e == cudaSuccess && !t32.empty()) e = launch_cfg_batches<BS, (BS == 32 ? 16 : 32), Tin, MODE>(t32, stream);
+  return e;
 }
 
 template <typename Tin, int MODE>
-cudaError_t launch_bs(const ActArgs& a, cudaStream_t stream) {
-  switch (a.block) {
-    case 32: return launch_tt<32, Tin, MODE>(a, stream);
-    case 64: return launch_tt<64, Tin, MODE>(a, stream);
-    case 128: return launch_tt<128, Tin, MODE>(a, stream);
-    case 256: return launch_tt<256, Tin, MODE>(a, stream);
-    default: return cudaErrorInvalidValue;
+cudaError_t launch_mode(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  static const int kBlocks[4] = {32, 64, 128, 256};
+  for (int b : kBlocks) {
+    std::vector<const ActArgs*> g;
+    for (const ActArgs* a : v)
+      if (a->block == b) g.push_back(a);
+    if (g.empty()) continue;
+    cudaError_t e;
+    switch (b) {
+      case 32: e = launch_bs<32, Tin, MODE>(g, stream); break;
+      case 64: e = launch_bs<64, Tin, MODE>(g, stream); break;
+      case 128: e = launch_bs<128, Tin, MODE>(g, stream); break;
+      default: e = launch_bs<256, Tin, MODE>(g, stream); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 template <typename Tin>
-cudaError_t launch_mode(const ActArgs& a, cudaStream_t stream) {
-  if (a.xq == nullptr) return launch_bs<Tin, kRotateOnly>(a, stream);
-  if (a.dynamic) return launch_bs<Tin, kDynamic>(a, stream);
-  return launch_bs<Tin, kTable>(a, stream);
+cudaError_t launch_dtype(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  std::vector<const ActArgs*> rot, dyn, tab;
+  for (const ActArgs* a : v) (a->xq == nullptr ? rot : a->dynamic ? dyn : tab).push_back(a);
+  cudaError_t e = cudaSuccess;
+  if (!rot.empty()) e = launch_mode<Tin, kRotateOnly>(rot, stream);
+  if (e == cudaSuccess && !dyn.empty()) e = launch_mode<Tin, kDynamic>(dyn, stream);
+  if (e == cudaSuccess && !tab.empty()) e = launch_mode<Tin, kTable>(tab, stream);
+  return e;
 }
 
 }  // namespace
 
+cudaError_t launch_rotate_quant_batch(const ActArgs* as, int n, cudaStream_t stream) {
+  std::vector<const ActArgs*> bf, f32;
+  for (int i = 0; i < n; ++i)
+    if (as[i].M > 0) (as[i].xdt == QVLA_DTYPE_BF16 ? bf : f32).push_back(&as[i]);
+  cudaError_t e = cudaSuccess;
+  if (!bf.empty()) e = launch_dtype<__nv_bfloat16>(bf, stream);
+  if (e == cudaSuccess && !f32.empty()) e = launch_dtype<float>(f32, stream);
+  return e;
+}
+
 cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream) {
-  if (a.xdt == QVLA_DTYPE_BF16) return launch_mode<__nv_bfloat16>(a, stream);
-  return launch_mode<float>(a, stream);
+  return launch_rotate_quant_batch(&a, 1, stream);
 }
 
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream) {

@@ -48,7 +48,7 @@ EXPORTED = (
     "qvla_status_str", "qvla_abi_version", "qvla_read_error_word", "qvla_packed_sizes",
     "qvla_pack_weights", "qvla_rotate_weights_f32", "qvla_quant_pack_weights_f32",
     "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
-    "qvla_w4a4_gemm_s32",
+    "qvla_w4a4_gemm_s32", "qvla_rotate_quant_act_batched", "qvla_w4a4_gemm_batched",
 )
 
 
@@ -58,7 +58,16 @@ class qvla_packed_linear(ctypes.Structure):
                 ("w_scale", c_void_p), ("bias", c_void_p)]
 
 
+class qvla_linear_problem(ctypes.Structure):
+    _fields_ = [("L", POINTER(qvla_packed_linear)), ("x", c_void_p), ("xdt", c_int32),
+                ("M", c_int32), ("ldx", c_int32), ("mode", c_int32), ("table", c_void_p),
+                ("T", c_int32), ("Lcount", c_int32), ("step_dev", c_void_p),
+                ("step_host", c_int32), ("layer", c_int32), ("xq", c_void_p), ("s_x", c_void_p),
+                ("y", c_void_p), ("ldy", c_int32)]
+
+
 _P = POINTER(qvla_packed_linear)
+_PP = POINTER(qvla_linear_problem)
 _sig = {
     "qvla_status_str": (ctypes.c_char_p, [c_int]),
     "qvla_abi_version": (c_int, []),
@@ -79,6 +88,8 @@ _sig = {
                                    c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "qvla_w4a4_gemm": (c_int, [c_void_p, c_void_p, c_int, _P, c_void_p, c_int, c_int, c_void_p]),
     "qvla_w4a4_gemm_s32": (c_int, [c_void_p, c_int, _P, c_void_p, c_int, c_void_p]),
+    "qvla_rotate_quant_act_batched": (c_int, [_PP, c_int, c_void_p]),
+    "qvla_w4a4_gemm_batched": (c_int, [_PP, c_int, c_int, c_void_p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -282,3 +293,44 @@ def from_host_packed(wq: np.ndarray, s_w: np.ndarray, perm: np.ndarray, rsvd: np
     t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(device)
     return PackedLinear(N, K, block, t(perm, np.int32), t(rsvd, np.float32), t(wq, np.uint8),
                         t(s_w, np.float32), None if bias is None else t(bias, np.float32))
+
+
+class LinearProblem:
+    """One independent linear of a batched call; keeps its tensors alive."""
+
+    def __init__(self, L: PackedLinear, x: Optional[torch.Tensor] = None,
+                 mode: int = QVLA_SCALE_DYNAMIC, table: Optional[torch.Tensor] = None,
+                 step=None, layer: int = 0, xq: Optional[torch.Tensor] = None,
+                 s_x: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None):
+        M = x.shape[0] if x is not None else xq.shape[0]
+        dev = (x if x is not None else xq).device
+        self.L, self.x, self.table, self.step = L, x, table, step
+        self.xq = xq if xq is not None else torch.empty(M, L.K // 2, dtype=torch.uint8, device=dev)
+        self.s_x = s_x if s_x is not None else torch.empty(M, dtype=torch.float32, device=dev)
+        self.y = y if y is not None else torch.empty(M, L.N, dtype=torch.bfloat16, device=dev)
+        T, Lc = (table.shape if table is not None else (0, 0))
+        sd, sh = _step_args(step)
+        self.c = qvla_linear_problem(
+            ctypes.pointer(L._s), x.data_ptr() if x is not None else None,
+            _dtype_code(x) if x is not None else QVLA_DTYPE_BF16, M,
+            x.stride(0) if x is not None else L.K, mode,
+            table.data_ptr() if table is not None else None, T, Lc,
+            sd.value if sd is not None else None, sh, layer, self.xq.data_ptr(),
+            self.s_x.data_ptr(), self.y.data_ptr(), self.y.stride(0))
+
+
+def _problem_array(problems):
+    arr = (qvla_linear_problem * len(problems))(*[p.c for p in problems])
+    return arr
+
+
+def qvla_rotate_quant_act_batched(problems, stream=None):
+    arr = _problem_array(problems)
+    _check(_lib.qvla_rotate_quant_act_batched(arr, len(problems), _stream(stream)),
+           "qvla_rotate_quant_act_batched")
+
+
+def qvla_w4a4_gemm_batched(problems, split_k: int = 0, stream=None):
+    arr = _problem_array(problems)
+    _check(_lib.qvla_w4a4_gemm_batched(arr, len(problems), split_k, _stream(stream)),
+           "qvla_w4a4_gemm_batched")
