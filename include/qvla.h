@@ -31,7 +31,15 @@
  *  - rot holds the R_SVD blocks, fp32 [nb][b][b]: rot[B][i][j] is row i,
  *    column j of R_SVD of block B.  The composite block rotation is
  *    R_B = R_SVD,B . H_b with H_b the Sylvester Hadamard matrix of order b
- *    scaled by 1/sqrt(b); H is never stored.
+ *    scaled by 1/sqrt(b); H is applied as a fast Walsh-Hadamard transform.
+ *  - rot_tc (optional, b = 64 or 128) holds R_B itself for the tensor-core
+ *    rotation: per block, R_B (computed in fp64) split into three bf16 parts
+ *    hi + mid + lo (each the bf16 rounding of what the previous parts leave),
+ *    each part stored as R_B^T (row j = output channel, its b inputs along
+ *    the row) in the 128-byte-swizzled K-major shared-memory image of the
+ *    tensor cores: 64-element K chunks of b rows x 128 bytes, the 16-byte
+ *    pieces of row j XOR-permuted by (j & 7).  uint16 bf16 bits,
+ *    [nb][3][b/64][b][64]; 6*K*b bytes.
  *  - Packed 4-bit codes: byte j of a row holds code 2j in its low nibble and
  *    code 2j+1 in its high nibble, 4-bit two's complement.  Weight codes lie
  *    in [-7, 7], activation codes in [-8, 7].
@@ -96,6 +104,7 @@ typedef struct {
   int32_t N, K, block;
   const int32_t* perm;      /* [K]  zigzag permutation                      */
   const float* rot;         /* [nb][b][b] R_SVD blocks                      */
+  const uint16_t* rot_tc;   /* tensor-core images of R_B, or NULL           */
   const uint8_t* wq;        /* [N][K/2] packed weight codes                 */
   const float* w_scale;     /* [N]  s_w                                      */
   const float* bias;        /* [N]  or NULL                                  */
@@ -109,11 +118,12 @@ int qvla_abi_version(void);
 qvla_status qvla_read_error_word(uint32_t* out, int clear);
 
 /* Byte sizes of the buffers a packed linear needs:
- *   *wq_bytes   = N * K / 2
- *   *rot_bytes  = 4 * K * block
- *   *ws_bytes   = workspace of qvla_pack_weights().                         */
+ *   *wq_bytes     = N * K / 2
+ *   *rot_bytes    = 4 * K * block
+ *   *rot_tc_bytes = 6 * K * block for block 64 or 128, else 0 (no image)
+ *   *ws_bytes     = workspace of qvla_pack_weights().  Any output may be NULL. */
 qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t* rot_bytes,
-                              size_t* ws_bytes);
+                              size_t* rot_tc_bytes, size_t* ws_bytes);
 
 /* ---------------------------------------------------------------------------
  * Offline pack ([PT]/[FR] Methodology 1: zigzag permutation by weight-column
@@ -129,7 +139,8 @@ qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t*
  *          eigenvectors are found on the host (cyclic Jacobi, fp64), ordered
  *          by descending eigenvalue with the largest-magnitude entry of each
  *          made positive.
- * Outputs (device): perm_out [K], rot_out [nb][b][b] fp32, wq_out [N][K/2],
+ * Outputs (device): perm_out [K], rot_out [nb][b][b] fp32, rot_tc_out (may be
+ *          NULL; ignored unless block is 64 or 128), wq_out [N][K/2],
  *          w_scale_out [N].  W' = W P R is formed in fp64 and
  *          rounded once to fp32 before RTN.
  * workspace device, >= ws_bytes from qvla_packed_sizes().
@@ -138,8 +149,8 @@ qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t*
  * ------------------------------------------------------------------------- */
 qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
                               const double* rsvd_in, int32_t* perm_out, float* rot_out,
-                              uint8_t* wq_out, float* w_scale_out, void* workspace,
-                              size_t ws_bytes, cudaStream_t stream);
+                              uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Device step of the pack: W'_f32 = fp32(W P R), computed in fp64 from fp64
  * R_SVD blocks.  W device fp32 [N][K]; perm device [K]; rsvd64 device fp64
@@ -161,7 +172,11 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
  *
  * x       device, [M][ldx] of `xdt` (ldx >= K, in elements).
  * L       host pointer to a packed linear (device pointers inside); only
- *         perm, rot, K and block are read.
+ *         perm, rot, rot_tc, K and block are read.  With bf16 input and a
+ *         rot_tc image the rotation runs on the tensor cores as one dense
+ *         product with R_B = R_SVD,B . H_b (three bf16 parts, fp32
+ *         accumulation in tensor memory); otherwise on the CUDA cores as the
+ *         R_SVD product followed by the fast Walsh-Hadamard transform.
  * table   device fp32 [T][Lcount], required for TABLE mode.
  * step_dev device int32 or NULL.  If non-NULL the step is read on the device
  *         (so one captured graph serves every denoising step); a step outside
@@ -170,13 +185,23 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
  *         the table ([ES]).  If NULL, `step_host` is used and checked on the
  *         host (QVLA_ERR_STEP_RANGE).
  * layer   column of the table; 0 <= layer < Lcount (checked on the host).
+ * workspace optional device scratch (see qvla_rotate_quant_workspace_bytes).
  * Outputs (device): xq [M][K/2] packed codes, s_x [M] fp32.
  * ------------------------------------------------------------------------- */
 qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
                                   const qvla_packed_linear* L, qvla_scale_mode mode,
                                   const float* table, int T, int Lcount, const int32_t* step_dev,
                                   int step_host, int layer, uint8_t* xq, float* s_x,
-                                  cudaStream_t stream);
+                                  void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Scratch that lets qvla_rotate_quant_act take its fastest route for large M
+ * (tensor-core rotation fed by TMA from a permuted copy of x): M * K * 2 bytes
+ * when that route applies (bf16 input, block 64 or 128, M > 64), else 0.
+ * Without it (workspace NULL or too small) the call still works, gathering
+ * the permuted inputs directly.  The scratch is only used while the call's
+ * kernels run; reusing it for another call on the same stream is safe.     */
+qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtype xdt,
+                                              size_t* bytes);
 
 /* The rotation alone, for parity checks: xr_out device fp32 [M][K] = the
  * same fp32 x' the fused kernel quantises.                                  */
@@ -241,6 +266,8 @@ typedef struct {
   float* s_x;                    /* device [M] scales: output, then input       */
   void* y;                       /* device bf16 [M][ldy] GEMM output            */
   int32_t ldy;
+  void* workspace;               /* optional rotate-quant scratch, or NULL      */
+  size_t ws_bytes;               /* (qvla_rotate_quant_workspace_bytes)         */
 } qvla_linear_problem;
 
 /* qvla_rotate_quant_act for every problem (reads x, writes xq and s_x). */

@@ -46,8 +46,11 @@ def test_status_strings_and_version():
 
 def test_packed_sizes_and_shape_errors():
     q = _lib_mod()
-    wq, rot, ws = q.qvla_packed_sizes(4096, 1024, 64)
+    wq, rot, tc, ws = q.qvla_packed_sizes(4096, 1024, 64)
     assert wq == 4096 * 1024 // 2 and rot == 1024 * 64 * 4 and ws > 4096 * 1024 * 4
+    assert tc == 6 * 1024 * 64
+    assert q.qvla_packed_sizes(256, 512, 256)[2] == 0          # no tensor-core image
+    assert q.qvla_packed_sizes(256, 512, 128)[2] == 6 * 512 * 128
     for args in ((4096, 1000, 64), (4096, 1024, 48), (0, 1024, 64), (16, 65536, 64),
                  (16, 1024, 512)):
         with pytest.raises(q.QvlaError) as e:
@@ -60,22 +63,22 @@ def test_argument_errors_before_any_cuda_call():
     lib = q._lib
     # null packed linear
     assert lib.qvla_rotate_quant_act(None, 1, 4, 64, None, 0, None, 0, 0, None, 0, 0, None,
-                                     None, None) == q.QVLA_ERR_ARG
-    L = q.qvla_packed_linear(128, 256, 64, 0, 0, 0, 0, None)
+                                     None, None, 0, None) == q.QVLA_ERR_ARG
+    L = q.qvla_packed_linear(128, 256, 64, 0, 0, None, 0, 0, None)
     assert lib.qvla_w4a4_gemm(None, None, 4, ctypes.byref(L), None, 128, 0, None) == q.QVLA_ERR_ARG
     # bad shape inside the struct
-    Lbad = q.qvla_packed_linear(128, 250, 64, 16, 16, 16, 16, None)
+    Lbad = q.qvla_packed_linear(128, 250, 64, 16, 16, None, 16, 16, None)
     assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lbad),
                                    ctypes.c_void_p(16), None) == q.QVLA_ERR_SHAPE
     # misaligned pointers
-    Lmis = q.qvla_packed_linear(128, 256, 64, 16, 24, 16, 16, None)
+    Lmis = q.qvla_packed_linear(128, 256, 64, 16, 24, None, 16, 16, None)
     assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lmis),
                                    ctypes.c_void_p(16), None) == q.QVLA_ERR_ALIGN
     # table mode: layer or host step outside the table -> STEP_RANGE, never a clamp
-    Lok = q.qvla_packed_linear(128, 256, 64, 16, 16, 16, 16, None)
+    Lok = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)
     args = lambda step, layer: (ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lok),
                                 q.QVLA_SCALE_TABLE, ctypes.c_void_p(16), 10, 12, None, step,
-                                layer, ctypes.c_void_p(16), ctypes.c_void_p(16), None)
+                                layer, ctypes.c_void_p(16), ctypes.c_void_p(16), None, 0, None)
     assert lib.qvla_rotate_quant_act(*args(10, 0)) == q.QVLA_ERR_STEP_RANGE
     assert lib.qvla_rotate_quant_act(*args(-1, 0)) == q.QVLA_ERR_STEP_RANGE
     assert lib.qvla_rotate_quant_act(*args(0, 12)) == q.QVLA_ERR_STEP_RANGE
@@ -85,10 +88,14 @@ def test_argument_errors_before_any_cuda_call():
                                   None) == q.QVLA_ERR_ARG
     # empty input is a no-op
     assert lib.qvla_rotate_quant_act(None, 1, 0, 256, ctypes.byref(Lok), 0, None, 0, 0, None, 0,
-                                     0, None, None, None) == q.QVLA_OK
+                                     0, None, None, None, 0, None) == q.QVLA_OK
+    # scratch size query: only the tensor-core route for more than 64 bf16 tokens uses it
+    assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 128) == 1024 * 2048 * 2
+    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64) == 0
+    assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 256) == 0
     assert lib.qvla_w4a4_gemm_s32(None, 0, ctypes.byref(Lok), None, 0, None) == q.QVLA_OK
     # split-K factor must be a power of two <= 16 and <= the number of 256-wide K tiles
-    Lw = q.qvla_packed_linear(128, 256, 64, 16, 16, 16, 16, None)
+    Lw = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)
     assert lib.qvla_w4a4_gemm_s32(ctypes.c_void_p(16), 4, ctypes.byref(Lw), ctypes.c_void_p(16),
                                   3, None) == q.QVLA_ERR_ARG
     assert lib.qvla_w4a4_gemm_s32(ctypes.c_void_p(16), 4, ctypes.byref(Lw), ctypes.c_void_p(16),
@@ -99,5 +106,6 @@ def test_pack_workspace_check():
     q = _lib_mod()
     lib = q._lib
     assert lib.qvla_pack_weights(ctypes.c_void_p(16), 64, 256, 64, None, None,
-                                 ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
-                                 ctypes.c_void_p(16), None, 0, None) == q.QVLA_ERR_WORKSPACE
+                                 ctypes.c_void_p(16), ctypes.c_void_p(16), None,
+                                 ctypes.c_void_p(16), ctypes.c_void_p(16), None, 0,
+                                 None) == q.QVLA_ERR_WORKSPACE

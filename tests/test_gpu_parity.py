@@ -63,6 +63,41 @@ def test_act_quant_from_fp32_is_bit_exact(q, M, K):
     no_device_error(q)
 
 
+def test_quant_near_rounding_boundaries_is_bit_exact(q):
+    """Values at, and one or two ulp around, every half-integer multiple of the
+    scale: the codes must equal clamp(rint(fp32(v / s))) exactly (ties to even),
+    including where a reciprocal multiply would round the other way."""
+    rows = []
+    for s in (np.float32(0.1), np.float32(0.0123), np.float32(3.7), np.float32(1e-3)):
+        v = []
+        for j in range(-9, 9):
+            c = np.float32((j + 0.5) * float(s))
+            for d in (-2, -1, 0, 1, 2):
+                v.append(c + np.float32(d) * np.spacing(c) if d else c)
+        v = np.array(v, np.float32)
+        # the row's max must pin s = max/7 exactly: append +-7 s and pad to 96
+        row = np.zeros(96, np.float32)
+        row[:len(v)] = v
+        row[-1] = np.float32(7) * s
+        rows.append(row)
+    xr = np.stack(rows)
+    # table mode (s taken as given) and dynamic mode (s = max/7)
+    for mode in ("table", "dynamic"):
+        if mode == "dynamic":
+            qr, sr = O.quantize_acts_dynamic_fp32(xr)
+            xq, sg = q.qvla_quant_act_f32(cu(xr), q.QVLA_SCALE_DYNAMIC)
+            assert np.array_equal(sg.cpu().numpy(), sr)
+            assert np.array_equal(xq.cpu().numpy(), O.pack_nibbles(qr))
+        else:
+            for i, s in enumerate((0.1, 0.0123, 3.7, 1e-3)):
+                tab = np.full((1, 1), s, np.float32)
+                qr, _ = O.quantize_acts_table_fp32(xr[i:i + 1], np.float32(s))
+                xq, _ = q.qvla_quant_act_f32(cu(xr[i:i + 1]), q.QVLA_SCALE_TABLE, table=cu(tab),
+                                             step=0, layer=0)
+                assert np.array_equal(xq.cpu().numpy(), O.pack_nibbles(qr)), s
+    no_device_error(q)
+
+
 @pytest.mark.parametrize("N,K", [(3, 64), (256, 256), (1000, 1024)])
 def test_weight_quant_from_fp32_is_bit_exact(q, N, K):
     Wr = I.weights(200 + N, N, K, n_outlier_rows=2)
@@ -112,10 +147,44 @@ def test_pack_parity(q, N, K, b):
 
 # ----------------------------------------------------- activation rotation
 
+@pytest.fixture(params=["auto", "fma"])
+def path(request, monkeypatch):
+    """auto: tensor cores where the linear has an image (bf16, block 64/128);
+    fma: always the CUDA-core rotation."""
+    monkeypatch.setenv("QVLA_ROTATE_PATH", request.param)
+    return request.param
+
+
+def _unswizzle_tc_image(img, nb, b):
+    """uint16 [nb*3*b*b] (128B-swizzled K-major R_B^T parts) -> float64 [nb, 3, b(i), b(j)]."""
+    img = img.reshape(nb, 3, b * b)
+    out = np.zeros((nb, 3, b, b))
+    i = np.arange(b)[:, None]
+    j = np.arange(b)[None, :]
+    kc, c = i // 64, (i % 64) // 8
+    off = kc * b * 64 + j * 64 + ((c ^ (j & 7)) * 8) + (i % 8)
+    bits = img[:, :, off].astype(np.uint32) << 16
+    return bits.view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("K,b", [(256, 64), (512, 128)])
+def test_tc_image_is_the_composite_rotation(q, K, b):
+    """The tensor-core image holds hi + mid + lo = R_SVD,B . H_b to ~2^-25."""
+    W = I.weights(450 + K, 96, K)
+    ref = O.pack_linear(W, b)
+    L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    parts = _unswizzle_tc_image(L.rot_tc.cpu().numpy().view(np.uint16), K // b, b)
+    recon = parts.sum(axis=1)
+    assert np.abs(recon - ref.R).max() <= 2e-8 * np.abs(ref.R).max()
+    assert np.abs(parts[:, 0] - ref.R).max() > 1e-5 * np.abs(ref.R).max()   # hi alone is coarse
+    no_device_error(q)
+
+
 @pytest.mark.parametrize("M,K,b,dt", [(16, 256, 64, "f32"), (50, 1024, 64, "bf16"),
                                       (5, 2048, 128, "bf16"), (3, 512, 32, "bf16"),
-                                      (9, 1024, 256, "bf16"), (2, 16384, 128, "bf16")])
-def test_rotation_fp32_vs_fp64(q, M, K, b, dt):
+                                      (9, 1024, 256, "bf16"), (2, 16384, 128, "bf16"),
+                                      (300, 1024, 64, "bf16"), (130, 512, 128, "bf16")])
+def test_rotation_fp32_vs_fp64(q, path, M, K, b, dt):
     W = I.weights(400 + K, 64, K)
     ref = O.pack_linear(W, b)
     L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
@@ -130,21 +199,29 @@ def test_rotation_fp32_vs_fp64(q, M, K, b, dt):
     (16, 256, 64, "f32", "dynamic"), (50, 1024, 64, "bf16", "table"),
     (50, 4096, 64, "bf16", "table"), (37, 2048, 128, "bf16", "dynamic"),
     (8, 1024, 32, "bf16", "dynamic"), (8, 1024, 256, "bf16", "table"),
-    (3, 16384, 128, "bf16", "dynamic")])
-def test_rotate_quant_end_to_end(q, M, K, b, dt, mode):
+    (3, 16384, 128, "bf16", "dynamic"), (300, 2048, 64, "bf16", "dynamic"),
+    (257, 1536, 64, "bf16", "table"), (200, 4096, 128, "bf16", "table")])
+@pytest.mark.parametrize("scratch", [False, True])
+def test_rotate_quant_end_to_end(q, path, scratch, M, K, b, dt, mode):
+    """scratch=True gives the call its workspace, which routes large bf16 inputs
+    through the permuted copy + TMA-fed tensor-core kernel."""
     W = I.weights(500 + K + b, 96, K)
     ref = O.pack_linear(W, b)
     L = q.qvla_pack_weights(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
     x = I.activations(501 + M, M, K, std=1.3, n_outlier_cols=4, dtype=dt)
     tab = I.scale_table(7, 10, 12, I.step_sigmas(10) * 1.3)
+    ws = None
+    if scratch:
+        nbytes = q.qvla_rotate_quant_workspace_bytes(M, K, b, x_dev(x[:1], dt).dtype)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
     if mode == "dynamic":
-        xq, s = q.qvla_rotate_quant_act(x_dev(x, dt), L, q.QVLA_SCALE_DYNAMIC)
+        xq, s = q.qvla_rotate_quant_act(x_dev(x, dt), L, q.QVLA_SCALE_DYNAMIC, workspace=ws)
         xr_ref, qx_ref, s_ref = O.rotate_quant_act(x, ref, "dynamic")
         np.testing.assert_allclose(s.cpu().numpy(), s_ref, rtol=2e-6)
     else:
         step = torch.tensor([4], dtype=torch.int32, device="cuda")
         xq, s = q.qvla_rotate_quant_act(x_dev(x, dt), L, q.QVLA_SCALE_TABLE, table=cu(tab),
-                                        step=step, layer=7)
+                                        step=step, layer=7, workspace=ws)
         xr_ref, qx_ref, s_ref = O.rotate_quant_act(x, ref, "table", tab, 4, 7)
         assert (s.cpu().numpy() == tab[4, 7]).all()
     check_codes_near_boundary(unpack(xq.cpu().numpy()), qx_ref, xr_ref, s_ref, "activations")

@@ -8,6 +8,8 @@
 // ("{Omega}-QVLA: Robust Quantization ...", Methodology 1: SVD rotation from
 // W = U S V^T, normalised Hadamard, block implementation with a zigzag
 // permutation by weight-column norm.)
+#include <cuda_bf16.h>
+
 #include "qvla_common.cuh"
 #include "qvla_internal.h"
 
@@ -139,7 +141,51 @@ __global__ void __launch_bounds__(256)
   for (int c = 0; c < C; ++c) dst[32 * c] = static_cast<float>(acc[c] * inv);
 }
 
+// Tensor-core image of the composite rotation: R_B = R_SVD,B . H_b in fp64,
+// split into bf16 parts hi + mid + lo (each the round-to-nearest bf16 of what
+// the previous parts leave), stored as R_B^T rows in the 128-byte-swizzled
+// K-major layout (see qvla.h).  One thread per element (i, j) of R_B.
+template <int BS>
+__global__ void __launch_bounds__(256)
+    rot_tc_image_kernel(const double* __restrict__ rsvd, uint16_t* __restrict__ img) {
+  const int B = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= BS * BS) return;
+  const int i = e / BS, j = e % BS;           // R_B[i][j]: input i, output j
+  const double* R = rsvd + static_cast<size_t>(B) * BS * BS;
+  const double inv = 1.0 / sqrt(static_cast<double>(BS));
+  double v = 0.0;
+  for (int k = 0; k < BS; ++k) {
+    const double h = (__popc(k & j) & 1) ? -inv : inv;
+    v = fma(R[i * BS + k], h, v);
+  }
+  uint16_t* base = img + static_cast<size_t>(B) * 3 * BS * BS;
+  const int kc = i / 64, c = (i % 64) / 8;
+  const size_t off = static_cast<size_t>(kc) * BS * 64 + j * 64 + ((c ^ (j & 7)) * 8) + (i % 8);
+  double r = v;
+#pragma unroll
+  for (int sp = 0; sp < 3; ++sp) {
+    const __nv_bfloat16 part = __double2bfloat16(r);
+    r -= static_cast<double>(__bfloat162float(part));
+    base[static_cast<size_t>(sp) * BS * BS + off] = __bfloat16_as_ushort(part);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_rot_tc_image(const double* rsvd64, int K, int block, uint16_t* img,
+                                cudaStream_t s) {
+  const int nb = K / block;
+  const dim3 grid((block * block + 255) / 256, nb);
+  if (block == 64) {
+    rot_tc_image_kernel<64><<<grid, 256, 0, s>>>(rsvd64, img);
+  } else if (block == 128) {
+    rot_tc_image_kernel<128><<<grid, 256, 0, s>>>(rsvd64, img);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_column_norms(const float* W, int N, int K, double* norms, cudaStream_t s) {
   column_norms_kernel<<<(K + 255) / 256, 256, 0, s>>>(W, N, K, norms);

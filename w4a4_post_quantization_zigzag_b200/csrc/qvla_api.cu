@@ -60,6 +60,7 @@ qvla_status check_linear(const qvla_packed_linear* L, bool need_weights) {
   if (!L->perm || !L->rot) return QVLA_ERR_ARG;
   if (need_weights && (!L->wq || !L->w_scale)) return QVLA_ERR_ARG;
   if (!aligned16(L->perm) || !aligned16(L->rot)) return QVLA_ERR_ALIGN;
+  if (L->rot_tc && !aligned16(L->rot_tc)) return QVLA_ERR_ALIGN;
   if (need_weights && (!aligned16(L->wq) || !aligned16(L->w_scale))) return QVLA_ERR_ALIGN;
   if (L->bias && !aligned16(L->bias)) return QVLA_ERR_ALIGN;
   return QVLA_OK;
@@ -224,12 +225,14 @@ qvla_status qvla_read_error_word(uint32_t* out, int clear) {
 }
 
 qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t* rot_bytes,
-                              size_t* ws_bytes) {
+                              size_t* rot_tc_bytes, size_t* ws_bytes) {
   qvla_status st = check_shape(N, K, block);
   if (st != QVLA_OK) return st;
   if (K % 32) return QVLA_ERR_SHAPE;
   if (wq_bytes) *wq_bytes = static_cast<size_t>(N) * K / 2;
   if (rot_bytes) *rot_bytes = static_cast<size_t>(K) * block * 4;
+  if (rot_tc_bytes)
+    *rot_tc_bytes = (block == 64 || block == 128) ? static_cast<size_t>(K) * block * 6 : 0;
   if (ws_bytes) *ws_bytes = pack_ws_bytes(N, K, block);
   return QVLA_OK;
 }
@@ -263,8 +266,8 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
 
 qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
                               const double* rsvd_in, int32_t* perm_out, float* rot_out,
-                              uint8_t* wq_out, float* w_scale_out, void* workspace,
-                              size_t ws_bytes, cudaStream_t stream) {
+                              uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream) {
   qvla_status st = check_shape(N, K, block);
   if (st != QVLA_OK) return st;
   if (K % 32) return QVLA_ERR_SHAPE;
@@ -335,6 +338,12 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
                       stream) != cudaSuccess)
     return QVLA_ERR_CUDA;
 
+  if (rot_tc_out && (block == 64 || block == 128)) {
+    if (!aligned16(rot_tc_out)) return QVLA_ERR_ALIGN;
+    if (launch_rot_tc_image(rsvd_dev, K, block, rot_tc_out, stream) != cudaSuccess)
+      return QVLA_ERR_CUDA;
+  }
+
   // 3. W' = fp32(W P R) in fp64, then RTN + packing
   if (launch_rotate_weights(W, N, K, block, perm_out, rsvd_dev, Wr, stream) != cudaSuccess)
     return QVLA_ERR_CUDA;
@@ -380,6 +389,7 @@ static qvla_status prepare_act(const void* x, qvla_dtype xdt, int M, int ldx,
   a.block = L->block;
   a.perm = L->perm;
   a.rot = L->rot;
+  a.rot_tc = (L->rot_tc && (L->block == 64 || L->block == 128)) ? L->rot_tc : nullptr;
   a.dynamic = mode == QVLA_SCALE_DYNAMIC;
   a.table = table;
   a.T = T;
@@ -396,12 +406,23 @@ qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
                                   const qvla_packed_linear* L, qvla_scale_mode mode,
                                   const float* table, int T, int Lcount, const int32_t* step_dev,
                                   int step_host, int layer, uint8_t* xq, float* s_x,
-                                  cudaStream_t stream) {
+                                  void* workspace, size_t ws_bytes, cudaStream_t stream) {
   ActArgs a;
   qvla_status st = prepare_act(x, xdt, M, ldx, L, mode, table, T, Lcount, step_dev, step_host,
                                layer, xq, s_x, &a);
   if (st != QVLA_OK || M == 0) return st;
+  a.ws = workspace;
+  a.ws_bytes = ws_bytes;
   return cuda_status(launch_rotate_quant(a, stream));
+}
+
+qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtype xdt,
+                                              size_t* bytes) {
+  if (!bytes) return QVLA_ERR_ARG;
+  if (M < 0 || K <= 0 || K > QVLA_MAX_K || !valid_block(block) || K % block) return QVLA_ERR_SHAPE;
+  const bool tc = xdt == QVLA_DTYPE_BF16 && (block == 64 || block == 128) && M > 64;
+  *bytes = tc ? static_cast<size_t>(M) * K * 2 : 0;
+  return QVLA_OK;
 }
 
 qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int n,
@@ -414,6 +435,8 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
                                  static_cast<qvla_scale_mode>(p.mode), p.table, p.T, p.Lcount,
                                  p.step_dev, p.step_host, p.layer, p.xq, p.s_x, &v[i]);
     if (st != QVLA_OK) return st;
+    v[i].ws = p.workspace;
+    v[i].ws_bytes = p.ws_bytes;
   }
   return cuda_status(launch_rotate_quant_batch(v.data(), n, stream));
 }
@@ -438,6 +461,7 @@ qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
   a.block = L->block;
   a.perm = L->perm;
   a.rot = L->rot;
+  a.rot_tc = (L->rot_tc && (L->block == 64 || L->block == 128)) ? L->rot_tc : nullptr;
   a.dynamic = 1;
   a.xr_out = xr_out;
   return cuda_status(launch_rotate_quant(a, stream));

@@ -22,6 +22,7 @@ struct ActArgs {
   int M, ldx, K, block;
   const int32_t* perm;
   const float* rot;
+  const uint16_t* rot_tc; // tensor-core image of R_B or nullptr
   int dynamic;            // 1: per-token absmax, 0: table
   const float* table;
   int T, Lcount;
@@ -30,6 +31,8 @@ struct ActArgs {
   uint8_t* xq;
   float* s_x;
   float* xr_out;          // rotate-only mode when non-null and xq == nullptr
+  void* ws;               // optional scratch for the permuted copy of x
+  size_t ws_bytes;
 };
 cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream);
 // independent linears in as few launches as possible (grouped by kernel config)
@@ -54,6 +57,8 @@ cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream);
 cudaError_t launch_column_norms(const float* W, int N, int K, double* norms, cudaStream_t s);
 cudaError_t launch_block_gram(const float* W, int N, int K, int block, const int32_t* perm,
                               double* gram, cudaStream_t s);
+cudaError_t launch_rot_tc_image(const double* rsvd64, int K, int block, uint16_t* img,
+                                cudaStream_t s);
 cudaError_t launch_rotate_weights(const float* W, int N, int K, int block, const int32_t* perm,
                                   const double* rsvd64, float* Wr, cudaStream_t s);
 

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
@@ -106,6 +107,75 @@ QVLA_DEVICE int quant_code(float v, float s, int qmin, int qmax) {
   return static_cast<int>(r);
 }
 
+// The same code as quant_code(v, s, ...), i.e. clamp(rint(fp32(v / s))), with
+// the IEEE division replaced by v * rs (rs = fp32(1 / s)) wherever that cannot
+// change the rounding: the product is within 2^-19 of the exact quotient for
+// |quotient| < 16 (two roundings of 2^-24 relative), so unless it lies within
+// 2^-18 of a half-integer both round to the same integer; near a half-integer
+// (about 1 element in 10^5) the exact division decides.  Quotients of 16 or
+// more clamp either way.
+// Kept out of line so the compiler cannot hoist the rare exact division into
+// the common path.
+__device__ __noinline__ float exact_rint_quotient(float v, float s) { return rintf(__fdiv_rn(v, s)); }
+
+QVLA_DEVICE int quant_code_fast(float v, float s, float rs, int qmin, int qmax) {
+  if (s == 0.f) return 0;
+  if (rs == 0.f) return quant_code(v, s, qmin, qmax);
+  const float q = v * rs;
+  float r = rintf(q);
+  if (fabsf(fabsf(q - r) - 0.5f) < 3.814697265625e-06f) r = exact_rint_quotient(v, s);
+  r = fminf(fmaxf(r, static_cast<float>(qmin)), static_cast<float>(qmax));
+  return static_cast<int>(r);
+}
+
+// Codes of N consecutive values, packed two per byte (value 2k in the low
+// nibble of byte k) into N/8 32-bit words: the same codes as quant_code, as
+// straight-line code (so the independent elements overlap) with the rare
+// near-half-integer elements redone by exact division afterwards.  The code's
+// 4-bit two's complement is read from the mantissa of code + 2^23 + 16.
+template <int N>
+QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float rs, int qmin, int qmax,
+                            uint32_t (&w)[N / 8]) {
+  static_assert(N % 8 == 0 && N <= 32, "8..32 values");
+  float c[N];
+  if (s == 0.f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) c[i] = 0.f;
+  } else if (rs == 0.f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) c[i] = exact_rint_quotient(v[i], s);
+  } else {
+    uint32_t near = 0u;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const float q = v[i] * rs;
+      c[i] = rintf(q);
+      near |= (fabsf(fabsf(q - c[i]) - 0.5f) < 3.814697265625e-06f ? 1u : 0u) << i;
+    }
+    if (near) {
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+        if ((near >> i) & 1u) c[i] = exact_rint_quotient(v[i], s);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < N / 8; ++k) w[k] = 0u;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float cl = fminf(fmaxf(c[i], static_cast<float>(qmin)), static_cast<float>(qmax));
+    const uint32_t nib = __float_as_uint(cl + 8388624.0f) & 15u;      // 2^23 + 16
+    w[i >> 3] |= nib << (4 * (i & 7));
+  }
+}
+
+// fp32(1 / s) for quant_code_fast, or 0 to force the exact path (s == 0 or a
+// reciprocal that overflows).
+QVLA_DEVICE float quant_recip(float s) {
+  if (s == 0.f) return 0.f;
+  const float rs = __frcp_rn(s);
+  return isfinite(rs) ? rs : 0.f;
+}
+
 QVLA_DEVICE float load_x(const float* p) { return __ldg(p); }
 QVLA_DEVICE float load_x(const __nv_bfloat16* p) {
   return __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p)))
@@ -167,9 +237,11 @@ QVLA_DEVICE void store_codes32(uint8_t* dst, int q, int lane) {
 // over the cluster along grid y instead.
 constexpr int kMaxBatch = 16;
 struct ActProblem {
+  CUtensorMap txp;            // permuted copy of x (tensor-core path with scratch)
   const void* x;
   const int32_t* perm;
   const float* rot;
+  const uint16_t* rot_tc;
   const float* table;
   const int32_t* step_dev;
   uint8_t* xq;
@@ -302,9 +374,10 @@ __global__ void __launch_bounds__(kThreads)
         for (int c = 0; c < C; ++c) dst[32 * c] = v[c];
       } else if (MODE == kTable) {
         uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS) / 2;
+        const float rs = quant_recip(s_tab);
 #pragma unroll
         for (int c = 0; c < C; ++c)
-          store_codes32(dst + 16 * c, quant_code(v[c], s_tab, -8, 7), lane);
+          store_codes32(dst + 16 * c, quant_code_fast(v[c], s_tab, rs, -8, 7), lane);
       } else {
         float mx = 0.f;
 #pragma unroll
@@ -352,6 +425,7 @@ __global__ void __launch_bounds__(kThreads)
   const int nch = nbc * BS;                    // channels held by this CTA (multiple of 32)
   for (int t = warp; t < ntok; t += kWarps) {
     const float s = scale_s[t];
+    const float rs = quant_recip(s);
     uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B0 * BS) / 2;
     for (int c0 = 0; c0 < nch; c0 += 256) {
       const int k = c0 + 8 * lane;            // 8 channels -> 4 bytes per lane
@@ -359,17 +433,361 @@ __global__ void __launch_bounds__(kThreads)
         const float4 a = *reinterpret_cast<const float4*>(keep + t * kpitch + k);
         const float4 b = *reinterpret_cast<const float4*>(keep + t * kpitch + k + 4);
         const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        uint32_t w = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int lo = quant_code(f[2 * q], s, -8, 7), hi = quant_code(f[2 * q + 1], s, -8, 7);
-          w |= static_cast<uint32_t>((lo & 15) | ((hi & 15) << 4)) << (8 * q);
-        }
-        *reinterpret_cast<uint32_t*>(dst + k / 2) = w;
+        uint32_t w[1];
+        quant_pack<8>(f, s, rs, -8, 7, w);
+        *reinterpret_cast<uint32_t*>(dst + k / 2) = w[0];
       }
     }
   }
   if (cs > 1) cluster_wait();                  // peers finished reading our maxima
+}
+
+// ===========================================================================
+// Tensor-core path (bf16 input, block 64 or 128).
+//
+// The block rotation is one dense product x'_B = x_B . R_B with the composite
+// R_B = R_SVD,B . H_b, on tcgen05 (kind::f16, fp32 accumulation in tensor
+// memory).  bf16 activations are exact in bf16; R_B is carried as three bf16
+// parts (hi + mid + lo, pack time), so the product has ~fp32 accuracy.
+// Per CTA: a tile of 128 tokens (the UMMA M dimension) and a run of blocks.
+//   warp 0      bulk-copies the R_B parts (pre-swizzled images) into a ring
+//   warp 1      issues the MMAs (3 parts x b/16 K-steps per block)
+//   warps 2-5   gather x[m, perm[B*b + i]] into a 128B-swizzled A tile
+//   warps 6-9   read the accumulator (one token per thread) and quantise
+// DYNAMIC mode runs the blocks twice: pass 0 takes each token's max |x'|
+// (reduced over the cluster that shares the row), pass 1 quantises.
+// ===========================================================================
+using EncodeTiledFnR = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+constexpr int kTcThreads = 320;
+constexpr int kTM = 128;
+
+template <int BS>
+struct TcCfg {
+  static constexpr int kAStage = kTM * BS * 2;          // bf16 A tile
+  static constexpr int kRStage = BS * BS * 2;           // one bf16 part of R_B^T
+  static constexpr int kAS = 2;
+  static constexpr int kRS = BS == 64 ? 6 : 4;
+  static constexpr int kTmemCols = 2 * BS;              // double-buffered fp32 accumulator
+  static constexpr int kSmem = kAS * kAStage + kRS * kRStage + 1024;
+};
+
+struct TcBars {
+  uint64_t full_a[2], empty_a[2], full_r[6], empty_r[6], acc_full[2], acc_empty[2];
+  uint32_t tmem;
+};
+
+QVLA_DEVICE void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int BS, int MODE, bool kTmaA>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    rotq_tc_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
+  using C = TcCfg<BS>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ TcBars bars;
+  __shared__ unsigned int amax_s[kTM];
+
+  int pi = 0;
+  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[pi + 1]) ++pi;
+  const ActProblem& P = batch.p[pi];
+  const __nv_bfloat16* __restrict__ x = static_cast<const __nv_bfloat16*>(P.x);
+  const int M = P.M, ldx = P.ldx, K = P.K;
+  const int local = static_cast<int>(blockIdx.x) - batch.cta_start[pi];
+  const int tile = local % P.gx;
+  const int group = MODE == kDynamic ? static_cast<int>(blockIdx.y) : local / P.gx;
+  const int m0 = tile * kTM;
+  const int ntok = min(kTM, M - m0);
+  const int nb = K / BS;
+  const int B0 = group * P.bpc;
+  const int nbc = max(0, min(P.bpc, nb - B0));
+  const int passes = MODE == kDynamic ? 2 : 1;
+  const int W = passes * nbc;                  // work items: (pass, block)
+  const int cs = MODE == kDynamic ? static_cast<int>(gridDim.y) : 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  uint8_t* const base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  uint8_t* const astage = base;
+  uint8_t* const rstage = base + C::kAS * C::kAStage;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.full_a[i], kTmaA ? 1 : 128);
+      mbar_init(&bars.empty_a[i], 1);
+      mbar_init(&bars.acc_full[i], 1);
+      mbar_init(&bars.acc_empty[i], 128);
+    }
+    for (int i = 0; i < C::kRS; ++i) {
+      mbar_init(&bars.full_r[i], 1);
+      mbar_init(&bars.empty_r[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem;
+  const bool epi = warp >= 6;
+  // cluster barrier phase 1 ("row maxima published"): threads that are not in
+  // the epilogue arrive once their pass-0 work is issued, so the epilogue's
+  // wait never depends on work that waits for the epilogue
+  bool arrived1 = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- R_B parts
+    if (lane == 0) {
+      for (int w = 0; w < W; ++w) {
+        const int B = B0 + w % nbc;
+        for (int sp = 0; sp < 3; ++sp) {
+          const int u = 3 * w + sp, rr = u % C::kRS;
+          if (!mbar_wait(&bars.empty_r[rr], ((u / C::kRS) & 1) ^ 1u, err)) break;
+          mbar_arrive_expect_tx(&bars.full_r[rr], C::kRStage);
+          bulk_copy_g2s(rstage + rr * C::kRStage,
+                        P.rot_tc + (static_cast<size_t>(B) * 3 + sp) * BS * BS, C::kRStage,
+                        &bars.full_r[rr]);
+        }
+        if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
+          cluster_arrive_relaxed();
+          arrived1 = true;
+        }
+      }
+      // never leave with copies in flight
+      const int U = 3 * W;
+      for (int u = U - C::kRS < 0 ? 0 : U - C::kRS; u < U; ++u)
+        mbar_wait(&bars.full_r[u % C::kRS], (u / C::kRS) & 1, err);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTM, BS);
+      const uint32_t a_base = smem_u32(astage), r_base = smem_u32(rstage);
+      for (int w = 0; w < W; ++w) {
+        const int as = w & 1, ab = w & 1;
+        if (!mbar_wait(&bars.full_a[as], (w >> 1) & 1, err)) break;
+        if (!mbar_wait(&bars.acc_empty[ab], ((w >> 1) & 1) ^ 1u, err)) break;
+        tc_fence_after();
+        for (int sp = 0; sp < 3; ++sp) {
+          const int u = 3 * w + sp, rr = u % C::kRS;
+          if (!mbar_wait(&bars.full_r[rr], (u / C::kRS) & 1, err)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < BS / 16; ++k) {
+            const int kc = k >> 2, kk = k & 3;
+            const uint64_t ad = smem_desc_kmajor_sw128(a_base + as * C::kAStage + kc * (kTM * 128) + kk * 32);
+            const uint64_t bd = smem_desc_kmajor_sw128(r_base + rr * C::kRStage + kc * (BS * 128) + kk * 32);
+            umma_bf16(tmem + ab * BS, ad, bd, idesc, (sp | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&bars.empty_r[rr]);
+        }
+        umma_commit(&bars.empty_a[as]);
+        umma_commit(&bars.acc_full[ab]);
+        if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
+          cluster_arrive_relaxed();
+          arrived1 = true;
+        }
+      }
+    }
+  } else if (!epi && kTmaA) {
+    // ------------------------------------------- A tiles by TMA (permuted x)
+    if (tid == 64) {
+      pdl_wait();
+      int issued = 0;
+      for (int w = 0; w < W; ++w) {
+        const int B = B0 + w % nbc, as = w & 1;
+        if (!mbar_wait(&bars.empty_a[as], ((w >> 1) & 1) ^ 1u, err)) break;
+        mbar_arrive_expect_tx(&bars.full_a[as], C::kAStage);
+#pragma unroll
+        for (int kc = 0; kc < BS / 64; ++kc)
+          tma_load_2d(astage + as * C::kAStage + kc * (kTM * 128), &P.txp, &bars.full_a[as],
+                      B * BS + kc * 64, m0);
+        ++issued;
+        if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
+          cluster_arrive_relaxed();
+          arrived1 = true;
+        }
+      }
+      for (int w = issued - 2 < 0 ? 0 : issued - 2; w < issued; ++w)
+        mbar_wait(&bars.full_a[w & 1], (w >> 1) & 1, err);
+    }
+  } else if (!epi) {
+    // ------------------------------------------------------------- gather
+    const int t = tid - 64;                    // token row of the tile
+    pdl_wait();
+    const bool valid = t < ntok;
+    const __nv_bfloat16* xrow = x + static_cast<size_t>(m0 + (valid ? t : 0)) * ldx;
+    for (int w = 0; w < W; ++w) {
+      const int B = B0 + w % nbc, as = w & 1;
+      const int32_t* pB = P.perm + static_cast<size_t>(B) * BS;
+      uint32_t v[BS / 2];
+#pragma unroll
+      for (int i = 0; i < BS; i += 2) {
+        uint32_t lo = 0, hi = 0;
+        if (valid) {
+          const int p0 = __ldg(pB + i), p1 = __ldg(pB + i + 1);
+          lo = __ldg(reinterpret_cast<const unsigned short*>(xrow) + (static_cast<unsigned>(p0) < static_cast<unsigned>(K) ? p0 : 0));
+          hi = __ldg(reinterpret_cast<const unsigned short*>(xrow) + (static_cast<unsigned>(p1) < static_cast<unsigned>(K) ? p1 : 0));
+        }
+        v[i / 2] = lo | (hi << 16);
+      }
+      if (!mbar_wait(&bars.empty_a[as], ((w >> 1) & 1) ^ 1u, err)) break;
+      uint8_t* at = astage + as * C::kAStage;
+#pragma unroll
+      for (int c8 = 0; c8 < BS / 8; ++c8) {
+        const int kc = c8 >> 3, c = c8 & 7;
+        *reinterpret_cast<uint4*>(at + kc * (kTM * 128) + t * 128 + ((c ^ (t & 7)) << 4)) =
+            make_uint4(v[4 * c8], v[4 * c8 + 1], v[4 * c8 + 2], v[4 * c8 + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars.full_a[as]);
+      if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
+        cluster_arrive_relaxed();
+        arrived1 = true;
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int t = q4 * 32 + lane;              // token row = TMEM lane
+    const bool valid = t < ntok;
+    pdl_wait();
+    pdl_launch_dependents();
+    float s = 0.f;
+    if (MODE == kTable) s = table_scale(P.table, P.T, P.Lcount, P.step_dev, P.step_host, P.layer, err);
+    float amax = 0.f;
+    bool reduced = false;
+    // row maximum over every CTA of the cluster that shares these tokens
+    // (once per thread, also when this CTA holds no block or gave up early)
+    auto reduce_rows = [&]() {
+      if (cs > 1) {
+        amax_s[t] = __float_as_uint(amax);
+        asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+        asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+        unsigned int mx = 0u;
+        const uint32_t a = smem_u32(&amax_s[t]);
+        for (int r2 = 0; r2 < cs; ++r2) {
+          uint32_t v;
+          asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                       : "=r"(v)
+                       : "r"(map_shared_rank(a, static_cast<uint32_t>(r2)))
+                       : "memory");
+          mx = max(mx, v);
+        }
+        cluster_arrive_relaxed();          // phase 2: done reading peers
+        amax = __uint_as_float(mx);
+      }
+      s = __fdiv_rn(amax, 7.0f);
+      reduced = true;
+    };
+    for (int w = 0; w < W; ++w) {
+      const int ab = w & 1, pass = w / nbc, B = B0 + w % nbc;
+      if (!mbar_wait(&bars.acc_full[ab], (w >> 1) & 1, err)) break;
+      tc_fence_after();
+      const float rs = quant_recip(s);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BS; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * BS + c0, r);
+        tmem_ld_wait();
+        if (MODE == kRotateOnly) {
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(P.xr_out + static_cast<size_t>(m0 + t) * K + B * BS + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                   __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
+        } else if (MODE == kDynamic && pass == 0) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(__uint_as_float(r[c])));
+        } else {
+          float f[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(r[c]);
+          uint32_t wv[4];
+          quant_pack<32>(f, s, rs, -8, 7, wv);
+          if (valid)
+            *reinterpret_cast<uint4*>(P.xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS + c0) / 2) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.acc_empty[ab]);
+      if (MODE == kDynamic && w == nbc - 1) reduce_rows();
+    }
+    if (MODE == kDynamic && !reduced) reduce_rows();
+    if (MODE != kRotateOnly && group == 0 && valid) P.s_x[m0 + t] = s;
+  }
+
+  if (MODE == kDynamic && cs > 1) {
+    if (!epi) {
+      if (!arrived1) cluster_arrive_relaxed();   // idle lanes, early exits
+      cluster_wait();                            // phase 1
+      cluster_arrive_relaxed();                  // phase 2
+    }
+    cluster_wait();                              // phase 2: peers done with our smem
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Permuted copy of bf16 rows: out[m][j] = x[m][perm[j]].  One CTA per row:
+// the row is staged in shared memory with 16-byte loads and written back in
+// permuted order with 16-byte stores (coalesced both ways).
+struct PermJob {
+  const __nv_bfloat16* x;
+  const int32_t* perm;
+  __nv_bfloat16* out;
+  int ldx, M, K;
+};
+struct PermBatch {
+  int n;
+  int row_start[kMaxBatch + 1];
+  PermJob j[kMaxBatch];
+};
+
+__global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermBatch batch) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  int ji = 0;
+  while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.row_start[ji + 1]) ++ji;
+  const PermJob& J = batch.j[ji];
+  const int row = static_cast<int>(blockIdx.x) - batch.row_start[ji];
+  const int K = J.K;
+  unsigned short* srow = reinterpret_cast<unsigned short*>(smem);
+  pdl_wait();
+  pdl_launch_dependents();
+  const uint4* src = reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(row) * J.ldx);
+  for (int i = threadIdx.x; i < K / 8; i += 256) reinterpret_cast<uint4*>(srow)[i] = __ldg(src + i);
+  __syncthreads();
+  uint4* dst = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(row) * K);
+  for (int i = threadIdx.x; i < K / 8; i += 256) {
+    const int4 p0 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
+    const int4 p1 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
+    const int p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int a = p[2 * q], b = p[2 * q + 1];
+      const uint32_t lo = srow[static_cast<unsigned>(a) < static_cast<unsigned>(K) ? a : 0];
+      const uint32_t hi = srow[static_cast<unsigned>(b) < static_cast<unsigned>(K) ? b : 0];
+      w[q] = lo | (hi << 16);
+    }
+    dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // Quantise fp32 rows (already rotated): one CTA per row.
@@ -400,10 +818,11 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   const float s = s_sh;
+  const float rs = quant_recip(s);
   uint8_t* dst = q_out + static_cast<size_t>(row) * (K / 2);
   for (int j = tid; j < K / 2; j += kThreads) {
-    const int q0 = quant_code(src[2 * j], s, qmin, qmax);
-    const int q1 = quant_code(src[2 * j + 1], s, qmin, qmax);
+    const int q0 = quant_code_fast(src[2 * j], s, rs, qmin, qmax);
+    const int q1 = quant_code_fast(src[2 * j + 1], s, rs, qmin, qmax);
     dst[j] = static_cast<uint8_t>((q0 & 15) | ((q1 & 15) << 4));
   }
   if (tid == 0) s_out[row] = s;
@@ -574,6 +993,238 @@ cudaError_t launch_mode(const std::vector<const ActArgs*>& v, cudaStream_t strea
   return cudaSuccess;
 }
 
+// ---------------------------------------------------------------- TC host
+template <int BS>
+int tc_ctas_per_sm() { return TcCfg<BS>::kSmem <= 110 * 1024 ? 2 : 1; }
+
+template <int BS>
+int tc_cluster(int M, int K) {
+  const int gx = (M + kTM - 1) / kTM, nb = K / BS;
+  const int slots = 148 * tc_ctas_per_sm<BS>();
+  int cs = 1;
+  while (cs < 16 && 2 * cs <= nb && gx * cs < slots) cs *= 2;
+  return cs;
+}
+
+// One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
+// mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
+bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
+  static EncodeTiledFnR enc = nullptr;
+  if (!enc) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    enc = reinterpret_cast<EncodeTiledFnR>(p);
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTM)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Permuted copies x_perm = x[:, perm] of the problems that have scratch.
+cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+    PermBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.n = n;
+    int rows = 0, kmax = 0;
+    for (int i = 0; i < n; ++i) {
+      const ActArgs& a = *v[i0 + i];
+      b.j[i].x = static_cast<const __nv_bfloat16*>(a.x);
+      b.j[i].perm = a.perm;
+      b.j[i].out = static_cast<__nv_bfloat16*>(a.ws);
+      b.j[i].ldx = a.ldx;
+      b.j[i].M = a.M;
+      b.j[i].K = a.K;
+      b.row_start[i] = rows;
+      rows += a.M;
+      kmax = std::max(kmax, a.K);
+    }
+    b.row_start[n] = rows;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           QVLA_MAX_K * 2);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(kmax) * 2;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, permute_rows_kernel, b);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
+template <int BS, int MODE, bool kTmaA>
+cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cudaStream_t stream) {
+  using C = TcCfg<BS>;
+  ActBatch batch;
+  std::memset(&batch, 0, sizeof(batch));
+  batch.n = n;
+  int ctas = 0;
+  for (int i = 0; i < n; ++i) {
+    const ActArgs& a = *as[i];
+    ActProblem& P = batch.p[i];
+    if (kTmaA && !make_xperm_map(&P.txp, a.ws, a.M, a.K)) return cudaErrorInvalidValue;
+    P.x = a.x;
+    P.perm = a.perm;
+    P.rot = a.rot;
+    P.rot_tc = a.rot_tc;
+    P.table = a.table;
+    P.step_dev = a.step_dev;
+    P.xq = a.xq;
+    P.s_x = a.s_x;
+    P.xr_out = a.xr_out;
+    P.M = a.M;
+    P.ldx = a.ldx;
+    P.K = a.K;
+    P.T = a.T;
+    P.Lcount = a.Lcount;
+    P.step_host = a.step_host;
+    P.layer = a.layer;
+    const int nb = a.K / BS;
+    P.gx = (a.M + kTM - 1) / kTM;
+    batch.cta_start[i] = ctas;
+    if (MODE == kDynamic) {
+      P.bpc = (nb + cs - 1) / cs;
+      ctas += P.gx;
+    } else {
+      P.bpc = std::min(G, nb);
+      ctas += P.gx * ((nb + P.bpc - 1) / P.bpc);
+    }
+  }
+  batch.cta_start[n] = ctas;
+  auto kern = rotq_tc_kernel<BS, MODE, kTmaA>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (MODE == kDynamic && cs > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = cs;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, batch, device_error_word());
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int BS, int MODE, bool kTmaA>
+cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  if (v.empty()) return cudaSuccess;
+  if (MODE == kDynamic) {
+    for (int cs = 1; cs <= 16; cs *= 2) {
+      std::vector<const ActArgs*> g;
+      for (const ActArgs* a : v)
+        if (tc_cluster<BS>(a->M, a->K) == cs) g.push_back(a);
+      for (size_t i0 = 0; i0 < g.size(); i0 += kMaxBatch) {
+        const int n = static_cast<int>(std::min<size_t>(kMaxBatch, g.size() - i0));
+        cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(g.data() + i0, n, 1, cs, stream);
+        if (e != cudaSuccess) return e;
+      }
+    }
+    return cudaSuccess;
+  }
+  // blocks per CTA: spread the batch's (token tile, block) pairs over one wave
+  long long pairs = 0;
+  for (const ActArgs* a : v) pairs += static_cast<long long>((a->M + kTM - 1) / kTM) * (a->K / BS);
+  const long long slots = 148LL * tc_ctas_per_sm<BS>();
+  const int G = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
+  for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+    cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, G, 1, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+bool tc_path_forced_off() {
+  const char* p = std::getenv("QVLA_ROTATE_PATH");
+  return p && std::strcmp(p, "fma") == 0;
+}
+
+// Token count from which the tensor-core rotation beats the CUDA-core one.
+constexpr int kTcMinM = 65;
+
+bool has_perm_scratch(const ActArgs* a) {
+  return a->ws != nullptr && a->ws_bytes >= static_cast<size_t>(a->M) * a->K * 2 &&
+         (reinterpret_cast<uintptr_t>(a->ws) & 15u) == 0;
+}
+
+// bf16 problems with a tensor-core image, block 64 / 128 and more than 64
+// tokens go to the tensor cores (through a permuted copy when the call gave
+// scratch for it, else gathering); returns the rest.
+cudaError_t launch_tc_subset(std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  if (tc_path_forced_off()) return cudaSuccess;
+  std::vector<const ActArgs*> rest, perm, g[2][3], t[2][3];
+  for (const ActArgs* a : v) {
+    if (a->rot_tc == nullptr || (a->block != 64 && a->block != 128) || a->M < kTcMinM) {
+      rest.push_back(a);
+      continue;
+    }
+    const int mode = a->xq == nullptr ? kRotateOnly : a->dynamic ? kDynamic : kTable;
+    const int bi = a->block == 64 ? 0 : 1;
+    if (has_perm_scratch(a)) {
+      perm.push_back(a);
+      t[bi][mode].push_back(a);
+    } else {
+      g[bi][mode].push_back(a);
+    }
+  }
+  cudaError_t e = launch_permute(perm, stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kTable, true>(t[0][kTable], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kDynamic, true>(t[0][kDynamic], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kRotateOnly, true>(t[0][kRotateOnly], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kTable, true>(t[1][kTable], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kDynamic, true>(t[1][kDynamic], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kRotateOnly, true>(t[1][kRotateOnly], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kTable, false>(g[0][kTable], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kDynamic, false>(g[0][kDynamic], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<64, kRotateOnly, false>(g[0][kRotateOnly], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kTable, false>(g[1][kTable], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kDynamic, false>(g[1][kDynamic], stream);
+  if (e == cudaSuccess) e = launch_tc_mode<128, kRotateOnly, false>(g[1][kRotateOnly], stream);
+  v.swap(rest);
+  return e;
+}
+
 template <typename Tin>
 cudaError_t launch_dtype(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   std::vector<const ActArgs*> rot, dyn, tab;
@@ -591,8 +1242,8 @@ cudaError_t launch_rotate_quant_batch(const ActArgs* as, int n, cudaStream_t str
   std::vector<const ActArgs*> bf, f32;
   for (int i = 0; i < n; ++i)
     if (as[i].M > 0) (as[i].xdt == QVLA_DTYPE_BF16 ? bf : f32).push_back(&as[i]);
-  cudaError_t e = cudaSuccess;
-  if (!bf.empty()) e = launch_dtype<__nv_bfloat16>(bf, stream);
+  cudaError_t e = launch_tc_subset(bf, stream);     // leaves the rest in bf
+  if (e == cudaSuccess && !bf.empty()) e = launch_dtype<__nv_bfloat16>(bf, stream);
   if (e == cudaSuccess && !f32.empty()) e = launch_dtype<float>(f32, stream);
   return e;
 }

@@ -49,12 +49,13 @@ EXPORTED = (
     "qvla_pack_weights", "qvla_rotate_weights_f32", "qvla_quant_pack_weights_f32",
     "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
     "qvla_w4a4_gemm_s32", "qvla_rotate_quant_act_batched", "qvla_w4a4_gemm_batched",
+    "qvla_rotate_quant_workspace_bytes",
 )
 
 
 class qvla_packed_linear(ctypes.Structure):
     _fields_ = [("N", c_int32), ("K", c_int32), ("block", c_int32),
-                ("perm", c_void_p), ("rot", c_void_p), ("wq", c_void_p),
+                ("perm", c_void_p), ("rot", c_void_p), ("rot_tc", c_void_p), ("wq", c_void_p),
                 ("w_scale", c_void_p), ("bias", c_void_p)]
 
 
@@ -63,7 +64,8 @@ class qvla_linear_problem(ctypes.Structure):
                 ("M", c_int32), ("ldx", c_int32), ("mode", c_int32), ("table", c_void_p),
                 ("T", c_int32), ("Lcount", c_int32), ("step_dev", c_void_p),
                 ("step_host", c_int32), ("layer", c_int32), ("xq", c_void_p), ("s_x", c_void_p),
-                ("y", c_void_p), ("ldy", c_int32)]
+                ("y", c_void_p), ("ldy", c_int32), ("workspace", c_void_p),
+                ("ws_bytes", c_size_t)]
 
 
 _P = POINTER(qvla_packed_linear)
@@ -73,16 +75,18 @@ _sig = {
     "qvla_abi_version": (c_int, []),
     "qvla_read_error_word": (c_int, [POINTER(c_uint32), c_int]),
     "qvla_packed_sizes": (c_int, [c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t),
-                                  POINTER(c_size_t)]),
+                                  POINTER(c_size_t), POINTER(c_size_t)]),
     "qvla_pack_weights": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
-                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                  c_void_p]),
     "qvla_rotate_weights_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
     "qvla_quant_pack_weights_f32": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p,
                                             c_void_p]),
     "qvla_rotate_quant_act": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_int, c_void_p, c_int,
                                       c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
-                                      c_void_p]),
+                                      c_void_p, c_size_t, c_void_p]),
+    "qvla_rotate_quant_workspace_bytes": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
     "qvla_rotate_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_void_p, c_void_p]),
     "qvla_quant_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_int,
                                    c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
@@ -134,20 +138,23 @@ def qvla_read_error_word(clear: bool = True) -> int:
     return int(v.value)
 
 
-def qvla_packed_sizes(N: int, K: int, block: int) -> Tuple[int, int, int]:
-    a, b, c = c_size_t(), c_size_t(), c_size_t()
-    _check(_lib.qvla_packed_sizes(N, K, block, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
-           "qvla_packed_sizes")
-    return a.value, b.value, c.value
+def qvla_packed_sizes(N: int, K: int, block: int) -> Tuple[int, int, int, int]:
+    """(wq_bytes, rot_bytes, rot_tc_bytes, workspace_bytes)."""
+    a, b, t, c = c_size_t(), c_size_t(), c_size_t(), c_size_t()
+    _check(_lib.qvla_packed_sizes(N, K, block, ctypes.byref(a), ctypes.byref(b), ctypes.byref(t),
+                                  ctypes.byref(c)), "qvla_packed_sizes")
+    return a.value, b.value, t.value, c.value
 
 
 class PackedLinear:
     """Device buffers of one packed linear plus the C struct that points at them."""
 
-    def __init__(self, N, K, block, perm, rot, wq, w_scale, bias=None):
+    def __init__(self, N, K, block, perm, rot, wq, w_scale, bias=None, rot_tc=None):
         self.N, self.K, self.block = int(N), int(K), int(block)
         self.perm, self.rot, self.wq, self.w_scale, self.bias = perm, rot, wq, w_scale, bias
+        self.rot_tc = rot_tc
         self._s = qvla_packed_linear(self.N, self.K, self.block, perm.data_ptr(), rot.data_ptr(),
+                                     rot_tc.data_ptr() if rot_tc is not None else None,
                                      wq.data_ptr(), w_scale.data_ptr(),
                                      bias.data_ptr() if bias is not None else None)
 
@@ -157,6 +164,7 @@ class PackedLinear:
 
     def device_bytes(self) -> int:
         n = sum(t.numel() * t.element_size() for t in (self.perm, self.rot, self.wq, self.w_scale))
+        n += self.rot_tc.numel() * 2 if self.rot_tc is not None else 0
         return n + (self.bias.numel() * 4 if self.bias is not None else 0)
 
 
@@ -166,10 +174,11 @@ def qvla_pack_weights(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] 
     """W: cuda fp32 [N, K].  perm_in: host int32 [K]; rsvd_in: host float64 [nb, b, b]."""
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
     N, K = W.shape
-    wq_b, rot_b, ws_b = qvla_packed_sizes(N, K, block)
+    wq_b, rot_b, tc_b, ws_b = qvla_packed_sizes(N, K, block)
     dev = W.device
     perm = torch.empty(K, dtype=torch.int32, device=dev)
     rot = torch.empty(rot_b // 4, dtype=torch.float32, device=dev)
+    rot_tc = torch.empty(tc_b // 2, dtype=torch.int16, device=dev) if tc_b else None
     wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
     s_w = torch.empty(N, dtype=torch.float32, device=dev)
     ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
@@ -183,12 +192,13 @@ def qvla_pack_weights(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] 
         assert rsvd_in.shape == (K // block, block, block)
         r_in = rsvd_in.ctypes.data_as(c_void_p)
     _check(_lib.qvla_pack_weights(_ptr(W), N, K, block, p_in, r_in, _ptr(perm), _ptr(rot),
-                                  _ptr(wq), _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
-           "qvla_pack_weights")
+                                  _ptr(rot_tc), _ptr(wq), _ptr(s_w), _ptr(ws), ws_b,
+                                  _stream(stream)), "qvla_pack_weights")
     if bias is not None:
         assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
         bias = bias.contiguous()
-    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias)
+    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias,
+                        rot_tc=rot_tc)
 
 
 def qvla_rotate_weights_f32(W: torch.Tensor, block: int, perm: torch.Tensor,
@@ -227,10 +237,19 @@ def _step_args(step):
     return None, int(step)
 
 
+def qvla_rotate_quant_workspace_bytes(M: int, K: int, block: int, dtype=torch.bfloat16) -> int:
+    b = c_size_t()
+    code = QVLA_DTYPE_BF16 if dtype == torch.bfloat16 else QVLA_DTYPE_F32
+    _check(_lib.qvla_rotate_quant_workspace_bytes(M, K, block, code, ctypes.byref(b)),
+           "qvla_rotate_quant_workspace_bytes")
+    return b.value
+
+
 def qvla_rotate_quant_act(x: torch.Tensor, L: PackedLinear, mode: int = QVLA_SCALE_DYNAMIC,
                           table: Optional[torch.Tensor] = None, step=None, layer: int = 0,
                           xq: Optional[torch.Tensor] = None, s_x: Optional[torch.Tensor] = None,
-                          stream=None):
+                          workspace: Optional[torch.Tensor] = None, stream=None):
+    """workspace: optional uint8 device scratch of qvla_rotate_quant_workspace_bytes() bytes."""
     M = x.shape[0]
     if xq is None:
         xq = torch.empty(M, L.K // 2, dtype=torch.uint8, device=x.device)
@@ -238,9 +257,11 @@ def qvla_rotate_quant_act(x: torch.Tensor, L: PackedLinear, mode: int = QVLA_SCA
         s_x = torch.empty(M, dtype=torch.float32, device=x.device)
     T, Lc = (table.shape if table is not None else (0, 0))
     sd, sh = _step_args(step)
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_lib.qvla_rotate_quant_act(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct, mode,
                                       _ptr(table), T, Lc, sd, sh, layer, _ptr(xq), _ptr(s_x),
-                                      _stream(stream)), "qvla_rotate_quant_act")
+                                      _ptr(workspace), ws_n, _stream(stream)),
+           "qvla_rotate_quant_act")
     return xq, s_x
 
 
@@ -301,7 +322,8 @@ class LinearProblem:
     def __init__(self, L: PackedLinear, x: Optional[torch.Tensor] = None,
                  mode: int = QVLA_SCALE_DYNAMIC, table: Optional[torch.Tensor] = None,
                  step=None, layer: int = 0, xq: Optional[torch.Tensor] = None,
-                 s_x: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None):
+                 s_x: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None):
         M = x.shape[0] if x is not None else xq.shape[0]
         dev = (x if x is not None else xq).device
         self.L, self.x, self.table, self.step = L, x, table, step
@@ -316,7 +338,10 @@ class LinearProblem:
             x.stride(0) if x is not None else L.K, mode,
             table.data_ptr() if table is not None else None, T, Lc,
             sd.value if sd is not None else None, sh, layer, self.xq.data_ptr(),
-            self.s_x.data_ptr(), self.y.data_ptr(), self.y.stride(0))
+            self.s_x.data_ptr(), self.y.data_ptr(), self.y.stride(0),
+            workspace.data_ptr() if workspace is not None else None,
+            workspace.numel() * workspace.element_size() if workspace is not None else 0)
+        self.workspace = workspace
 
 
 def _problem_array(problems):
