@@ -203,6 +203,31 @@ qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
 qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtype xdt,
                                               size_t* bytes);
 
+/* qvla_rotate_quant_act without any allocation by the caller or the library.
+ * (No counterpart in the paper: this is a deployment convenience.)
+ * For callers that cannot allocate device memory when they run a layer --
+ * an inference loop that must not call cudaMalloc once it is running (a
+ * robot control loop with a hard cycle budget, code that is being captured
+ * into a CUDA graph, a host application that hands out no allocator) -- the
+ * scratch the fast large-M route needs (qvla_rotate_quant_workspace_bytes)
+ * lives in a fixed array inside the library, QVLA_NOALLOC_SCRATCH_BYTES bytes
+ * per device, kept for as long as the library is loaded.  Arguments and
+ * results are those of qvla_rotate_quant_act.
+ *  - A call whose scratch need exceeds QVLA_NOALLOC_SCRATCH_BYTES returns
+ *    QVLA_ERR_WORKSPACE and does nothing.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array: calls that may run at the
+ *    same time on the GPU (different streams, no ordering) race on it.  The
+ *    array keeps the last call's contents; nothing in it needs to start at
+ *    zero (each call writes every byte it later reads).                    */
+#define QVLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+qvla_status qvla_rotate_quant_act_noalloc(const void* x, qvla_dtype xdt, int M, int ldx,
+                                          const qvla_packed_linear* L, qvla_scale_mode mode,
+                                          const float* table, int T, int Lcount,
+                                          const int32_t* step_dev, int step_host, int layer,
+                                          uint8_t* xq, float* s_x, cudaStream_t stream);
+
 /* The rotation alone, for parity checks: xr_out device fp32 [M][K] = the
  * same fp32 x' the fused kernel quantises.                                  */
 qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,

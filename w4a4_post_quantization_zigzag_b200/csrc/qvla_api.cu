@@ -425,6 +425,61 @@ qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtyp
   return QVLA_OK;
 }
 
+}  // extern "C"
+
+// Scratch of qvla_rotate_quant_act_noalloc, for callers that cannot allocate
+// device memory while they run: a fixed array in the library's module, one per
+// device that loads it, held until the process exits.  Host code must not pass
+// the symbol itself to a kernel (in host code it is only a stand-in for the
+// device array); the entry point looks up its device address per device.
+static __device__ __align__(256) unsigned char g_qvla_noalloc_scratch[QVLA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the scratch array for the current device, looked up once
+// per device with that device current.
+qvla_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QVLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_qvla_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return QVLA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return QVLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qvla_status qvla_rotate_quant_act_noalloc(const void* x, qvla_dtype xdt, int M, int ldx,
+                                          const qvla_packed_linear* L, qvla_scale_mode mode,
+                                          const float* table, int T, int Lcount,
+                                          const int32_t* step_dev, int step_host, int layer,
+                                          uint8_t* xq, float* s_x, cudaStream_t stream) {
+  ActArgs a;
+  qvla_status st = prepare_act(x, xdt, M, ldx, L, mode, table, T, Lcount, step_dev, step_host,
+                               layer, xq, s_x, &a);
+  if (st != QVLA_OK || M == 0) return st;
+  size_t need = 0;
+  if ((st = qvla_rotate_quant_workspace_bytes(M, L->K, L->block, xdt, &need)) != QVLA_OK)
+    return st;
+  if (need > QVLA_NOALLOC_SCRATCH_BYTES) return QVLA_ERR_WORKSPACE;
+  if (need > 0) {
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != QVLA_OK) return st;
+    a.ws = scratch;
+    a.ws_bytes = QVLA_NOALLOC_SCRATCH_BYTES;
+  }
+  return cuda_status(launch_rotate_quant(a, stream));
+}
+
 qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int n,
                                           cudaStream_t stream) {
   if (n < 0 || (n > 0 && !probs)) return QVLA_ERR_ARG;

@@ -49,8 +49,10 @@ EXPORTED = (
     "qvla_pack_weights", "qvla_rotate_weights_f32", "qvla_quant_pack_weights_f32",
     "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
     "qvla_w4a4_gemm_s32", "qvla_rotate_quant_act_batched", "qvla_w4a4_gemm_batched",
-    "qvla_rotate_quant_workspace_bytes",
+    "qvla_rotate_quant_workspace_bytes", "qvla_rotate_quant_act_noalloc",
 )
+
+QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class qvla_packed_linear(ctypes.Structure):
@@ -87,6 +89,9 @@ _sig = {
                                       c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
     "qvla_rotate_quant_workspace_bytes": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
+    "qvla_rotate_quant_act_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_int, c_void_p,
+                                              c_int, c_int, c_void_p, c_int, c_int, c_void_p,
+                                              c_void_p, c_void_p]),
     "qvla_rotate_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_void_p, c_void_p]),
     "qvla_quant_act_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_int,
                                    c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
@@ -262,6 +267,24 @@ def qvla_rotate_quant_act(x: torch.Tensor, L: PackedLinear, mode: int = QVLA_SCA
                                       _ptr(table), T, Lc, sd, sh, layer, _ptr(xq), _ptr(s_x),
                                       _ptr(workspace), ws_n, _stream(stream)),
            "qvla_rotate_quant_act")
+    return xq, s_x
+
+
+def qvla_rotate_quant_act_noalloc(x: torch.Tensor, L: PackedLinear, xq: torch.Tensor,
+                                  s_x: torch.Tensor, mode: int = QVLA_SCALE_DYNAMIC,
+                                  table: Optional[torch.Tensor] = None, step=None,
+                                  layer: int = 0, stream=None):
+    """qvla_rotate_quant_act for callers that cannot allocate device memory:
+    the outputs are given, and the scratch is the library's fixed per-device
+    array (at most QVLA_NOALLOC_SCRATCH_BYTES).  Calls that may overlap on the
+    GPU race on that array."""
+    M = x.shape[0]
+    T, Lc = (table.shape if table is not None else (0, 0))
+    sd, sh = _step_args(step)
+    _check(_lib.qvla_rotate_quant_act_noalloc(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct,
+                                              mode, _ptr(table), T, Lc, sd, sh, layer, _ptr(xq),
+                                              _ptr(s_x), _stream(stream)),
+           "qvla_rotate_quant_act_noalloc")
     return xq, s_x
 
 
