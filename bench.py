@@ -65,6 +65,19 @@ def make_workload(name):
             "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
 
 
+def kernel_nodes(raw_graph):
+    """Kernel nodes of a captured CUDA graph (every one a launch of this library)."""
+    from cuda.bindings import runtime as rt
+    if isinstance(raw_graph, int):
+        raw_graph = rt.cudaGraph_t(init_value=raw_graph)
+    err, _, n = rt.cudaGraphGetNodes(raw_graph)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    err, nodes, n = rt.cudaGraphGetNodes(raw_graph, n)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+    return sum(k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel for k in kinds)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -274,11 +287,15 @@ def run_ours(args):
     xq = [torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev) for l in wl.linears]
     sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
     ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
+    # scratch of the tensor-core rotation route (more than 64 bf16 tokens), one
+    # per linear since a batched launch runs them together
+    wss = [torch.empty(max(Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
+                       dtype=torch.uint8, device=dev) for l in wl.linears]
     nl = len(wl.linears)
     # one problem set per denoising step: same packed weights and buffers, the
     # step's own inputs and device step index
     probs = [[Q.LinearProblem(L, xs[t][i], mode, table=table, step=steps_dev[t:t + 1],
-                              layer=lin.layer, xq=xq[i], s_x=sx[i], y=ys[i])
+                              layer=lin.layer, xq=xq[i], s_x=sx[i], y=ys[i], workspace=wss[i])
               for i, (lin, L) in enumerate(zip(wl.linears, packs))] for t in range(T)]
 
     def step_batched(t, rec=None):
@@ -294,27 +311,30 @@ def run_ours(args):
     def step_per_linear(t):
         for i, (lin, L) in enumerate(zip(wl.linears, packs)):
             Q.qvla_rotate_quant_act(xs[t][i], L, mode, table=table, step=steps_dev[t:t + 1],
-                                    layer=lin.layer, xq=xq[i], s_x=sx[i])
+                                    layer=lin.layer, xq=xq[i], s_x=sx[i], workspace=wss[i])
             Q.qvla_w4a4_gemm(xq[i], sx[i], L, y=ys[i])
 
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def capture(fn):
-        gs = []
+        """One graph per denoising step; also returns the kernel nodes in each."""
+        gs, nk = [], []
         for t in range(T):
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g, stream=stream):
                 fn(t)
+            nk.append(kernel_nodes(g.raw_cuda_graph()))
+            g.instantiate()
             gs.append(g)
-        return gs
+        return gs, nk
 
     with torch.cuda.stream(stream):
         step_batched(0)               # first calls resolve attributes outside capture
         step_per_linear(0)
         torch.cuda.synchronize()
-        graphs = capture(step_batched)
-        graphs_pl = capture(step_per_linear)
+        graphs, kernels_per_step = capture(step_batched)
+        graphs_pl, _ = capture(step_per_linear)
     torch.cuda.synchronize()
     assert Q.qvla_read_error_word(clear=True) == 0
 
@@ -436,7 +456,8 @@ def run_ours(args):
         "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3},
         "per_linear_launches_us_per_step": per_linear_us,
         "pack_s": pack_s,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": sum(kernels_per_step[i % T] for i in range(args.steps)),
+        "kernels_per_step": kernels_per_step[0],
         "e2e": e2e,
     }
     if sampler:
