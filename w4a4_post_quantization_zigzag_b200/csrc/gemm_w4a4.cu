@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(tmap_x);
   }
   if (warp == 1) {
+    __syncwarp();                  // tcgen05 alloc/ld/st/dealloc are warp-wide
     tmem_alloc(&bars.tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
@@ -296,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------- epilogue
-    const bool have = ok && mbar_wait(&bars.acc_full, 0, err);
+    // one outcome per warp, and a converged warp for the warp-wide loads
+    const bool have = __all_sync(0xffffffffu, ok && mbar_wait(&bars.acc_full, 0, err));
     tc_fence_after();
     pdl_launch_dependents();
     if (have) {
@@ -348,7 +351,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (S == 1 && acc_out == nullptr) {
         fence_proxy_async_smem();
         named_barrier(1, kWorkers);
-        if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0, m0);
+        if (n0 + kBM <= N || (N & 7) == 0) {
+          if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0, m0);
+        } else {
+          // a tile cut by N with N % 8 != 0: plain stores, not a TMA box
+          // reaching past N
+          for (int e = wt; e < NT * kBM; e += kWorkers) {
+            const int c = e / kBM, nx = e % kBM;
+            if (n0 + nx < N && m0 + c < M)
+              y[static_cast<size_t>(m0 + c) * ldy + n0 + nx] = otile[c * kBM + nx];
+          }
+        }
       }
     }
     tc_fence_before();
@@ -386,12 +399,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (acc_out == nullptr) {
         fence_proxy_async_smem();
         named_barrier(1, kWorkers);
-        if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0 + static_cast<int>(rank) * rpr, m0);
+        const int nr = n0 + static_cast<int>(rank) * rpr;
+        if (nr + rpr <= N || (N & 7) == 0) {
+          if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, nr, m0);
+        } else {
+          for (int e = wt; e < NT * rpr; e += kWorkers) {
+            const int c = e / rpr, nx = e % rpr;
+            if (nr + nx < N && m0 + c < M)
+              y[static_cast<size_t>(m0 + c) * ldy + nr + nx] = otile[c * rpr + nx];
+          }
+        }
       }
     }
   }
 
   if (warp == 1) {
+    __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
     tmem_dealloc(tmem_d, C::kTmemCols);
   }
@@ -566,6 +589,20 @@ cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cud
 
 }  // namespace
 
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
+                   uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int gemm_choose_split(int M, int N, int K) {
   const int nt = token_tile(M);
   if (nt == 256) return 1;
@@ -576,15 +613,32 @@ int gemm_choose_split(int M, int N, int K) {
   return S;
 }
 
+// QVLA_GEMM_PATH=rows sends the automatic-split linears of up to 64 tokens
+// to the persistent row-split kernel (gemm_w4a4_rows.cu); by default they
+// stay on the one-tile-per-CTA kernel with cluster split-K, which measures
+// faster on the DiT action-head shapes (a row-split tile pays its per-K-tile
+// overheads once per part).
+bool rows_path_selected() {
+  const char* p = std::getenv("QVLA_GEMM_PATH");
+  return p && std::strcmp(p, "rows") == 0;
+}
+
 cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream) {
-  // group by token tile (a template parameter of the kernel)
+  // group by token tile (a template parameter of the kernel); up to 64 tokens
+  // the persistent row-split kernel serves the automatic split choice
   static const int kTiles[5] = {16, 32, 64, 128, 256};
+  const bool rows = split_k == 0 && rows_path_selected();
   for (int t : kTiles) {
     std::vector<const GemmArgs*> grp;
     for (int i = 0; i < n; ++i)
       if (gs[i].M > 0 && token_tile(gs[i].M) == t) grp.push_back(&gs[i]);
     if (grp.empty()) continue;
     cudaError_t e;
+    if (rows && t <= 64) {
+      e = launch_w4a4_gemm_rows(grp.data(), static_cast<int>(grp.size()), t, stream);
+      if (e != cudaSuccess) return e;
+      continue;
+    }
     switch (t) {
       case 16: e = launch_nt_batches<16>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
       case 32: e = launch_nt_batches<32>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;

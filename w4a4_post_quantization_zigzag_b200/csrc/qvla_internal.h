@@ -2,6 +2,7 @@
 // translation units.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -76,6 +77,15 @@ struct GemmArgs {
   int split_k;
 };
 cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream);
+// persistent small-M GEMM (gemm_w4a4_rows.cu): M <= 64, no split-K;
+// `nt` is the token tile (16, 32 or 64) shared by every problem of the launch
+cudaError_t launch_w4a4_gemm_rows(const GemmArgs* const* gs, int n, int nt, cudaStream_t stream);
+
+// 2-D tiled tensor map over a row-major array (`inner` elements per row,
+// `outer` rows, row pitch `pitch` bytes), box `box_inner` x `box_outer`.
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
+                   uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle);
 // independent linears in as few launches as possible (grouped by token tile)
 cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream);
 int gemm_choose_split(int M, int N, int K);

@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    __syncwarp();                  // tcgen05 alloc/ld/dealloc are warp-wide
     tmem_alloc(&bars.tmem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -692,7 +693,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     for (int w = 0; w < W; ++w) {
       const int ab = w & 1, pass = w / nbc, B = B0 + w % nbc;
-      if (!mbar_wait(&bars.acc_full[ab], (w >> 1) & 1, err)) break;
+      // one outcome per warp, and a converged warp for the warp-wide loads
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.acc_full[ab], (w >> 1) & 1, err))) break;
       tc_fence_after();
       const float rs = quant_recip(s);
 #pragma unroll 1
@@ -740,6 +742,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
