@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem_d = bars.tmem_base;
   // split-K: announce that this CTA runs; remote shared-memory stores wait for
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
 
-  __syncthreads();
+  cta_sync();
 
   if (S > 1) {
     // ------------------------------------------- cluster split-K reduction
@@ -577,6 +577,9 @@ int choose_splits(const GemmArgs* const* gs, int n, int split_k, int* splits) {
 
 template <int NT>
 cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cudaStream_t stream) {
+  // (Giving the deepest linears of a batch a launch of their own, with their
+  // own split-K factor, balances the K walk per CTA but measured slower on
+  // the DiT shapes: each extra launch costs more than the imbalance.)
   for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
     const int m = std::min(kMaxBatch, n - i0);
     int splits[kMaxBatch];

@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
 
-  __syncthreads();
+  cta_sync();
   if (warp == 1) {
     __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();

@@ -175,8 +175,18 @@ QVLA_DEVICE void bulk_wait_read0() {
 QVLA_DEVICE void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Barrier over `count` threads (a multiple of 32) on hardware barrier `id`.
+// The non-aligned form: a warp may arrive diverged (after a branch taken by
+// one lane, or after per-lane waits that end in different iterations).
 QVLA_DEVICE void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Block-wide barrier after code where a warp may have diverged (one-lane
+// roles such as the TMA producer or the MMA issuer): the warp reconverges
+// first, so that it arrives at the barrier as a whole.
+QVLA_DEVICE void cta_sync() {
+  __syncwarp();
+  __syncthreads();
 }
 
 // Barrier over `count` threads on hardware barrier `id` that also returns
@@ -185,7 +195,7 @@ QVLA_DEVICE bool named_barrier_all(int id, int count, bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "barrier.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(count)
       : "memory");

@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kThreads)
   float s_tab = 0.f;
   if (MODE == kTable)
     s_tab = table_scale(P.table, P.T, P.Lcount, P.step_dev, P.step_host, P.layer, err);
-  __syncthreads();   // perm_s visible
+  cta_sync();   // perm_s visible
 
   const int jp = tid % G::NJP, tg = tid / G::NJP;
   for (int bl = 0; bl < nbc; ++bl) {
@@ -341,27 +341,44 @@ __global__ void __launch_bounds__(kThreads)
       } else {
         cp_async_wait<0>();
       }
-      __syncthreads();
+      cta_sync();
       const float* Rc = rbuf + (g & 1) * G::kChunkFloats;
 #pragma unroll 4
       for (int ii = 0; ii < G::RCH; ++ii) {
         const float2 r = *reinterpret_cast<const float2*>(Rc + ii * BS + 2 * jp);
         const float* xrow = xg + (ch * G::RCH + ii) * TT + tg * TPT;
+        // the thread's TPT tokens in as few (warp-broadcast) loads as possible
+        float xv[TPT];
+        if constexpr (TPT % 4 == 0) {
+#pragma unroll
+          for (int u = 0; u < TPT; u += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(xrow + u);
+            xv[u] = q.x; xv[u + 1] = q.y; xv[u + 2] = q.z; xv[u + 3] = q.w;
+          }
+        } else if constexpr (TPT % 2 == 0) {
+#pragma unroll
+          for (int u = 0; u < TPT; u += 2) {
+            const float2 q = *reinterpret_cast<const float2*>(xrow + u);
+            xv[u] = q.x; xv[u + 1] = q.y;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < TPT; ++u) xv[u] = xrow[u];
+        }
 #pragma unroll
         for (int u = 0; u < TPT; ++u) {
-          const float xv = xrow[u];
-          acc[u][0] = fmaf(r.x, xv, acc[u][0]);
-          acc[u][1] = fmaf(r.y, xv, acc[u][1]);
+          acc[u][0] = fmaf(r.x, xv[u], acc[u][0]);
+          acc[u][1] = fmaf(r.y, xv[u], acc[u][1]);
         }
       }
-      __syncthreads();   // chunk buffer (g & 1) may be refilled next
+      cta_sync();   // chunk buffer (g & 1) may be refilled next
     }
     // 3. stage the products token-major (over the gather buffer)
 #pragma unroll
     for (int u = 0; u < TPT; ++u)
       *reinterpret_cast<float2*>(xg + (tg * TPT + u) * BS + 2 * jp) =
           make_float2(acc[u][0], acc[u][1]);
-    __syncthreads();
+    cta_sync();
     // 4. Hadamard factor per token, then quantise / keep / store
     for (int t = warp; t < ntok; t += kWarps) {
       float v[C];
@@ -390,7 +407,7 @@ __global__ void __launch_bounds__(kThreads)
         if (lane == 0) atomicMax(&amax_s[t], __float_as_uint(mx));
       }
     }
-    __syncthreads();   // gather buffer reused by the next block
+    cta_sync();   // gather buffer reused by the next block
   }
 
   if (MODE == kTable) {
@@ -420,7 +437,7 @@ __global__ void __launch_bounds__(kThreads)
   } else if (tid < TT) {
     scale_s[tid] = __fdiv_rn(__uint_as_float(amax_s[tid]), 7.0f);
   }
-  __syncthreads();
+  cta_sync();
   if (blockIdx.y == 0 && tid < ntok) s_x[m0 + tid] = scale_s[tid];
   const int nch = nbc * BS;                    // channels held by this CTA (multiple of 32)
   for (int t = warp; t < ntok; t += kWarps) {
@@ -537,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem = bars.tmem;
   const bool epi = warp >= 6;
@@ -740,7 +757,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     cluster_wait();                              // phase 2: peers done with our smem
   }
-  __syncthreads();
+  cta_sync();
   if (warp == 1) {
     __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
@@ -775,7 +792,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant
   pdl_launch_dependents();
   const uint4* src = reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(row) * J.ldx);
   for (int i = threadIdx.x; i < K / 8; i += 256) reinterpret_cast<uint4*>(srow)[i] = __ldg(src + i);
-  __syncthreads();
+  cta_sync();
   uint4* dst = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(row) * K);
   for (int i = threadIdx.x; i < K / 8; i += 256) {
     const int4 p0 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
@@ -810,7 +827,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if ((tid & 31) == 0) red[tid >> 5] = mx;
-    __syncthreads();
+    cta_sync();
     if (tid == 0) {
       float m = 0.f;
       for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w]);
@@ -819,7 +836,7 @@ __global__ void __launch_bounds__(kThreads)
   } else if (tid == 0) {
     s_sh = table_scale(table, T, Lcount, step_dev, step_host, layer, err);
   }
-  __syncthreads();
+  cta_sync();
   const float s = s_sh;
   const float rs = quant_recip(s);
   uint8_t* dst = q_out + static_cast<size_t>(row) * (K / 2);
@@ -834,7 +851,7 @@ __global__ void __launch_bounds__(kThreads)
 // Grid of one problem: token tiles gx, CTAs per token tile (block groups, or
 // the cluster size in DYNAMIC mode) and rotation blocks per CTA.
 template <int BS, int TT, int MODE>
-void problem_grid(int M, int K, int* gx, int* per_tile, int* bpc) {
+void problem_grid(int M, int K, int* gx, int* per_tile, int* bpc, int min_bpc = 1) {
   const int nb = K / BS;
   *gx = (M + TT - 1) / TT;
   if (MODE == kDynamic) {
@@ -848,7 +865,7 @@ void problem_grid(int M, int K, int* gx, int* per_tile, int* bpc) {
     const int target = 2 * 148;
     int g = (target + *gx - 1) / *gx;
     g = g < 1 ? 1 : (g > nb ? nb : g);
-    *bpc = (nb + g - 1) / g;
+    *bpc = std::min(nb, std::max((nb + g - 1) / g, min_bpc));
     *per_tile = (nb + *bpc - 1) / *bpc;
   }
 }
@@ -856,7 +873,7 @@ void problem_grid(int M, int K, int* gx, int* per_tile, int* bpc) {
 // Launches up to kMaxBatch problems that share (BS, TT, Tin, MODE) and, in
 // DYNAMIC mode, the cluster size.
 template <int BS, int TT, typename Tin, int MODE>
-cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream) {
+cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream, int min_bpc = 1) {
   ActBatch batch;
   std::memset(&batch, 0, sizeof(batch));
   batch.n = n;
@@ -864,7 +881,7 @@ cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream) {
   for (int i = 0; i < n; ++i) {
     const ActArgs& a = *as[i];
     int gx, per_tile, bpc;
-    problem_grid<BS, TT, MODE>(a.M, a.K, &gx, &per_tile, &bpc);
+    problem_grid<BS, TT, MODE>(a.M, a.K, &gx, &per_tile, &bpc, min_bpc);
     ActProblem& P = batch.p[i];
     P.x = a.x;
     P.perm = a.perm;
@@ -936,9 +953,24 @@ cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream) {
 template <int BS, int TT, typename Tin, int MODE>
 cudaError_t launch_cfg_batches(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   if (MODE != kDynamic) {
+    // Each problem alone would be cut into ~2 CTAs per SM; a batch of them
+    // shares the GPU, so the blocks per CTA are raised until the launch fits
+    // in one wave (4 resident CTAs per SM), rather than leave a second wave
+    // of a few CTAs.
     for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
       const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
-      cudaError_t e = launch_group<BS, TT, Tin, MODE>(v.data() + i0, n, stream);
+      int min_bpc = 1;
+      for (;;) {
+        int ctas = 0;
+        for (int i = 0; i < n; ++i) {
+          int gx, per_tile, bpc;
+          problem_grid<BS, TT, MODE>(v[i0 + i]->M, v[i0 + i]->K, &gx, &per_tile, &bpc, min_bpc);
+          ctas += gx * per_tile;
+        }
+        if (ctas <= 4 * 148 || min_bpc >= 64) break;
+        min_bpc *= 2;
+      }
+      cudaError_t e = launch_group<BS, TT, Tin, MODE>(v.data() + i0, n, stream, min_bpc);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
