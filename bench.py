@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--workload", default="dit_mlp_stack",
                    choices=["dit_mlp_stack", "dit_denoise_loop", "backbone_prefill",
                             "single_linear"])
+    p.add_argument("--rotation", default="composite", choices=["composite", "hadamard"],
+                   help="composite: R = R_SVD.H (the method); hadamard: R_SVD = I variant")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-steps", type=int, default=0,
                    help="oracle steps for the CPU baseline (0: sized to ~15 s)")
@@ -60,9 +62,13 @@ def parse():
     return p.parse_args()
 
 
-def make_workload(name):
-    return {"dit_mlp_stack": I.dit_mlp_stack, "dit_denoise_loop": I.dit_denoise_loop,
-            "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
+def make_workload(name, rotation="composite"):
+    wl = {"dit_mlp_stack": I.dit_mlp_stack, "dit_denoise_loop": I.dit_denoise_loop,
+          "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
+    if rotation == "hadamard":
+        wl.name += "_hadamard_only"
+    wl.rotation = rotation
+    return wl
 
 
 def kernel_nodes(raw_graph):
@@ -185,7 +191,8 @@ def oracle_step(wl, packs, xs, t):
 
 def oracle_setup(wl, steps):
     from oracle import qvla_oracle as O
-    packs = [O.pack_linear(l.make_w(), l.block, bias=l.make_bias()) for l in wl.linears]
+    pack = O.pack_linear_hadamard if getattr(wl, "rotation", "") == "hadamard" else O.pack_linear
+    packs = [pack(l.make_w(), l.block, bias=l.make_bias()) for l in wl.linears]
     xs = [[l.make_x(seed_offset=t, std=(float(wl.sigmas[t]) if wl.sigmas is not None else None))
            for l in wl.linears] for t in range(steps)]
     return packs, xs
@@ -221,7 +228,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.rotation)
     packs, xs = oracle_setup(wl, min(max(1, wl.steps), 2))
     for i in range(args.warmup):
         oracle_step(wl, packs, xs, i % len(xs))
@@ -261,7 +268,7 @@ def run_ours(args):
     B.build()
     from w4a4_post_quantization_zigzag_b200 import qvla as Q
 
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.rotation)
     T = max(1, wl.steps)
     table = torch.from_numpy(wl.table).to(dev) if wl.table is not None else None
     steps_dev = torch.arange(T, dtype=torch.int32, device=dev)
@@ -273,7 +280,8 @@ def run_ours(args):
     packs = []
     for lin in wl.linears:
         W = torch.from_numpy(lin.make_w()).to(dev)
-        packs.append(Q.qvla_pack_weights(W, lin.block, bias=torch.from_numpy(lin.make_bias()).to(dev)))
+        pack = Q.qvla_pack_weights_hadamard if wl.rotation == "hadamard" else Q.qvla_pack_weights
+        packs.append(pack(W, lin.block, bias=torch.from_numpy(lin.make_bias()).to(dev)))
         del W
     torch.cuda.synchronize()
     pack_s = time.perf_counter() - t0
@@ -352,12 +360,13 @@ def run_ours(args):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    def timed_replays(gs, n):
+    def timed_replays(gs, n, flush_l2=True):
         starts = [ev() for _ in range(n)]
         ends = [ev() for _ in range(n)]
         with torch.cuda.stream(stream):
             for i in range(n):
-                l2_flush()
+                if flush_l2:
+                    l2_flush()
                 starts[i].record()
                 gs[i % T].replay()
                 ends[i].record()
@@ -389,6 +398,11 @@ def run_ours(args):
     s2, e2 = timed_replays(graphs_pl, args.steps)
     torch.cuda.synchronize()
     per_linear_us = sum(a.elapsed_time(b) for a, b in zip(s2, e2)) * 1e3 / args.steps
+
+    # ---- the batched step with a warm L2 (no flush between steps; informational)
+    sw_, ew_ = timed_replays(graphs, args.steps, flush_l2=False)
+    torch.cuda.synchronize()
+    warm_us = sum(a.elapsed_time(b) for a, b in zip(sw_, ew_)) * 1e3 / args.steps
 
     # ---- per-kernel breakdown: eager launches with events on the launching
     # stream; a GPU sleep ahead of the events keeps host enqueue time out
@@ -432,7 +446,8 @@ def run_ours(args):
     gemm_bytes = sum(l.N * l.K // 2 + l.M * l.K // 2 + 2 * l.M * l.N + 4 * l.M + 8 * l.N
                      for l in wl.linears)
     rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + l.M * l.K // 2 + 4 * l.M
-                    + 4 * l.K * l.block + 4 * l.K for l in wl.linears)
+                    + (4 * l.K * l.block if wl.rotation != "hadamard" else 0) + 4 * l.K
+                    for l in wl.linears)
     t_gemm = sum(kgemm) / args.steps          # ms per step (one batched launch)
     t_rot = sum(krot) / args.steps
     dom = "w4a4_gemm" if t_gemm >= t_rot else "rotate_quant"
@@ -452,13 +467,17 @@ def run_ours(args):
         "metric": METRIC, "value": us_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": {"workload": wl.name, "tokens_M": wl.linears[0].M,
+        "config": {"workload": wl.name, "rotation": wl.rotation, "tokens_M": wl.linears[0].M,
                    "linears_per_step": nl, "denoise_steps_T": T,
                    "block": wl.linears[0].block, "scale": wl.mode,
                    "l2": "flushed before every timed step (512 MB written, then read back: cold, clean L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single"},
         "roofline": roof,
         "tops": ops / (ms_per_step * 1e-3) / 1e12,
+        "tops_frac_int8": ops / (ms_per_step * 1e-3) / 1e12 / (2.0 * bf16_tf),
+        "int8_peak_tops": {"value": 2.0 * bf16_tf,
+                           "source": f"2 x bf16_tflops ({peak_src}; dense int8 : bf16 = 2 : 1)"},
+        "l2_warm_us_per_step": warm_us,
         "weight_gbs": wl.packed_weight_bytes() / (ms_per_step * 1e-3) / 1e9,
         "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3},
         "per_linear_launches_us_per_step": per_linear_us,

@@ -103,8 +103,10 @@ typedef enum { QVLA_SCALE_DYNAMIC = 0, QVLA_SCALE_TABLE = 1 } qvla_scale_mode;
 typedef struct {
   int32_t N, K, block;
   const int32_t* perm;      /* [K]  zigzag permutation                      */
-  const float* rot;         /* [nb][b][b] R_SVD blocks                      */
-  const uint16_t* rot_tc;   /* tensor-core images of R_B, or NULL           */
+  const float* rot;         /* [nb][b][b] R_SVD blocks, or NULL: R_SVD = I  */
+                            /* (Hadamard-only rotation, R_B = H_b)           */
+  const uint16_t* rot_tc;   /* tensor-core images of R_B, or NULL (must be  */
+                            /* NULL when rot is NULL)                        */
   const uint8_t* wq;        /* [N][K/2] packed weight codes                 */
   const float* w_scale;     /* [N]  s_w                                      */
   const float* bias;        /* [N]  or NULL                                  */
@@ -152,6 +154,24 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
                               uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
                               void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Offline pack of the Hadamard-only variant: R_SVD = I for every block, so
+ * R_B = H_b ("FoldQuantVLA" page: Hadamard rotation of weights and
+ * activations; the composite-rotation ablation of "{Omega}-QVLA"
+ * Methodology 1, SVD factor removed).  The zigzag permutation is kept:
+ * perm_in host int32 [K] or NULL (computed as in qvla_pack_weights()).
+ * Outputs (device): perm_out [K], wq_out [N][K/2], w_scale_out [N];
+ * W' = W P H is formed in fp64 and rounded once to fp32 before RTN.  The
+ * packed linear built from these has rot = NULL and rot_tc = NULL; the
+ * activation side then applies only the fast Walsh-Hadamard transform.
+ * workspace device, >= ws_bytes from qvla_packed_sizes().  Blocks the calling
+ * thread (one synchronisation for the host-side sort, one at the end).
+ * ------------------------------------------------------------------------- */
+qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
+                                       const int32_t* perm_in, int32_t* perm_out, uint8_t* wq_out,
+                                       float* w_scale_out, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream);
+
 /* Device step of the pack: W'_f32 = fp32(W P R), computed in fp64 from fp64
  * R_SVD blocks.  W device fp32 [N][K]; perm device [K]; rsvd64 device fp64
  * [nb][b][b]; Wr_out device fp32 [N][K].  Asynchronous.                    */
@@ -172,7 +192,9 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
  *
  * x       device, [M][ldx] of `xdt` (ldx >= K, in elements).
  * L       host pointer to a packed linear (device pointers inside); only
- *         perm, rot, rot_tc, K and block are read.  With bf16 input and a
+ *         perm, rot, rot_tc, K and block are read.  rot = NULL (Hadamard-only
+ *         linear): the gathered block goes straight to the fast Walsh-Hadamard
+ *         transform, no R_SVD product.  With bf16 input and a
  *         rot_tc image the rotation runs on the tensor cores as one dense
  *         product with R_B = R_SVD,B . H_b (three bf16 parts, fp32
  *         accumulation in tensor memory); otherwise on the CUDA cores as the

@@ -267,6 +267,17 @@ class PackedLinear:
         return pack_nibbles(self.qw)
 
 
+def pack_linear_hadamard(W: np.ndarray, block: int, bias=None, perm=None) -> PackedLinear:
+    """Hadamard-only variant: R_SVD = I for every block, so R_B = H_b and
+    x'_B = H x_B ("FoldQuantVLA": Hadamard rotation of weights and activations;
+    the composite rotation of "{Omega}-QVLA" Methodology 1 without its SVD
+    factor).  The zigzag permutation is kept."""
+    if perm is None:
+        perm = zigzag_permutation(W, block)
+    nb = np.asarray(W).shape[1] // block
+    return pack_linear(W, block, bias=bias, perm=perm, rsvd=np.stack([np.eye(block)] * nb))
+
+
 def pack_linear(W: np.ndarray, block: int, bias=None, perm=None, rsvd=None) -> PackedLinear:
     """Offline pack: zigzag P, per-block R_SVD, R = R_SVD.H, W' = W P R, then RTN
     of fp32(W').  `perm` / `rsvd` may be given to pin the non-unique parts."""

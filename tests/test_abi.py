@@ -70,6 +70,10 @@ def test_argument_errors_before_any_cuda_call():
     Lbad = q.qvla_packed_linear(128, 250, 64, 16, 16, None, 16, 16, None)
     assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lbad),
                                    ctypes.c_void_p(16), None) == q.QVLA_ERR_SHAPE
+    # a tensor-core image without R_SVD blocks (rot NULL means R_SVD = I)
+    Lhad = q.qvla_packed_linear(128, 256, 64, 16, 0, 16, 16, 16, None)
+    assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lhad),
+                                   ctypes.c_void_p(16), None) == q.QVLA_ERR_ARG
     # misaligned pointers
     Lmis = q.qvla_packed_linear(128, 256, 64, 16, 24, None, 16, 16, None)
     assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lmis),

@@ -140,6 +140,46 @@ def test_rotation_preserves_the_product():
     assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-9
 
 
+# -------------------------------------- Hadamard-only variant (R_SVD = I)
+
+@pytest.mark.parametrize("K,b", [(256, 32), (512, 64), (1024, 128), (512, 256)])
+def test_hadamard_only_pack_uses_the_library_hadamard(K, b):
+    """R_B is SciPy's Sylvester Hadamard matrix scaled by 1/sqrt(b), entry for
+    entry, and the zigzag permutation is the one the full method uses."""
+    from scipy.linalg import hadamard as scipy_hadamard
+    W = I.weights(7000 + K + b, 64, K, col_spread=10.0).astype(np.float64)
+    pk = O.pack_linear_hadamard(W, b)
+    Hs = scipy_hadamard(b).astype(np.float64) / np.sqrt(b)
+    assert pk.R.shape == (K // b, b, b)
+    for B in range(K // b):
+        assert np.array_equal(pk.R[B], Hs)
+    assert np.array_equal(pk.perm, O.zigzag_permutation(W, b))
+    # W' = W P H block by block, against a dense product built from SciPy's H
+    Wp = W[:, pk.perm]
+    dense = np.concatenate([Wp[:, B * b:(B + 1) * b] @ Hs for B in range(K // b)], axis=1)
+    np.testing.assert_allclose(pk.Wr, dense, rtol=0, atol=1e-12)
+
+
+def test_hadamard_only_preserves_the_product_and_codes_range():
+    """(W P H)(H^T P^T x) = W x, and the activation side is H applied to the
+    gathered block (the fast Walsh-Hadamard transform)."""
+    from scipy.linalg import hadamard as scipy_hadamard
+    wl = I.single_linear()
+    lin = wl.linears[0]
+    W, x = lin.make_w().astype(np.float64), lin.make_x().astype(np.float64)
+    pk = O.pack_linear_hadamard(W, lin.block)
+    xr = O.rotate_activations(x, pk.perm, pk.R)
+    ref = x @ W.T
+    assert np.linalg.norm(xr @ pk.Wr.T - ref) / np.linalg.norm(ref) <= 1e-9
+    b = lin.block
+    Hs = scipy_hadamard(b).astype(np.float64) / np.sqrt(b)
+    xp = x[:, pk.perm]
+    for B in range(lin.K // b):
+        np.testing.assert_allclose(xr[:, B * b:(B + 1) * b], xp[:, B * b:(B + 1) * b] @ Hs,
+                                   rtol=0, atol=1e-12)
+    assert pk.qw.min() >= -7 and pk.qw.max() <= 7
+
+
 # ------------------------------------------------ dense brute force (tiny)
 
 def _dense_P(perm):

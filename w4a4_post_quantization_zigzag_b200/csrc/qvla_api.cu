@@ -57,9 +57,10 @@ qvla_status check_linear(const qvla_packed_linear* L, bool need_weights) {
   if (!L) return QVLA_ERR_ARG;
   qvla_status st = check_shape(L->N, L->K, L->block);
   if (st != QVLA_OK) return st;
-  if (!L->perm || !L->rot) return QVLA_ERR_ARG;
+  // rot == NULL: Hadamard-only linear (R_SVD = I), which has no tensor-core image
+  if (!L->perm || (!L->rot && L->rot_tc)) return QVLA_ERR_ARG;
   if (need_weights && (!L->wq || !L->w_scale)) return QVLA_ERR_ARG;
-  if (!aligned16(L->perm) || !aligned16(L->rot)) return QVLA_ERR_ALIGN;
+  if (!aligned16(L->perm) || (L->rot && !aligned16(L->rot))) return QVLA_ERR_ALIGN;
   if (L->rot_tc && !aligned16(L->rot_tc)) return QVLA_ERR_ALIGN;
   if (need_weights && (!aligned16(L->wq) || !aligned16(L->w_scale))) return QVLA_ERR_ALIGN;
   if (L->bias && !aligned16(L->bias)) return QVLA_ERR_ALIGN;
@@ -264,17 +265,21 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
   return cuda_status(launch_quant_rows(a, stream));
 }
 
-qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
-                              const double* rsvd_in, int32_t* perm_out, float* rot_out,
-                              uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
-                              void* workspace, size_t ws_bytes, cudaStream_t stream) {
+// The pack.  hadamard_only: R_SVD = I for every block (no Gram matrices, no
+// eigensolve; rot_out and rot_tc_out are not written).
+static qvla_status pack_impl(const float* W, int N, int K, int block, const int32_t* perm_in,
+                             const double* rsvd_in, bool hadamard_only, int32_t* perm_out,
+                             float* rot_out, uint16_t* rot_tc_out, uint8_t* wq_out,
+                             float* w_scale_out, void* workspace, size_t ws_bytes,
+                             cudaStream_t stream) {
   qvla_status st = check_shape(N, K, block);
   if (st != QVLA_OK) return st;
   if (K % 32) return QVLA_ERR_SHAPE;
-  if (!W || !perm_out || !rot_out || !wq_out || !w_scale_out) return QVLA_ERR_ARG;
+  if (!W || !perm_out || (!rot_out && !hadamard_only) || !wq_out || !w_scale_out)
+    return QVLA_ERR_ARG;
   if (!workspace || ws_bytes < pack_ws_bytes(N, K, block)) return QVLA_ERR_WORKSPACE;
-  if (!aligned16(W) || !aligned16(perm_out) || !aligned16(rot_out) || !aligned16(wq_out) ||
-      !aligned16(w_scale_out) || !aligned16(workspace))
+  if (!aligned16(W) || !aligned16(perm_out) || (rot_out && !aligned16(rot_out)) ||
+      !aligned16(wq_out) || !aligned16(w_scale_out) || !aligned16(workspace))
     return QVLA_ERR_ALIGN;
   const int nb = K / block;
   const size_t bb = static_cast<size_t>(block) * block;
@@ -309,8 +314,11 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
     return QVLA_ERR_CUDA;
 
   // 2. R_SVD per block
-  std::vector<double> rs(nb * bb);
-  if (rsvd_in) {
+  std::vector<double> rs(nb * bb, 0.0);
+  if (hadamard_only) {
+    for (int B = 0; B < nb; ++B)
+      for (int i = 0; i < block; ++i) rs[B * bb + static_cast<size_t>(i) * block + i] = 1.0;
+  } else if (rsvd_in) {
     std::memcpy(rs.data(), rsvd_in, rs.size() * sizeof(double));
   } else {
     if (launch_block_gram(W, N, K, block, perm_out, gram, stream) != cudaSuccess)
@@ -334,11 +342,11 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
   for (size_t i = 0; i < rs.size(); ++i) rs32[i] = static_cast<float>(rs[i]);
   if (cudaMemcpyAsync(rsvd_dev, rs.data(), rs.size() * sizeof(double), cudaMemcpyHostToDevice,
                       stream) != cudaSuccess ||
-      cudaMemcpyAsync(rot_out, rs32.data(), rs32.size() * sizeof(float), cudaMemcpyHostToDevice,
-                      stream) != cudaSuccess)
+      (!hadamard_only && cudaMemcpyAsync(rot_out, rs32.data(), rs32.size() * sizeof(float),
+                                         cudaMemcpyHostToDevice, stream) != cudaSuccess))
     return QVLA_ERR_CUDA;
 
-  if (rot_tc_out && (block == 64 || block == 128)) {
+  if (!hadamard_only && rot_tc_out && (block == 64 || block == 128)) {
     if (!aligned16(rot_tc_out)) return QVLA_ERR_ALIGN;
     if (launch_rot_tc_image(rsvd_dev, K, block, rot_tc_out, stream) != cudaSuccess)
       return QVLA_ERR_CUDA;
@@ -360,6 +368,22 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
   // host staging vectors must outlive the copies
   if (cudaStreamSynchronize(stream) != cudaSuccess) return QVLA_ERR_CUDA;
   return QVLA_OK;
+}
+
+qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int32_t* perm_in,
+                              const double* rsvd_in, int32_t* perm_out, float* rot_out,
+                              uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, perm_out, rot_out, rot_tc_out, wq_out,
+                   w_scale_out, workspace, ws_bytes, stream);
+}
+
+qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
+                                       const int32_t* perm_in, int32_t* perm_out, uint8_t* wq_out,
+                                       float* w_scale_out, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream) {
+  return pack_impl(W, N, K, block, perm_in, nullptr, true, perm_out, nullptr, nullptr, wq_out,
+                   w_scale_out, workspace, ws_bytes, stream);
 }
 
 // Validates one rotate-quantise call and fills its launch arguments.

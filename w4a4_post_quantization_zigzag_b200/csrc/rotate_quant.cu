@@ -300,7 +300,9 @@ __global__ void __launch_bounds__(kThreads)
   // ---- prologue: weight-side data, independent of the previous kernel
   for (int e = tid; e < nbc * BS; e += kThreads) perm_s[e] = __ldg(perm + B0 * BS + e);
   if (tid < TT) amax_s[tid] = 0u;
-  const int nchunks = nbc * G::NCH;
+  // no R_SVD blocks: the Hadamard-only rotation (R_SVD = I), x'_B = H x_B
+  const bool hadamard_only = rot == nullptr;
+  const int nchunks = hadamard_only ? 0 : nbc * G::NCH;
   auto issue_chunk = [&](int g) {
     const int bl = g / G::NCH, ch = g % G::NCH;
     const float* src = rot + (static_cast<size_t>(B0 + bl) * BS + ch * G::RCH) * BS;
@@ -329,11 +331,21 @@ __global__ void __launch_bounds__(kThreads)
         v = load_x(x + static_cast<size_t>(m0 + t) * ldx + p);
       xg[e] = v;
     }
-    // 2. dense product over R chunks
+    // 2. dense product over R chunks (the gathered inputs themselves when
+    // R_SVD = I)
     float acc[TPT][2];
 #pragma unroll
     for (int u = 0; u < TPT; ++u) acc[u][0] = acc[u][1] = 0.f;
-    for (int ch = 0; ch < G::NCH; ++ch) {
+    if (hadamard_only) {
+      cta_sync();   // the gather is complete
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) {
+        acc[u][0] = xg[(2 * jp) * TT + tg * TPT + u];
+        acc[u][1] = xg[(2 * jp + 1) * TT + tg * TPT + u];
+      }
+      cta_sync();   // every thread has read its inputs before they are overwritten
+    }
+    for (int ch = 0; ch < (hadamard_only ? 0 : G::NCH); ++ch) {
       const int g = bl * G::NCH + ch;
       if (g + 1 < nchunks) {
         issue_chunk(g + 1);

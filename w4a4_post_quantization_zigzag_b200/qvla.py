@@ -50,6 +50,7 @@ EXPORTED = (
     "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
     "qvla_w4a4_gemm_s32", "qvla_rotate_quant_act_batched", "qvla_w4a4_gemm_batched",
     "qvla_rotate_quant_workspace_bytes", "qvla_rotate_quant_act_noalloc",
+    "qvla_pack_weights_hadamard",
 )
 
 QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -81,6 +82,8 @@ _sig = {
     "qvla_pack_weights": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                   c_void_p]),
+    "qvla_pack_weights_hadamard": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qvla_rotate_weights_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
     "qvla_quant_pack_weights_f32": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p,
@@ -158,7 +161,8 @@ class PackedLinear:
         self.N, self.K, self.block = int(N), int(K), int(block)
         self.perm, self.rot, self.wq, self.w_scale, self.bias = perm, rot, wq, w_scale, bias
         self.rot_tc = rot_tc
-        self._s = qvla_packed_linear(self.N, self.K, self.block, perm.data_ptr(), rot.data_ptr(),
+        self._s = qvla_packed_linear(self.N, self.K, self.block, perm.data_ptr(),
+                                     rot.data_ptr() if rot is not None else None,
                                      rot_tc.data_ptr() if rot_tc is not None else None,
                                      wq.data_ptr(), w_scale.data_ptr(),
                                      bias.data_ptr() if bias is not None else None)
@@ -168,7 +172,8 @@ class PackedLinear:
         return ctypes.byref(self._s)
 
     def device_bytes(self) -> int:
-        n = sum(t.numel() * t.element_size() for t in (self.perm, self.rot, self.wq, self.w_scale))
+        n = sum(t.numel() * t.element_size() for t in (self.perm, self.rot, self.wq, self.w_scale)
+                if t is not None)
         n += self.rot_tc.numel() * 2 if self.rot_tc is not None else 0
         return n + (self.bias.numel() * 4 if self.bias is not None else 0)
 
@@ -204,6 +209,31 @@ def qvla_pack_weights(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] 
         bias = bias.contiguous()
     return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias,
                         rot_tc=rot_tc)
+
+
+def qvla_pack_weights_hadamard(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
+                               perm_in: Optional[np.ndarray] = None, stream=None) -> PackedLinear:
+    """Hadamard-only pack (R_SVD = I): the packed linear has rot = rot_tc = None."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    wq_b, _, _, ws_b = qvla_packed_sizes(N, K, block)
+    dev = W.device
+    perm = torch.empty(K, dtype=torch.int32, device=dev)
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    p_in = None
+    if perm_in is not None:
+        perm_in = np.ascontiguousarray(perm_in, dtype=np.int32)
+        assert perm_in.shape == (K,)
+        p_in = perm_in.ctypes.data_as(c_void_p)
+    _check(_lib.qvla_pack_weights_hadamard(_ptr(W), N, K, block, p_in, _ptr(perm), _ptr(wq),
+                                           _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
+           "qvla_pack_weights_hadamard")
+    if bias is not None:
+        assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
+        bias = bias.contiguous()
+    return PackedLinear(N, K, block, perm, None, wq, s_w, bias, rot_tc=None)
 
 
 def qvla_rotate_weights_f32(W: torch.Tensor, block: int, perm: torch.Tensor,
