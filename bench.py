@@ -50,8 +50,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="dit_mlp_stack",
-                   choices=["dit_mlp_stack", "dit_denoise_loop", "backbone_prefill",
-                            "single_linear"])
+                   choices=["dit_mlp_stack", "dit_mlp_stack_fused", "dit_denoise_loop",
+                            "backbone_prefill", "single_linear"])
     p.add_argument("--rotation", default="composite", choices=["composite", "hadamard"],
                    help="composite: R = R_SVD.H (the method); hadamard: R_SVD = I variant")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -64,6 +64,7 @@ def parse():
 
 def make_workload(name, rotation="composite"):
     wl = {"dit_mlp_stack": I.dit_mlp_stack, "dit_denoise_loop": I.dit_denoise_loop,
+          "dit_mlp_stack_fused": lambda: I.dit_mlp_stack(fuse_gate_up=True),
           "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
     if rotation == "hadamard":
         wl.name += "_hadamard_only"

@@ -74,6 +74,20 @@ def test_dit_mlp_stack_step_full_size(q):
         _check_sampled(lin, x, ref, p, rows, "table", wl.table, t)
 
 
+def test_dit_mlp_stack_gate_up_fused_full_size(q):
+    """Shared-input fusion: gate and up as one 1024->8192 linear (one
+    permutation and rotation from the concatenated weights, one activation
+    pass), in the batched launches of the fused step."""
+    wl = I.dit_mlp_stack(fuse_gate_up=True)
+    assert [l.N for l in wl.linears[:2]] == [8192, 1024] and len(wl.linears) == 8
+    t = 4
+    xs = [l.make_x(seed_offset=t, std=float(wl.sigmas[t])) for l in wl.linears]
+    refs, probs = _run_batched(q, wl.linears, xs, "table", wl.table, t, scratch=False)
+    rows = np.random.default_rng(3).choice(wl.linears[0].M, 5, replace=False)
+    for lin, x, ref, p in zip(wl.linears[:2], xs, refs, probs):
+        _check_sampled(lin, x, ref, p, rows, "table", wl.table, t)
+
+
 def test_backbone_prefill_full_size(q):
     wl = I.backbone_prefill()
     xs = [l.make_x() for l in wl.linears]

@@ -180,24 +180,31 @@ def single_linear(seed: int = 0) -> Workload:
 
 
 def dit_mlp_stack(seed: int = 1, layers: int = 4, M: int = 50, hidden: int = 1024,
-                  ffn: int = 4096, steps: int = 10, block: int = 64) -> Workload:
+                  ffn: int = 4096, steps: int = 10, block: int = 64,
+                  fuse_gate_up: bool = False) -> Workload:
     """DiT action-head MLP stack: 50 action tokens x batch 1, hidden 1024,
     gate/up 1024->4096 and down 4096->1024, 4 layers, bf16 activations;
     10 denoising steps with a static act_scale_table[10][12]; activation std
     drifts 0.5 -> 3.0 across steps; block 64.  Every linear draws its own input
-    (the MLP nonlinearity between up/gate and down is not part of the layer)."""
+    (the MLP nonlinearity between up/gate and down is not part of the layer).
+
+    fuse_gate_up: gate and up, which read the same input in the MLP, become one
+    linear 1024->8192 (concatenated weights, one permutation and rotation, one
+    activation pass); 8 linears and a table [10][8] per step."""
     lins = []
     li = 0
+    shapes = ((("gate_up", hidden, 2 * ffn), ("down", ffn, hidden)) if fuse_gate_up else
+              (("gate", hidden, ffn), ("up", hidden, ffn), ("down", ffn, hidden)))
     for layer in range(layers):
-        for j, (nm, K, N) in enumerate((("gate", hidden, ffn), ("up", hidden, ffn),
-                                        ("down", ffn, hidden))):
+        for j, (nm, K, N) in enumerate(shapes):
             s = seed * 100000 + li * 10
             lins.append(Linear(f"l{layer}.{nm}", M=M, K=K, N=N, block=block, x_seed=s,
                                w_seed=s + 1, b_seed=s + 2, layer=li))
             li += 1
     sig = step_sigmas(steps)
     tab = scale_table(seed * 100000 + 99, steps, len(lins), sig)
-    return Workload(f"dit_mlp_stack_M{M}_h{hidden}_f{ffn}_L{layers}_T{steps}_b{block}",
+    tag = "_gateup_fused" if fuse_gate_up else ""
+    return Workload(f"dit_mlp_stack_M{M}_h{hidden}_f{ffn}_L{layers}_T{steps}_b{block}{tag}",
                     lins, mode="table", steps=steps, table=tab, sigmas=sig)
 
 
