@@ -61,9 +61,12 @@ struct Cfg {
   static constexpr int kTmemCols = NT < 32 ? 32 : NT;
   static constexpr int kRedPitch = NT + 4;             // int32 per row of the split-K buffer
   static constexpr int kStageBytes = kPS * kPStageBytes + kUS * kUStageBytes;
-  static constexpr int kRecvBytes = kBM * kRedPitch * 4;   // split-K receive buffer
-  static constexpr int kSmemBytes = kStageBytes + 1024;    // + kRecvBytes when split
-  static constexpr bool kCanSplit = kSmemBytes + kRecvBytes <= 227 * 1024;
+  // split-K receive buffer and the owner's output rows (at most 64 of them,
+  // S >= 2), both placed over the stage memory once every CTA of the cluster
+  // is done with its stages
+  static constexpr int kRecvBytes = kBM * kRedPitch * 4;
+  static constexpr int kSmemBytes = kStageBytes + 1024;
+  static constexpr bool kCanSplit = kRecvBytes + NT * 64 * 2 <= kStageBytes;
 };
 
 struct Barriers {
@@ -159,9 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   cta_sync();
   tc_fence_after();
   const uint32_t tmem_d = bars.tmem_base;
-  // split-K: announce that this CTA runs; remote shared-memory stores wait for
-  // every CTA of the cluster to have done so
-  if (S > 1) cluster_arrive_relaxed();
+  // split-K: every thread arrives on the cluster barrier once it is done with
+  // the stage memory (the producer after its last load has landed, the MMA
+  // issuer after its last MMA has completed, the workers after the
+  // accumulator is final); partial sums are pushed into the owner's stage
+  // memory only after the whole cluster has arrived
   bool cluster_waited = false;
 
   if (warp == 0) {
@@ -202,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = issued - C::kPS < 0 ? 0 : issued - C::kPS; i < issued; ++i)
         mbar_wait(&bars.full_p[i % C::kPS], (i / C::kPS) & 1, err);
     }
+    if (S > 1) cluster_arrive_relaxed();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -228,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&bars.acc_full);
       mbar_wait(&bars.acc_full, 0, err);   // tensor memory is freed only after this
     }
+    if (S > 1) cluster_arrive_relaxed();
   } else {
     // --------------------------------------------------- unpack (4 warps)
     const int wt = tid - 64;   // 0..127
@@ -301,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one outcome per warp, and a converged warp for the warp-wide loads
     const bool have = __all_sync(0xffffffffu, ok && mbar_wait(&bars.acc_full, 0, err));
     tc_fence_after();
+    if (S > 1) cluster_arrive_relaxed();
     pdl_launch_dependents();
     if (have) {
       // split-K: this CTA's partial rows go to the receive buffer of the CTA
@@ -309,8 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rpr = kBM / S;
       const uint32_t owner = static_cast<uint32_t>(nl / rpr);
       const uint32_t recv_row =
-          smem_u32(base + C::kStageBytes) +
-          static_cast<uint32_t>(((split * rpr + nl % rpr) * C::kRedPitch) * 4);
+          smem_u32(base) + static_cast<uint32_t>(((split * rpr + nl % rpr) * C::kRedPitch) * 4);
       const uint32_t remote_row = S > 1 ? map_shared_rank(recv_row, owner) : 0u;
       if (S > 1) {
         cluster_wait();
@@ -377,9 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int wt = tid - 64;
       const uint32_t rank = cluster_ctarank();
       const int rpr = kBM / S;                     // channel rows reduced by this CTA
-      const int32_t* recv = reinterpret_cast<const int32_t*>(base + C::kStageBytes);
-      // output tile [NT tokens][rpr channels] for one TMA store of this CTA's rows
-      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base);
+      const int32_t* recv = reinterpret_cast<const int32_t*>(base);
+      // output tile [NT tokens][rpr channels] for one TMA store of this CTA's
+      // rows, after the receive buffer
+      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base + C::kRecvBytes);
       for (int e = wt; e < rpr * NT; e += kWorkers) {
         const int lr = e % rpr;
         const int col = e / rpr;
@@ -504,8 +512,7 @@ cudaError_t launch_group(const GemmArgs* const* gs, const int* splits, int n, in
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C_::kCanSplit ? C_::kSmemBytes + C_::kRecvBytes : C_::kSmemBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
@@ -514,7 +521,7 @@ cudaError_t launch_group(const GemmArgs* const* gs, const int* splits, int n, in
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C_::kSmemBytes + (C > 1 ? C_::kRecvBytes : 0);
+  cfg.dynamicSmemBytes = C_::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -552,23 +559,39 @@ int choose_splits(const GemmArgs* const* gs, int n, int split_k, int* splits) {
     for (int i = 0; i < n; ++i) splits[i] = split_k;
     return split_k;
   }
-  // (Splitting only the long-K problems of a batch balances the K walk, but
-  // the split-K receive buffer then halves the CTAs per SM for the whole
-  // launch, which costs more than it gains; so the automatic factor is
-  // uniform.)
-  int min_nkt = 1 << 30;
-  for (int i = 0; i < n; ++i) min_nkt = std::min(min_nkt, (gs[i]->K + kKP - 1) / kKP);
-  int C = 1;
+  int min_nkt = 1 << 30, max_nkt = 0;
+  for (int i = 0; i < n; ++i) {
+    const int nkt = (gs[i]->K + kKP - 1) / kKP;
+    min_nkt = std::min(min_nkt, nkt);
+    max_nkt = std::max(max_nkt, nkt);
+  }
   for (int i = 0; i < n; ++i) splits[i] = 1;
+  if (NT <= 64 && max_nkt > 2 * min_nkt) {
+    // Weight-streaming launches (few tokens): linears more than twice as deep
+    // in K as the shallowest of the launch are split over a cluster of C
+    // CTAs, so that no CTA walks more than about twice the K tiles of the
+    // shallowest; the others stay whole.  (The split costs no extra shared
+    // memory: partial sums land in the stage memory of the owner once the
+    // cluster is done with its stages.)  With many tokens the launch already
+    // has several waves of CTAs and splitting measured slower.
+    int C = 1;
+    while (C < 8 && max_nkt > 2 * min_nkt * C) C *= 2;
+    for (int i = 0; i < n; ++i) {
+      const int nkt = (gs[i]->K + kKP - 1) / kKP;
+      if (nkt > 2 * min_nkt && C <= nkt) splits[i] = C;
+    }
+    return C;
+  }
+  // similar depths: one factor for all, raised while the launch has fewer
+  // CTAs than SMs
+  int C = 1;
   auto total = [&]() {
     int t = 0;
     for (int i = 0; i < n; ++i)
       t += ((gs[i]->N + kBM - 1) / kBM) * ((gs[i]->M + NT - 1) / NT) * splits[i];
     return t;
   };
-  bool uniform = true;
-  for (int i = 0; i < n; ++i) uniform = uniform && splits[i] == C;
-  while (uniform && C < 8 && total() < 148 && 2 * C <= min_nkt) {
+  while (C < 8 && total() < 148 && 2 * C <= min_nkt) {
     C *= 2;
     for (int i = 0; i < n; ++i) splits[i] = C;
   }
@@ -584,7 +607,18 @@ cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cud
     const int m = std::min(kMaxBatch, n - i0);
     int splits[kMaxBatch];
     const int C = choose_splits<NT>(gs + i0, m, split_k, splits);
-    cudaError_t e = launch_group<NT>(gs + i0, splits, m, C, stream);
+    // CTAs are dispatched in index order: the split (deepest) linears first,
+    // so that a partial second wave holds only short CTAs
+    const GemmArgs* order[kMaxBatch];
+    int osplit[kMaxBatch];
+    int k = 0;
+    for (int pass = 0; pass < 2; ++pass)
+      for (int i = 0; i < m; ++i)
+        if ((splits[i] > 1) == (pass == 0)) {
+          order[k] = gs[i0 + i];
+          osplit[k++] = splits[i];
+        }
+    cudaError_t e = launch_group<NT>(order, osplit, m, C, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
