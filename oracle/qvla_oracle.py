@@ -49,6 +49,11 @@ import numpy as np
 
 WEIGHT_QMAX = 7
 ACT_QMIN, ACT_QMAX = -8, 7
+# W8A8 variant ("FoldQuantVLA": attention-output and FFN-down projections kept
+# at W8A8): symmetric per-channel 8-bit weights, per-token dynamic 8-bit
+# activations; the same RTN rule with the 8-bit ranges.
+WEIGHT_QMAX8 = 127
+ACT_QMIN8, ACT_QMAX8 = -128, 127
 
 
 # --------------------------------------------------------------------------
@@ -174,23 +179,25 @@ def _rtn_codes(v32: np.ndarray, s32: np.ndarray, qmin: int, qmax: int) -> np.nda
     return q.astype(np.int8)
 
 
-def quantize_weights_fp32(Wr32: np.ndarray):
+def quantize_weights_fp32(Wr32: np.ndarray, qmax: int = WEIGHT_QMAX):
     """Symmetric per-output-channel RTN of fp32 rotated weights [N, K].
-    s_w[n] = fp32(max_k |W'[n,k]| / 7), codes in [-7, 7]."""
+    s_w[n] = fp32(max_k |W'[n,k]| / qmax), codes in [-qmax, qmax] (qmax 7 for
+    the 4-bit weights, 127 for the W8A8 variant)."""
     Wr32 = np.asarray(Wr32, dtype=np.float32)
     amax = np.max(np.abs(Wr32), axis=1)
-    s = np.divide(amax, np.float32(WEIGHT_QMAX), dtype=np.float32)
-    q = _rtn_codes(Wr32, s[:, None], -WEIGHT_QMAX, WEIGHT_QMAX)
+    s = np.divide(amax, np.float32(qmax), dtype=np.float32)
+    q = _rtn_codes(Wr32, s[:, None], -qmax, qmax)
     return q, s
 
 
-def quantize_acts_dynamic_fp32(xr32: np.ndarray):
+def quantize_acts_dynamic_fp32(xr32: np.ndarray, qmin: int = ACT_QMIN, qmax: int = ACT_QMAX):
     """Per-token dynamic RTN of fp32 rotated activations [M, K].
-    s_x[m] = fp32(max_k |x'[m,k]| / 7), codes clamped to [-8, 7]."""
+    s_x[m] = fp32(max_k |x'[m,k]| / qmax), codes clamped to [qmin, qmax]
+    ([-8, 7] for 4-bit activations, [-128, 127] for the W8A8 variant)."""
     xr32 = np.asarray(xr32, dtype=np.float32)
     amax = np.max(np.abs(xr32), axis=1) if xr32.shape[1] else np.zeros(xr32.shape[0], np.float32)
-    s = np.divide(amax, np.float32(ACT_QMAX), dtype=np.float32)
-    q = _rtn_codes(xr32, s[:, None], ACT_QMIN, ACT_QMAX)
+    s = np.divide(amax, np.float32(qmax), dtype=np.float32)
+    q = _rtn_codes(xr32, s[:, None], qmin, qmax)
     return q, s
 
 
@@ -258,12 +265,15 @@ def dequantize(acc: np.ndarray, s_x: np.ndarray, s_w: np.ndarray, bias=None) -> 
 class PackedLinear:
     """What the offline pack step produces for one linear (all on the host)."""
 
-    def __init__(self, perm, rsvd, R, Wr, qw, s_w, bias):
+    def __init__(self, perm, rsvd, R, Wr, qw, s_w, bias, bits=4):
         self.perm, self.rsvd, self.R, self.Wr = perm, rsvd, R, Wr
-        self.qw, self.s_w, self.bias = qw, s_w, bias
+        self.qw, self.s_w, self.bias, self.bits = qw, s_w, bias, bits
 
     @property
     def wq(self):
+        """Packed weight bytes: two 4-bit codes per byte, or one int8 code."""
+        if self.bits == 8:
+            return np.asarray(self.qw, dtype=np.int8).view(np.uint8)
         return pack_nibbles(self.qw)
 
 
@@ -278,17 +288,20 @@ def pack_linear_hadamard(W: np.ndarray, block: int, bias=None, perm=None) -> Pac
     return pack_linear(W, block, bias=bias, perm=perm, rsvd=np.stack([np.eye(block)] * nb))
 
 
-def pack_linear(W: np.ndarray, block: int, bias=None, perm=None, rsvd=None) -> PackedLinear:
+def pack_linear(W: np.ndarray, block: int, bias=None, perm=None, rsvd=None,
+                bits: int = 4) -> PackedLinear:
     """Offline pack: zigzag P, per-block R_SVD, R = R_SVD.H, W' = W P R, then RTN
-    of fp32(W').  `perm` / `rsvd` may be given to pin the non-unique parts."""
+    of fp32(W') to 4-bit codes (8-bit for the W8A8 variant).  `perm` / `rsvd`
+    may be given to pin the non-unique parts."""
     if perm is None:
         perm = zigzag_permutation(W, block)
     if rsvd is None:
         rsvd = svd_rotation_blocks(W, perm, block)
     R = composite_blocks(rsvd)
     Wr = rotate_weights(W, perm, R)
-    qw, s_w = quantize_weights_fp32(Wr.astype(np.float32))
-    return PackedLinear(perm, rsvd, R, Wr, qw, s_w, bias)
+    qw, s_w = quantize_weights_fp32(Wr.astype(np.float32),
+                                    WEIGHT_QMAX8 if bits == 8 else WEIGHT_QMAX)
+    return PackedLinear(perm, rsvd, R, Wr, qw, s_w, bias, bits)
 
 
 def rotate_quant_act(x: np.ndarray, pk: PackedLinear, mode: str = "dynamic",
@@ -296,15 +309,16 @@ def rotate_quant_act(x: np.ndarray, pk: PackedLinear, mode: str = "dynamic",
     """Activation side in double, quantised like the fp32 path but from the
     double x' (the end-to-end reference).  Returns (x' double, codes, s_x double)."""
     xr = rotate_activations(x, pk.perm, pk.R)
+    qmin, qmax = (ACT_QMIN8, ACT_QMAX8) if pk.bits == 8 else (ACT_QMIN, ACT_QMAX)
     if mode == "dynamic":
-        s = np.max(np.abs(xr), axis=1) / ACT_QMAX
+        s = np.max(np.abs(xr), axis=1) / qmax
     elif mode == "table":
         s = np.full(xr.shape[0], float(table_scale(table, step, layer)))
     else:
         raise ValueError(mode)
     with np.errstate(divide="ignore", invalid="ignore"):
         r = np.rint(xr / np.where(s == 0, 1.0, s)[:, None])
-    q = np.where((s == 0)[:, None], 0, np.clip(r, ACT_QMIN, ACT_QMAX)).astype(np.int8)
+    q = np.where((s == 0)[:, None], 0, np.clip(r, qmin, qmax)).astype(np.int16)
     return xr, q, s
 
 

@@ -266,6 +266,47 @@ def test_rtn_brute_force_and_ranges():
             assert qw[n, k] == _brute_rtn(W[n, k], sw[n], -7, 7)
 
 
+def test_rtn_8bit_brute_force_and_ranges():
+    """The W8A8 reading: the same RTN rule with the 8-bit ranges, checked
+    element by element against scalar fp32 arithmetic."""
+    x = I.activations(15, 6, 64, n_outlier_cols=2, dtype="f32")
+    q, s = O.quantize_acts_dynamic_fp32(x, O.ACT_QMIN8, O.ACT_QMAX8)
+    for m in range(x.shape[0]):
+        assert s[m] == np.float32(np.float32(np.abs(x[m]).max()) / np.float32(127))
+        for k in range(x.shape[1]):
+            assert q[m, k] == _brute_rtn(x[m, k], s[m], -128, 127)
+        assert np.abs(q[m]).max() == 127              # the token max lands on +-127
+    W = I.weights(16, 8, 64, n_outlier_rows=2)
+    W[2] = 0.0
+    qw, sw = O.quantize_weights_fp32(W, O.WEIGHT_QMAX8)
+    assert qw.min() >= -127 and qw.max() <= 127
+    for n in range(W.shape[0]):
+        if sw[n] == 0:
+            assert not qw[n].any()
+        else:
+            assert np.abs(qw[n]).max() == 127
+            # every code is within half a step of the value it stands for
+            err = np.abs(W[n].astype(np.float64) - qw[n] * np.float64(sw[n]))
+            assert err.max() <= 0.5 * sw[n] * (1 + 1e-6)
+        for k in range(W.shape[1]):
+            assert qw[n, k] == _brute_rtn(W[n, k], sw[n], -127, 127)
+
+
+def test_w8a8_layer_tracks_the_fp_layer_more_closely_than_w4a4():
+    wl = I.single_linear()
+    lin = wl.linears[0]
+    W, x, b = lin.make_w(), lin.make_x(), lin.make_bias()
+    ref = x.astype(np.float64) @ W.astype(np.float64).T + b
+    errs = {}
+    for bits in (4, 8):
+        pk = O.pack_linear(W, lin.block, bias=b, bits=bits)
+        out = O.linear_forward(x.astype(np.float64), pk)
+        assert pk.bits == bits and np.abs(out["qx"]).max() <= (127 if bits == 8 else 8)
+        errs[bits] = np.linalg.norm(out["y"] - ref) / np.linalg.norm(ref)
+    assert errs[8] < errs[4] / 8
+    assert O.pack_linear(W, lin.block, bits=8).wq.shape == (lin.N, lin.K)
+
+
 def test_table_lookup_rejects_out_of_range():
     tab = np.ones((8, 3), np.float32)
     assert O.table_scale(tab, 7, 2) == 1.0
