@@ -54,6 +54,9 @@ def parse():
                             "backbone_prefill", "single_linear"])
     p.add_argument("--rotation", default="composite", choices=["composite", "hadamard"],
                    help="composite: R = R_SVD.H (the method); hadamard: R_SVD = I variant")
+    p.add_argument("--precision", default="w4a4", choices=["w4a4", "w8a8", "mix"],
+                   help="w8a8: every linear W8A8 (dynamic per-token 8-bit activations); "
+                        "mix: the down projections W8A8, the rest W4A4")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-steps", type=int, default=0,
                    help="oracle steps for the CPU baseline (0: sized to ~15 s)")
@@ -278,10 +281,15 @@ def run_ours(args):
     # pack (offline step, timed for information)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
+    # which linears run W8A8 (dynamic 8-bit activations, one launch sequence
+    # each) and which W4A4 (batched)
+    w8 = [args.precision == "w8a8" or (args.precision == "mix" and lin.name.endswith("down"))
+          for lin in wl.linears]
     packs = []
-    for lin in wl.linears:
+    for lin, is8 in zip(wl.linears, w8):
         W = torch.from_numpy(lin.make_w()).to(dev)
-        pack = Q.qvla_pack_weights_hadamard if wl.rotation == "hadamard" else Q.qvla_pack_weights
+        pack = (Q.qvla_pack_weights_w8 if is8 else
+                Q.qvla_pack_weights_hadamard if wl.rotation == "hadamard" else Q.qvla_pack_weights)
         packs.append(pack(W, lin.block, bias=torch.from_numpy(lin.make_bias()).to(dev)))
         del W
     torch.cuda.synchronize()
@@ -293,32 +301,53 @@ def run_ours(args):
                                                               if wl.sigmas is not None else None)))
                 .to(xdt).pin_memory() for l in wl.linears] for t in range(T)]
     xs = [[x.to(dev) for x in row] for row in xs_host]
-    xq = [torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev) for l in wl.linears]
+    xq = [torch.empty(l.M, l.K, dtype=torch.int8, device=dev) if is8 else
+          torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev)
+          for l, is8 in zip(wl.linears, w8)]
     sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
     ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
     # scratch of the tensor-core rotation route (more than 64 bf16 tokens), one
     # per linear since a batched launch runs them together
-    wss = [torch.empty(max(Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
-                       dtype=torch.uint8, device=dev) for l in wl.linears]
+    wss = [torch.empty(max(l.M * l.K * 4 if is8 else
+                           Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
+                       dtype=torch.uint8, device=dev) for l, is8 in zip(wl.linears, w8)]
     nl = len(wl.linears)
     # one problem set per denoising step: same packed weights and buffers, the
     # step's own inputs and device step index
     probs = [[Q.LinearProblem(L, xs[t][i], mode, table=table, step=steps_dev[t:t + 1],
                               layer=lin.layer, xq=xq[i], s_x=sx[i], y=ys[i], workspace=wss[i])
-              for i, (lin, L) in enumerate(zip(wl.linears, packs))] for t in range(T)]
+              for i, (lin, L) in enumerate(zip(wl.linears, packs)) if not w8[i]]
+             for t in range(T)]
+    idx8 = [i for i in range(len(wl.linears)) if w8[i]]
+
+    def w8_linears(t, phase):
+        for i in idx8:
+            if phase == 0:
+                Q.qvla_rotate_quant_act_a8(xs[t][i], packs[i], xq8=xq[i], s_x=sx[i],
+                                           workspace=wss[i])
+            else:
+                Q.qvla_w8a8_gemm(xq[i], sx[i], packs[i], y=ys[i])
 
     def step_batched(t, rec=None):
         if rec is not None:
             rec[0].record()
-        Q.qvla_rotate_quant_act_batched(probs[t])
+        if probs[t]:
+            Q.qvla_rotate_quant_act_batched(probs[t])
+        w8_linears(t, 0)
         if rec is not None:
             rec[1].record()
-        Q.qvla_w4a4_gemm_batched(probs[t])
+        if probs[t]:
+            Q.qvla_w4a4_gemm_batched(probs[t])
+        w8_linears(t, 1)
         if rec is not None:
             rec[2].record()
 
     def step_per_linear(t):
         for i, (lin, L) in enumerate(zip(wl.linears, packs)):
+            if w8[i]:
+                Q.qvla_rotate_quant_act_a8(xs[t][i], L, xq8=xq[i], s_x=sx[i], workspace=wss[i])
+                Q.qvla_w8a8_gemm(xq[i], sx[i], L, y=ys[i])
+                continue
             Q.qvla_rotate_quant_act(xs[t][i], L, mode, table=table, step=steps_dev[t:t + 1],
                                     layer=lin.layer, xq=xq[i], s_x=sx[i], workspace=wss[i])
             Q.qvla_w4a4_gemm(xq[i], sx[i], L, y=ys[i])
@@ -444,11 +473,13 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel
     hbm, bf16_tf, peak_src = load_peaks()
-    gemm_bytes = sum(l.N * l.K // 2 + l.M * l.K // 2 + 2 * l.M * l.N + 4 * l.M + 8 * l.N
-                     for l in wl.linears)
-    rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + l.M * l.K // 2 + 4 * l.M
+    cb = [1.0 if is8 else 0.5 for is8 in w8]          # code bytes per element
+    gemm_bytes = sum(int(l.N * l.K * c) + int(l.M * l.K * c) + 2 * l.M * l.N + 4 * l.M + 8 * l.N
+                     for l, c in zip(wl.linears, cb))
+    rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + int(l.M * l.K * c) + 4 * l.M
                     + (4 * l.K * l.block if wl.rotation != "hadamard" else 0) + 4 * l.K
-                    for l in wl.linears)
+                    for l, c in zip(wl.linears, cb))
+    weight_bytes = sum(int(l.N * l.K * c) + 8 * l.N for l, c in zip(wl.linears, cb))
     t_gemm = sum(kgemm) / args.steps          # ms per step (one batched launch)
     t_rot = sum(krot) / args.steps
     dom = "w4a4_gemm" if t_gemm >= t_rot else "rotate_quant"
@@ -468,7 +499,8 @@ def run_ours(args):
         "metric": METRIC, "value": us_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": {"workload": wl.name, "rotation": wl.rotation, "tokens_M": wl.linears[0].M,
+        "config": {"workload": wl.name, "rotation": wl.rotation, "precision": args.precision,
+                   "w8a8_linears": len(idx8), "tokens_M": wl.linears[0].M,
                    "linears_per_step": nl, "denoise_steps_T": T,
                    "block": wl.linears[0].block, "scale": wl.mode,
                    "l2": "flushed before every timed step (512 MB written, then read back: cold, clean L2)",
@@ -479,7 +511,7 @@ def run_ours(args):
         "int8_peak_tops": {"value": 2.0 * bf16_tf,
                            "source": f"2 x bf16_tflops ({peak_src}; dense int8 : bf16 = 2 : 1)"},
         "l2_warm_us_per_step": warm_us,
-        "weight_gbs": wl.packed_weight_bytes() / (ms_per_step * 1e-3) / 1e9,
+        "weight_gbs": weight_bytes / (ms_per_step * 1e-3) / 1e9,
         "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3},
         "per_linear_launches_us_per_step": per_linear_us,
         "pack_s": pack_s,

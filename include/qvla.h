@@ -172,6 +172,50 @@ qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
                                        float* w_scale_out, void* workspace, size_t ws_bytes,
                                        cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * W8A8 variant ("FoldQuantVLA" page: attention-output and FFN-down
+ * projections kept at W8A8, native integer execution).  The same zigzag
+ * permutation and composite rotation as qvla_pack_weights(); weights
+ * quantised symmetric per output channel to 8 bits: s_w[n] = fp32(max_k
+ * |W'[n,k]| / 127), q = clamp(rint(W'/s_w), -127, 127).
+ * Outputs (device): perm_out [K], rot_out [nb][b][b] fp32, wq_out [N][K]
+ * int8 (one code per byte: N * K bytes, not the N * K / 2 of
+ * qvla_packed_sizes()), w_scale_out [N].  No tensor-core image: a packed
+ * linear built from these has rot_tc = NULL, and its wq must only be given to
+ * qvla_w8a8_gemm() / qvla_w8a8_gemm_s32().  Other arguments and the blocking
+ * behaviour as qvla_pack_weights().
+ * ------------------------------------------------------------------------- */
+qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const int32_t* perm_in,
+                                 const double* rsvd_in, int32_t* perm_out, float* rot_out,
+                                 uint8_t* wq_out, float* w_scale_out, void* workspace,
+                                 size_t ws_bytes, cudaStream_t stream);
+
+/* W8A8 activations: the rotation of qvla_rotate_act_f32() into `workspace`
+ * (fp32 [M][K], M * K * 4 bytes, see qvla_rotate_quant_a8_workspace_bytes),
+ * then per-token dynamic 8-bit RTN: s_x[m] = fp32(max_k |x'[m,k]| / 127),
+ * q = clamp(rint(x'/s_x), -128, 127), one int8 code per byte.
+ * x, xdt, ldx, L as in qvla_rotate_quant_act().  Outputs (device): xq8
+ * [M][K] int8, s_x [M] fp32.  Asynchronous (two launches).                 */
+qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int ldx,
+                                     const qvla_packed_linear* L, int8_t* xq8, float* s_x,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Scratch of qvla_rotate_quant_act_a8(): M * K * 4 bytes.                   */
+qvla_status qvla_rotate_quant_a8_workspace_bytes(int M, int K, size_t* bytes);
+
+/* W8A8 GEMM: acc[m,n] = sum_k xq8[m,k] wq[n,k] (int8 x int8 -> int32, exact
+ * for K <= QVLA_MAX_K), y = bf16(fp32(s_x[m] s_w[n]) * acc + b[n]) — the W4A4
+ * epilogue.  xq8 device [M][K] int8 from qvla_rotate_quant_act_a8(); L from
+ * qvla_pack_weights_w8() (wq [N][K] int8); y device bf16 [M][ldy] (ldy >= N,
+ * ldy * 2 a multiple of 16).  The int8 codes go to the tensor cores as they
+ * are (no unpack).  Asynchronous.                                          */
+qvla_status qvla_w8a8_gemm(const int8_t* xq8, const float* s_x, int M,
+                           const qvla_packed_linear* L, void* y, int ldy, cudaStream_t stream);
+
+/* The int32 accumulators of qvla_w8a8_gemm() into acc [M][N] (tests).       */
+qvla_status qvla_w8a8_gemm_s32(const int8_t* xq8, int M, const qvla_packed_linear* L,
+                               int32_t* acc, cudaStream_t stream);
+
 /* Device step of the pack: W'_f32 = fp32(W P R), computed in fp64 from fp64
  * R_SVD blocks.  W device fp32 [N][K]; perm device [K]; rsvd64 device fp64
  * [nb][b][b]; Wr_out device fp32 [N][K].  Asynchronous.                    */

@@ -268,7 +268,7 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
 // The pack.  hadamard_only: R_SVD = I for every block (no Gram matrices, no
 // eigensolve; rot_out and rot_tc_out are not written).
 static qvla_status pack_impl(const float* W, int N, int K, int block, const int32_t* perm_in,
-                             const double* rsvd_in, bool hadamard_only, int32_t* perm_out,
+                             const double* rsvd_in, bool hadamard_only, int bits, int32_t* perm_out,
                              float* rot_out, uint16_t* rot_tc_out, uint8_t* wq_out,
                              float* w_scale_out, void* workspace, size_t ws_bytes,
                              cudaStream_t stream) {
@@ -359,9 +359,10 @@ static qvla_status pack_impl(const float* W, int N, int K, int block, const int3
   q.xr = Wr;
   q.rows = N;
   q.K = K;
-  q.qmin = -7;
-  q.qmax = 7;
+  q.qmin = bits == 8 ? -127 : -7;
+  q.qmax = bits == 8 ? 127 : 7;
   q.dynamic = 1;
+  q.bits = bits;
   q.q_out = wq_out;
   q.s_out = w_scale_out;
   if (launch_quant_rows(q, stream) != cudaSuccess) return QVLA_ERR_CUDA;
@@ -374,16 +375,24 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
                               const double* rsvd_in, int32_t* perm_out, float* rot_out,
                               uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
                               void* workspace, size_t ws_bytes, cudaStream_t stream) {
-  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, perm_out, rot_out, rot_tc_out, wq_out,
-                   w_scale_out, workspace, ws_bytes, stream);
+  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, 4, perm_out, rot_out, rot_tc_out,
+                   wq_out, w_scale_out, workspace, ws_bytes, stream);
+}
+
+qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const int32_t* perm_in,
+                                 const double* rsvd_in, int32_t* perm_out, float* rot_out,
+                                 uint8_t* wq_out, float* w_scale_out, void* workspace,
+                                 size_t ws_bytes, cudaStream_t stream) {
+  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, 8, perm_out, rot_out, nullptr,
+                   wq_out, w_scale_out, workspace, ws_bytes, stream);
 }
 
 qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
                                        const int32_t* perm_in, int32_t* perm_out, uint8_t* wq_out,
                                        float* w_scale_out, void* workspace, size_t ws_bytes,
                                        cudaStream_t stream) {
-  return pack_impl(W, N, K, block, perm_in, nullptr, true, perm_out, nullptr, nullptr, wq_out,
-                   w_scale_out, workspace, ws_bytes, stream);
+  return pack_impl(W, N, K, block, perm_in, nullptr, true, 4, perm_out, nullptr, nullptr,
+                   wq_out, w_scale_out, workspace, ws_bytes, stream);
 }
 
 // Validates one rotate-quantise call and fills its launch arguments.
@@ -520,6 +529,40 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
   return cuda_status(launch_rotate_quant_batch(v.data(), n, stream));
 }
 
+qvla_status qvla_rotate_quant_a8_workspace_bytes(int M, int K, size_t* bytes) {
+  if (!bytes) return QVLA_ERR_ARG;
+  if (M < 0 || K <= 0 || K > QVLA_MAX_K) return QVLA_ERR_SHAPE;
+  *bytes = static_cast<size_t>(M) * K * 4;
+  return QVLA_OK;
+}
+
+qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int ldx,
+                                     const qvla_packed_linear* L, int8_t* xq8, float* s_x,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  qvla_status st = check_linear(L, false);
+  if (st != QVLA_OK) return st;
+  if (M < 0) return QVLA_ERR_SHAPE;
+  if (M == 0) return QVLA_OK;
+  if (!xq8 || !s_x) return QVLA_ERR_ARG;
+  if (!aligned16(xq8) || !aligned16(s_x)) return QVLA_ERR_ALIGN;
+  if (!workspace || ws_bytes < static_cast<size_t>(M) * L->K * 4) return QVLA_ERR_WORKSPACE;
+  float* xr = static_cast<float*>(workspace);
+  // 1. the rotation (fp32 x' into the workspace)
+  if ((st = qvla_rotate_act_f32(x, xdt, M, ldx, L, xr, stream)) != QVLA_OK) return st;
+  // 2. per-token dynamic 8-bit RTN
+  QuantArgs q = {};
+  q.xr = xr;
+  q.rows = M;
+  q.K = L->K;
+  q.qmin = -128;
+  q.qmax = 127;
+  q.dynamic = 1;
+  q.bits = 8;
+  q.q_out = reinterpret_cast<uint8_t*>(xq8);
+  q.s_out = s_x;
+  return cuda_status(launch_quant_rows(q, stream));
+}
+
 qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
                                 const qvla_packed_linear* L, float* xr_out, cudaStream_t stream) {
   qvla_status st = check_linear(L, false);
@@ -648,6 +691,28 @@ qvla_status qvla_w4a4_gemm_batched(const qvla_linear_problem* probs, int n, int 
   qvla_status st = check_sm100();
   if (st != QVLA_OK) return st;
   return cuda_status(launch_w4a4_gemm_batch(v.data(), n, split_k, stream));
+}
+
+static qvla_status w8a8_common(const int8_t* xq8, const float* s_x, int M,
+                               const qvla_packed_linear* L, void* y, int ldy, int32_t* acc,
+                               cudaStream_t stream) {
+  GemmArgs g;
+  qvla_status st = prepare_gemm(reinterpret_cast<const uint8_t*>(xq8), s_x, M, L, y, ldy, acc, 0,
+                                &g);
+  if (st != QVLA_OK || M == 0) return st;
+  if ((st = check_sm100()) != QVLA_OK) return st;
+  return cuda_status(launch_w8a8_gemm(g, stream));
+}
+
+qvla_status qvla_w8a8_gemm(const int8_t* xq8, const float* s_x, int M,
+                           const qvla_packed_linear* L, void* y, int ldy, cudaStream_t stream) {
+  if (M > 0 && !y) return QVLA_ERR_ARG;
+  return w8a8_common(xq8, s_x, M, L, y, ldy, nullptr, stream);
+}
+
+qvla_status qvla_w8a8_gemm_s32(const int8_t* xq8, int M, const qvla_packed_linear* L,
+                               int32_t* acc, cudaStream_t stream) {
+  return w8a8_common(xq8, nullptr, M, L, nullptr, 0, acc, stream);
 }
 
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,

@@ -49,8 +49,9 @@ struct QuantArgs {
   int T, Lcount;
   const int32_t* step_dev;
   int step_host, layer;
-  uint8_t* q_out;
+  uint8_t* q_out;          // [rows][K/2] packed 4-bit codes, or [rows][K] int8 when bits == 8
   float* s_out;
+  int bits;                // 4 (default when 0) or 8
 };
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream);
 
@@ -89,5 +90,8 @@ bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, ui
 // independent linears in as few launches as possible (grouped by token tile)
 cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream);
 int gemm_choose_split(int M, int N, int K);
+// W8A8 variant (gemm_w8a8.cu): int8 codes [M][K] and [N][K] straight into the
+// tensor cores (xq and wq hold one int8 code per byte; split_k is ignored)
+cudaError_t launch_w8a8_gemm(const GemmArgs& g, cudaStream_t stream);
 
 }  // namespace qvla

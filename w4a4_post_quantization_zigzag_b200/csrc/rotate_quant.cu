@@ -827,7 +827,7 @@ __global__ void __launch_bounds__(kThreads)
     quant_rows_kernel(const float* __restrict__ xr, int K, int qmin, int qmax, int dynamic,
                       const float* __restrict__ table, int T, int Lcount,
                       const int32_t* __restrict__ step_dev, int step_host, int layer,
-                      uint8_t* __restrict__ q_out, float* __restrict__ s_out,
+                      uint8_t* __restrict__ q_out, float* __restrict__ s_out, int bits,
                       unsigned int* err) {
   __shared__ float red[kWarps];
   __shared__ float s_sh;
@@ -850,6 +850,14 @@ __global__ void __launch_bounds__(kThreads)
   }
   cta_sync();
   const float s = s_sh;
+  if (bits == 8) {
+    // one int8 code per byte, decided by the IEEE fp32 division itself
+    int8_t* dst8 = reinterpret_cast<int8_t*>(q_out) + static_cast<size_t>(row) * K;
+    for (int j = tid; j < K; j += kThreads)
+      dst8[j] = static_cast<int8_t>(quant_code(src[j], s, qmin, qmax));
+    if (tid == 0) s_out[row] = s;
+    return;
+  }
   const float rs = quant_recip(s);
   uint8_t* dst = q_out + static_cast<size_t>(row) * (K / 2);
   for (int j = tid; j < K / 2; j += kThreads) {
@@ -1303,7 +1311,7 @@ cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream) {
   quant_rows_kernel<<<a.rows, kThreads, 0, stream>>>(a.xr, a.K, a.qmin, a.qmax, a.dynamic,
                                                      a.table, a.T, a.Lcount, a.step_dev,
                                                      a.step_host, a.layer, a.q_out, a.s_out,
-                                                     device_error_word());
+                                                     a.bits == 8 ? 8 : 4, device_error_word());
   return cudaGetLastError();
 }
 

@@ -50,7 +50,8 @@ EXPORTED = (
     "qvla_rotate_quant_act", "qvla_rotate_act_f32", "qvla_quant_act_f32", "qvla_w4a4_gemm",
     "qvla_w4a4_gemm_s32", "qvla_rotate_quant_act_batched", "qvla_w4a4_gemm_batched",
     "qvla_rotate_quant_workspace_bytes", "qvla_rotate_quant_act_noalloc",
-    "qvla_pack_weights_hadamard",
+    "qvla_pack_weights_hadamard", "qvla_pack_weights_w8", "qvla_rotate_quant_act_a8",
+    "qvla_rotate_quant_a8_workspace_bytes", "qvla_w8a8_gemm", "qvla_w8a8_gemm_s32",
 )
 
 QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -84,6 +85,13 @@ _sig = {
                                   c_void_p]),
     "qvla_pack_weights_hadamard": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qvla_pack_weights_w8": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qvla_rotate_quant_act_a8": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_void_p, c_void_p,
+                                         c_void_p, c_size_t, c_void_p]),
+    "qvla_rotate_quant_a8_workspace_bytes": (c_int, [c_int, c_int, POINTER(c_size_t)]),
+    "qvla_w8a8_gemm": (c_int, [c_void_p, c_void_p, c_int, _P, c_void_p, c_int, c_void_p]),
+    "qvla_w8a8_gemm_s32": (c_int, [c_void_p, c_int, _P, c_void_p, c_void_p]),
     "qvla_rotate_weights_f32": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
     "qvla_quant_pack_weights_f32": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p,
@@ -234,6 +242,74 @@ def qvla_pack_weights_hadamard(W: torch.Tensor, block: int, bias: Optional[torch
         assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
         bias = bias.contiguous()
     return PackedLinear(N, K, block, perm, None, wq, s_w, bias, rot_tc=None)
+
+
+def qvla_pack_weights_w8(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
+                         perm_in: Optional[np.ndarray] = None,
+                         rsvd_in: Optional[np.ndarray] = None, stream=None) -> PackedLinear:
+    """W8A8 variant: the same P and R, int8 weight codes wq [N, K]."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    _, rot_b, _, ws_b = qvla_packed_sizes(N, K, block)
+    dev = W.device
+    perm = torch.empty(K, dtype=torch.int32, device=dev)
+    rot = torch.empty(rot_b // 4, dtype=torch.float32, device=dev)
+    wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    p_in = r_in = None
+    if perm_in is not None:
+        perm_in = np.ascontiguousarray(perm_in, dtype=np.int32)
+        assert perm_in.shape == (K,)
+        p_in = perm_in.ctypes.data_as(c_void_p)
+    if rsvd_in is not None:
+        rsvd_in = np.ascontiguousarray(rsvd_in, dtype=np.float64)
+        assert rsvd_in.shape == (K // block, block, block)
+        r_in = rsvd_in.ctypes.data_as(c_void_p)
+    _check(_lib.qvla_pack_weights_w8(_ptr(W), N, K, block, p_in, r_in, _ptr(perm), _ptr(rot),
+                                     _ptr(wq), _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
+           "qvla_pack_weights_w8")
+    if bias is not None:
+        assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
+        bias = bias.contiguous()
+    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias)
+
+
+def qvla_rotate_quant_act_a8(x: torch.Tensor, L: PackedLinear,
+                             xq8: Optional[torch.Tensor] = None,
+                             s_x: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None):
+    """8-bit per-token dynamic codes xq8 [M, K] int8 and s_x [M]."""
+    M = x.shape[0]
+    if xq8 is None:
+        xq8 = torch.empty(M, L.K, dtype=torch.int8, device=x.device)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(M * L.K * 4, 16), dtype=torch.uint8, device=x.device)
+    _check(_lib.qvla_rotate_quant_act_a8(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct,
+                                         _ptr(xq8), _ptr(s_x), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)), "qvla_rotate_quant_act_a8")
+    return xq8, s_x
+
+
+def qvla_w8a8_gemm(xq8: torch.Tensor, s_x: torch.Tensor, L: PackedLinear,
+                   y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M = xq8.shape[0]
+    if y is None:
+        y = torch.empty(M, L.N, dtype=torch.bfloat16, device=xq8.device)
+    _check(_lib.qvla_w8a8_gemm(_ptr(xq8), _ptr(s_x), M, L.struct, _ptr(y), y.stride(0),
+                               _stream(stream)), "qvla_w8a8_gemm")
+    return y
+
+
+def qvla_w8a8_gemm_s32(xq8: torch.Tensor, L: PackedLinear, stream=None) -> torch.Tensor:
+    M = xq8.shape[0]
+    acc = torch.empty(M, L.N, dtype=torch.int32, device=xq8.device)
+    _check(_lib.qvla_w8a8_gemm_s32(_ptr(xq8), M, L.struct, _ptr(acc), _stream(stream)),
+           "qvla_w8a8_gemm_s32")
+    return acc
 
 
 def qvla_rotate_weights_f32(W: torch.Tensor, block: int, perm: torch.Tensor,
