@@ -304,6 +304,78 @@ def pack_linear(W: np.ndarray, block: int, bias=None, perm=None, rsvd=None,
     return PackedLinear(perm, rsvd, R, Wr, qw, s_w, bias, bits)
 
 
+# --------------------------------------------------------------------------
+# GPTQ weight rounding (the pages' LLM pack: "build_gptq_weights" with the
+# composite rotation, 4-bit weights, block 128, damping 0.05): an alternative
+# to round-to-nearest that quantises the rotated weight columns one at a time
+# and moves each column's rounding error onto the columns not yet quantised,
+# weighted by the inverse Hessian of the layer's calibration inputs.
+# --------------------------------------------------------------------------
+
+def gptq_hessian(xr_cal: np.ndarray) -> np.ndarray:
+    """H = X'^T X' (K x K, double) of rotated calibration activations [T, K]."""
+    X = np.asarray(xr_cal, dtype=np.float64)
+    return X.T @ X
+
+
+def gptq_inverse_factor(H: np.ndarray, damp: float = 0.05):
+    """The upper Cholesky factor U of (H + damp * mean(diag H) * I)^-1 (so that
+    U^T U is that inverse), after giving dead inputs (H[i,i] == 0) a unit
+    diagonal.  Returns (U, dead)."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    dead = np.diag(H) == 0
+    H[dead, dead] = 1.0
+    K = H.shape[0]
+    H[np.arange(K), np.arange(K)] += damp * np.mean(np.diag(H))
+    Hinv = np.linalg.inv(H)
+    # upper factor: Hinv = U^T U  <=>  U = L^T with Hinv = L L^T
+    U = np.linalg.cholesky(Hinv).T
+    return U, dead
+
+
+def gptq_quantize(Wr32: np.ndarray, U: np.ndarray, dead=None, qmax: int = WEIGHT_QMAX):
+    """GPTQ rounding of fp32 rotated weights [N, K] with the inverse factor U.
+
+    The per-row scale is the RTN one, s = fp32(max |W'[n,:]| / qmax).  Column
+    by column, in order: q = clamp(rint(w / s), -qmax, qmax) in double, the
+    error e = (w - q s) / U[j, j], and every later column k takes
+    w_k -= e * U[j, k] (the block size of the pages only groups these updates
+    and leaves the result unchanged).  Returns (codes int8 [N, K], s fp32 [N])."""
+    W = np.asarray(Wr32, dtype=np.float32)
+    s = np.divide(np.max(np.abs(W), axis=1), np.float32(qmax), dtype=np.float32)
+    Wc = W.astype(np.float64)
+    if dead is not None:
+        Wc[:, np.asarray(dead, bool)] = 0.0
+    s64 = s.astype(np.float64)
+    safe = np.where(s64 == 0, 1.0, s64)
+    N, K = Wc.shape
+    Q = np.zeros((N, K), dtype=np.int8)
+    for j in range(K):
+        w = Wc[:, j]
+        q = np.where(s64 == 0, 0.0, np.clip(np.rint(w / safe), -qmax, qmax))
+        Q[:, j] = q.astype(np.int8)
+        e = (w - q * s64) / U[j, j]
+        if j + 1 < K:
+            Wc[:, j + 1:] -= e[:, None] * U[j, j + 1:][None, :]
+    return Q, s
+
+
+def pack_linear_gptq(W: np.ndarray, block: int, x_cal: np.ndarray, bias=None, perm=None,
+                     rsvd=None, damp: float = 0.05, U=None) -> PackedLinear:
+    """Offline pack with GPTQ rounding: zigzag P and composite R as
+    pack_linear, the Hessian from the rotated calibration activations, codes
+    by gptq_quantize.  `U` may be given (the inverse factor) to pin it."""
+    pk = pack_linear(W, block, bias=bias, perm=perm, rsvd=rsvd)
+    dead = None
+    if U is None:
+        xr = rotate_activations(np.asarray(x_cal, np.float64), pk.perm, pk.R)
+        U, dead = gptq_inverse_factor(gptq_hessian(xr), damp)
+    qw, s_w = gptq_quantize(pk.Wr.astype(np.float32), U, dead)
+    pk.qw, pk.s_w = qw, s_w
+    pk.U = U
+    return pk
+
+
 def rotate_quant_act(x: np.ndarray, pk: PackedLinear, mode: str = "dynamic",
                      table=None, step: int = 0, layer: int = 0):
     """Activation side in double, quantised like the fp32 path but from the

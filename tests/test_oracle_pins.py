@@ -307,6 +307,65 @@ def test_w8a8_layer_tracks_the_fp_layer_more_closely_than_w4a4():
     assert O.pack_linear(W, lin.block, bits=8).wq.shape == (lin.N, lin.K)
 
 
+# ------------------------------------------------------------------- GPTQ
+
+def test_gptq_with_an_identity_hessian_is_round_to_nearest():
+    """No correlation between inputs: the inverse factor is diagonal, no error
+    moves between columns, and GPTQ rounds like RTN."""
+    W = I.weights(40, 16, 64, n_outlier_rows=2).astype(np.float32)
+    U, dead = O.gptq_inverse_factor(np.eye(64), damp=0.05)
+    np.testing.assert_allclose(U, np.eye(64) / np.sqrt(1.05), rtol=1e-14, atol=0)
+    q, s = O.gptq_quantize(W, U, dead)
+    q_rtn, s_rtn = O.quantize_weights_fp32(W)
+    assert np.array_equal(s, s_rtn) and np.array_equal(q, q_rtn)
+
+
+def test_gptq_two_columns_by_hand():
+    """K = 2 written out: damped H, its inverse and that inverse's upper
+    Cholesky factor in closed form, then the two GPTQ steps."""
+    H = np.array([[2.0, 0.9], [0.9, 1.5]])
+    damp = 0.05
+    mean = (H[0, 0] + H[1, 1]) / 2
+    a, b, c = H[0, 0] + damp * mean, H[0, 1], H[1, 1] + damp * mean
+    det = a * c - b * b
+    i00, i01, i11 = c / det, -b / det, a / det            # inverse of [[a, b], [b, c]]
+    u00 = np.sqrt(i00)
+    u01 = i01 / u00
+    u11 = np.sqrt(i11 - u01 * u01)
+    U, _ = O.gptq_inverse_factor(H, damp)
+    np.testing.assert_allclose(U, [[u00, u01], [0.0, u11]], rtol=1e-13, atol=1e-15)
+    W = np.array([[0.70, -0.45], [0.10, 0.33], [-0.5, 0.5]], dtype=np.float32)
+    q, s = O.gptq_quantize(W, U)
+    for n in range(3):
+        sn = float(np.float32(np.float32(np.abs(W[n]).max()) / np.float32(7)))
+        w0, w1 = float(W[n, 0]), float(W[n, 1])
+        q0 = min(7, max(-7, round(w0 / sn)))               # Python round: half to even
+        e = (w0 - q0 * sn) / u00
+        q1 = min(7, max(-7, round((w1 - e * u01) / sn)))
+        assert (q[n, 0], q[n, 1]) == (q0, q1)
+
+
+def test_gptq_dead_input_column_is_zero():
+    W = I.weights(41, 8, 32).astype(np.float32)
+    X = I.activations(42, 40, 32, dtype="f32").astype(np.float64)
+    X[:, 5] = 0.0                                         # input 5 never active
+    U, dead = O.gptq_inverse_factor(O.gptq_hessian(X))
+    assert dead[5] and dead.sum() == 1
+    q, _ = O.gptq_quantize(W, U, dead)
+    assert not q[:, 5].any()
+
+
+def test_gptq_lowers_the_calibration_output_error():
+    W = I.weights(43, 128, 256, col_spread=10.0)
+    x = I.activations(44, 300, 256, n_outlier_cols=3, dtype="f32")
+    g = O.pack_linear_gptq(W, 64, x)
+    r = O.pack_linear(W, 64)
+    xr = O.rotate_activations(x.astype(np.float64), g.perm, g.R)
+    err = lambda pk: np.linalg.norm((pk.Wr - pk.qw * pk.s_w[:, None].astype(np.float64)) @ xr.T)
+    assert err(g) < 0.8 * err(r)
+    assert np.abs(g.qw).max() <= 7 and np.array_equal(g.s_w, r.s_w)
+
+
 def test_table_lookup_rejects_out_of_range():
     tab = np.ones((8, 3), np.float32)
     assert O.table_scale(tab, 7, 2) == 1.0
