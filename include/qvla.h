@@ -190,6 +190,49 @@ qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const 
                                  uint8_t* wq_out, float* w_scale_out, void* workspace,
                                  size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * GPTQ rounding of rotated weights ("Omega-QVLA: Nen VLA W4A4 tren Edge",
+ * "Build LLM pack": the LLM pack's 4-bit weights come from GPTQ on the
+ * composite-rotated weights, block 128, damping 0.05).  Host only, fp64.
+ *   H  = X'^T X' of the rotated calibration rows X' (K x K);
+ *   dead inputs (H[i][i] == 0) get H[i][i] = 1 and a zero weight column;
+ *   U  = upper Cholesky factor of (H + damp * mean(diag H) * I)^-1;
+ *   per row: s = fp32(max_k |W'[n,k]| / 7) (the RTN scale); for j = 0..K-1:
+ *     q_j = clamp(rint(w_j / s), -7, 7); e = (w_j - q_j s) / U[j][j];
+ *     w_k -= e U[j][k] for k > j.
+ * The pages' block size only groups the lazy updates; it does not change the
+ * result, and here every update is applied as its column is done.
+ *
+ * qvla_gptq_quantize_host: Wr host fp32 [N][K] (rotated weights W' = W P R);
+ * H host fp64 [K][K] (symmetric) or NULL when u_in is given; u_in host fp64
+ * [K][K] upper factor U (used as is; then H and damp are ignored) or NULL;
+ * q_out host int8 [N][K] codes in [-7, 7]; s_out host fp32 [N].  K <= 4096
+ * (QVLA_ERR_SHAPE otherwise: the work is K x K fp64 on the host);
+ * QVLA_ERR_ARG if a factorisation fails.  Synchronous, multithreaded.
+ * ------------------------------------------------------------------------- */
+qvla_status qvla_gptq_quantize_host(const float* Wr, int N, int K, const double* H, double damp,
+                                    const double* u_in, int8_t* q_out, float* s_out);
+
+/* H = X'^T X' in fp64 (K x K, row-major, symmetric) of the rotated
+ * calibration rows xr host fp32 [T][K], into H_out host fp64 [K][K] (the
+ * Hessian the GPTQ entry points factorise).  K <= 4096.  Synchronous.       */
+qvla_status qvla_gptq_hessian_host(const float* xr, int T, int K, double* H_out);
+
+/* Offline pack with GPTQ weights: as qvla_pack_weights() (same perm_in,
+ * rsvd_in, outputs, workspace and blocking behaviour), but wq_out and
+ * w_scale_out hold the GPTQ codes of W' instead of the RTN codes.  The
+ * calibration rows x_cal (device, xdt F32 or BF16, [T][K] dense) are
+ * rotated on the device with P and R (as qvla_rotate_act_f32(), into
+ * cal_workspace, >= T * K * 4 bytes) and H is formed on the host in fp64.
+ * u_in host fp64 [K][K] or NULL: a given U skips the calibration (x_cal,
+ * T and cal_workspace may then be NULL / 0).  damp >= 0.  K <= 4096.        */
+qvla_status qvla_pack_weights_gptq(const float* W, int N, int K, int block, const void* x_cal,
+                                   qvla_dtype xdt, int T, double damp, const int32_t* perm_in,
+                                   const double* rsvd_in, const double* u_in, int32_t* perm_out,
+                                   float* rot_out, uint16_t* rot_tc_out, uint8_t* wq_out,
+                                   float* w_scale_out, void* workspace, size_t ws_bytes,
+                                   void* cal_workspace, size_t cal_ws_bytes, cudaStream_t stream);
+
 /* W8A8 activations: the rotation of qvla_rotate_act_f32() into `workspace`
  * (fp32 [M][K], M * K * 4 bytes, see qvla_rotate_quant_a8_workspace_bytes),
  * then per-token dynamic 8-bit RTN: s_x[m] = fp32(max_k |x'[m,k]| / 127),

@@ -26,6 +26,7 @@ LIB = os.path.join(HERE, "libqvla.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
+         "-Xcompiler", "-ffp-contract=off",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]
 
 

@@ -379,6 +379,89 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
                    wq_out, w_scale_out, workspace, ws_bytes, stream);
 }
 
+qvla_status qvla_gptq_hessian_host(const float* xr, int T, int K, double* H_out) {
+  if (T <= 0 || K <= 0 || K > 4096) return QVLA_ERR_SHAPE;
+  if (!xr || !H_out) return QVLA_ERR_ARG;
+  std::vector<double> H;
+  gptq_hessian(xr, T, K, H);
+  std::memcpy(H_out, H.data(), H.size() * sizeof(double));
+  return QVLA_OK;
+}
+
+qvla_status qvla_gptq_quantize_host(const float* Wr, int N, int K, const double* H, double damp,
+                                    const double* u_in, int8_t* q_out, float* s_out) {
+  if (N <= 0 || K <= 0 || K > 4096) return QVLA_ERR_SHAPE;
+  if (!Wr || !q_out || !s_out || (!H && !u_in) || !(damp >= 0.0)) return QVLA_ERR_ARG;
+  std::vector<double> U;
+  std::vector<char> dead;
+  const double* u = u_in;
+  if (!u) {
+    if (!gptq_inverse_factor(H, K, damp, U, dead)) return QVLA_ERR_ARG;
+    u = U.data();
+  }
+  gptq_quantize_rows(Wr, N, K, u, dead.empty() ? nullptr : dead.data(), 7, q_out, s_out);
+  return QVLA_OK;
+}
+
+qvla_status qvla_pack_weights_gptq(const float* W, int N, int K, int block, const void* x_cal,
+                                   qvla_dtype xdt, int T, double damp, const int32_t* perm_in,
+                                   const double* rsvd_in, const double* u_in, int32_t* perm_out,
+                                   float* rot_out, uint16_t* rot_tc_out, uint8_t* wq_out,
+                                   float* w_scale_out, void* workspace, size_t ws_bytes,
+                                   void* cal_workspace, size_t cal_ws_bytes,
+                                   cudaStream_t stream) {
+  if (K > 4096) return QVLA_ERR_SHAPE;                 // fp64 K x K work on the host
+  if (!u_in) {
+    if (!x_cal || T <= 0 || (xdt != QVLA_DTYPE_F32 && xdt != QVLA_DTYPE_BF16))
+      return QVLA_ERR_ARG;
+    if (!cal_workspace || cal_ws_bytes < static_cast<size_t>(T) * K * 4) return QVLA_ERR_WORKSPACE;
+  }
+  // 1. permutation, R_SVD, rotated weights (and RTN codes, replaced below)
+  qvla_status st = pack_impl(W, N, K, block, perm_in, rsvd_in, false, 4, perm_out, rot_out,
+                             rot_tc_out, wq_out, w_scale_out, workspace, ws_bytes, stream);
+  if (st != QVLA_OK) return st;
+  const int nb = K / block;
+  const size_t bb = static_cast<size_t>(block) * block;
+  const size_t off = (static_cast<size_t>(K) * 8 + 2 * nb * bb * 8 + 255) & ~static_cast<size_t>(255);
+  std::vector<float> Wr(static_cast<size_t>(N) * K);
+  if (cudaStreamSynchronize(stream) != cudaSuccess ||
+      cudaMemcpy(Wr.data(), static_cast<uint8_t*>(workspace) + off, Wr.size() * 4,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+  // 2. the inverse factor of the damped Hessian of the rotated calibration rows
+  std::vector<double> U;
+  std::vector<char> dead;
+  const double* u = u_in;
+  if (!u) {
+    qvla_packed_linear Lc = {N, K, block, perm_out, rot_out, nullptr, wq_out, w_scale_out, nullptr};
+    float* xr_dev = static_cast<float*>(cal_workspace);
+    if ((st = qvla_rotate_act_f32(x_cal, xdt, T, K, &Lc, xr_dev, stream)) != QVLA_OK) return st;
+    std::vector<float> xr(static_cast<size_t>(T) * K);
+    if (cudaStreamSynchronize(stream) != cudaSuccess ||
+        cudaMemcpy(xr.data(), xr_dev, xr.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return QVLA_ERR_CUDA;
+    std::vector<double> H;
+    gptq_hessian(xr.data(), T, K, H);
+    if (!gptq_inverse_factor(H.data(), K, damp, U, dead)) return QVLA_ERR_ARG;
+    u = U.data();
+  }
+  // 3. GPTQ codes, packed two per byte
+  std::vector<int8_t> q(static_cast<size_t>(N) * K);
+  std::vector<float> s(N);
+  gptq_quantize_rows(Wr.data(), N, K, u, dead.empty() ? nullptr : dead.data(), 7, q.data(),
+                     s.data());
+  std::vector<uint8_t> packed(static_cast<size_t>(N) * K / 2);
+  for (size_t i = 0; i < packed.size(); ++i)
+    packed[i] = static_cast<uint8_t>((q[2 * i] & 15) | ((q[2 * i + 1] & 15) << 4));
+  if (cudaMemcpyAsync(wq_out, packed.data(), packed.size(), cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(w_scale_out, s.data(), s.size() * 4, cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return QVLA_ERR_CUDA;
+  return QVLA_OK;
+}
+
 qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const int32_t* perm_in,
                                  const double* rsvd_in, int32_t* perm_out, float* rot_out,
                                  uint8_t* wq_out, float* w_scale_out, void* workspace,

@@ -4,6 +4,8 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <vector>
 #include <stdint.h>
 
 #include "../../include/qvla.h"
@@ -54,6 +56,19 @@ struct QuantArgs {
   int bits;                // 4 (default when 0) or 8
 };
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream);
+
+// ---- GPTQ rounding on the host (gptq_host.cu)
+// H = X'^T X' (fp64, K x K) of T rotated calibration rows xr [T][K].
+void gptq_hessian(const float* xr, int T, int K, std::vector<double>& H);
+// U = upper Cholesky factor of (H + damp * mean(diag H) * I)^-1 after giving
+// dead inputs (H[i][i] == 0, flagged in `dead`) a unit diagonal; false if a
+// factorisation fails.
+bool gptq_inverse_factor(const double* H, int K, double damp, std::vector<double>& U,
+                         std::vector<char>& dead);
+// codes [N][K] (one int8 each) and fp32 scales [N] of fp32 rotated weights;
+// `dead` may be null.
+void gptq_quantize_rows(const float* Wr, int N, int K, const double* U, const char* dead, int qmax,
+                        int8_t* q, float* s);
 
 // ---- pack helpers (pack_kernels.cu)
 cudaError_t launch_column_norms(const float* W, int N, int K, double* norms, cudaStream_t s);

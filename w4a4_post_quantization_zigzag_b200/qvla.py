@@ -52,6 +52,7 @@ EXPORTED = (
     "qvla_rotate_quant_workspace_bytes", "qvla_rotate_quant_act_noalloc",
     "qvla_pack_weights_hadamard", "qvla_pack_weights_w8", "qvla_rotate_quant_act_a8",
     "qvla_rotate_quant_a8_workspace_bytes", "qvla_w8a8_gemm", "qvla_w8a8_gemm_s32",
+    "qvla_gptq_quantize_host", "qvla_pack_weights_gptq", "qvla_gptq_hessian_host",
 )
 
 QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -87,6 +88,13 @@ _sig = {
                                            c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qvla_pack_weights_w8": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qvla_gptq_hessian_host": (c_int, [c_void_p, c_int, c_int, c_void_p]),
+    "qvla_gptq_quantize_host": (c_int, [c_void_p, c_int, c_int, c_void_p, ctypes.c_double,
+                                        c_void_p, c_void_p, c_void_p]),
+    "qvla_pack_weights_gptq": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_int,
+                                       ctypes.c_double, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                       c_void_p, c_size_t, c_void_p]),
     "qvla_rotate_quant_act_a8": (c_int, [c_void_p, c_int, c_int, c_int, _P, c_void_p, c_void_p,
                                          c_void_p, c_size_t, c_void_p]),
     "qvla_rotate_quant_a8_workspace_bytes": (c_int, [c_int, c_int, POINTER(c_size_t)]),
@@ -242,6 +250,81 @@ def qvla_pack_weights_hadamard(W: torch.Tensor, block: int, bias: Optional[torch
         assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
         bias = bias.contiguous()
     return PackedLinear(N, K, block, perm, None, wq, s_w, bias, rot_tc=None)
+
+
+def _host_f64(a, shape):
+    if a is None:
+        return None, None
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    assert a.shape == shape
+    return a, a.ctypes.data_as(c_void_p)
+
+
+def qvla_gptq_hessian_host(xr: np.ndarray) -> np.ndarray:
+    """H = X'^T X' (fp64 [K, K]) of host fp32 rotated calibration rows [T, K]."""
+    xr = np.ascontiguousarray(xr, dtype=np.float32)
+    T, K = xr.shape
+    H = np.empty((K, K), np.float64)
+    _check(_lib.qvla_gptq_hessian_host(xr.ctypes.data_as(c_void_p), T, K,
+                                       H.ctypes.data_as(c_void_p)), "qvla_gptq_hessian_host")
+    return H
+
+
+def qvla_gptq_quantize_host(Wr: np.ndarray, H: Optional[np.ndarray] = None, damp: float = 0.05,
+                            U: Optional[np.ndarray] = None):
+    """GPTQ codes of host fp32 rotated weights Wr [N, K]; returns (int8 [N, K], fp32 [N])."""
+    Wr = np.ascontiguousarray(Wr, dtype=np.float32)
+    N, K = Wr.shape
+    H, h_p = _host_f64(H, (K, K))
+    U, u_p = _host_f64(U, (K, K))
+    q = np.empty((N, K), np.int8)
+    s = np.empty(N, np.float32)
+    _check(_lib.qvla_gptq_quantize_host(Wr.ctypes.data_as(c_void_p), N, K, h_p, float(damp), u_p,
+                                        q.ctypes.data_as(c_void_p), s.ctypes.data_as(c_void_p)),
+           "qvla_gptq_quantize_host")
+    return q, s
+
+
+def qvla_pack_weights_gptq(W: torch.Tensor, block: int, x_cal: Optional[torch.Tensor] = None,
+                           damp: float = 0.05, bias: Optional[torch.Tensor] = None,
+                           perm_in: Optional[np.ndarray] = None,
+                           rsvd_in: Optional[np.ndarray] = None, U: Optional[np.ndarray] = None,
+                           stream=None) -> PackedLinear:
+    """As qvla_pack_weights, with GPTQ weight codes (calibration rows x_cal [T, K] on the device,
+    fp32 or bf16, or a given inverse-Hessian factor U)."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    wq_b, rot_b, tc_b, ws_b = qvla_packed_sizes(N, K, block)
+    dev = W.device
+    perm = torch.empty(K, dtype=torch.int32, device=dev)
+    rot = torch.empty(rot_b // 4, dtype=torch.float32, device=dev)
+    rot_tc = torch.empty(tc_b // 2, dtype=torch.int16, device=dev) if tc_b else None
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    p_in = None
+    if perm_in is not None:
+        perm_in = np.ascontiguousarray(perm_in, dtype=np.int32)
+        assert perm_in.shape == (K,)
+        p_in = perm_in.ctypes.data_as(c_void_p)
+    rsvd_in, r_in = _host_f64(rsvd_in, (K // block, block, block))
+    U, u_p = _host_f64(U, (K, K))
+    T, xdt, cal, cal_b = 0, QVLA_DTYPE_F32, None, 0
+    if x_cal is not None:
+        assert x_cal.is_cuda and x_cal.is_contiguous() and x_cal.dim() == 2 and x_cal.shape[1] == K
+        xdt = _dtype_code(x_cal)
+        T = x_cal.shape[0]
+        cal = torch.empty(T * K, dtype=torch.float32, device=dev)
+        cal_b = T * K * 4
+    _check(_lib.qvla_pack_weights_gptq(_ptr(W), N, K, block, _ptr(x_cal), xdt, T, float(damp),
+                                       p_in, r_in, u_p, _ptr(perm), _ptr(rot), _ptr(rot_tc),
+                                       _ptr(wq), _ptr(s_w), _ptr(ws), ws_b, _ptr(cal), cal_b,
+                                       _stream(stream)), "qvla_pack_weights_gptq")
+    if bias is not None:
+        assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
+        bias = bias.contiguous()
+    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias,
+                        rot_tc=rot_tc)
 
 
 def qvla_pack_weights_w8(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
