@@ -285,7 +285,9 @@ qvla_status qvla_quant_pack_weights_f32(const float* Wr, int N, int K, uint8_t* 
  *         rot_tc image the rotation runs on the tensor cores as one dense
  *         product with R_B = R_SVD,B . H_b (three bf16 parts, fp32
  *         accumulation in tensor memory); otherwise on the CUDA cores as the
- *         R_SVD product followed by the fast Walsh-Hadamard transform.
+ *         R_SVD product followed by the fast Walsh-Hadamard transform
+ *         (fp32 input at block 64 in TABLE mode: one dense product with the
+ *         fp32 sum of the image's three parts).
  * table   device fp32 [T][Lcount], required for TABLE mode.
  * step_dev device int32 or NULL.  If non-NULL the step is read on the device
  *         (so one captured graph serves every denoising step); a step outside
@@ -303,9 +305,9 @@ qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
                                   int step_host, int layer, uint8_t* xq, float* s_x,
                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Scratch that lets qvla_rotate_quant_act take its fastest route for large M
+/* Scratch that lets qvla_rotate_quant_act take its fastest route
  * (tensor-core rotation fed by TMA from a permuted copy of x): M * K * 2 bytes
- * when that route applies (bf16 input, block 64 or 128, M > 64), else 0.
+ * when that route applies (bf16 input, block 64 or 128, M > 0), else 0.
  * Without it (workspace NULL or too small) the call still works, gathering
  * the permuted inputs directly.  The scratch is only used while the call's
  * kernels run; reusing it for another call on the same stream is safe.     */

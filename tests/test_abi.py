@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -93,9 +94,11 @@ def test_argument_errors_before_any_cuda_call():
     # empty input is a no-op
     assert lib.qvla_rotate_quant_act(None, 1, 0, 256, ctypes.byref(Lok), 0, None, 0, 0, None, 0,
                                      0, None, None, None, 0, None) == q.QVLA_OK
-    # scratch size query: only the tensor-core route for more than 64 bf16 tokens uses it
+    # scratch size query: the tensor-core route (bf16, block 64 / 128) uses it
     assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 128) == 1024 * 2048 * 2
-    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64) == 0
+    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64) == 50 * 2048 * 2
+    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64, torch.float32) == 0
+    assert q.qvla_rotate_quant_workspace_bytes(0, 2048, 64) == 0
     assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 256) == 0
     assert lib.qvla_w4a4_gemm_s32(None, 0, ctypes.byref(Lok), None, 0, None) == q.QVLA_OK
     # split-K factor must be a power of two <= 16 and <= the number of 256-wide K tiles

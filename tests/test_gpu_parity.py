@@ -149,8 +149,10 @@ def test_pack_parity(q, N, K, b):
 
 @pytest.fixture(params=["auto", "fma"])
 def path(request, monkeypatch):
-    """auto: tensor cores where the linear has an image (bf16, block 64/128);
-    fma: always the CUDA-core rotation."""
+    """auto: tensor cores where the linear has an image (bf16, block 64/128),
+    else the CUDA-core kernels (the composite-R_B one for fp32 input at block
+    64 in table / rotate-only mode); fma: always the R_SVD + Walsh-Hadamard
+    CUDA-core kernel."""
     monkeypatch.setenv("QVLA_ROTATE_PATH", request.param)
     return request.param
 
@@ -183,7 +185,9 @@ def test_tc_image_is_the_composite_rotation(q, K, b):
 @pytest.mark.parametrize("M,K,b,dt", [(16, 256, 64, "f32"), (50, 1024, 64, "bf16"),
                                       (5, 2048, 128, "bf16"), (3, 512, 32, "bf16"),
                                       (9, 1024, 256, "bf16"), (2, 16384, 128, "bf16"),
-                                      (300, 1024, 64, "bf16"), (130, 512, 128, "bf16")])
+                                      (300, 1024, 64, "bf16"), (130, 512, 128, "bf16"),
+                                      (33, 512, 64, "f32"), (100, 1024, 64, "f32"),
+                                      (1, 4096, 64, "bf16")])
 def test_rotation_fp32_vs_fp64(q, path, M, K, b, dt):
     W = I.weights(400 + K, 64, K)
     ref = O.pack_linear(W, b)
@@ -200,7 +204,8 @@ def test_rotation_fp32_vs_fp64(q, path, M, K, b, dt):
     (50, 4096, 64, "bf16", "table"), (37, 2048, 128, "bf16", "dynamic"),
     (8, 1024, 32, "bf16", "dynamic"), (8, 1024, 256, "bf16", "table"),
     (3, 16384, 128, "bf16", "dynamic"), (300, 2048, 64, "bf16", "dynamic"),
-    (257, 1536, 64, "bf16", "table"), (200, 4096, 128, "bf16", "table")])
+    (257, 1536, 64, "bf16", "table"), (200, 4096, 128, "bf16", "table"),
+    (1, 256, 64, "bf16", "table"), (33, 512, 64, "f32", "table"), (100, 1024, 64, "f32", "table")])
 @pytest.mark.parametrize("scratch", [False, True])
 def test_rotate_quant_end_to_end(q, path, scratch, M, K, b, dt, mode):
     """scratch=True gives the call its workspace, which routes large bf16 inputs

@@ -536,7 +536,7 @@ qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtyp
                                               size_t* bytes) {
   if (!bytes) return QVLA_ERR_ARG;
   if (M < 0 || K <= 0 || K > QVLA_MAX_K || !valid_block(block) || K % block) return QVLA_ERR_SHAPE;
-  const bool tc = xdt == QVLA_DTYPE_BF16 && (block == 64 || block == 128) && M > 64;
+  const bool tc = xdt == QVLA_DTYPE_BF16 && (block == 64 || block == 128) && M > 0;
   *bytes = tc ? static_cast<size_t>(M) * K * 2 : 0;
   return QVLA_OK;
 }

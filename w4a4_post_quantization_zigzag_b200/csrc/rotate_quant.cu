@@ -472,6 +472,142 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ===========================================================================
+// Composite CUDA-core path (block 64, TABLE and rotate-only modes, a linear
+// that carries the tensor-core image of R_B, input the tensor-core route does
+// not take: fp32).
+//
+// x'_B = x_B . R_B with the composite R_B = R_SVD,B . H_b itself: the image's
+// three bf16 parts are summed in fp32 ((hi + mid) + lo, within one fp32 ulp
+// of R_B), so no Walsh-Hadamard step follows the product.  One CTA = 32
+// tokens x one rotation block at a time, 128 threads, each holding a
+// 4-channel x 4-token register tile (16 fp32 FMA per two 16-byte shared
+// loads); codes are formed and stored straight from the registers.
+// ===========================================================================
+constexpr int kCThreads = 128;
+constexpr int kCBS = 64;
+constexpr int kCTT = 32;
+
+QVLA_DEVICE void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+
+template <typename Tin, int MODE>
+__global__ void __launch_bounds__(kCThreads)
+    rotq_comp_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
+  __shared__ __align__(16) float comp[kCBS * kCBS];     // R_B[i][j], input-major, swizzled
+  __shared__ __align__(16) float xg[kCBS * kCTT];       // x[t][perm[i]] at [i][t]
+  __shared__ int32_t perm_s[kCBS];
+
+  int pi = 0;
+  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[pi + 1]) ++pi;
+  const ActProblem& P = batch.p[pi];
+  const Tin* __restrict__ x = static_cast<const Tin*>(P.x);
+  const int M = P.M, ldx = P.ldx, K = P.K;
+  const int local = static_cast<int>(blockIdx.x) - batch.cta_start[pi];
+  const int tile = local % P.gx;
+  const int group = local / P.gx;
+  const int m0 = tile * kCTT;
+  const int ntok = min(kCTT, M - m0);
+  const int nb = K / kCBS;
+  const int B0 = group * P.bpc;
+  const int nbc = max(0, min(P.bpc, nb - B0));
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j0 = (warp & 1) * 32 + (lane & 7) * 4;      // four output channels
+  const int t0 = (warp >> 1) * 16 + (lane >> 3) * 4;    // four tokens
+
+  float s_tab = 0.f;
+  for (int bl = 0; bl < nbc; ++bl) {
+    const int B = B0 + bl;
+    // 1. R_B from the image (weights: for the first block this runs before
+    // the wait on the previous kernel).  A 16-byte chunk q of part sp holds
+    // inputs 8c..8c+7 of output j = q / 8, c = (q % 8) ^ (j % 8); a warp
+    // reads 32 consecutive chunks.  R_B[i][j] lands in row i at the 4-float
+    // granule (j / 4) ^ (i / 8 % 8): the transposing stores of a warp and the
+    // product's 16-byte reads both hit 32 different banks.
+    const uint4* img = reinterpret_cast<const uint4*>(P.rot_tc + static_cast<size_t>(B) * 3 * kCBS * kCBS);
+#pragma unroll
+    for (int q = tid; q < kCBS * 8; q += kCThreads) {
+      const int j = q >> 3, c = (q & 7) ^ (j & 7);
+      const int col = 4 * ((j >> 2) ^ c) + (j & 3);
+      const uint4 h = __ldg(img + q), m = __ldg(img + 512 + q), l = __ldg(img + 1024 + q);
+      const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, mw[4] = {m.x, m.y, m.z, m.w},
+                     lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float h0, h1, m0f, m1f, l0, l1;
+        bf16x2_to_f32(hw[k], h0, h1);
+        bf16x2_to_f32(mw[k], m0f, m1f);
+        bf16x2_to_f32(lw[k], l0, l1);
+        comp[(8 * c + 2 * k) * kCBS + col] = (h0 + m0f) + l0;
+        comp[(8 * c + 2 * k + 1) * kCBS + col] = (h1 + m1f) + l1;
+      }
+    }
+    if (tid < kCBS) perm_s[tid] = __ldg(P.perm + static_cast<size_t>(B) * kCBS + tid);
+    if (bl == 0) {
+      pdl_wait();
+      pdl_launch_dependents();
+      if (MODE == kTable)
+        s_tab = table_scale(P.table, P.T, P.Lcount, P.step_dev, P.step_host, P.layer, err);
+    }
+    cta_sync();   // perm_s and comp complete
+    // 2. gather the block's inputs, token-contiguous
+#pragma unroll
+    for (int e = tid; e < kCBS * kCTT; e += kCThreads) {
+      const int i = e / kCTT, t = e % kCTT;
+      const int p = perm_s[i];
+      float v = 0.f;
+      if (t < ntok && static_cast<unsigned>(p) < static_cast<unsigned>(K))
+        v = load_x(x + static_cast<size_t>(m0 + t) * ldx + p);
+      xg[e] = v;
+    }
+    cta_sync();
+    // 3. acc[u][c] = sum_i x[t0 + u][i] R_B[i][j0 + c], in input order
+    float acc[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[u][c] = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < kCBS; ++i) {
+      const float4 r = *reinterpret_cast<const float4*>(comp + i * kCBS + 4 * ((j0 >> 2) ^ ((i >> 3) & 7)));
+      const float4 xv = *reinterpret_cast<const float4*>(xg + i * kCTT + t0);
+      const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[u][0] = fmaf(xs[u], r.x, acc[u][0]);
+        acc[u][1] = fmaf(xs[u], r.y, acc[u][1]);
+        acc[u][2] = fmaf(xs[u], r.z, acc[u][2]);
+        acc[u][3] = fmaf(xs[u], r.w, acc[u][3]);
+      }
+    }
+    // 4. codes (or rotated values) straight from the registers
+    if (MODE == kRotateOnly) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (t0 + u < ntok)
+          *reinterpret_cast<float4*>(P.xr_out + static_cast<size_t>(m0 + t0 + u) * K + B * kCBS + j0) =
+              make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    } else {
+      const float rs = quant_recip(s_tab);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u >= ntok) continue;
+        uint32_t w = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          w |= static_cast<uint32_t>(quant_code_fast(acc[u][c], s_tab, rs, -8, 7) & 15) << (4 * c);
+        *reinterpret_cast<uint16_t*>(P.xq + static_cast<size_t>(m0 + t0 + u) * (K / 2) + (B * kCBS + j0) / 2) =
+            static_cast<uint16_t>(w);
+      }
+    }
+    cta_sync();   // comp, xg and perm_s are refilled for the next block
+  }
+  if (MODE == kTable && group == 0 && tid < ntok) P.s_x[m0 + tid] = s_tab;
+}
+
+// ===========================================================================
 // Tensor-core path (bf16 input, block 64 or 128).
 //
 // The block rotation is one dense product x'_B = x_B . R_B with the composite
@@ -1018,12 +1154,78 @@ int token_tile_for(int M, int K, int BS, int mode) {
   return (M <= 16 || BS == 32 || (mode == kDynamic && K > 8192)) ? 16 : 32;
 }
 
+bool rsvd_path_forced() {
+  const char* p = std::getenv("QVLA_ROTATE_PATH");
+  return p && std::strcmp(p, "fma") == 0;
+}
+
+// Composite-path launches: every (token tile, block) pair of the batch gets a
+// CTA while they fit eight per SM; beyond that each CTA walks several blocks.
+template <typename Tin, int MODE>
+cudaError_t launch_comp(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  long long pairs = 0;
+  for (const ActArgs* a : v) pairs += static_cast<long long>((a->M + kCTT - 1) / kCTT) * (a->K / kCBS);
+  const long long slots = 8LL * 148;
+  const int bpc = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
+  for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+    ActBatch batch;
+    std::memset(&batch, 0, sizeof(batch));
+    batch.n = n;
+    int ctas = 0;
+    for (int i = 0; i < n; ++i) {
+      const ActArgs& a = *v[i0 + i];
+      ActProblem& P = batch.p[i];
+      P.x = a.x;
+      P.perm = a.perm;
+      P.rot = a.rot;
+      P.rot_tc = a.rot_tc;
+      P.table = a.table;
+      P.step_dev = a.step_dev;
+      P.xq = a.xq;
+      P.s_x = a.s_x;
+      P.xr_out = a.xr_out;
+      P.M = a.M;
+      P.ldx = a.ldx;
+      P.K = a.K;
+      P.T = a.T;
+      P.Lcount = a.Lcount;
+      P.step_host = a.step_host;
+      P.layer = a.layer;
+      P.gx = (a.M + kCTT - 1) / kCTT;
+      P.bpc = std::min(bpc, a.K / kCBS);
+      batch.cta_start[i] = ctas;
+      ctas += P.gx * ((a.K / kCBS + P.bpc - 1) / P.bpc);
+    }
+    batch.cta_start[n] = ctas;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas, 1, 1);
+    cfg.blockDim = dim3(kCThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, rotq_comp_kernel<Tin, MODE>, batch, device_error_word());
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
 template <int BS, typename Tin, int MODE>
 cudaError_t launch_bs(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
-  std::vector<const ActArgs*> t16, t32;
-  for (const ActArgs* a : v) (token_tile_for(a->M, a->K, BS, MODE) == 16 ? t16 : t32).push_back(a);
+  std::vector<const ActArgs*> comp, t16, t32;
+  for (const ActArgs* a : v) {
+    if (BS == kCBS && MODE != kDynamic && a->rot_tc != nullptr && !rsvd_path_forced())
+      comp.push_back(a);
+    else
+      (token_tile_for(a->M, a->K, BS, MODE) == 16 ? t16 : t32).push_back(a);
+  }
   cudaError_t e = cudaSuccess;
-  if (!t16.empty()) e = launch_cfg_batches<BS, 16, Tin, MODE>(t16, stream);
+  if (!comp.empty()) e = launch_comp<Tin, MODE>(comp, stream);
+  if (e == cudaSuccess && !t16.empty()) e = launch_cfg_batches<BS, 16, Tin, MODE>(t16, stream);
   if (e == cudaSuccess && !t32.empty()) e = launch_cfg_batches<BS, (BS == 32 ? 16 : 32), Tin, MODE>(t32, stream);
   return e;
 }
@@ -1235,16 +1437,19 @@ bool tc_path_forced_off() {
   return p && std::strcmp(p, "fma") == 0;
 }
 
-// Token count from which the tensor-core rotation beats the CUDA-core one.
-constexpr int kTcMinM = 65;
+// Token count from which the tensor-core rotation beats the CUDA-core ones:
+// every M (50 tokens x 12 linears of a DiT step, table mode: 19.5 us through
+// the permuted copy, 25.6 us gathering, against 27.7 us for the composite
+// CUDA-core kernel and 31.7 us for the R_SVD + Walsh-Hadamard one).
+constexpr int kTcMinM = 1;
 
 bool has_perm_scratch(const ActArgs* a) {
   return a->ws != nullptr && a->ws_bytes >= static_cast<size_t>(a->M) * a->K * 2 &&
          (reinterpret_cast<uintptr_t>(a->ws) & 15u) == 0;
 }
 
-// bf16 problems with a tensor-core image, block 64 / 128 and more than 64
-// tokens go to the tensor cores (through a permuted copy when the call gave
+// bf16 problems with a tensor-core image and block 64 / 128 go to the tensor
+// cores (through a permuted copy when the call gave
 // scratch for it, else gathering); returns the rest.
 cudaError_t launch_tc_subset(std::vector<const ActArgs*>& v, cudaStream_t stream) {
   if (tc_path_forced_off()) return cudaSuccess;
