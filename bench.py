@@ -306,9 +306,10 @@ def run_ours(args):
           for l, is8 in zip(wl.linears, w8)]
     sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
     ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
-    # scratch of the tensor-core rotation route (more than 64 bf16 tokens), one
-    # per linear since a batched launch runs them together
-    wss = [torch.empty(max(l.M * l.K * 4 if is8 else
+    # scratch of the tensor-core rotation route (the permuted copy of x; for a
+    # W8A8 linear also its fp32 rotated rows), one per linear since a batched
+    # launch runs them together
+    wss = [torch.empty(max(Q.qvla_rotate_quant_a8_workspace_bytes(l.M, l.K) if is8 else
                            Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
                        dtype=torch.uint8, device=dev) for l, is8 in zip(wl.linears, w8)]
     nl = len(wl.linears)

@@ -234,16 +234,23 @@ qvla_status qvla_pack_weights_gptq(const float* W, int N, int K, int block, cons
                                    void* cal_workspace, size_t cal_ws_bytes, cudaStream_t stream);
 
 /* W8A8 activations: the rotation of qvla_rotate_act_f32() into `workspace`
- * (fp32 [M][K], M * K * 4 bytes, see qvla_rotate_quant_a8_workspace_bytes),
- * then per-token dynamic 8-bit RTN: s_x[m] = fp32(max_k |x'[m,k]| / 127),
- * q = clamp(rint(x'/s_x), -128, 127), one int8 code per byte.
- * x, xdt, ldx, L as in qvla_rotate_quant_act().  Outputs (device): xq8
- * [M][K] int8, s_x [M] fp32.  Asynchronous (two launches).                 */
+ * (fp32 [M][K] at its start, M * K * 4 bytes), then per-token dynamic 8-bit
+ * RTN: s_x[m] = fp32(max_k |x'[m,k]| / 127), q = clamp(rint(x'/s_x), -128,
+ * 127), one int8 code per byte.  When the workspace holds M * K * 6 bytes
+ * (qvla_rotate_quant_a8_workspace_bytes) the last M * K * 2 take the
+ * permuted copy of x that the tensor-core rotation reads through TMA (bf16
+ * input and a linear that carries a tensor-core image, block 64 / 128; the
+ * packs of qvla_pack_weights_w8() carry none, so their rotation runs on the
+ * CUDA cores and leaves that part unused); with M * K * 4 the rotation
+ * gathers instead (same result).  x, xdt, ldx, L as in qvla_rotate_quant_act().  Outputs
+ * (device): xq8 [M][K] int8, s_x [M] fp32.  Asynchronous (two or three
+ * launches).                                                               */
 qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int ldx,
                                      const qvla_packed_linear* L, int8_t* xq8, float* s_x,
                                      void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Scratch of qvla_rotate_quant_act_a8(): M * K * 4 bytes.                   */
+/* Scratch of qvla_rotate_quant_act_a8() for its fastest route: M * K * 6
+ * bytes (M * K * 4 is the minimum).                                         */
 qvla_status qvla_rotate_quant_a8_workspace_bytes(int M, int K, size_t* bytes);
 
 /* W8A8 GEMM: acc[m,n] = sum_k xq8[m,k] wq[n,k] (int8 x int8 -> int32, exact

@@ -100,6 +100,8 @@ def test_argument_errors_before_any_cuda_call():
     assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64, torch.float32) == 0
     assert q.qvla_rotate_quant_workspace_bytes(0, 2048, 64) == 0
     assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 256) == 0
+    # the W8A8 activation entry: fp32 rows plus the permuted copy
+    assert q.qvla_rotate_quant_a8_workspace_bytes(50, 1024) == 50 * 1024 * 6
     assert lib.qvla_w4a4_gemm_s32(None, 0, ctypes.byref(Lok), None, 0, None) == q.QVLA_OK
     # split-K factor must be a power of two <= 16 and <= the number of 256-wide K tiles
     Lw = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)

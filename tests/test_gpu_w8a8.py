@@ -67,6 +67,24 @@ def test_a8_activation_codes(q, M, K, b, dt):
     assert q.qvla_read_error_word(clear=True) == 0
 
 
+@pytest.mark.parametrize("M,K,b", [(50, 4096, 64), (3, 1024, 128), (200, 2048, 64)])
+def test_a8_routes_agree(q, M, K, b):
+    """A workspace of M*K*6 bytes (room for the permuted copy) and the minimum
+    M*K*4 give identical codes and scales."""
+    W = I.weights(9450 + K, 64, K)
+    ref = O.pack_linear(W, b, bits=8)
+    L = q.qvla_pack_weights_w8(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd)
+    x = cu(I.activations(9451 + M, M, K, std=1.3, n_outlier_cols=4)).to(torch.bfloat16)
+    assert q.qvla_rotate_quant_a8_workspace_bytes(M, K) == M * K * 6
+    big = torch.empty(M * K * 6, dtype=torch.uint8, device="cuda")
+    small = torch.empty(M * K * 4, dtype=torch.uint8, device="cuda")
+    a, sa = q.qvla_rotate_quant_act_a8(x, L, workspace=big)
+    b8, sb = q.qvla_rotate_quant_act_a8(x, L, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b8) and torch.equal(sa, sb)
+    assert q.qvla_read_error_word(clear=True) == 0
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (16, 384, 512), (50, 1024, 4096),
                                    (64, 4096, 1024), (100, 256, 2048), (300, 1000, 1056),
                                    (520, 256, 2048), (33, 8, 32768)])

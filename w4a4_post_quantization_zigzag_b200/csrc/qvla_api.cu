@@ -193,6 +193,11 @@ size_t pack_ws_bytes(int N, int K, int block) {
 
 using namespace qvla;
 
+// The rotation of qvla_rotate_act_f32 with an optional permuted-copy scratch.
+static qvla_status rotate_act_impl(const void* x, qvla_dtype xdt, int M, int ldx,
+                                   const qvla_packed_linear* L, float* xr_out, void* perm_ws,
+                                   size_t perm_ws_bytes, cudaStream_t stream);
+
 extern "C" {
 
 const char* qvla_status_str(qvla_status s) {
@@ -615,7 +620,7 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
 qvla_status qvla_rotate_quant_a8_workspace_bytes(int M, int K, size_t* bytes) {
   if (!bytes) return QVLA_ERR_ARG;
   if (M < 0 || K <= 0 || K > QVLA_MAX_K) return QVLA_ERR_SHAPE;
-  *bytes = static_cast<size_t>(M) * K * 4;
+  *bytes = static_cast<size_t>(M) * K * 6;
   return QVLA_OK;
 }
 
@@ -628,10 +633,16 @@ qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int l
   if (M == 0) return QVLA_OK;
   if (!xq8 || !s_x) return QVLA_ERR_ARG;
   if (!aligned16(xq8) || !aligned16(s_x)) return QVLA_ERR_ALIGN;
-  if (!workspace || ws_bytes < static_cast<size_t>(M) * L->K * 4) return QVLA_ERR_WORKSPACE;
+  const size_t xr_bytes = static_cast<size_t>(M) * L->K * 4;
+  if (!workspace || ws_bytes < xr_bytes) return QVLA_ERR_WORKSPACE;
   float* xr = static_cast<float*>(workspace);
-  // 1. the rotation (fp32 x' into the workspace)
-  if ((st = qvla_rotate_act_f32(x, xdt, M, ldx, L, xr, stream)) != QVLA_OK) return st;
+  // 1. the rotation (fp32 x' into the workspace; the permuted copy of x that
+  // the tensor-core route reads goes after it when the workspace has room)
+  const size_t perm_bytes = static_cast<size_t>(M) * L->K * 2;
+  void* perm_ws = ws_bytes >= xr_bytes + perm_bytes ? static_cast<uint8_t*>(workspace) + xr_bytes : nullptr;
+  if ((st = rotate_act_impl(x, xdt, M, ldx, L, xr, perm_ws, perm_ws ? perm_bytes : 0, stream)) !=
+      QVLA_OK)
+    return st;
   // 2. per-token dynamic 8-bit RTN
   QuantArgs q = {};
   q.xr = xr;
@@ -648,6 +659,16 @@ qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int l
 
 qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
                                 const qvla_packed_linear* L, float* xr_out, cudaStream_t stream) {
+  return rotate_act_impl(x, xdt, M, ldx, L, xr_out, nullptr, 0, stream);
+}
+
+}  // extern "C"
+
+// The rotation alone; perm_ws (or NULL) holds the permuted copy of x that the
+// tensor-core route reads through TMA.
+static qvla_status rotate_act_impl(const void* x, qvla_dtype xdt, int M, int ldx,
+                                   const qvla_packed_linear* L, float* xr_out, void* perm_ws,
+                                   size_t perm_ws_bytes, cudaStream_t stream) {
   qvla_status st = check_linear(L, false);
   if (st != QVLA_OK) return st;
   if (M < 0) return QVLA_ERR_SHAPE;
@@ -669,8 +690,12 @@ qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
   a.rot_tc = (L->rot_tc && (L->block == 64 || L->block == 128)) ? L->rot_tc : nullptr;
   a.dynamic = 1;
   a.xr_out = xr_out;
+  a.ws = perm_ws;
+  a.ws_bytes = perm_ws_bytes;
   return cuda_status(launch_rotate_quant(a, stream));
 }
+
+extern "C" {
 
 qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mode,
                                const float* table, int T, int Lcount, const int32_t* step_dev,

@@ -358,6 +358,13 @@ def qvla_pack_weights_w8(W: torch.Tensor, block: int, bias: Optional[torch.Tenso
     return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias)
 
 
+def qvla_rotate_quant_a8_workspace_bytes(M: int, K: int) -> int:
+    b = c_size_t()
+    _check(_lib.qvla_rotate_quant_a8_workspace_bytes(M, K, ctypes.byref(b)),
+           "qvla_rotate_quant_a8_workspace_bytes")
+    return b.value
+
+
 def qvla_rotate_quant_act_a8(x: torch.Tensor, L: PackedLinear,
                              xq8: Optional[torch.Tensor] = None,
                              s_x: Optional[torch.Tensor] = None,
@@ -369,7 +376,8 @@ def qvla_rotate_quant_act_a8(x: torch.Tensor, L: PackedLinear,
     if s_x is None:
         s_x = torch.empty(M, dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = torch.empty(max(M * L.K * 4, 16), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(max(qvla_rotate_quant_a8_workspace_bytes(M, L.K), 16),
+                                dtype=torch.uint8, device=x.device)
     _check(_lib.qvla_rotate_quant_act_a8(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct,
                                          _ptr(xq8), _ptr(s_x), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(),
