@@ -40,3 +40,18 @@ def test_product_arm_fails_without_a_gpu():
     r = _run(["--steps", "1", "--warmup", "0"])
     assert r.returncode != 0
     assert not any(l.startswith("{") for l in r.stdout.splitlines()), "no number without a GPU"
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Two ranks: rank 0 alone runs the oracle and prints; the other exits 0."""
+    port = 29600 + (os.getpid() % 300)
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
