@@ -1154,6 +1154,8 @@ int token_tile_for(int M, int K, int BS, int mode) {
   return (M <= 16 || BS == 32 || (mode == kDynamic && K > 8192)) ? 16 : 32;
 }
 
+// QVLA_ROTATE_PATH=fma: every problem on the R_SVD + Walsh-Hadamard
+// CUDA-core kernel (no tensor cores, no composite kernel), for tests.
 bool rsvd_path_forced() {
   const char* p = std::getenv("QVLA_ROTATE_PATH");
   return p && std::strcmp(p, "fma") == 0;
@@ -1432,11 +1434,6 @@ cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t st
   return cudaSuccess;
 }
 
-bool tc_path_forced_off() {
-  const char* p = std::getenv("QVLA_ROTATE_PATH");
-  return p && std::strcmp(p, "fma") == 0;
-}
-
 // Token count from which the tensor-core rotation beats the CUDA-core ones:
 // every M (50 tokens x 12 linears of a DiT step, table mode: 19.5 us through
 // the permuted copy, 25.6 us gathering, against 27.7 us for the composite
@@ -1452,7 +1449,7 @@ bool has_perm_scratch(const ActArgs* a) {
 // cores (through a permuted copy when the call gave
 // scratch for it, else gathering); returns the rest.
 cudaError_t launch_tc_subset(std::vector<const ActArgs*>& v, cudaStream_t stream) {
-  if (tc_path_forced_off()) return cudaSuccess;
+  if (rsvd_path_forced()) return cudaSuccess;
   std::vector<const ActArgs*> rest, perm, g[2][3], t[2][3];
   for (const ActArgs* a : v) {
     if (a->rot_tc == nullptr || (a->block != 64 && a->block != 128) || a->M < kTcMinM) {
