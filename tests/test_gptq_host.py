@@ -37,7 +37,8 @@ def _recon_error(Wr, qw, s, xr):
 
 
 @pytest.mark.parametrize("N,K,block,T", [(40, 128, 32, 300), (96, 512, 64, 700),
-                                         (7, 256, 128, 64), (64, 1024, 128, 1500)])
+                                         (7, 256, 128, 64), (64, 1024, 128, 1500),
+                                         (32, 256, 64, 100)])     # T < K: H singular
 def test_given_factor_bit_identical(q, N, K, block, T):
     pk, xr = _case(2100 + K, N, K, block, T)
     U, dead = O.gptq_inverse_factor(O.gptq_hessian(xr), 0.05)
@@ -48,7 +49,8 @@ def test_given_factor_bit_identical(q, N, K, block, T):
 
 
 @pytest.mark.parametrize("N,K,block,T,dead", [(96, 512, 64, 700, ()), (33, 256, 32, 100, (3, 200)),
-                                              (64, 1024, 128, 1500, (0,))])
+                                              (64, 1024, 128, 1500, (0,)),
+                                              (48, 512, 64, 200, ())])   # T < K: damping makes H definite
 def test_own_factor_matches_oracle(q, N, K, block, T, dead):
     pk, xr = _case(2200 + K, N, K, block, T, dead)
     H = O.gptq_hessian(xr)
