@@ -118,3 +118,36 @@ def test_pack_workspace_check():
                                  ctypes.c_void_p(16), ctypes.c_void_p(16), None,
                                  ctypes.c_void_p(16), ctypes.c_void_p(16), None, 0,
                                  None) == q.QVLA_ERR_WORKSPACE
+
+
+def test_variant_entry_points_reject_bad_arguments():
+    """The Hadamard-only, W8A8 and GPTQ entry points validate on the host,
+    before any CUDA call (no GPU here)."""
+    q = _lib_mod()
+    lib = q._lib
+    P = ctypes.c_void_p(16)
+    big = 1 << 30
+    # GPTQ pack: K beyond the host factorisation's limit; neither calibration
+    # rows nor a factor; calibration scratch too small for T x K fp32 rows
+    assert lib.qvla_pack_weights_gptq(P, 64, 8192, 64, P, 1, 100, 0.05, None, None, None, P, P,
+                                      None, P, P, P, big, P, big, None) == q.QVLA_ERR_SHAPE
+    assert lib.qvla_pack_weights_gptq(P, 64, 256, 64, None, 1, 0, 0.05, None, None, None, P, P,
+                                      None, P, P, P, big, None, 0, None) == q.QVLA_ERR_ARG
+    assert lib.qvla_pack_weights_gptq(P, 64, 256, 64, P, 1, 100, 0.05, None, None, None, P, P,
+                                      None, P, P, P, big, P, 100 * 256 * 4 - 1,
+                                      None) == q.QVLA_ERR_WORKSPACE
+    # Hadamard-only and W8 packs: a block size outside {32, 64, 128, 256}
+    assert lib.qvla_pack_weights_hadamard(P, 64, 256, 48, None, P, P, P, P, big,
+                                          None) == q.QVLA_ERR_SHAPE
+    assert lib.qvla_pack_weights_w8(P, 64, 256, 48, None, None, P, P, P, P, P, big,
+                                    None) == q.QVLA_ERR_SHAPE
+    # 8-bit activations: no packed linear; workspace below the M x K fp32 rows
+    L = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)
+    assert lib.qvla_rotate_quant_act_a8(P, 1, 4, 256, None, P, P, P, big,
+                                        None) == q.QVLA_ERR_ARG
+    assert lib.qvla_rotate_quant_act_a8(P, 1, 4, 256, ctypes.byref(L), P, P, P, 4 * 256 * 4 - 1,
+                                        None) == q.QVLA_ERR_WORKSPACE
+    # W8A8 GEMM: no output; no packed linear; nothing to do for M = 0
+    assert lib.qvla_w8a8_gemm(P, P, 4, ctypes.byref(L), None, 256, None) == q.QVLA_ERR_ARG
+    assert lib.qvla_w8a8_gemm_s32(P, 4, None, P, None) == q.QVLA_ERR_ARG
+    assert lib.qvla_w8a8_gemm_s32(None, 0, ctypes.byref(L), None, None) == q.QVLA_OK
