@@ -327,7 +327,7 @@ qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtyp
  * an inference loop that must not call cudaMalloc once it is running (a
  * robot control loop with a hard cycle budget, code that is being captured
  * into a CUDA graph, a host application that hands out no allocator) -- the
- * scratch the fast large-M route needs (qvla_rotate_quant_workspace_bytes)
+ * scratch the tensor-core route needs (qvla_rotate_quant_workspace_bytes)
  * lives in a fixed array inside the library, QVLA_NOALLOC_SCRATCH_BYTES bytes
  * per device, kept for as long as the library is loaded.  Arguments and
  * results are those of qvla_rotate_quant_act.
