@@ -14,7 +14,7 @@ kernel.  L2 is flushed (512 MB written, then read back) before every timed step,
 streams its packed weights from HBM.
 
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on the
-same workload instead (the reference arm).
+same workload instead (the reference arm: the pages publish no code to run).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
 """

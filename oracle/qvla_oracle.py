@@ -26,7 +26,7 @@ Sources (web pages on the method; page title, then section):
         Models via Consistent Folding" (radar.vhtltd.com): dynamic per-token
         activation quantisation.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * Layouts follow PyTorch Linear: W is [N, K] (out x in), x is [M, K].
   * R_SVD of a block is the matrix of right singular vectors of that block of
     W (eigenvectors of its Gram matrix), columns ordered by descending singular

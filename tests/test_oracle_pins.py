@@ -426,6 +426,107 @@ def test_end_to_end_quantised_layer_is_close_to_fp_layer():
     assert err_rot < err_plain
 
 
+# ------------------------------------- end-to-end activation quantiser
+
+def _golden_pack(g):
+    """The hand-worked linear: the fixture's permutation, R_SVD = I in every
+    block (so R_B is the normalised Hadamard matrix), given weight codes."""
+    b = g["block"]
+    nb = g["K"] // b
+    rsvd = np.stack([np.eye(b)] * nb)
+    return O.PackedLinear(np.array(g["perm"]), rsvd, O.composite_blocks(rsvd), None,
+                          np.array(g["qw"], np.int8), np.array(g["s_w"], np.float32),
+                          np.array(g["bias"], np.float64))
+
+
+def _golden_act_mismatches(g):
+    """Which parts of the hand-worked case the oracle's end-to-end quantiser
+    (rotate_quant_act) and layer (linear_forward) fail to reproduce."""
+    pk = _golden_pack(g)
+    x = np.array(g["x"], np.float64)
+    table = np.array(g["table"], np.float32)
+    bad = []
+    xr, q, s = O.rotate_quant_act(x, pk, "table", table, g["step"], g["layer"])
+    if not np.array_equal(xr, np.array(g["xr"], np.float64)):
+        bad.append("xr")
+    if q.tolist() != g["table_codes"] or not np.all(s == g["table_s"]):
+        bad.append("table codes")
+    out = O.linear_forward(x, pk, "table", table, g["step"], g["layer"])
+    if out["acc"].tolist() != g["table_acc"] or not np.allclose(out["y"], g["table_y"],
+                                                              rtol=0, atol=1e-15):
+        bad.append("table layer")
+    xr, q, s = O.rotate_quant_act(x, pk, "dynamic")
+    want_s = [n / d for n, d in g["dynamic_s_fraction"]]
+    if q.tolist() != g["dynamic_codes"] or not np.allclose(s, want_s, rtol=1e-15, atol=0):
+        bad.append("dynamic codes")
+    out = O.linear_forward(x, pk, "dynamic")
+    want_y = [[n / d for n, d in row] for row in g["dynamic_y_fraction"]]
+    if out["acc"].tolist() != g["dynamic_acc"] or not np.allclose(out["y"], want_y,
+                                                                rtol=1e-14, atol=1e-15):
+        bad.append("dynamic layer")
+    return bad
+
+
+def test_end_to_end_quantiser_golden():
+    assert _golden_act_mismatches(gold("act_quant_cases.json")) == []
+
+
+@pytest.mark.parametrize("mode", ["dynamic", "table"])
+def test_end_to_end_quantiser_follows_the_fp32_rule(mode):
+    """rotate_quant_act quantises the double x'; its codes must be the pinned
+    fp32 rule applied to fp32(x') except within 1e-5 of a rounding boundary
+    (where both roundings are correct), and its dynamic scale must be the
+    token's max |x'| / 7 (scalar loop)."""
+    lin = I.single_linear().linears[0]
+    W = lin.make_w()
+    pk = O.pack_linear(W, lin.block)
+    x = I.activations(21, 64, 256, n_outlier_cols=4, dtype="f32").astype(np.float64)
+    table = np.array([[0.9, 0.8], [0.5, 0.7]], np.float32)
+    xr, q, s = O.rotate_quant_act(x, pk, mode, table, 1, 0)
+    # x' is x P R with the dense matrices (pinned above)
+    np.testing.assert_allclose(xr, x @ _dense_P(pk.perm) @ _dense_R(pk.R), rtol=0, atol=1e-12)
+    xr32 = xr.astype(np.float32)
+    if mode == "dynamic":
+        q32, _ = O.quantize_acts_dynamic_fp32(xr32)
+        for m in range(x.shape[0]):
+            amax = 0.0
+            for v in xr[m]:
+                amax = max(amax, abs(float(v)))
+            assert s[m] == amax / 7.0
+            assert np.abs(q[m]).max() == 7 and q[m].min() >= -7   # -8 needs a table scale
+    else:
+        q32, _ = O.quantize_acts_table_fp32(xr32, np.float32(table[1, 0]))
+        assert np.all(s == float(np.float32(table[1, 0])))
+        assert q.min() == -8 and q.max() == 7                       # saturates both ways
+    d = q.astype(np.int64) - q32.astype(np.int64)
+    rows, cols = np.nonzero(d)
+    assert np.abs(d).max(initial=0) <= 1
+    t = xr[rows, cols] / s[rows]
+    assert (np.abs(t - np.floor(t) - 0.5) < 1e-5).all()
+    assert len(rows) <= max(1, 1e-4 * q.size)
+
+
+def test_end_to_end_pins_catch_planted_mistakes(monkeypatch):
+    """A dynamic divisor of 8, a clamp to [-7, 7], a transposed table read and
+    a dropped permutation each break the hand-worked case."""
+    g = gold("act_quant_cases.json")
+    assert _golden_act_mismatches(g) == []
+    with monkeypatch.context() as mp:
+        mp.setattr(O, "ACT_QMAX", 8)
+        assert "dynamic codes" in _golden_act_mismatches(g)
+    with monkeypatch.context() as mp:
+        mp.setattr(O, "ACT_QMIN", -7)
+        assert "table codes" in _golden_act_mismatches(g)
+    with monkeypatch.context() as mp:
+        mp.setattr(O, "table_scale", lambda tab, step, layer: np.float32(tab[layer, step]))
+        assert "table codes" in _golden_act_mismatches(g)
+    rot = O.rotate_activations
+    with monkeypatch.context() as mp:
+        mp.setattr(O, "rotate_activations", lambda x, perm, R: rot(x, np.arange(len(perm)), R))
+        assert "xr" in _golden_act_mismatches(g)
+    assert _golden_act_mismatches(g) == []
+
+
 # ------------------------------------------------------ planted mistakes
 
 def test_pins_catch_planted_mistakes():
