@@ -333,14 +333,16 @@ def gptq_inverse_factor(H: np.ndarray, damp: float = 0.05):
     return U, dead
 
 
-def gptq_quantize(Wr32: np.ndarray, U: np.ndarray, dead=None, qmax: int = WEIGHT_QMAX):
+def gptq_quantize(Wr32: np.ndarray, U: np.ndarray, dead=None, qmax: int = WEIGHT_QMAX,
+                  quotients: bool = False):
     """GPTQ rounding of fp32 rotated weights [N, K] with the inverse factor U.
 
     The per-row scale is the RTN one, s = fp32(max |W'[n,:]| / qmax).  Column
     by column, in order: q = clamp(rint(w / s), -qmax, qmax) in double, the
     error e = (w - q s) / U[j, j], and every later column k takes
     w_k -= e * U[j, k] (the block size of the pages only groups these updates
-    and leaves the result unchanged).  Returns (codes int8 [N, K], s fp32 [N])."""
+    and leaves the result unchanged).  Returns (codes int8 [N, K], s fp32 [N]),
+    and with `quotients` also the double w / s that each code rounded."""
     W = np.asarray(Wr32, dtype=np.float32)
     s = np.divide(np.max(np.abs(W), axis=1), np.float32(qmax), dtype=np.float32)
     Wc = W.astype(np.float64)
@@ -350,14 +352,16 @@ def gptq_quantize(Wr32: np.ndarray, U: np.ndarray, dead=None, qmax: int = WEIGHT
     safe = np.where(s64 == 0, 1.0, s64)
     N, K = Wc.shape
     Q = np.zeros((N, K), dtype=np.int8)
+    T = np.zeros((N, K), dtype=np.float64)
     for j in range(K):
         w = Wc[:, j]
+        T[:, j] = w / safe
         q = np.where(s64 == 0, 0.0, np.clip(np.rint(w / safe), -qmax, qmax))
         Q[:, j] = q.astype(np.int8)
         e = (w - q * s64) / U[j, j]
         if j + 1 < K:
             Wc[:, j + 1:] -= e[:, None] * U[j, j + 1:][None, :]
-    return Q, s
+    return (Q, s, T) if quotients else (Q, s)
 
 
 def pack_linear_gptq(W: np.ndarray, block: int, x_cal: np.ndarray, bias=None, perm=None,
@@ -372,7 +376,7 @@ def pack_linear_gptq(W: np.ndarray, block: int, x_cal: np.ndarray, bias=None, pe
         U, dead = gptq_inverse_factor(gptq_hessian(xr), damp)
     qw, s_w = gptq_quantize(pk.Wr.astype(np.float32), U, dead)
     pk.qw, pk.s_w = qw, s_w
-    pk.U = U
+    pk.U, pk.dead = U, dead
     return pk
 
 

@@ -48,3 +48,27 @@ def check_y(y_gpu, y_ref, what="y"):
     worst = float((err - lim).max()) if err.size else 0.0
     assert (err <= lim).all(), f"{what}: {int((err > lim).sum())} outputs outside tolerance " \
                                f"(worst excess {worst:.3g})"
+
+
+def check_gptq_flips(q_gpu, q_ref, t_ref, boundary, max_frac, what="GPTQ codes"):
+    """GPTQ codes from a factor that differs from the oracle's by rounding.
+
+    The error feedback carries a flipped code along its row, so only the
+    first flip of each row is a rounding decision of its own: it must differ
+    by 1 and lie where the oracle's quotient w/s is within `boundary` of a
+    half-integer.  Later flips in that row follow from it.  Returns the
+    number of flipped codes (at most max_frac of them, and at least 1
+    allowed)."""
+    q_gpu = np.asarray(q_gpu, np.int64)
+    q_ref = np.asarray(q_ref, np.int64)
+    d = q_gpu - q_ref
+    n = int((d != 0).sum())
+    for r in np.nonzero((d != 0).any(axis=1))[0]:
+        j = int(np.argmax(d[r] != 0))
+        t = float(t_ref[r, j])
+        dist = abs(t - (np.floor(t) + 0.5))
+        assert abs(int(d[r, j])) == 1, f"{what}: row {r} first flip differs by {d[r, j]}"
+        assert dist < boundary, (f"{what}: row {r} first flip at column {j} is {dist:.3g} "
+                                 f"from a rounding boundary")
+    assert n <= max(1, max_frac * q_ref.size), f"{what}: {n} flips of {q_ref.size}"
+    return n

@@ -2,9 +2,11 @@
 rotates the calibration rows, and the library rounds W' with GPTQ.  Against
 the oracle's GPTQ pack of the same weights and calibration rows:
   * scales bit-identical (GPTQ keeps the RTN scale);
-  * codes equal except for a bounded number of flips (W' and the rotated
-    calibration rows differ from the oracle's fp64 ones by rounding, and the
-    error feedback carries a flip along its row);
+  * codes identical when the oracle's inverse factor U is passed in;
+  * with the library's own factor (fp32-rotated calibration rows, so H and U
+    differ from the oracle's by rounding) every row's first flipped code
+    sits at a rounding boundary of the oracle's quotient, and the flips
+    are few (the error feedback carries a flip along its row);
   * the calibration output error no worse than the oracle's codes';
   * end to end, a GPTQ-packed linear through the W4A4 path within the bf16
     tolerance of the oracle's dequantisation of the same codes."""
@@ -14,7 +16,7 @@ import torch
 
 from oracle import qvla_oracle as O
 from w4a4_post_quantization_zigzag_b200 import inputs as I
-from _parity import check_codes_near_boundary, check_y
+from _parity import check_codes_near_boundary, check_gptq_flips, check_y
 
 pytestmark = pytest.mark.gpu
 
@@ -53,12 +55,9 @@ def test_gptq_pack_given_factor(q, N, K, b, T):
     torch.cuda.synchronize()
     assert np.array_equal(pk.w_scale.cpu().numpy().view(np.uint32), ref.s_w.view(np.uint32))
     qg = O.unpack_nibbles(pk.wq.cpu().numpy())
-    flips = int((qg != ref.qw).sum())
-    assert flips <= max(4, qg.size // 500), f"{flips} code flips"
-    assert np.abs(qg.astype(int) - ref.qw).max() <= 1
-    xr = O.rotate_activations(x.astype(np.float64), ref.perm, ref.R)
-    Wr32 = ref.Wr.astype(np.float32)
-    assert _recon_error(Wr32, qg, ref.s_w, xr) <= 1.01 * _recon_error(Wr32, ref.qw, ref.s_w, xr)
+    # W' on the device is bit-exact and the column loop with the same U is a
+    # fixed sequence of fp64 operations: no code may differ
+    assert int((qg != ref.qw).sum()) == 0, "code flips with the oracle's own factor"
     assert q.qvla_read_error_word(clear=True) == 0
 
 
@@ -72,8 +71,11 @@ def test_gptq_pack_with_calibration(q, N, K, b, T, dt):
     torch.cuda.synchronize()
     assert np.array_equal(pk.w_scale.cpu().numpy().view(np.uint32), ref.s_w.view(np.uint32))
     qg = O.unpack_nibbles(pk.wq.cpu().numpy())
-    flips = int((qg != ref.qw).sum())
-    assert flips <= max(4, qg.size // 500), f"{flips} code flips"
+    # the device rotates the calibration rows in fp32 (x' within ~2e-6 of each
+    # row's max), so H and U differ from the oracle's at ~1e-6 relative and
+    # a row's first flip must sit within 1e-3 of a rounding boundary
+    _, _, t_ref = O.gptq_quantize(ref.Wr.astype(np.float32), ref.U, ref.dead, quotients=True)
+    check_gptq_flips(qg, ref.qw, t_ref, boundary=1e-3, max_frac=2e-3)
     xr = O.rotate_activations(x.astype(np.float64), ref.perm, ref.R)
     Wr32 = ref.Wr.astype(np.float32)
     e_g = _recon_error(Wr32, qg, ref.s_w, xr)
@@ -99,6 +101,7 @@ def test_gptq_linear_end_to_end(q):
     qx = O.unpack_nibbles(xq.cpu().numpy()).astype(np.int64)
     check_codes_near_boundary(qx, out["qx"], out["xr"], out["s_x"], "activation codes")
     qw = O.unpack_nibbles(L.wq.cpu().numpy()).astype(np.int64)
-    assert int((qw != ref.qw).sum()) <= qw.size // 500
+    _, _, t_ref = O.gptq_quantize(ref.Wr.astype(np.float32), ref.U, ref.dead, quotients=True)
+    check_gptq_flips(qw, ref.qw, t_ref, boundary=1e-3, max_frac=2e-3)
     check_y(y.float().cpu().numpy(), O.dequantize(O.int_gemm(qx, qw), out["s_x"], ref.s_w, bias))
     assert q.qvla_read_error_word(clear=True) == 0
