@@ -114,10 +114,23 @@ typedef struct {
 
 const char* qvla_status_str(qvla_status s);
 int qvla_abi_version(void);
+/* SHA-256 (64 hex digits) of the sources this library was built from, as
+ * the build computed it; "unstamped" for a build that set none.            */
+const char* qvla_source_hash(void);
 
 /* Reads the current device's error word into *out and, if clear != 0, resets
  * it to 0.  Synchronises the device.  Returns QVLA_ERR_CUDA on a CUDA error. */
 qvla_status qvla_read_error_word(uint32_t* out, int clear);
+
+/* Self-test of the kernels' failure path (no page counterpart: it checks this
+ * library's promise that a kernel never hangs).  Launches one warp that holds
+ * tensor memory and waits, with the same bounded wait every kernel here uses,
+ * on a barrier nothing arrives on; after limit_ns nanoseconds it gives up,
+ * sets QVLA_DEVERR_TIMEOUT in the error word, frees its tensor memory and
+ * returns.  The context stays usable.  limit_ns in [1e3, 1e7], else
+ * QVLA_ERR_ARG.  Asynchronous on `stream`; read the outcome with
+ * qvla_read_error_word().                                                   */
+qvla_status qvla_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 
 /* Byte sizes of the buffers a packed linear needs:
  *   *wq_bytes     = N * K / 2
@@ -393,7 +406,10 @@ qvla_status qvla_w4a4_gemm_s32(const uint8_t* xq, int M, const qvla_packed_linea
  * Linears are grouped by kernel configuration (rotation block, token tile,
  * input type, scale mode); each launch takes up to 16 of them.  Results are
  * identical to calling the single-linear entry points one by one.  No two
- * problems may share an output buffer.
+ * problems may share an output buffer, and their workspaces must not
+ * overlap (the problems of one call run at the same time): the batched
+ * rotate-quantise returns QVLA_ERR_ARG when two non-NULL workspace ranges
+ * [workspace, workspace + ws_bytes) intersect.
  * ------------------------------------------------------------------------- */
 typedef struct {
   const qvla_packed_linear* L;   /* host pointer to the packed linear          */

@@ -151,3 +151,22 @@ def test_variant_entry_points_reject_bad_arguments():
     assert lib.qvla_w8a8_gemm(P, P, 4, ctypes.byref(L), None, 256, None) == q.QVLA_ERR_ARG
     assert lib.qvla_w8a8_gemm_s32(P, 4, None, P, None) == q.QVLA_ERR_ARG
     assert lib.qvla_w8a8_gemm_s32(None, 0, ctypes.byref(L), None, None) == q.QVLA_OK
+
+
+def test_selftest_wait_limit_is_checked_on_the_host():
+    """Out-of-range wait limits are rejected before anything is launched."""
+    q = _lib_mod()
+    for ns in (0, 999, 10_000_001):
+        with pytest.raises(q.QvlaError) as e:
+            q.qvla_selftest_wait_timeout(ns, stream=0)
+        assert e.value.code == q.QVLA_ERR_ARG
+
+
+def test_library_carries_the_hash_of_its_sources():
+    """build() rebuilds on any change of content (not of file times), and the
+    loaded library reports the hash of exactly the sources on disk."""
+    from w4a4_post_quantization_zigzag_b200 import build
+    q = _lib_mod()
+    h = build.source_hash()
+    assert len(h) == 64 and q.qvla_source_hash() == h == build.library_stamp()
+    assert build.up_to_date()

@@ -56,6 +56,32 @@ def test_noalloc_matches_the_allocating_entry_point_twice(q, M, K, b, mode):
     assert q.qvla_read_error_word(clear=True) == 0
 
 
+def test_noalloc_runs_the_permuted_copy_route(q):
+    """The fixed array must really serve as the scratch: the call has to launch
+    the permuted-copy kernel (without usable scratch the route would gather
+    instead and give the same bits, so equal outputs alone do not show it).
+    Kernel names come from the PyTorch profiler's CUDA activity trace."""
+    M, K, b = 64, 1024, 64
+    L = _packed(q, 128, K, b, 9300)
+    x = torch.from_numpy(I.activations(9301, M, K, n_outlier_cols=3)).cuda().to(torch.bfloat16)
+    xq = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    q.qvla_rotate_quant_act_noalloc(x, L, xq, sx)            # first call: set-up outside the trace
+    torch.cuda.synchronize()
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        q.qvla_rotate_quant_act_noalloc(x, L, xq, sx)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    if not names:
+        pytest.skip("no CUDA activity trace in this process")
+    assert any("permute_rows_kernel" in n for n in names), names
+    ref_q, ref_s = q.qvla_rotate_quant_act(x, L)
+    torch.cuda.synchronize()
+    assert torch.equal(xq, ref_q) and torch.equal(sx, ref_s)
+    assert q.qvla_read_error_word(clear=True) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_array(q):
     M, K, b = 1024, 16384, 128                # needs 32 MiB of scratch
     assert q.qvla_rotate_quant_workspace_bytes(M, K, b) > q.QVLA_NOALLOC_SCRATCH_BYTES

@@ -5,13 +5,16 @@
 Every ``csrc/*.cu`` file is compiled for ``-gencode arch=compute_100a,code=sm_100a``
 (relocatable objects are not needed: kernels in different files share only the
 device error word, whose address is passed as a kernel argument) and linked into
-one library next to this file.  Objects are rebuilt only when a source or header
-is newer than the library.
+one library next to this file.  A SHA-256 of every source, header and of this
+script is compiled into the library (``qvla_source_hash()``); the library is
+rebuilt whenever the stamp it carries differs from the hash of the files on
+disk, so a reused binary is always the one these sources produce.
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -46,11 +49,36 @@ def _deps():
         os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
 
 
+STAMP_PREFIX = b"QVLA_SOURCE_SHA256="
+
+
+def source_hash() -> str:
+    """SHA-256 over the build inputs (path relative to the repository, then
+    content), in a fixed order."""
+    h = hashlib.sha256()
+    for d in sorted(set(_deps())):
+        h.update(os.path.relpath(d, ROOT).encode() + b"\0")
+        with open(d, "rb") as f:
+            h.update(f.read())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
+def library_stamp(path: str = LIB):
+    """The source hash compiled into a built library, or None."""
+    if not os.path.exists(path):
+        return None
+    with open(path, "rb") as f:
+        data = f.read()
+    i = data.find(STAMP_PREFIX)
+    if i < 0:
+        return None
+    j = i + len(STAMP_PREFIX)
+    return data[j:j + 64].decode("ascii", "replace")
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
-        return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in _deps())
+    return library_stamp() == source_hash()
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
@@ -59,6 +87,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra.append(f'-DQVLA_SOURCE_SHA256="{source_hash()}"')
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")

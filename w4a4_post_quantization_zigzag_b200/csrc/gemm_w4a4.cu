@@ -435,17 +435,15 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -509,15 +507,14 @@ cudaError_t launch_group(const GemmArgs* const* gs, const int* splits, int n, in
   }
   batch.tile_start[n] = ctas;
   auto kern = w4a4_gemm_kernel<NT>;
-  static bool attr_set = false;
-  cudaError_t e;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [&]() {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -650,32 +647,15 @@ int gemm_choose_split(int M, int N, int K) {
   return S;
 }
 
-// QVLA_GEMM_PATH=rows sends the automatic-split linears of up to 64 tokens
-// to the persistent row-split kernel (gemm_w4a4_rows.cu); by default they
-// stay on the one-tile-per-CTA kernel with cluster split-K, which measures
-// faster on the DiT action-head shapes (a row-split tile pays its per-K-tile
-// overheads once per part).
-bool rows_path_selected() {
-  const char* p = std::getenv("QVLA_GEMM_PATH");
-  return p && std::strcmp(p, "rows") == 0;
-}
-
 cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream) {
-  // group by token tile (a template parameter of the kernel); up to 64 tokens
-  // the persistent row-split kernel serves the automatic split choice
+  // group by token tile (a template parameter of the kernel)
   static const int kTiles[5] = {16, 32, 64, 128, 256};
-  const bool rows = split_k == 0 && rows_path_selected();
   for (int t : kTiles) {
     std::vector<const GemmArgs*> grp;
     for (int i = 0; i < n; ++i)
       if (gs[i].M > 0 && token_tile(gs[i].M) == t) grp.push_back(&gs[i]);
     if (grp.empty()) continue;
     cudaError_t e;
-    if (rows && t <= 64) {
-      e = launch_w4a4_gemm_rows(grp.data(), static_cast<int>(grp.size()), t, stream);
-      if (e != cudaSuccess) return e;
-      continue;
-    }
     switch (t) {
       case 16: e = launch_nt_batches<16>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
       case 32: e = launch_nt_batches<32>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;

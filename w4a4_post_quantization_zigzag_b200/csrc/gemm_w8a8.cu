@@ -218,13 +218,11 @@ cudaError_t launch_nt(const GemmArgs& g, cudaStream_t stream) {
   P.tiles_n = (g.N + kBM - 1) / kBM;
   const int tiles = P.tiles_n * ((g.M + NT - 1) / NT);
   auto kern = w8a8_gemm_kernel<NT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  });
+  if (e != cudaSuccess) return e;
   kern<<<tiles, kThreads, C::kSmem, stream>>>(P, device_error_word());
   return cudaGetLastError();
 }

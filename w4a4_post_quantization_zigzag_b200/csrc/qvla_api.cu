@@ -31,6 +31,32 @@ unsigned int* device_error_word() {
   return addr[dev];
 }
 
+namespace {
+// One warp: holds tensor memory and an mbarrier that nothing ever arrives on,
+// waits on it with the production bounded wait, gives up after limit_ns,
+// then frees its tensor memory and returns.  The wait expiring is the
+// expected outcome: it must set QVLA_DEVERR_TIMEOUT and nothing else.
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(uint64_t limit_ns,
+                                                                   unsigned int* err) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_slot;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  tmem_alloc(&tmem_slot, 32);
+  tmem_relinquish();
+  tc_fence_before();
+  __syncwarp();
+  tc_fence_after();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, err, limit_ns);
+  __syncwarp();
+  tc_fence_after();
+  tmem_dealloc(tmem_slot, 32);
+}
+}  // namespace
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = std::getenv("QVLA_PDL");
@@ -217,6 +243,15 @@ const char* qvla_status_str(qvla_status s) {
 
 int qvla_abi_version(void) { return QVLA_ABI_VERSION; }
 
+#ifndef QVLA_SOURCE_SHA256
+#define QVLA_SOURCE_SHA256 "unstamped"
+#endif
+// The build stamps the hash of its inputs here; the prefix lets a build
+// script find it in the file without loading the library.
+__attribute__((used)) static const char kSourceStamp[] = "QVLA_SOURCE_SHA256=" QVLA_SOURCE_SHA256;
+
+const char* qvla_source_hash(void) { return kSourceStamp + sizeof("QVLA_SOURCE_SHA256=") - 1; }
+
 qvla_status qvla_read_error_word(uint32_t* out, int clear) {
   if (!out) return QVLA_ERR_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return QVLA_ERR_CUDA;
@@ -228,6 +263,14 @@ qvla_status qvla_read_error_word(uint32_t* out, int clear) {
     if (cudaMemcpyToSymbol(g_qvla_error_word, &z, sizeof(z)) != cudaSuccess) return QVLA_ERR_CUDA;
   }
   return QVLA_OK;
+}
+
+qvla_status qvla_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > 10000000ull) return QVLA_ERR_ARG;
+  unsigned int* err = device_error_word();
+  if (!err) return QVLA_ERR_CUDA;
+  bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, err);
+  return cuda_status(cudaGetLastError());
 }
 
 qvla_status qvla_packed_sizes(int N, int K, int block, size_t* wq_bytes, size_t* rot_bytes,
@@ -614,6 +657,13 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
     v[i].ws = p.workspace;
     v[i].ws_bytes = p.ws_bytes;
   }
+  // the problems run concurrently: their scratch ranges must be disjoint
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(v[i].ws), b0 = reinterpret_cast<uintptr_t>(v[j].ws);
+      if (!a0 || !b0) continue;
+      if (a0 < b0 + v[j].ws_bytes && b0 < a0 + v[i].ws_bytes) return QVLA_ERR_ARG;
+    }
   return cuda_status(launch_rotate_quant_batch(v.data(), n, stream));
 }
 

@@ -83,13 +83,16 @@ QVLA_DEVICE bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t 
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// sets QVLA_DEVERR_TIMEOUT) if it has not completed within kWaitLimitNs.
-QVLA_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
+// sets QVLA_DEVERR_TIMEOUT) if it has not completed within `limit_ns`
+// (kWaitLimitNs unless a caller asks for less).
+QVLA_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
+                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint32_t hint = limit_ns < 100000ull ? static_cast<uint32_t>(limit_ns) : 100000u;
   for (;;) {
-    if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
       report(err, QVLA_DEVERR_TIMEOUT);
       return false;
     }

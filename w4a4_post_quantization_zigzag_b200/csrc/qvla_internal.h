@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <vector>
 #include <stdint.h>
 
@@ -17,6 +18,22 @@ unsigned int* device_error_word();
 
 // Programmatic dependent launch on/off (environment QVLA_PDL=0 turns it off).
 bool pdl_enabled();
+
+// Runs `set` (kernel attribute calls, which bind to the current device only)
+// once per device: bit d of `done` records device d.  Concurrent first calls
+// may both run `set`, which is harmless (it sets the same values).  Devices
+// past 63 run it on every call.
+template <typename F>
+cudaError_t once_per_device(std::atomic<unsigned long long>& done, F set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ---- activation rotate + quantise (rotate_quant.cu)
 struct ActArgs {
@@ -93,9 +110,6 @@ struct GemmArgs {
   int split_k;
 };
 cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream);
-// persistent small-M GEMM (gemm_w4a4_rows.cu): M <= 64, no split-K;
-// `nt` is the token tile (16, 32 or 64) shared by every problem of the launch
-cudaError_t launch_w4a4_gemm_rows(const GemmArgs* const* gs, int n, int nt, cudaStream_t stream);
 
 // 2-D tiled tensor map over a row-major array (`inner` elements per row,
 // `outer` rows, row pitch `pitch` bytes), box `box_inner` x `box_outer`.

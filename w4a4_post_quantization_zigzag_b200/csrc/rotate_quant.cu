@@ -1069,16 +1069,15 @@ cudaError_t launch_group(const ActArgs* const* as, int n, cudaStream_t stream, i
   const size_t smem = Smem<BS, TT>::bytes(bpc_max, MODE == kDynamic);
   if (smem > static_cast<size_t>(kSmemCap)) return cudaErrorInvalidConfiguration;
   auto kern = rotq_kernel<BS, TT, Tin, MODE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
+  static std::atomic<unsigned long long> attr_done{0};
+  {
+    cudaError_t e = once_per_device(attr_done, [&]() {
+      cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
+      if (r == cudaSuccess && MODE == kDynamic)
+        r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      return r;
+    });
     if (e != cudaSuccess) return e;
-    if (MODE == kDynamic) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-    }
-    attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);
@@ -1268,15 +1267,15 @@ int tc_cluster(int M, int K) {
 // One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
 // mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
 bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
-  static EncodeTiledFnR enc = nullptr;
-  if (!enc) {
+  static const EncodeTiledFnR enc = []() -> EncodeTiledFnR {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
         q != cudaDriverEntryPointSuccess)
-      return false;
-    enc = reinterpret_cast<EncodeTiledFnR>(p);
-  }
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFnR>(p);
+  }();
+  if (!enc) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
   const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTM)};
@@ -1307,13 +1306,13 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
       kmax = std::max(kmax, a.K);
     }
     b.row_start[n] = rows;
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           QVLA_MAX_K * 2);
+    static std::atomic<unsigned long long> attr_done{0};
+    {
+      cudaError_t e = once_per_device(attr_done, []() {
+        return cudaFuncSetAttribute(permute_rows_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, QVLA_MAX_K * 2);
+      });
       if (e != cudaSuccess) return e;
-      attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(rows, 1, 1);
@@ -1371,13 +1370,15 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
   }
   batch.cta_start[n] = ctas;
   auto kern = rotq_tc_kernel<BS, MODE, kTmaA>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  static std::atomic<unsigned long long> attr_done{0};
+  {
+    cudaError_t e = once_per_device(attr_done, [&]() {
+      cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      return r;
+    });
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);

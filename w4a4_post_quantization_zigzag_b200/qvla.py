@@ -24,6 +24,21 @@ if not os.path.exists(LIB_PATH):
                       "`python -m w4a4_post_quantization_zigzag_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
+
+def _check_stamp():
+    """The loaded library must be the build of the sources next to it."""
+    from . import build as _build
+    _lib.qvla_source_hash.restype = ctypes.c_char_p
+    have = _lib.qvla_source_hash().decode()
+    want = _build.source_hash()
+    if have != want:
+        raise ImportError(f"{LIB_PATH} was built from other sources (stamp {have[:12]}, "
+                          f"sources {want[:12]}): rebuild it with "
+                          "`python -m w4a4_post_quantization_zigzag_b200.build`")
+
+
+_check_stamp()
+
 QVLA_OK = 0
 QVLA_ERR_ARG = 1
 QVLA_ERR_SHAPE = 2
@@ -53,6 +68,7 @@ EXPORTED = (
     "qvla_pack_weights_hadamard", "qvla_pack_weights_w8", "qvla_rotate_quant_act_a8",
     "qvla_rotate_quant_a8_workspace_bytes", "qvla_w8a8_gemm", "qvla_w8a8_gemm_s32",
     "qvla_gptq_quantize_host", "qvla_pack_weights_gptq", "qvla_gptq_hessian_host",
+    "qvla_selftest_wait_timeout", "qvla_source_hash",
 )
 
 QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -78,7 +94,9 @@ _PP = POINTER(qvla_linear_problem)
 _sig = {
     "qvla_status_str": (ctypes.c_char_p, [c_int]),
     "qvla_abi_version": (c_int, []),
+    "qvla_source_hash": (ctypes.c_char_p, []),
     "qvla_read_error_word": (c_int, [POINTER(c_uint32), c_int]),
+    "qvla_selftest_wait_timeout": (c_int, [ctypes.c_uint64, c_void_p]),
     "qvla_packed_sizes": (c_int, [c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t),
                                   POINTER(c_size_t), POINTER(c_size_t)]),
     "qvla_pack_weights": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
@@ -139,6 +157,10 @@ def qvla_abi_version() -> int:
     return _lib.qvla_abi_version()
 
 
+def qvla_source_hash() -> str:
+    return _lib.qvla_source_hash().decode()
+
+
 def _check(rc: int, where: str):
     if rc != QVLA_OK:
         raise QvlaError(rc, where)
@@ -160,6 +182,13 @@ def qvla_read_error_word(clear: bool = True) -> int:
     v = c_uint32(0)
     _check(_lib.qvla_read_error_word(ctypes.byref(v), int(clear)), "qvla_read_error_word")
     return int(v.value)
+
+
+def qvla_selftest_wait_timeout(limit_ns: int = 50_000, stream=None):
+    """Launch the failure-path self-test: a wait that nothing ends, bounded
+    by limit_ns; the error word then holds QVLA_DEVERR_TIMEOUT."""
+    _check(_lib.qvla_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "qvla_selftest_wait_timeout")
 
 
 def qvla_packed_sizes(N: int, K: int, block: int) -> Tuple[int, int, int, int]:
@@ -429,6 +458,22 @@ def _dtype_code(x: torch.Tensor) -> int:
     raise TypeError(f"unsupported activation dtype {x.dtype}")
 
 
+def _expect(t: torch.Tensor, dtype, shape, device, name: str):
+    """Caller-given buffers: the kernels write exactly this shape, densely."""
+    if (t.dtype != dtype or tuple(t.shape) != tuple(shape) or t.device != device
+            or not t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)} "
+                         f"on {device}, got {t.dtype} {tuple(t.shape)} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _expect_rows(x: torch.Tensor, K: int, name: str = "x"):
+    """Token rows [M, K] with unit stride along K (any row pitch)."""
+    if x.dim() != 2 or x.shape[1] != K or (x.numel() and x.stride(1) != 1):
+        raise ValueError(f"{name}: expected [M, {K}] rows with unit stride along K, "
+                         f"got shape {tuple(x.shape)} strides {tuple(x.stride())}")
+
+
 def _step_args(step):
     """int -> checked on the host; cuda int32 tensor -> read on the device."""
     if step is None:
@@ -452,11 +497,14 @@ def qvla_rotate_quant_act(x: torch.Tensor, L: PackedLinear, mode: int = QVLA_SCA
                           xq: Optional[torch.Tensor] = None, s_x: Optional[torch.Tensor] = None,
                           workspace: Optional[torch.Tensor] = None, stream=None):
     """workspace: optional uint8 device scratch of qvla_rotate_quant_workspace_bytes() bytes."""
+    _expect_rows(x, L.K)
     M = x.shape[0]
     if xq is None:
         xq = torch.empty(M, L.K // 2, dtype=torch.uint8, device=x.device)
     if s_x is None:
         s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    _expect(xq, torch.uint8, (M, L.K // 2), x.device, "xq")
+    _expect(s_x, torch.float32, (M,), x.device, "s_x")
     T, Lc = (table.shape if table is not None else (0, 0))
     sd, sh = _step_args(step)
     ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -475,7 +523,10 @@ def qvla_rotate_quant_act_noalloc(x: torch.Tensor, L: PackedLinear, xq: torch.Te
     the outputs are given, and the scratch is the library's fixed per-device
     array (at most QVLA_NOALLOC_SCRATCH_BYTES).  Calls that may overlap on the
     GPU race on that array."""
+    _expect_rows(x, L.K)
     M = x.shape[0]
+    _expect(xq, torch.uint8, (M, L.K // 2), x.device, "xq")
+    _expect(s_x, torch.float32, (M,), x.device, "s_x")
     T, Lc = (table.shape if table is not None else (0, 0))
     sd, sh = _step_args(step)
     _check(_lib.qvla_rotate_quant_act_noalloc(_ptr(x), _dtype_code(x), M, x.stride(0), L.struct,
