@@ -5,13 +5,18 @@ Default workload: the DiT action-head MLP stack (50 action tokens x batch 1,
 hidden 1024, gate/up 1024->4096 and down 4096->1024, 4 layers, bf16 input,
 10 denoising steps, per-step scale table [10][12], rotation block 64).
 One timed step = one denoising step = 12 rotated W4A4 linears: one batched
-rotate-quantise launch for all 12, then one batched W4A4 GEMM launch for all 12
-(the step's linears are independent: each draws its own input), replayed from a
-CUDA graph.  The same step with one launch per kernel and linear is reported
+rotate-quantise call for all 12 (it also writes the int8 image of the codes
+that the GEMM reads), then one batched W4A4 GEMM launch for all 12 (the
+step's linears are independent: each draws its own input), replayed from a
+CUDA graph.  The same step with one call per kernel and linear is reported
 beside it.
 The activation step index is a device scalar read by the rotate-quantise
-kernel.  L2 is flushed (512 MB written, then read back) before every timed step, so every step
-streams its packed weights from HBM.
+kernel.  L2 is flushed (512 MB written, then read back) before every timed
+step, so every step streams its packed weights and rotations from HBM.
+
+Besides the headline workload, the same line carries shorter measurements
+of the backbone prefill linears (1024 tokens, 2048<->16384) and of the full
+DiT denoise loop (512 tokens, 16 layers) under "secondary".
 
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on the
 same workload instead (the reference arm: the pages publish no code to run).
@@ -34,40 +39,47 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-import numpy as np  # noqa: E402
+import numpy as np  # noqa: E402,F401
 
 from w4a4_post_quantization_zigzag_b200 import inputs as I  # noqa: E402
 
 METRIC = "µs per DiT denoise step"
 UNIT = "us/step"
 L2_FLUSH_BYTES = 512 << 20
+WORKLOADS = ("dit_mlp_stack", "dit_mlp_stack_fused", "dit_denoise_loop",
+             "dit_denoise_loop_fused", "backbone_prefill", "single_linear")
+SECONDARY = ("backbone_prefill", "dit_denoise_loop")
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="dit_mlp_stack",
-                   choices=["dit_mlp_stack", "dit_mlp_stack_fused", "dit_denoise_loop",
-                            "backbone_prefill", "single_linear"])
+    p.add_argument("--workload", default="dit_mlp_stack", choices=WORKLOADS)
     p.add_argument("--rotation", default="composite", choices=["composite", "hadamard"],
                    help="composite: R = R_SVD.H (the method); hadamard: R_SVD = I variant")
     p.add_argument("--precision", default="w4a4", choices=["w4a4", "w8a8", "mix"],
                    help="w8a8: every linear W8A8 (dynamic per-token 8-bit activations); "
                         "mix: the down projections W8A8, the rest W4A4")
+    p.add_argument("--no-image", action="store_true",
+                   help="batched GEMM unpacks the packed codes instead of reading the image")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true")
+    p.add_argument("--secondary-steps", type=int, default=3)
     p.add_argument("--cpu-sample-steps", type=int, default=0,
                    help="oracle steps for the CPU baseline (0: sized to ~15 s)")
     p.add_argument("--quick", action="store_true",
-                   help="skip clocks, e2e and the CPU baseline (for profiler runs)")
-    return p.parse_args()
+                   help="skip clocks, e2e, the CPU baseline and the secondary workloads "
+                        "(for profiler runs)")
+    return p.parse_args(argv)
 
 
 def make_workload(name, rotation="composite"):
     wl = {"dit_mlp_stack": I.dit_mlp_stack, "dit_denoise_loop": I.dit_denoise_loop,
           "dit_mlp_stack_fused": lambda: I.dit_mlp_stack(fuse_gate_up=True),
+          "dit_denoise_loop_fused": lambda: I.dit_denoise_loop(fuse_qkv=True),
           "backbone_prefill": I.backbone_prefill, "single_linear": I.single_linear}[name]()
     if rotation == "hadamard":
         wl.name += "_hadamard_only"
@@ -89,6 +101,8 @@ def kernel_nodes(raw_graph):
 
 
 def load_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, source) from the machine's measured peaks,
+    else the recipe's fallback figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
@@ -106,6 +120,7 @@ class ClockSampler:
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
+        self.out = ""
 
     def __enter__(self):
         try:
@@ -118,7 +133,6 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.out = ""
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -180,6 +194,46 @@ def job_time_per_unit(total_ms: float, steps: int, world: int) -> float:
     return total_ms * 1e3 / (steps * world)
 
 
+# ------------------------------------------------------- roofline arithmetic
+def algorithmic_work(wl, w8, rotation="composite"):
+    """Per-step algorithmic bytes and ops of the two kernels (the work the
+    method must do, not what an implementation happens to move):
+      GEMM: N*K*c weights + M*K*c codes + 2*M*N bf16 out + 4*M s_x + 8*N s_w
+            and bias (c = bytes per code: 1/2 for 4-bit, 1 for 8-bit);
+            ops 2*M*N*K.
+      rotate-quantise: e_x*M*K input + M*K*c codes + 4*M scales + 4*K*b
+            R_SVD (fp32; none for the Hadamard-only variant) + 4*K perm."""
+    cb = [1.0 if is8 else 0.5 for is8 in w8]
+    gemm_bytes = sum(int(l.N * l.K * c) + int(l.M * l.K * c) + 2 * l.M * l.N + 4 * l.M + 8 * l.N
+                     for l, c in zip(wl.linears, cb))
+    gemm_ops = sum(2 * l.M * l.N * l.K for l in wl.linears)
+    rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + int(l.M * l.K * c) + 4 * l.M
+                    + (4 * l.K * l.block if rotation != "hadamard" else 0) + 4 * l.K
+                    for l, c in zip(wl.linears, cb))
+    weight_bytes = sum(int(l.N * l.K * c) + 8 * l.N for l, c in zip(wl.linears, cb))
+    return gemm_bytes, gemm_ops, rot_bytes, weight_bytes
+
+
+def roofline_entry(kernel, t_ms, nbytes, ops, hbm_gbs, int8_tops, peak_src, workload):
+    """Achieved vs peak for one kernel's per-step launch(es).  The bound is the
+    larger of bytes / HBM bandwidth and ops / int8 tensor peak."""
+    t_hbm = nbytes / (hbm_gbs * 1e9)
+    t_ten = ops / (int8_tops * 1e12) if ops else 0.0
+    if t_ten > t_hbm:
+        ach = ops / (t_ms * 1e-3) / 1e12
+        ent = {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": int8_tops,
+               "unit": "TOPS", "frac": ach / int8_tops,
+               "peak_source": f"2 x bf16_tflops ({peak_src}; dense int8 : bf16 = 2 : 1)"}
+    else:
+        ach = nbytes / (t_ms * 1e-3) / 1e9
+        ent = {"kernel": kernel, "bound": "hbm", "achieved": ach, "peak": hbm_gbs,
+               "unit": "GB/s", "frac": ach / hbm_gbs, "peak_source": f"hbm_gbs ({peak_src})"}
+    ent.update({"traffic": recorded_traffic(kernel, workload),
+                "algorithmic_bytes_per_launch": nbytes, "ops_per_launch": ops,
+                "avg_launch_us": t_ms * 1e3})
+    return ent
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_step(wl, packs, xs, t):
     from oracle import qvla_oracle as O
@@ -202,6 +256,13 @@ def oracle_setup(wl, steps):
     return packs, xs
 
 
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -209,6 +270,11 @@ def blas_threads():
         return max(n) if n else 1
     except Exception:
         return 1
+
+
+THREADING_NOTE = ("numpy fp64 rotation products and Gram eigensolves on the BLAS/LAPACK "
+                  "threads; the fp32 RTN, the int64 GEMM (numpy integer matmul, no BLAS) "
+                  "and the dequantisation on one core")
 
 
 def cpu_baseline(wl, sample_steps):
@@ -223,7 +289,8 @@ def cpu_baseline(wl, sample_steps):
         if (sample_steps and n >= sample_steps) or (not sample_steps and (el > 12.0 or n >= 50)):
             break
     us = el / n * 1e6
-    return {"value": us, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": us, "unit": UNIT, "cores": host_cores(), "blas_threads": blas_threads(),
+            "threading": THREADING_NOTE, "kind": "oracle",
             "sample": f"{n} full denoise step(s) of {wl.name} ({len(wl.linears)} linears each); "
                       f"numpy fp64 rotation, fp32 RTN, int64 GEMM, fp64 dequant"}
 
@@ -246,7 +313,8 @@ def run_reference(args):
             "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name},
-            "cpu_baseline": {"value": us, "unit": UNIT, "cores": blas_threads(),
+            "cpu_baseline": {"value": us, "unit": UNIT, "cores": host_cores(),
+                             "blas_threads": blas_threads(), "threading": THREADING_NOTE,
                              "kind": "oracle",
                              "sample": f"each step: one full denoise step of {wl.name}"},
             "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -255,106 +323,137 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------- ours
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
+class DeviceStep:
+    """One workload on the device: packed linears, per-step inputs (device
+    resident; each step's inputs are one contiguous buffer, mirrored in pinned
+    host memory), outputs (one contiguous buffer), scratch, and the batched and
+    per-linear step functions."""
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    from w4a4_post_quantization_zigzag_b200 import build as B
-    B.build()
-    from w4a4_post_quantization_zigzag_b200 import qvla as Q
-
-    wl = make_workload(args.workload, args.rotation)
-    T = max(1, wl.steps)
-    table = torch.from_numpy(wl.table).to(dev) if wl.table is not None else None
-    steps_dev = torch.arange(T, dtype=torch.int32, device=dev)
-    mode = Q.QVLA_SCALE_TABLE if wl.mode == "table" else Q.QVLA_SCALE_DYNAMIC
-
-    # pack (offline step, timed for information)
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    # which linears run W8A8 (dynamic 8-bit activations, one launch sequence
-    # each) and which W4A4 (batched)
-    w8 = [args.precision == "w8a8" or (args.precision == "mix" and lin.name.endswith("down"))
-          for lin in wl.linears]
-    packs = []
-    for lin, is8 in zip(wl.linears, w8):
-        W = torch.from_numpy(lin.make_w()).to(dev)
-        pack = (Q.qvla_pack_weights_w8 if is8 else
-                Q.qvla_pack_weights_hadamard if wl.rotation == "hadamard" else Q.qvla_pack_weights)
-        packs.append(pack(W, lin.block, bias=torch.from_numpy(lin.make_bias()).to(dev)))
-        del W
-    torch.cuda.synchronize()
-    pack_s = time.perf_counter() - t0
-
-    # per-step inputs (device resident) and outputs
-    xdt = torch.bfloat16 if wl.linears[0].x_dtype == "bf16" else torch.float32
-    xs_host = [[torch.from_numpy(l.make_x(seed_offset=t, std=(float(wl.sigmas[t])
-                                                              if wl.sigmas is not None else None)))
-                .to(xdt).pin_memory() for l in wl.linears] for t in range(T)]
-    xs = [[x.to(dev) for x in row] for row in xs_host]
-    xq = [torch.empty(l.M, l.K, dtype=torch.int8, device=dev) if is8 else
-          torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev)
-          for l, is8 in zip(wl.linears, w8)]
-    sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
-    ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in wl.linears]
-    # scratch of the tensor-core rotation route (the permuted copy of x; for a
-    # W8A8 linear also its fp32 rotated rows), one per linear since a batched
-    # launch runs them together
-    wss = [torch.empty(max(Q.qvla_rotate_quant_a8_workspace_bytes(l.M, l.K) if is8 else
-                           Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
-                       dtype=torch.uint8, device=dev) for l, is8 in zip(wl.linears, w8)]
-    nl = len(wl.linears)
-    # one problem set per denoising step: same packed weights and buffers, the
-    # step's own inputs and device step index
-    probs = [[Q.LinearProblem(L, xs[t][i], mode, table=table, step=steps_dev[t:t + 1],
-                              layer=lin.layer, xq=xq[i], s_x=sx[i], y=ys[i], workspace=wss[i])
-              for i, (lin, L) in enumerate(zip(wl.linears, packs)) if not w8[i]]
-             for t in range(T)]
-    idx8 = [i for i in range(len(wl.linears)) if w8[i]]
-
-    def w8_linears(t, phase):
-        for i in idx8:
-            if phase == 0:
-                Q.qvla_rotate_quant_act_a8(xs[t][i], packs[i], xq8=xq[i], s_x=sx[i],
-                                           workspace=wss[i])
+    def __init__(self, wl, Q, dev, precision="w4a4", image=True, pack_fn=None):
+        """pack_fn(lin, W, bias) -> packed linear replaces the default pack
+        (tests pass one that feeds the oracle's permutation and R_SVD)."""
+        import torch
+        self.wl, self.Q, self.dev = wl, Q, dev
+        self.T = T = max(1, wl.steps)
+        self.table = torch.from_numpy(wl.table).to(dev) if wl.table is not None else None
+        self.steps_dev = torch.arange(T, dtype=torch.int32, device=dev)
+        self.mode = Q.QVLA_SCALE_TABLE if wl.mode == "table" else Q.QVLA_SCALE_DYNAMIC
+        self.w8 = [precision == "w8a8" or (precision == "mix" and lin.name.endswith("down"))
+                   for lin in wl.linears]
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        self.packs = []
+        for lin, is8 in zip(wl.linears, self.w8):
+            W = torch.from_numpy(lin.make_w()).to(dev)
+            b = torch.from_numpy(lin.make_bias()).to(dev)
+            if pack_fn is not None:
+                self.packs.append(pack_fn(lin, W, b))
             else:
-                Q.qvla_w8a8_gemm(xq[i], sx[i], packs[i], y=ys[i])
+                pack = (Q.qvla_pack_weights_w8 if is8 else
+                        Q.qvla_pack_weights_hadamard if wl.rotation == "hadamard" else
+                        Q.qvla_pack_weights)
+                self.packs.append(pack(W, lin.block, bias=b))
+            del W
+        torch.cuda.synchronize()
+        self.pack_s = time.perf_counter() - t0
 
-    def step_batched(t, rec=None):
+        xdt = torch.bfloat16 if wl.linears[0].x_dtype == "bf16" else torch.float32
+
+        def carve(flat, shapes):
+            """Row-major views [r, c] of a flat buffer, each 16-byte aligned."""
+            out, off = [], 0
+            step = 16 // flat.element_size()
+            for r, c in shapes:
+                out.append(flat[off:off + r * c].view(r, c))
+                off += r * c + (-(r * c)) % step
+            return out
+
+        def total(shapes, esz):
+            step = 16 // esz
+            return sum(r * c + (-(r * c)) % step for r, c in shapes)
+
+        xshapes = [(l.M, l.K) for l in wl.linears]
+        xtot = total(xshapes, 2 if xdt == torch.bfloat16 else 4)
+        self.x_host, self.x_dev, self.xs = [], [], []
+        for t in range(T):
+            hb = torch.empty(xtot, dtype=xdt).pin_memory()
+            std = float(wl.sigmas[t]) if wl.sigmas is not None else None
+            for v, l in zip(carve(hb, xshapes), wl.linears):
+                v.copy_(torch.from_numpy(l.make_x(seed_offset=t, std=std)).to(xdt))
+            db = hb.to(dev)
+            self.x_host.append(hb)
+            self.x_dev.append(db)
+            self.xs.append(carve(db, xshapes))
+        yshapes = [(l.M, l.N) for l in wl.linears]
+        self.y_dev = torch.empty(total(yshapes, 2), dtype=torch.bfloat16, device=dev)
+        self.ys = carve(self.y_dev, yshapes)
+        self.xq = [torch.empty(l.M, l.K, dtype=torch.int8, device=dev) if is8 else
+                   torch.empty(l.M, l.K // 2, dtype=torch.uint8, device=dev)
+                   for l, is8 in zip(wl.linears, self.w8)]
+        self.sx = [torch.empty(l.M, dtype=torch.float32, device=dev) for l in wl.linears]
+        # scratch of the tensor-core rotation route (the permuted copy of x; for a
+        # W8A8 linear also its fp32 rotated rows), one per linear since a batched
+        # launch runs them together
+        self.wss = [torch.empty(max(Q.qvla_rotate_quant_a8_workspace_bytes(l.M, l.K) if is8 else
+                                    Q.qvla_rotate_quant_workspace_bytes(l.M, l.K, l.block), 16),
+                                dtype=torch.uint8, device=dev)
+                    for l, is8 in zip(wl.linears, self.w8)]
+        # the int8 image of each W4A4 linear's codes: written by the batched
+        # rotate-quantise, read by the batched GEMM
+        self.img = [torch.empty(l.M, l.K, dtype=torch.int8, device=dev)
+                    if (image and not is8) else None for l, is8 in zip(wl.linears, self.w8)]
+        self.probs = [[Q.LinearProblem(L, self.xs[t][i], self.mode, table=self.table,
+                                       step=self.steps_dev[t:t + 1], layer=lin.layer,
+                                       xq=self.xq[i], s_x=self.sx[i], y=self.ys[i],
+                                       workspace=self.wss[i], xq8=self.img[i])
+                       for i, (lin, L) in enumerate(zip(wl.linears, self.packs)) if not self.w8[i]]
+                      for t in range(T)]
+        self.idx8 = [i for i in range(len(wl.linears)) if self.w8[i]]
+
+    def w8_linears(self, t, phase):
+        Q = self.Q
+        for i in self.idx8:
+            if phase == 0:
+                Q.qvla_rotate_quant_act_a8(self.xs[t][i], self.packs[i], xq8=self.xq[i],
+                                           s_x=self.sx[i], workspace=self.wss[i])
+            else:
+                Q.qvla_w8a8_gemm(self.xq[i], self.sx[i], self.packs[i], y=self.ys[i])
+
+    def step_batched(self, t, rec=None):
+        Q = self.Q
         if rec is not None:
             rec[0].record()
-        if probs[t]:
-            Q.qvla_rotate_quant_act_batched(probs[t])
-        w8_linears(t, 0)
+        if self.probs[t]:
+            Q.qvla_rotate_quant_act_batched(self.probs[t])
+        self.w8_linears(t, 0)
         if rec is not None:
             rec[1].record()
-        if probs[t]:
-            Q.qvla_w4a4_gemm_batched(probs[t])
-        w8_linears(t, 1)
+        if self.probs[t]:
+            Q.qvla_w4a4_gemm_batched(self.probs[t])
+        self.w8_linears(t, 1)
         if rec is not None:
             rec[2].record()
 
-    def step_per_linear(t):
-        for i, (lin, L) in enumerate(zip(wl.linears, packs)):
-            if w8[i]:
-                Q.qvla_rotate_quant_act_a8(xs[t][i], L, xq8=xq[i], s_x=sx[i], workspace=wss[i])
-                Q.qvla_w8a8_gemm(xq[i], sx[i], L, y=ys[i])
+    def step_per_linear(self, t):
+        Q = self.Q
+        for i, (lin, L) in enumerate(zip(self.wl.linears, self.packs)):
+            if self.w8[i]:
+                Q.qvla_rotate_quant_act_a8(self.xs[t][i], L, xq8=self.xq[i], s_x=self.sx[i],
+                                           workspace=self.wss[i])
+                Q.qvla_w8a8_gemm(self.xq[i], self.sx[i], L, y=self.ys[i])
                 continue
-            Q.qvla_rotate_quant_act(xs[t][i], L, mode, table=table, step=steps_dev[t:t + 1],
-                                    layer=lin.layer, xq=xq[i], s_x=sx[i], workspace=wss[i])
-            Q.qvla_w4a4_gemm(xq[i], sx[i], L, y=ys[i])
+            Q.qvla_rotate_quant_act(self.xs[t][i], L, self.mode, table=self.table,
+                                    step=self.steps_dev[t:t + 1], layer=lin.layer, xq=self.xq[i],
+                                    s_x=self.sx[i], workspace=self.wss[i])
+            Q.qvla_w4a4_gemm(self.xq[i], self.sx[i], L, y=self.ys[i])
 
-    stream = torch.cuda.Stream(device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+def measure(ds, stream, steps, warmup, *, per_linear=True, warm=True, e2e=False,
+            sampler=None, barrier=None):
+    """Graph-replayed timing of one DeviceStep; returns a dict (ms values)."""
+    import torch
+    Q, T = ds.Q, ds.T
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=ds.dev)
 
     def l2_flush():
         """Cold L2 for the next step: write a buffer four times the L2, then
@@ -376,20 +475,16 @@ def run_ours(args):
         return gs, nk
 
     with torch.cuda.stream(stream):
-        step_batched(0)               # first calls resolve attributes outside capture
-        step_per_linear(0)
+        ds.step_batched(0)               # first calls resolve attributes outside capture
+        if per_linear:
+            ds.step_per_linear(0)
         torch.cuda.synchronize()
-        graphs, kernels_per_step = capture(step_batched)
-        graphs_pl, _ = capture(step_per_linear)
+        graphs, kernels_per_step = capture(ds.step_batched)
+        graphs_pl = capture(ds.step_per_linear)[0] if per_linear else None
     torch.cuda.synchronize()
     assert Q.qvla_read_error_word(clear=True) == 0
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    barrier = barrier or torch.cuda.synchronize
 
     def timed_replays(gs, n, flush_l2=True):
         starts = [ev() for _ in range(n)]
@@ -403,130 +498,186 @@ def run_ours(args):
                 ends[i].record()
         return starts, ends
 
-    # ---- warm-up
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
+        for i in range(warmup):
             l2_flush()
             graphs[i % T].replay()
-            l2_flush()
-            graphs_pl[i % T].replay()
-    # ---- timed steps: graph replay of the batched step, L2 flushed before each
-    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(gpu_uuid) if not args.quick else None
+            if graphs_pl:
+                l2_flush()
+                graphs_pl[i % T].replay()
     barrier()
     if sampler:
         sampler.__enter__()
-    starts, ends = timed_replays(graphs, args.steps)
+    starts, ends = timed_replays(graphs, steps)
     barrier()
     if sampler:
         sampler.__exit__()
-    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    tot_ms = max_over_ranks(sum(per_step_ms), dev)
-    ms_per_step = tot_ms / args.steps
-    us_job = job_time_per_unit(tot_ms, args.steps, world)
-
-    # ---- the same steps, one launch per kernel and linear (informational)
-    s2, e2 = timed_replays(graphs_pl, args.steps)
-    torch.cuda.synchronize()
-    per_linear_us = sum(a.elapsed_time(b) for a, b in zip(s2, e2)) * 1e3 / args.steps
-
-    # ---- the batched step with a warm L2 (no flush between steps; informational)
-    sw_, ew_ = timed_replays(graphs, args.steps, flush_l2=False)
-    torch.cuda.synchronize()
-    warm_us = sum(a.elapsed_time(b) for a, b in zip(sw_, ew_)) * 1e3 / args.steps
-
-    # ---- per-kernel breakdown: eager launches with events on the launching
-    # stream; a GPU sleep ahead of the events keeps host enqueue time out
+    out = {"step_ms": [a.elapsed_time(b) for a, b in zip(starts, ends)],
+           "kernels_per_step": kernels_per_step}
+    if graphs_pl:
+        s2, e2 = timed_replays(graphs_pl, steps)
+        torch.cuda.synchronize()
+        out["per_linear_ms"] = sum(a.elapsed_time(b) for a, b in zip(s2, e2)) / steps
+    if warm:
+        sw, ew = timed_replays(graphs, steps, flush_l2=False)
+        torch.cuda.synchronize()
+        out["warm_ms"] = sum(a.elapsed_time(b) for a, b in zip(sw, ew)) / steps
+    # per-kernel breakdown: eager calls with events on the launching stream; a
+    # GPU sleep ahead of the events keeps host enqueue time out
     krot, kgemm = [], []
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
+        for i in range(steps):
             rec = [ev(), ev(), ev()]
             l2_flush()
             torch.cuda._sleep(2_000_000)
-            step_batched(i % T, rec)
+            ds.step_batched(i % T, rec)
             stream.synchronize()
             krot.append(rec[0].elapsed_time(rec[1]))
             kgemm.append(rec[1].elapsed_time(rec[2]))
     assert Q.qvla_read_error_word(clear=True) == 0
-
-    # ---- end to end: pinned-host inputs in, outputs back, every step
-    e2e = None
-    if not args.quick:
-        y_host = [torch.empty(l.M, l.N, dtype=torch.bfloat16).pin_memory() for l in wl.linears]
-        h2d = sum(x.numel() * x.element_size() for x in xs_host[0])
-        d2h = sum(y.numel() * y.element_size() for y in y_host)
+    out["rot_ms"] = sum(krot) / steps
+    out["gemm_ms"] = sum(kgemm) / steps
+    if e2e:
+        # end to end: each step's inputs copied in from pinned host memory (one
+        # contiguous copy), the step replayed, all outputs copied back (one
+        # contiguous copy), inside the timed region
+        y_host = torch.empty(ds.y_dev.shape, dtype=ds.y_dev.dtype).pin_memory()
         e0, e1 = ev(), ev()
         barrier()
         with torch.cuda.stream(stream):
             e0.record()
-            for i in range(args.steps):
+            for i in range(steps):
                 t = i % T
-                for x_d, x_h in zip(xs[t], xs_host[t]):
-                    x_d.copy_(x_h, non_blocking=True)
+                ds.x_dev[t].copy_(ds.x_host[t], non_blocking=True)
                 graphs[t].replay()
-                for y_d, y_h in zip(ys, y_host):
-                    y_h.copy_(y_d, non_blocking=True)
+                y_host.copy_(ds.y_dev, non_blocking=True)
             e1.record()
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        out["e2e_ms"] = e0.elapsed_time(e1)
+        out["h2d_bytes"] = ds.x_host[0].numel() * ds.x_host[0].element_size()
+        out["d2h_bytes"] = y_host.numel() * y_host.element_size()
+    del graphs, graphs_pl
+    return out
+
+
+def secondary_line(name, Q, dev, stream, steps, peaks):
+    """Shorter measurement of another workload (graph replay, L2 flushed)."""
+    import torch
+    hbm, bf16_tf, src = peaks
+    wl = make_workload(name)
+    ds = DeviceStep(wl, Q, dev)
+    m = measure(ds, stream, steps, 2, per_linear=False, warm=False)
+    us = sum(m["step_ms"]) / steps * 1e3
+    gb, gops, rb, _ = algorithmic_work(wl, ds.w8)
+    r = {"workload": wl.name, "value": us, "unit": UNIT, "steps": steps,
+         "kernels_us_per_step": {"rotate_quant": m["rot_ms"] * 1e3,
+                                 "w4a4_gemm": m["gemm_ms"] * 1e3},
+         "tops": gops / (us * 1e-6) / 1e12,
+         "rooflines": [roofline_entry("rotate_quant", m["rot_ms"], rb, 0, hbm, 2 * bf16_tf, src,
+                                      wl.name),
+                       roofline_entry("w4a4_gemm", m["gemm_ms"], gb, gops, hbm, 2 * bf16_tf,
+                                      src, wl.name)],
+         "kernels_per_step": m["kernels_per_step"][0],
+         "pack_s": ds.pack_s}
+    del ds
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return r
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from w4a4_post_quantization_zigzag_b200 import build as B
+    B.build()
+    from w4a4_post_quantization_zigzag_b200 import qvla as Q
+
+    wl = make_workload(args.workload, args.rotation)
+    ds = DeviceStep(wl, Q, dev, args.precision, image=not args.no_image)
+    stream = torch.cuda.Stream(device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_uuid) if not args.quick else None
+    m = measure(ds, stream, args.steps, args.warmup, e2e=not args.quick, sampler=sampler,
+                barrier=barrier)
+    tot_ms = max_over_ranks(sum(m["step_ms"]), dev)
+    ms_per_step = tot_ms / args.steps
+    us_job = job_time_per_unit(tot_ms, args.steps, world)
+    e2e = None
+    if "e2e_ms" in m:
+        e2e_ms = max_over_ranks(m["e2e_ms"], dev)
         e2e = {"value": job_time_per_unit(e2e_ms, args.steps, world), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": m["h2d_bytes"], "d2h_bytes_per_step": m["d2h_bytes"]}
 
-    # ---- roofline of the dominant kernel
-    hbm, bf16_tf, peak_src = load_peaks()
-    cb = [1.0 if is8 else 0.5 for is8 in w8]          # code bytes per element
-    gemm_bytes = sum(int(l.N * l.K * c) + int(l.M * l.K * c) + 2 * l.M * l.N + 4 * l.M + 8 * l.N
-                     for l, c in zip(wl.linears, cb))
-    rot_bytes = sum((2 if l.x_dtype == "bf16" else 4) * l.M * l.K + int(l.M * l.K * c) + 4 * l.M
-                    + (4 * l.K * l.block if wl.rotation != "hadamard" else 0) + 4 * l.K
-                    for l, c in zip(wl.linears, cb))
-    weight_bytes = sum(int(l.N * l.K * c) + 8 * l.N for l, c in zip(wl.linears, cb))
-    t_gemm = sum(kgemm) / args.steps          # ms per step (one batched launch)
-    t_rot = sum(krot) / args.steps
-    dom = "w4a4_gemm" if t_gemm >= t_rot else "rotate_quant"
-    if dom == "w4a4_gemm":
-        per_launch_bytes, per_launch_ms = gemm_bytes, t_gemm
-    else:
-        per_launch_bytes, per_launch_ms = rot_bytes, t_rot
-    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
-    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "peak_source": f"hbm_gbs ({peak_src})",
-            "traffic": recorded_traffic(dom, wl.name),
-            "algorithmic_bytes_per_launch": per_launch_bytes,
-            "avg_launch_us": per_launch_ms * 1e3}
-
+    # ---- rooflines: every kernel of the step, the dominant one on top
+    peaks = load_peaks()
+    hbm, bf16_tf, peak_src = peaks
+    gb, gops, rb, wb = algorithmic_work(wl, ds.w8, wl.rotation)
+    roofs = [roofline_entry("rotate_quant", m["rot_ms"], rb, 0, hbm, 2 * bf16_tf, peak_src,
+                            wl.name),
+             roofline_entry("w4a4_gemm", m["gemm_ms"], gb, gops, hbm, 2 * bf16_tf, peak_src,
+                            wl.name)]
+    dom = max(roofs, key=lambda r: r["avg_launch_us"])
     ops = wl.ops_per_step()
+    kps = m["kernels_per_step"]
     line = {
         "metric": METRIC, "value": us_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
         "config": {"workload": wl.name, "rotation": wl.rotation, "precision": args.precision,
-                   "w8a8_linears": len(idx8), "tokens_M": wl.linears[0].M,
-                   "linears_per_step": nl, "denoise_steps_T": T,
+                   "w8a8_linears": len(ds.idx8), "tokens_M": wl.linears[0].M,
+                   "linears_per_step": len(wl.linears), "denoise_steps_T": ds.T,
                    "block": wl.linears[0].block, "scale": wl.mode,
-                   "l2": "flushed before every timed step (512 MB written, then read back: cold, clean L2)",
+                   "gemm_activations": "packed codes" if args.no_image else "int8 image",
+                   "l2": "flushed before every timed step (512 MB written, then read back: "
+                         "cold, clean L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single"},
-        "roofline": roof,
+        "roofline": dom,
+        "rooflines": roofs,
         "tops": ops / (ms_per_step * 1e-3) / 1e12,
         "tops_frac_int8": ops / (ms_per_step * 1e-3) / 1e12 / (2.0 * bf16_tf),
         "int8_peak_tops": {"value": 2.0 * bf16_tf,
                            "source": f"2 x bf16_tflops ({peak_src}; dense int8 : bf16 = 2 : 1)"},
-        "l2_warm_us_per_step": warm_us,
-        "weight_gbs": weight_bytes / (ms_per_step * 1e-3) / 1e9,
-        "kernels_us_per_step": {"rotate_quant": t_rot * 1e3, "w4a4_gemm": t_gemm * 1e3},
-        "per_linear_launches_us_per_step": per_linear_us,
-        "pack_s": pack_s,
-        "gpu_launches": sum(kernels_per_step[i % T] for i in range(args.steps)),
-        "kernels_per_step": kernels_per_step[0],
+        "weight_gbs": wb / (ms_per_step * 1e-3) / 1e9,
+        "kernels_us_per_step": {"rotate_quant": m["rot_ms"] * 1e3,
+                                "w4a4_gemm": m["gemm_ms"] * 1e3},
+        "per_linear_launches_us_per_step": m.get("per_linear_ms", 0.0) * 1e3,
+        "l2_warm_us_per_step": m.get("warm_ms", 0.0) * 1e3,
+        "pack_s": ds.pack_s,
+        "gpu_launches": sum(kps[i % ds.T] for i in range(args.steps)),
+        "kernels_per_step": kps[0],
+        "source_hash": Q.qvla_source_hash()[:16],
         "e2e": e2e,
     }
     if sampler:
         line["clocks"] = sampler.summary()
+    del ds
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if not args.quick and not args.no_secondary and args.workload == "dit_mlp_stack" \
+            and args.rotation == "composite" and args.precision == "w4a4":
+        # every rank runs the same secondary work (no collectives inside)
+        line["secondary"] = [secondary_line(n, Q, dev, stream, args.secondary_steps, peaks)
+                             for n in SECONDARY]
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_steps)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs, graphs_pl
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

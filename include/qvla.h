@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define QVLA_ABI_VERSION 1
+#define QVLA_ABI_VERSION 2
 #define QVLA_MAX_K 32768
 
 typedef enum {
@@ -105,8 +105,8 @@ typedef struct {
   const int32_t* perm;      /* [K]  zigzag permutation                      */
   const float* rot;         /* [nb][b][b] R_SVD blocks, or NULL: R_SVD = I  */
                             /* (Hadamard-only rotation, R_B = H_b)           */
-  const uint16_t* rot_tc;   /* tensor-core images of R_B, or NULL (must be  */
-                            /* NULL when rot is NULL)                        */
+  const uint16_t* rot_tc;   /* tensor-core images of R_B, or NULL (with rot */
+                            /* NULL: the image of R_B = H_b)                 */
   const uint8_t* wq;        /* [N][K/2] packed weight codes                 */
   const float* w_scale;     /* [N]  s_w                                      */
   const float* bias;        /* [N]  or NULL                                  */
@@ -173,15 +173,18 @@ qvla_status qvla_pack_weights(const float* W, int N, int K, int block, const int
  * activations; the composite-rotation ablation of "{Omega}-QVLA"
  * Methodology 1, SVD factor removed).  The zigzag permutation is kept:
  * perm_in host int32 [K] or NULL (computed as in qvla_pack_weights()).
- * Outputs (device): perm_out [K], wq_out [N][K/2], w_scale_out [N];
- * W' = W P H is formed in fp64 and rounded once to fp32 before RTN.  The
- * packed linear built from these has rot = NULL and rot_tc = NULL; the
- * activation side then applies only the fast Walsh-Hadamard transform.
+ * Outputs (device): perm_out [K], rot_tc_out (optional, NULL to skip: the
+ * tensor-core image of R_B = H_b for blocks 64 / 128, rot_tc_bytes of
+ * qvla_packed_sizes()), wq_out [N][K/2], w_scale_out [N]; W' = W P H is
+ * formed in fp64 and rounded once to fp32 before RTN.  The packed linear
+ * built from these has rot = NULL; with the image, bf16 activations take the
+ * tensor-core rotation, otherwise the fast Walsh-Hadamard transform alone.
  * workspace device, >= ws_bytes from qvla_packed_sizes().  Blocks the calling
  * thread (one synchronisation for the host-side sort, one at the end).
  * ------------------------------------------------------------------------- */
 qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
-                                       const int32_t* perm_in, int32_t* perm_out, uint8_t* wq_out,
+                                       const int32_t* perm_in, int32_t* perm_out,
+                                       uint16_t* rot_tc_out, uint8_t* wq_out,
                                        float* w_scale_out, void* workspace, size_t ws_bytes,
                                        cudaStream_t stream);
 
@@ -193,15 +196,17 @@ qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
  * |W'[n,k]| / 127), q = clamp(rint(W'/s_w), -127, 127).
  * Outputs (device): perm_out [K], rot_out [nb][b][b] fp32, wq_out [N][K]
  * int8 (one code per byte: N * K bytes, not the N * K / 2 of
- * qvla_packed_sizes()), w_scale_out [N].  No tensor-core image: a packed
- * linear built from these has rot_tc = NULL, and its wq must only be given to
- * qvla_w8a8_gemm() / qvla_w8a8_gemm_s32().  Other arguments and the blocking
- * behaviour as qvla_pack_weights().
+ * qvla_packed_sizes()), w_scale_out [N], and optionally rot_tc_out (the
+ * tensor-core image of R_B as in qvla_pack_weights(), NULL to skip; with it
+ * the activation rotation of qvla_rotate_quant_act_a8() runs on the tensor
+ * cores).  Its wq must only be given to qvla_w8a8_gemm() /
+ * qvla_w8a8_gemm_s32().  Other arguments and the blocking behaviour as
+ * qvla_pack_weights().
  * ------------------------------------------------------------------------- */
 qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const int32_t* perm_in,
                                  const double* rsvd_in, int32_t* perm_out, float* rot_out,
-                                 uint8_t* wq_out, float* w_scale_out, void* workspace,
-                                 size_t ws_bytes, cudaStream_t stream);
+                                 uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
+                                 void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * GPTQ rounding of rotated weights ("Omega-QVLA: Nen VLA W4A4 tren Edge",
@@ -252,10 +257,9 @@ qvla_status qvla_pack_weights_gptq(const float* W, int N, int K, int block, cons
  * 127), one int8 code per byte.  When the workspace holds M * K * 6 bytes
  * (qvla_rotate_quant_a8_workspace_bytes) the last M * K * 2 take the
  * permuted copy of x that the tensor-core rotation reads through TMA (bf16
- * input and a linear that carries a tensor-core image, block 64 / 128; the
- * packs of qvla_pack_weights_w8() carry none, so their rotation runs on the
- * CUDA cores and leaves that part unused); with M * K * 4 the rotation
- * gathers instead (same result).  x, xdt, ldx, L as in qvla_rotate_quant_act().  Outputs
+ * input and a linear that carries a tensor-core image, block 64 / 128; a
+ * pack without the image rotates on the CUDA cores and leaves that part
+ * unused); with M * K * 4 the rotation gathers instead (same result).  x, xdt, ldx, L as in qvla_rotate_quant_act().  Outputs
  * (device): xq8 [M][K] int8, s_x [M] fp32.  Asynchronous (two or three
  * launches).                                                               */
 qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int ldx,
@@ -375,19 +379,20 @@ qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mo
  * W4A4 GEMM with fused dequantisation:
  *   acc[m,n] = sum_k q_x[m,k] q_w[n,k]            (exact, int32)
  *   y[m,n]   = bf16( fp32(s_x[m] * s_w[n]) * fp32(acc) + b[n] )
- * int4 codes are unpacked to 8-bit in shared memory and multiplied on the
- * tcgen05 tensor cores (kind::i8, int32 accumulators in tensor memory).
- * Each code q is unpacked as the int8 value 16*q (a nibble moved into the
- * high half of its byte), so the tensor cores accumulate 256*acc exactly
- * (|256*acc| <= 256*64*K < 2^31 for K <= QVLA_MAX_K) and the epilogue
- * shifts it back.
- * Small M uses split-K over a thread-block cluster with the partial sums
- * reduced through distributed shared memory (no workspace).
+ * The int4 weight codes are unpacked to 8-bit values in tensor memory and
+ * multiplied on the tcgen05 tensor cores (kind::i8, A operand from tensor
+ * memory, int32 accumulators in tensor memory); the activation codes are
+ * unpacked in shared memory (or read as the int8 image, see
+ * qvla_linear_problem.xq8).  Each code q enters as the int8 value 16*q (a
+ * nibble moved into the high half of its byte), so the tensor cores
+ * accumulate 256*acc exactly (|256*acc| <= 256*64*K < 2^31 for
+ * K <= QVLA_MAX_K) and the epilogue shifts it back.
+ * One persistent CTA per SM walks a list of 128-channel x (16..128)-token
+ * tiles that the host deals out longest first; no workspace.
  * xq device [M][K/2]; s_x device [M]; y device bf16 [M][ldy].
- * split_k: 0 = automatic, else 1, 2, 4, 8 or 16, at most ceil(K / 256)
- * (K is consumed in 256-wide tiles; split s takes a contiguous run of them).
- * Split-K applies for M <= 128; larger M always runs unsplit (its token
- * tiles supply the parallelism), whatever split_k says.
+ * split_k: 0, 1, 2, 4, 8 or 16, at most ceil(K / 256); accepted for source
+ * compatibility and otherwise ignored (the tile schedule balances the work;
+ * results do not depend on it).
  * N may be any positive size; ragged M, N and K tails are zero-filled.      */
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
                            const qvla_packed_linear* L, void* y, int ldy, int split_k,
@@ -427,7 +432,20 @@ typedef struct {
   int32_t ldy;
   void* workspace;               /* optional rotate-quant scratch, or NULL      */
   size_t ws_bytes;               /* (qvla_rotate_quant_workspace_bytes)         */
+  int8_t* xq8;                   /* optional device [M][K] int8 image of the    */
+                                 /* codes (see below), or NULL                  */
 } qvla_linear_problem;
+
+/* The int8 image of the activation codes (xq8), the GEMM's B operand as the
+ * tensor cores take it: byte k of a row is 16 * q[j] with, inside every
+ * aligned group of 32 codes, the 16 even-indexed codes first and then the 16
+ * odd-indexed ones (k = 32g + i holds code 32g + 2i for i < 16 and code
+ * 32g + 2(i - 16) + 1 otherwise).  It is a fixed rearrangement of xq: each
+ * packed byte's low nibble moves to the high half of one image byte and its
+ * high nibble to another.  When a problem gives xq8, the batched
+ * rotate-quantise writes it next to xq and s_x, and the batched GEMM reads
+ * its activations from it (one TMA box straight into the MMA layout) instead
+ * of unpacking xq; the results are identical.  Row pitch K, 16-byte aligned. */
 
 /* qvla_rotate_quant_act for every problem (reads x, writes xq and s_x). */
 qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int n,

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     q = _lib_mod()
-    assert q.qvla_abi_version() == 1
+    assert q.qvla_abi_version() == 2
     for code in range(9):
         assert q.qvla_status_str(code)
     assert q.qvla_status_str(q.QVLA_ERR_STEP_RANGE).startswith("denoising step")
@@ -71,9 +71,9 @@ def test_argument_errors_before_any_cuda_call():
     Lbad = q.qvla_packed_linear(128, 250, 64, 16, 16, None, 16, 16, None)
     assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lbad),
                                    ctypes.c_void_p(16), None) == q.QVLA_ERR_SHAPE
-    # a tensor-core image without R_SVD blocks (rot NULL means R_SVD = I)
-    Lhad = q.qvla_packed_linear(128, 256, 64, 16, 0, 16, 16, 16, None)
-    assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lhad),
+    # no permutation
+    Lnop = q.qvla_packed_linear(128, 256, 64, 0, 16, 16, 16, 16, None)
+    assert lib.qvla_rotate_act_f32(ctypes.c_void_p(16), 1, 4, 256, ctypes.byref(Lnop),
                                    ctypes.c_void_p(16), None) == q.QVLA_ERR_ARG
     # misaligned pointers
     Lmis = q.qvla_packed_linear(128, 256, 64, 16, 24, None, 16, 16, None)
@@ -137,9 +137,9 @@ def test_variant_entry_points_reject_bad_arguments():
                                       None, P, P, P, big, P, 100 * 256 * 4 - 1,
                                       None) == q.QVLA_ERR_WORKSPACE
     # Hadamard-only and W8 packs: a block size outside {32, 64, 128, 256}
-    assert lib.qvla_pack_weights_hadamard(P, 64, 256, 48, None, P, P, P, P, big,
+    assert lib.qvla_pack_weights_hadamard(P, 64, 256, 48, None, P, None, P, P, P, big,
                                           None) == q.QVLA_ERR_SHAPE
-    assert lib.qvla_pack_weights_w8(P, 64, 256, 48, None, None, P, P, P, P, P, big,
+    assert lib.qvla_pack_weights_w8(P, 64, 256, 48, None, None, P, P, None, P, P, P, big,
                                     None) == q.QVLA_ERR_SHAPE
     # 8-bit activations: no packed linear; workspace below the M x K fp32 rows
     L = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)

@@ -39,7 +39,7 @@ def _lines(exe):
 
 def test_c_program_against_the_header(exe):
     d = _lines(exe)
-    assert d["abi"] == ["1", "1"]
+    assert d["abi"] == ["2", "2"]
     assert d["status"][0].startswith("ok") or "OK" in d["status"][0].upper()
     assert d["sizes"] == ["0", str(256 * 1024 // 2), str(4 * 1024 * 64), str(6 * 1024 * 64)]
     assert d["badshape"] == ["2"]                                   # QVLA_ERR_SHAPE

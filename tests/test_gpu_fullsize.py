@@ -23,9 +23,10 @@ def q():
     return qvla
 
 
-def _run_batched(q, lins, xs, mode, table=None, step=0, scratch=True):
+def _run_batched(q, lins, xs, mode, table=None, step=0, scratch=True, image=False):
     """Pack every linear (GPU pack fed the oracle's permutation and R_SVD),
-    run the batched rotate-quantise and GEMM; return oracle packs and problems."""
+    run the batched rotate-quantise and GEMM (with `image`, the GEMM reads the
+    int8 image of the codes); return oracle packs and problems."""
     refs, probs = [], []
     steps = torch.tensor([step], dtype=torch.int32, device="cuda")
     tab = torch.from_numpy(table).cuda() if table is not None else None
@@ -42,7 +43,7 @@ def _run_batched(q, lins, xs, mode, table=None, step=0, scratch=True):
             ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
         md = q.QVLA_SCALE_TABLE if mode == "table" else q.QVLA_SCALE_DYNAMIC
         kw = dict(table=tab, step=steps, layer=lin.layer) if mode == "table" else {}
-        probs.append(q.LinearProblem(L, xd, md, workspace=ws, **kw))
+        probs.append(q.LinearProblem(L, xd, md, workspace=ws, xq8=True if image else None, **kw))
         refs.append(ref)
     q.qvla_rotate_quant_act_batched(probs)
     q.qvla_w4a4_gemm_batched(probs)
@@ -88,10 +89,25 @@ def test_dit_mlp_stack_gate_up_fused_full_size(q):
         _check_sampled(lin, x, ref, p, rows, "table", wl.table, t)
 
 
+def test_dit_denoise_loop_qkv_fused_layer_full_size(q):
+    """Shared-input fusion: q, k and v as one 1536->4608 linear (one
+    permutation and rotation from the concatenated weights, one activation
+    pass), with o, up and down of the same layer in the batched launches."""
+    wl = I.dit_denoise_loop(fuse_qkv=True)
+    lins = wl.linears[:4]                                   # qkv, o, up, down of layer 0
+    assert [(l.K, l.N) for l in lins] == [(1536, 4608), (1536, 1536), (1536, 6144), (6144, 1536)]
+    t = 5
+    xs = [l.make_x(seed_offset=t, std=float(wl.sigmas[t])) for l in lins]
+    refs, probs = _run_batched(q, lins, xs, "table", wl.table, t, image=True)
+    rows = np.random.default_rng(4).choice(lins[0].M, 5, replace=False)
+    for lin, x, ref, p in zip(lins, xs, refs, probs):
+        _check_sampled(lin, x, ref, p, rows, "table", wl.table, t)
+
+
 def test_backbone_prefill_full_size(q):
     wl = I.backbone_prefill()
     xs = [l.make_x() for l in wl.linears]
-    refs, probs = _run_batched(q, wl.linears, xs, "dynamic")
+    refs, probs = _run_batched(q, wl.linears, xs, "dynamic", image=True)
     rows = np.sort(np.random.default_rng(1).choice(1024, 6, replace=False))
     rows[-1] = 1023                                         # the ragged last tile's edge
     for lin, x, ref, p in zip(wl.linears, xs, refs, probs):

@@ -32,7 +32,8 @@ def test_hadamard_pack_parity(q, N, K, b):
     W = I.weights(8000 + K + b, N, K, n_outlier_rows=3, col_spread=10.0)
     ref = O.pack_linear_hadamard(W, b)
     pk = q.qvla_pack_weights_hadamard(cu(W), b)
-    assert pk.rot is None and pk.rot_tc is None
+    # R_SVD = I: no R_SVD blocks; the tensor-core image of R_B = H_b for b 64 / 128
+    assert pk.rot is None and (pk.rot_tc is not None) == (b in (64, 128))
     assert np.array_equal(pk.perm.cpu().numpy(), ref.perm)
     assert np.array_equal(pk.w_scale.cpu().numpy().view(np.uint32), ref.s_w.view(np.uint32))
     flips = check_codes_near_boundary(unpack(pk.wq.cpu().numpy()), ref.qw, ref.Wr,
@@ -41,13 +42,18 @@ def test_hadamard_pack_parity(q, N, K, b):
     assert q.qvla_read_error_word(clear=True) == 0
 
 
-@pytest.mark.parametrize("M,K,b,dt", [(16, 256, 64, "f32"), (50, 1024, 64, "bf16"),
-                                      (3, 512, 32, "bf16"), (9, 1024, 256, "bf16"),
-                                      (300, 2048, 128, "bf16")])
-def test_hadamard_rotation_fp32_vs_fp64(q, M, K, b, dt):
+@pytest.mark.parametrize("M,K,b,dt,image", [(16, 256, 64, "f32", True), (50, 1024, 64, "bf16", True),
+                                            (50, 1024, 64, "bf16", False),
+                                            (3, 512, 32, "bf16", True), (9, 1024, 256, "bf16", True),
+                                            (300, 2048, 128, "bf16", True),
+                                            (300, 2048, 128, "bf16", False)])
+def test_hadamard_rotation_fp32_vs_fp64(q, M, K, b, dt, image):
+    """bf16 at blocks 64 / 128 with the image: the tensor-core route (R_B = H_b
+    in three bf16 parts, of which only the first is non-zero); without it, or
+    for fp32 input and blocks 32 / 256: the Walsh-Hadamard transform alone."""
     W = I.weights(8100 + K, 64, K)
     ref = O.pack_linear_hadamard(W, b)
-    L = q.qvla_pack_weights_hadamard(cu(W), b, perm_in=ref.perm.astype(np.int32))
+    L = q.qvla_pack_weights_hadamard(cu(W), b, perm_in=ref.perm.astype(np.int32), image=image)
     x = I.activations(8101 + M, M, K, n_outlier_cols=3, dtype=dt)
     xd = cu(x) if dt == "f32" else cu(x).to(torch.bfloat16)
     xr = q.qvla_rotate_act_f32(xd, L).cpu().numpy().astype(np.float64)

@@ -7,35 +7,48 @@
 // W4A16?": weights and activations both 4-bit so the product runs on integer
 // tensor cores; "FoldQuantVLA": native integer W4A4 execution.)
 //
-// sm_100a has no 4-bit integer MMA, so each CTA
-//   1. TMA-loads packed int4 tiles (128 bytes of K per row, 128B swizzle) of
-//      the weights [128 rows] and the activations [NT rows] into a ring of
-//      shared-memory stages (one elected producer thread);
-//   2. unpacks them with four warps into 128-byte-swizzled K-major UMMA
-//      operand rows: every code q becomes the int8 value 16*q (its nibble moved into
-//      the high half of the byte: `w & 0xF0F0F0F0` for odd codes,
-//      `(w << 4) & 0xF0F0F0F0` for even codes).  Even codes of a 32-code
-//      group fill the first 16-byte K chunk and odd codes the second; both
-//      operands use the same K order, so the dot product is unchanged;
-//   3. issues tcgen05.mma kind::i8 (M=128 weight rows, N=NT tokens, K=32)
-//      from one thread into an int32 accumulator in tensor memory, which
-//      therefore holds 256*acc exactly;
-//   4. reads the accumulator back with tcgen05.ld (one output channel per
-//      thread, tokens along registers), applies the epilogue into a bf16
-//      shared-memory tile and writes it back with one TMA tensor store.
-// Weights take the UMMA M slot and tokens the N slot for every M, so the small
-// token counts of a DiT action chunk (16-64) still fill a 128-row MMA.
-// Small M adds split-K over a thread-block cluster along grid z: every CTA of
-// the cluster owns a contiguous run of 256-wide K tiles, and the int32 partial
-// tiles are summed through distributed shared memory (exact, no workspace).
+// sm_100a has no 4-bit integer MMA.  Every code q runs through
+// tcgen05.mma kind::i8 as the int8 value 16*q (its nibble moved into the high
+// half of the byte: `w & 0xF0F0F0F0` takes the odd codes of a packed word,
+// `(w << 4) & 0xF0F0F0F0` the even ones), so the int32 accumulator holds
+// 256*acc exactly and the epilogue shifts it back.  Inside every group of 32
+// codes both operands carry the even codes first, then the odd ones; the dot
+// product is unchanged.
+//
+// One persistent CTA per SM, warp-specialised (320 threads):
+//   warp 0      TMA producer: per pipeline stage (128 of K) a 128-row box of
+//               packed weights and an NT-token box of activation codes go into
+//               a ring of shared-memory stages;
+//   warp 1      MMA issuer: tcgen05.mma with A (weights) read from tensor
+//               memory and B (activations) from shared memory; int32
+//               accumulators in tensor memory, two buffers when they fit;
+//   warps 2-5   unpack: each thread owns one weight row (one tensor-memory
+//               lane), reads the row's 64 packed bytes of the stage and stores
+//               its 128 int8 values into a ring of tensor-memory A stages
+//               (tcgen05.st), so the weights never make a second trip through
+//               shared memory; with nibble-packed activations these warps also
+//               unpack the B tile into a 128-byte-swizzled shared-memory tile;
+//   warps 6-9   epilogue: tcgen05.ld of the accumulator (one output channel per
+//               thread), dequantise, add the bias, round to bf16, stage
+//               32-token chunks in shared memory, TMA tensor stores.
+// The activation operand is either the int8 image of the codes written by the
+// rotate-quantise step (16*q, the same order inside each 32-code group; a TMA
+// box lands directly in the MMA layout) or the nibble-packed codes.
+// Tiles (128 weight rows x NT tokens x all of K) are dealt to the CTAs on the
+// host, longest first to the least-loaded CTA, and travel in the kernel
+// parameters; a CTA walks its list with one continuous pipeline, so the next
+// tile's loads and unpacking overlap the current tile's MMAs and the previous
+// tile's epilogue.
 //
 // All waits are bounded (2 s) and flag QVLA_DEVERR_TIMEOUT instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <queue>
 #include <vector>
 
 #include "qvla_common.cuh"
@@ -44,387 +57,397 @@
 namespace qvla {
 namespace {
 
-constexpr int kBM = 128;                  // weight rows per tile (UMMA M)
-constexpr int kKP = 256;                  // K per packed stage (128 bytes per row)
-constexpr int kKU = 128;                  // K per unpacked stage (128 int8 per row)
-constexpr int kRowP = kKP / 2;            // packed bytes per row per stage
-constexpr int kThreads = 192;             // warp0 TMA, warp1 MMA, warps2-5 unpack+epilogue
-constexpr int kWorkers = 128;
+constexpr int kBM = 128;                  // weight rows per tile (UMMA M, tensor-memory lanes)
+constexpr int kKS = 128;                  // K per pipeline stage
+constexpr int kAPack = kKS / 2;           // packed weight bytes per row per stage
+constexpr int kACols = kKS / 4;           // tensor-memory columns of one unpacked A stage
+constexpr int kSA = 8;                    // A stages in tensor memory
+constexpr int kThreads = 320;
+constexpr int kOutSlots = 4;              // output staging ring (32-token chunks)
+constexpr int kTmemCols = 512;
+constexpr int kMaxBatch = 16;
+constexpr int kMaxTiles = 2048;
+constexpr int kMaxCtas = 160;
+constexpr uint32_t kFull = 0xffffffffu;
 
-template <int NT>
+template <int NT, bool kImage>
 struct Cfg {
-  static constexpr int kRows = kBM + NT;
-  static constexpr int kPStageBytes = kRows * kRowP;   // packed: A rows then B rows
-  static constexpr int kUStageBytes = kRows * kKU;     // unpacked int8
-  static constexpr int kPS = 2;
-  static constexpr int kUS = 2;
-  static constexpr int kTmemCols = NT < 32 ? 32 : NT;
-  static constexpr int kRedPitch = NT + 4;             // int32 per row of the split-K buffer
-  static constexpr int kStageBytes = kPS * kPStageBytes + kUS * kUStageBytes;
-  // split-K receive buffer and the owner's output rows (at most 64 of them,
-  // S >= 2), both placed over the stage memory once every CTA of the cluster
-  // is done with its stages
-  static constexpr int kRecvBytes = kBM * kRedPitch * 4;
-  static constexpr int kSmemBytes = kStageBytes + 1024;
-  static constexpr bool kCanSplit = kRecvBytes + NT * 64 * 2 <= kStageBytes;
+  static constexpr int kAcc = NT >= 256 ? 1 : 2;                  // accumulator buffers
+  static constexpr int kAccCols = NT < 32 ? 32 : NT;
+  static constexpr int kACol0 = kAcc * kAccCols;                 // first A-stage column
+  static constexpr int kABytes = kBM * kAPack;                   // packed weight box
+  static constexpr int kBBytes = NT * (kImage ? kKS : kAPack);   // activation box
+  static constexpr int kUBytes = kImage ? 0 : NT * kKS;          // unpacked activations
+  static constexpr int kStage = kABytes + kBBytes + kUBytes;
+  static constexpr int kCh = NT < 32 ? NT : 32;                  // tokens per output chunk
+  static constexpr int kOutBytes = kOutSlots * kCh * kBM * 2;
+  static constexpr int kRing = (200 * 1024 - kOutBytes) / kStage;
+  static constexpr int kS = kRing > 8 ? 8 : kRing;
+  // at least 116 KB, so that two CTAs never share an SM (each takes all of
+  // tensor memory)
+  static constexpr int kNeed = kS * kStage + kOutBytes + 1024;
+  static constexpr int kSmem = kNeed < 116 * 1024 ? 116 * 1024 : kNeed;
+  static_assert(kACol0 + kSA * kACols <= kTmemCols, "tensor memory");
+  static_assert(kStage % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "alignment");
+  static_assert(kS >= 2, "pipeline depth");
 };
 
 struct Barriers {
-  uint64_t full_p[4], empty_p[4], full_u[4], empty_u[4], acc_full;
-  uint32_t tmem_base;
+  uint64_t full[8], empty[8];              // shared-memory stages
+  uint64_t a_full[kSA], a_empty[kSA];      // tensor-memory A stages
+  uint64_t acc_full[2], acc_empty[2];      // accumulators
+  uint64_t drain;
+  uint32_t tmem;
 };
 
-// One linear of a batched launch.  Independent linears (different weights,
-// inputs and outputs) share one launch; CTAs are numbered problem by problem.
-constexpr int kMaxBatch = 16;
-struct GemmProblem {
-  CUtensorMap tw;                 // packed weights  [N][K/2]
-  CUtensorMap tx;                 // packed codes    [M][K/2]
-  CUtensorMap ty;                 // bf16 output [M][ldy], box = (128/S channels) x NT tokens
+// One linear of a launch.  Its tiles are numbered n-tile fastest (tiles that
+// share an activation box are neighbours), from tile_base on.
+struct Problem {
+  CUtensorMap tw;                 // packed weights [N][K/2]: box 64 B x 128 rows, 64B swizzle
+  CUtensorMap tx;                 // activations: int8 image [M][K] (box 128 x NT, 128B
+                                  // swizzle) or packed [M][K/2] (box 64 x NT, 64B swizzle)
+  CUtensorMap ty;                 // bf16 output [M][ldy]: box 128 channels x kCh tokens
   const float* s_x;
   const float* s_w;
   const float* bias;
   __nv_bfloat16* y;
-  int32_t* acc;
+  int32_t* acc;                   // int32 [M][N] accumulators instead of y (or null)
   int M, N, K, ldy;
   int tiles_n;                    // ceil(N / 128)
-  int tiles;                      // tiles_n * ceil(M / NT)
-  int S;                          // split-K factor: 1 or the launch's cluster size
+  int nks;                        // K stages: ceil(K / 128)
+  int tile_base;                  // first tile of this problem in the launch
 };
-struct GemmBatch {
+struct Batch {
   int n;
-  int tile_start[kMaxBatch + 1];  // prefix sums of tiles_n * tiles_m
-  GemmProblem p[kMaxBatch];
+  int tile_start[kMaxBatch + 1];  // launch tile ids of each problem
+  uint16_t cta_begin[kMaxCtas + 1];
+  uint16_t order[kMaxTiles];      // launch tile ids, CTA by CTA
+  Problem p[kMaxBatch];
+};
+
+struct Tile {
+  int p, n0, m0;
 };
 
 template <int NT>
+QVLA_DEVICE Tile decode(const Batch& b, int t) {
+  int p = 0;
+  while (p + 1 < b.n && t >= b.tile_start[p + 1]) ++p;
+  const int local = t - b.tile_start[p] + b.p[p].tile_base;
+  const int tn = b.p[p].tiles_n;
+  return Tile{p, (local % tn) * kBM, (local / tn) * NT};
+}
+
+// Wait until at most N bulk groups of this thread still read shared memory.
+template <int N>
+QVLA_DEVICE void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+template <int NT>
+QVLA_DEVICE void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[NT < 32 ? NT : 32]) {
+  if constexpr (NT < 32) {
+    tmem_ld16(taddr, r);
+  } else {
+    tmem_ld32(taddr, r);
+  }
+}
+
+template <int NT, bool kImage>
 __global__ void __launch_bounds__(kThreads, 1)
-    w4a4_gemm_kernel(const __grid_constant__ GemmBatch batch, unsigned int* err) {
-  using C = Cfg<NT>;
+    w4a4_gemm_kernel(const __grid_constant__ Batch batch, unsigned int* err) {
+  using C = Cfg<NT, kImage>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
-  __shared__ __align__(16) float bars_sx[NT];   // s_x of this token tile
-
-  int pi = 0;
-  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.tile_start[pi + 1]) ++pi;
-  const GemmProblem& P = batch.p[pi];
-  const CUtensorMap* tmap_w = &P.tw;
-  const CUtensorMap* tmap_x = &P.tx;
-  const int M = P.M, N = P.N, K = P.K, ldy = P.ldy;
-  const float* __restrict__ s_x = P.s_x;
-  const float* __restrict__ s_w = P.s_w;
-  const float* __restrict__ bias = P.bias;
-  __nv_bfloat16* __restrict__ y = P.y;
-  int32_t* __restrict__ acc_out = P.acc;
-  const int local = static_cast<int>(blockIdx.x) - batch.tile_start[pi];
-  // A problem with S > 1 spans whole clusters (S consecutive CTAs share a
-  // tile, one K range each); a problem with S == 1 is padded to whole
-  // clusters, and the padding CTAs leave at once (they take part in no
-  // cluster barrier: only split problems use them).
-  const int S = P.S;
-  if (local >= P.tiles * S) return;
-  const int tile = local / S;
-  const int split = local % S;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = (tile % P.tiles_n) * kBM;
-  const int m0 = (tile / P.tiles_n) * NT;
-  const int nkt = (K + kKP - 1) / kKP;
-  const int kt0 = split * nkt / S, kt1 = (split + 1) * nkt / S;
-  const int nk = kt1 - kt0;
+  const int t_begin = batch.cta_begin[blockIdx.x];
+  const int t_end = batch.cta_begin[blockIdx.x + 1];
 
-  // 1024-byte aligned stage memory (128B-swizzled TMA destinations)
+  // 1024-byte aligned stage memory (swizzled TMA destinations)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* const base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-  uint8_t* const pstage = base;
-  uint8_t* const ustage = base + C::kPS * C::kPStageBytes;
+  uint8_t* const stages = base;
+  __nv_bfloat16* const outs = reinterpret_cast<__nv_bfloat16*>(base + C::kS * C::kStage);
 
   if (tid == 0) {
-    for (int s = 0; s < C::kPS; ++s) {
-      mbar_init(&bars.full_p[s], 1);
-      mbar_init(&bars.empty_p[s], kWorkers);
+    for (int s = 0; s < C::kS; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 5);          // four unpack warps + the MMA commit
     }
-    for (int u = 0; u < C::kUS; ++u) {
-      mbar_init(&bars.full_u[u], kWorkers);
-      mbar_init(&bars.empty_u[u], 1);
+    for (int a = 0; a < kSA; ++a) {
+      mbar_init(&bars.a_full[a], 4);
+      mbar_init(&bars.a_empty[a], 1);
     }
-    mbar_init(&bars.acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.acc_full[b], 1);
+      mbar_init(&bars.acc_empty[b], 4);
+    }
+    mbar_init(&bars.drain, 1);
     fence_mbar_init();
-    tma_prefetch_desc(tmap_w);
-    tma_prefetch_desc(tmap_x);
+    for (int p = 0; p < batch.n; ++p) {
+      tma_prefetch_desc(&batch.p[p].tw);
+      tma_prefetch_desc(&batch.p[p].tx);
+    }
   }
   if (warp == 1) {
     __syncwarp();                  // tcgen05 alloc/ld/st/dealloc are warp-wide
-    tmem_alloc(&bars.tmem_base, C::kTmemCols);
+    tmem_alloc(&bars.tmem, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   cta_sync();
   tc_fence_after();
-  const uint32_t tmem_d = bars.tmem_base;
-  // split-K: every thread arrives on the cluster barrier once it is done with
-  // the stage memory (the producer after its last load has landed, the MMA
-  // issuer after its last MMA has completed, the workers after the
-  // accumulator is final); partial sums are pushed into the owner's stage
-  // memory only after the whole cluster has arrived
-  bool cluster_waited = false;
+  const uint32_t tmem = bars.tmem;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      bool ok = true;
-      int issued = 0;
+      constexpr uint32_t kTx = C::kABytes + C::kBBytes;
+      constexpr int kBX = kImage ? kKS : kAPack;          // activation box x step
       // Weights do not depend on the previous kernel in the stream: the first
-      // stages' weight tiles are requested before waiting for it (programmatic
-      // dependent launch), the activation tiles after.
-      const int pre = nk < C::kPS ? nk : C::kPS;
-      // the whole weight range of this CTA is requested into L2 at once, so
-      // HBM streaming is not limited by the depth of the stage ring
-      for (int i = pre; i < nk; ++i) tma_prefetch_l2_2d(tmap_w, (kt0 + i) * kRowP, n0);
-      for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&bars.full_p[i], C::kPStageBytes);
-        tma_load_2d(pstage + i * C::kPStageBytes, tmap_w, &bars.full_p[i], (kt0 + i) * kRowP, n0);
+      // ring's worth of weight boxes are requested before waiting for it
+      // (programmatic dependent launch), the activation boxes after.
+      int pre = 0;
+      {
+        int i = t_begin, ks = 0;
+        while (pre < C::kS && i < t_end) {
+          const Tile tr = decode<NT>(batch, batch.order[i]);
+          const Problem& P = batch.p[tr.p];
+          mbar_arrive_expect_tx(&bars.full[pre], kTx);
+          tma_load_2d(stages + pre * C::kStage, &P.tw, &bars.full[pre], ks * kAPack, tr.n0);
+          ++pre;
+          if (++ks == P.nks) {
+            ks = 0;
+            ++i;
+          }
+        }
       }
       pdl_wait();
-      for (int i = 0; i < pre; ++i) {
-        tma_load_2d(pstage + i * C::kPStageBytes + kBM * kRowP, tmap_x, &bars.full_p[i],
-                    (kt0 + i) * kRowP, m0);
-        ++issued;
+      bool ok = true;
+      int g = 0;
+      for (int i = t_begin; i < t_end && ok; ++i) {
+        const Tile tr = decode<NT>(batch, batch.order[i]);
+        const Problem& P = batch.p[tr.p];
+        // the tile's weight boxes past the ring depth go to L2 now, so HBM
+        // streaming is not limited by the ring
+        for (int ks = C::kS; ks < P.nks; ++ks) tma_prefetch_l2_2d(&P.tw, ks * kAPack, tr.n0);
+        for (int ks = 0; ks < P.nks; ++ks, ++g) {
+          const int s = g % C::kS;
+          uint8_t* st = stages + s * C::kStage;
+          if (g >= pre) {
+            if (g >= C::kS) {
+              ok = mbar_wait(&bars.empty[s], ((g / C::kS) - 1) & 1, err);
+              if (!ok) break;
+            }
+            mbar_arrive_expect_tx(&bars.full[s], kTx);
+            tma_load_2d(st, &P.tw, &bars.full[s], ks * kAPack, tr.n0);
+          }
+          tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kBX, tr.m0);
+        }
       }
-      for (int i = pre; i < nk && ok; ++i) {
-        const int s = i % C::kPS;
-        const uint32_t ph = (i / C::kPS) & 1;
-        ok = mbar_wait(&bars.empty_p[s], ph ^ 1u, err);
-        if (!ok) break;
-        uint8_t* dst = pstage + s * C::kPStageBytes;
-        mbar_arrive_expect_tx(&bars.full_p[s], C::kPStageBytes);
-        const int xbyte = (kt0 + i) * kRowP;
-        tma_load_2d(dst, tmap_w, &bars.full_p[s], xbyte, n0);
-        tma_load_2d(dst + kBM * kRowP, tmap_x, &bars.full_p[s], xbyte, m0);
-        ++issued;
-      }
-      // never leave with copies in flight: wait for the last load of each stage
-      for (int i = issued - C::kPS < 0 ? 0 : issued - C::kPS; i < issued; ++i)
-        mbar_wait(&bars.full_p[i % C::kPS], (i / C::kPS) & 1, err);
+      // never leave with copies in flight: the last load of every stage has landed
+      for (int j = g - C::kS < 0 ? 0 : g - C::kS; j < g; ++j)
+        mbar_wait(&bars.full[j % C::kS], (j / C::kS) & 1, err);
     }
-    if (S > 1) cluster_arrive_relaxed();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(kBM, NT);
-      const uint32_t u_base = smem_u32(ustage);
       bool ok = true;
-      for (int j = 0; j < 2 * nk && ok; ++j) {
-        const int u = j % C::kUS;
-        ok = mbar_wait(&bars.full_u[u], (j / C::kUS) & 1, err);
-        if (!ok) break;
+      int g = 0, tc = 0;
+      for (int i = t_begin; i < t_end && ok; ++i, ++tc) {
+        const Tile tr = decode<NT>(batch, batch.order[i]);
+        const int nks = batch.p[tr.p].nks;
+        const int b = tc % C::kAcc, use = tc / C::kAcc;
+        if (use >= 1) {
+          ok = mbar_wait(&bars.acc_empty[b], (use - 1) & 1, err);
+          if (!ok) break;
+        }
         tc_fence_after();
-        const uint32_t a0 = u_base + u * C::kUStageBytes;
-        const uint32_t b0 = a0 + kBM * kKU;
+        const uint32_t d = tmem + static_cast<uint32_t>(b * C::kAccCols);
+        for (int ks = 0; ks < nks; ++ks, ++g) {
+          const int s = g % C::kS, a = g % kSA;
+          ok = mbar_wait(&bars.a_full[a], (g / kSA) & 1, err);
+          if (ok && kImage) ok = mbar_wait(&bars.full[s], (g / C::kS) & 1, err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bs =
+              smem_u32(stages + s * C::kStage + C::kABytes + (kImage ? 0 : C::kBBytes));
+          const uint32_t at = tmem + static_cast<uint32_t>(C::kACol0 + a * kACols);
 #pragma unroll
-        for (int q = 0; q < kKU / 32; ++q) {
-          // bytes [32q, 32q+32) of every 128-byte row: the even and the odd
-          // codes of packed chunk q of this half stage
-          const uint64_t ad = smem_desc_kmajor_sw128(a0 + 32 * q);
-          const uint64_t bd = smem_desc_kmajor_sw128(b0 + 32 * q);
-          umma_i8(tmem_d, ad, bd, idesc, (j > 0 || q > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars.empty_u[u]);
-      }
-      umma_commit(&bars.acc_full);
-      mbar_wait(&bars.acc_full, 0, err);   // tensor memory is freed only after this
-    }
-    if (S > 1) cluster_arrive_relaxed();
-  } else {
-    // --------------------------------------------------- unpack (4 warps)
-    const int wt = tid - 64;   // 0..127
-    // epilogue operands, loaded early so their latency hides under the main
-    // loop (s_x comes from the previous kernel in the stream)
-    pdl_wait();
-    float* sx_s = reinterpret_cast<float*>(bars_sx);
-    if (acc_out == nullptr)
-      for (int c = wt; c < NT; c += kWorkers) sx_s[c] = (m0 + c < M) ? __ldg(s_x + m0 + c) : 0.f;
-    const int quarter = warp & 3;
-    const int nl = quarter * 32 + lane;          // local output channel (TMEM lane)
-    const int n = n0 + nl;
-    const float sw = (acc_out == nullptr && n < N) ? __ldg(s_w + n) : 0.f;
-    const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
-    constexpr int kItems = (C::kRows * 4 + kWorkers - 1) / kWorkers;
-    bool ok = true;
-    for (int i = 0; i < nk && ok; ++i) {
-      const int s = i % C::kPS;
-      ok = mbar_wait(&bars.full_p[s], (i / C::kPS) & 1, err);
-      if (!ok) break;
-      const uint8_t* ps = pstage + s * C::kPStageBytes;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = 2 * i + h;
-        const int u = j % C::kUS;
-        // all packed loads of this half stage first (independent), then the
-        // nibble moves and the swizzled 16-byte stores
-        uint4 w[kItems];
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-          const int it = wt + k * kWorkers;
-          if (it < C::kRows * 4) {
-            const int row = ((it >> 5) << 3) + (it & 7);   // A rows, then B rows
-            const int cl = (it >> 3) & 3;                  // packed 16-byte chunk of the half
-            w[k] = *reinterpret_cast<const uint4*>(ps + row * kRowP +
-                                                   (((4 * h + cl) ^ (row & 7)) << 4));
+          for (int kk = 0; kk < kKS / 32; ++kk) {
+            // 32 codes of K: A columns [8kk, 8kk+8) of the stage, B bytes
+            // [32kk, 32kk+32) of every 128-byte row
+            const uint64_t bd = smem_desc_kmajor_sw128(bs + 32 * kk);
+            umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
           }
+          umma_commit(&bars.a_empty[a]);
+          umma_commit(&bars.empty[s]);
         }
-        ok = mbar_wait(&bars.empty_u[u], ((j / C::kUS) & 1) ^ 1u, err);
         if (!ok) break;
-        uint8_t* us = ustage + u * C::kUStageBytes;
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-          const int it = wt + k * kWorkers;
-          if (it < C::kRows * 4) {
-            const int row = ((it >> 5) << 3) + (it & 7);
-            const int cl = (it >> 3) & 3;
-            uint4 ev, od;
-            ev.x = (w[k].x << 4) & 0xF0F0F0F0u;
-            ev.y = (w[k].y << 4) & 0xF0F0F0F0u;
-            ev.z = (w[k].z << 4) & 0xF0F0F0F0u;
-            ev.w = (w[k].w << 4) & 0xF0F0F0F0u;
-            od.x = w[k].x & 0xF0F0F0F0u;
-            od.y = w[k].y & 0xF0F0F0F0u;
-            od.z = w[k].z & 0xF0F0F0F0u;
-            od.w = w[k].w & 0xF0F0F0F0u;
-            // 128-byte swizzled K-major rows (A rows 0..127, then B rows):
-            // chunk 2cl holds the even codes, 2cl+1 the odd codes
-            uint8_t* rowp = us + row * kKU;
-            *reinterpret_cast<uint4*>(rowp + (((2 * cl) ^ (row & 7)) << 4)) = ev;
-            *reinterpret_cast<uint4*>(rowp + (((2 * cl + 1) ^ (row & 7)) << 4)) = od;
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars.full_u[u]);
+        umma_commit(&bars.acc_full[b]);
       }
-      mbar_arrive(&bars.empty_p[s]);
+      umma_commit(&bars.drain);
+      mbar_wait(&bars.drain, 0, err);   // tensor memory is freed only after this
     }
-
-    // ---------------------------------------------------------- epilogue
-    // one outcome per warp, and a converged warp for the warp-wide loads
-    const bool have = __all_sync(0xffffffffu, ok && mbar_wait(&bars.acc_full, 0, err));
-    tc_fence_after();
-    if (S > 1) cluster_arrive_relaxed();
-    pdl_launch_dependents();
-    if (have) {
-      // split-K: this CTA's partial rows go to the receive buffer of the CTA
-      // that owns them (rows [r*128/S, (r+1)*128/S) belong to cluster rank r),
-      // slot `split`, as fire-and-forget distributed-shared-memory stores
-      const int rpr = kBM / S;
-      const uint32_t owner = static_cast<uint32_t>(nl / rpr);
-      const uint32_t recv_row =
-          smem_u32(base) + static_cast<uint32_t>(((split * rpr + nl % rpr) * C::kRedPitch) * 4);
-      const uint32_t remote_row = S > 1 ? map_shared_rank(recv_row, owner) : 0u;
-      if (S > 1) {
-        cluster_wait();
-        cluster_waited = true;
-      }
-      // bf16 output tile [NT tokens][128 channels] in the (now idle) stage
-      // memory, written back by one TMA tensor store
-      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base);
-#pragma unroll 1
-      for (int c0 = 0; c0 < NT; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
-        tmem_ld_wait();
-        if (S > 1) {
+  } else if (warp < 6) {
+    // ------------------------------------------------------- unpack (4 warps)
+    const int q4 = warp & 3;                       // tensor-memory lane quarter
+    const int row = q4 * 32 + lane;                // weight row of the tile
+    const int wt = tid - 64;                       // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    constexpr int kBItems = (NT * 4 + 127) / 128;  // packed activation chunks per thread
+    bool ok = true;
+    int g = 0;
+    for (int i = t_begin; i < t_end && ok; ++i) {
+      const int nks = batch.p[decode<NT>(batch, batch.order[i]).p].nks;
+      for (int ks = 0; ks < nks; ++ks, ++g) {
+        const int s = g % C::kS, a = g % kSA;
+        // warp-uniform outcome: the tensor-memory stores below are warp-wide
+        ok = __all_sync(kFull, mbar_wait(&bars.full[s], (g / C::kS) & 1, err));
+        if (!ok) break;
+        const uint32_t st = smem_u32(stages + s * C::kStage);
+        // the row's 64 packed bytes; 64-byte swizzle: 16-byte chunk c of row r
+        // sits at chunk c ^ ((r >> 1) & 3)
+        uint4 w[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_shared_cluster_v4(remote_row + (c0 + 4 * q) * 4,
-                                 make_int4(static_cast<int>(r[4 * q]), static_cast<int>(r[4 * q + 1]),
-                                           static_cast<int>(r[4 * q + 2]),
-                                           static_cast<int>(r[4 * q + 3])));
-        } else if (acc_out) {
-          if (n < N) {
+        for (int c = 0; c < 4; ++c) w[c] = lds128(st + row * kAPack + ((c ^ ((row >> 1) & 3)) << 4));
+        if constexpr (!kImage) {
+          // activation chunk e: code row br = e % NT, 32-code group c = e / NT
+          // (consecutive threads take consecutive rows: conflict-free)
+          const uint32_t bp = st + C::kABytes, bu = st + C::kABytes + C::kBBytes;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int m = m0 + c0 + c;
-              if (m < M) acc_out[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(r[c]) >> 8;
+          for (int k = 0; k < kBItems; ++k) {
+            const int e = wt + k * 128;
+            if (e < NT * 4) {
+              const int br = e % NT, c = e / NT;
+              const uint4 v = lds128(bp + br * kAPack + ((c ^ ((br >> 1) & 3)) << 4));
+              uint4 ev, od;
+              ev.x = (v.x << 4) & 0xF0F0F0F0u;
+              ev.y = (v.y << 4) & 0xF0F0F0F0u;
+              ev.z = (v.z << 4) & 0xF0F0F0F0u;
+              ev.w = (v.w << 4) & 0xF0F0F0F0u;
+              od.x = v.x & 0xF0F0F0F0u;
+              od.y = v.y & 0xF0F0F0F0u;
+              od.z = v.z & 0xF0F0F0F0u;
+              od.w = v.w & 0xF0F0F0F0u;
+              // 128-byte swizzled K-major row: chunk 2c even codes, 2c+1 odd codes
+              sts128(bu + br * kKS + (((2 * c) ^ (br & 7)) << 4), ev);
+              sts128(bu + br * kKS + (((2 * c + 1) ^ (br & 7)) << 4), od);
             }
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float sc = sx_s[c0 + c] * sw;
-            const int32_t a = static_cast<int32_t>(r[c]) >> 8;
-            otile[(c0 + c) * kBM + nl] = __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
-          }
         }
-      }
-      if (S == 1 && acc_out == nullptr) {
-        fence_proxy_async_smem();
-        named_barrier(1, kWorkers);
-        if (n0 + kBM <= N || (N & 7) == 0) {
-          if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, n0, m0);
-        } else {
-          // a tile cut by N with N % 8 != 0: plain stores, not a TMA box
-          // reaching past N
-          for (int e = wt; e < NT * kBM; e += kWorkers) {
-            const int c = e / kBM, nx = e % kBM;
-            if (n0 + nx < N && m0 + c < M)
-              y[static_cast<size_t>(m0 + c) * ldy + n0 + nx] = otile[c * kBM + nx];
-          }
+        if (g >= kSA) {
+          ok = __all_sync(kFull, mbar_wait(&bars.a_empty[a], ((g / kSA) - 1) & 1, err));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        // 32 columns: for packed chunk c, columns [8c, 8c+4) the even codes of
+        // its four words, [8c+4, 8c+8) the odd codes
+        uint32_t av[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          av[8 * c + 0] = (w[c].x << 4) & 0xF0F0F0F0u;
+          av[8 * c + 1] = (w[c].y << 4) & 0xF0F0F0F0u;
+          av[8 * c + 2] = (w[c].z << 4) & 0xF0F0F0F0u;
+          av[8 * c + 3] = (w[c].w << 4) & 0xF0F0F0F0u;
+          av[8 * c + 4] = w[c].x & 0xF0F0F0F0u;
+          av[8 * c + 5] = w[c].y & 0xF0F0F0F0u;
+          av[8 * c + 6] = w[c].z & 0xF0F0F0F0u;
+          av[8 * c + 7] = w[c].w & 0xF0F0F0F0u;
+        }
+        tmem_st32(tmem + lane_base + static_cast<uint32_t>(C::kACol0 + a * kACols), av);
+        tmem_st_wait();
+        if constexpr (!kImage) fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars.a_full[a]);
+          mbar_arrive(&bars.empty[s]);
         }
       }
     }
-    tc_fence_before();
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;                // output channel of the tile
+    const int et = tid - 192;                      // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    pdl_wait();                                    // s_x comes from the previous kernel
+    bool ok = true;
+    int tc = 0, chunk = 0;
+    for (int i = t_begin; i < t_end && ok; ++i, ++tc) {
+      const Tile tr = decode<NT>(batch, batch.order[i]);
+      const Problem& P = batch.p[tr.p];
+      const int b = tc % C::kAcc, use = tc / C::kAcc;
+      // one outcome for all four epilogue warps (they share named barriers)
+      ok = named_barrier_all(2, 128, mbar_wait(&bars.acc_full[b], use & 1, err));
+      if (!ok) break;
+      tc_fence_after();
+      const int n = tr.n0 + row;
+      const bool nv = n < P.N;
+      const float sw = (P.acc == nullptr && nv) ? __ldg(P.s_w + n) : 0.f;
+      const float bn = (P.bias != nullptr && nv) ? __ldg(P.bias + n) : 0.f;
+      const bool tma = tr.n0 + kBM <= P.N || (P.N & 7) == 0;
+      const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(b * C::kAccCols);
+#pragma unroll 1
+      for (int c0 = 0; c0 < NT; c0 += C::kCh) {
+        uint32_t r[C::kCh];
+        tmem_ld_chunk<NT>(tacc + c0, r);
+        tmem_ld_wait();
+        if (c0 + C::kCh >= NT) {
+          // the accumulator may be reused once every warp has read it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.acc_empty[b]);
+        }
+        if (P.acc != nullptr) {
+          if (nv) {
+#pragma unroll
+            for (int j = 0; j < C::kCh; ++j) {
+              const int m = tr.m0 + c0 + j;
+              if (m < P.M) P.acc[static_cast<size_t>(m) * P.N + n] = static_cast<int32_t>(r[j]) >> 8;
+            }
+          }
+          continue;
+        }
+        __nv_bfloat16* ot = outs + (chunk % kOutSlots) * (C::kCh * kBM);
+        // the store that last read this slot has finished reading it
+        if (et == 0) bulk_wait_read<kOutSlots - 1>();
+        named_barrier(1, 128);
+#pragma unroll
+        for (int j = 0; j < C::kCh; ++j) {
+          const int m = tr.m0 + c0 + j;
+          const float sx = m < P.M ? __ldg(P.s_x + m) : 0.f;
+          const int32_t a = static_cast<int32_t>(r[j]) >> 8;
+          ot[j * kBM + row] = __float2bfloat16_rn(fmaf(sx * sw, static_cast<float>(a), bn));
+        }
+        fence_proxy_async_smem();
+        named_barrier(1, 128);
+        if (tma) {
+          if (et == 0) tma_store_2d(&P.ty, ot, tr.n0, tr.m0 + c0);
+        } else {
+          // a tile cut by N with N % 8 != 0: plain stores, no box past N
+          for (int e = et; e < C::kCh * kBM; e += 128) {
+            const int c = e / kBM, nx = e % kBM;
+            if (tr.n0 + nx < P.N && tr.m0 + c0 + c < P.M)
+              P.y[static_cast<size_t>(tr.m0 + c0 + c) * P.ldy + tr.n0 + nx] = ot[c * kBM + nx];
+          }
+        }
+        if (et == 0) bulk_commit();                // one group per chunk, maybe empty
+        ++chunk;
+      }
+    }
+    if (et == 0) bulk_wait0();
+    pdl_launch_dependents();
   }
 
   cta_sync();
-
-  if (S > 1) {
-    // ------------------------------------------- cluster split-K reduction
-    if (!cluster_waited) cluster_wait();
-    cluster_sync();                  // every partial tile has landed
-    if (warp >= 2) {
-      const int wt = tid - 64;
-      const uint32_t rank = cluster_ctarank();
-      const int rpr = kBM / S;                     // channel rows reduced by this CTA
-      const int32_t* recv = reinterpret_cast<const int32_t*>(base);
-      // output tile [NT tokens][rpr channels] for one TMA store of this CTA's
-      // rows, after the receive buffer
-      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(base + C::kRecvBytes);
-      for (int e = wt; e < rpr * NT; e += kWorkers) {
-        const int lr = e % rpr;
-        const int col = e / rpr;
-        int32_t sum = 0;
-        for (int src = 0; src < S; ++src) sum += recv[(src * rpr + lr) * C::kRedPitch + col];
-        const int nl = rank * rpr + lr;
-        const int n = n0 + nl, m = m0 + col;
-        const int32_t a = sum >> 8;
-        if (acc_out) {
-          if (n < N && m < M) acc_out[static_cast<size_t>(m) * N + n] = a;
-        } else {
-          const float sc = n < N ? bars_sx[col] * __ldg(s_w + n) : 0.f;
-          const float bn = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.f;
-          otile[col * rpr + lr] = __float2bfloat16_rn(fmaf(sc, static_cast<float>(a), bn));
-        }
-      }
-      if (acc_out == nullptr) {
-        fence_proxy_async_smem();
-        named_barrier(1, kWorkers);
-        const int nr = n0 + static_cast<int>(rank) * rpr;
-        if (nr + rpr <= N || (N & 7) == 0) {
-          if (wt == 0) tma_store_2d_and_wait(&P.ty, otile, nr, m0);
-        } else {
-          for (int e = wt; e < NT * rpr; e += kWorkers) {
-            const int c = e / rpr, nx = e % rpr;
-            if (nr + nx < N && m0 + c < M)
-              y[static_cast<size_t>(m0 + c) * ldy + nr + nx] = otile[c * rpr + nx];
-          }
-        }
-      }
-    }
-  }
-
   if (warp == 1) {
     __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
-    tmem_dealloc(tmem_d, C::kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -447,175 +470,184 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// rows x (K/2) bytes, row pitch K/2; box = 128 bytes x box_rows, 128B swizzle.
-bool make_packed_map(CUtensorMap* map, const uint8_t* ptr, int rows, int K, int box_rows) {
+bool encode(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
+            uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+            CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promo) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowP), static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(ptr), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [M][ldy] output; box = box_n channels x box_m tokens, no swizzle.
-bool make_output_map(CUtensorMap* map, void* ptr, int M, int N, int ldy, int box_n, int box_m) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldy) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_n), static_cast<cuuint32_t>(box_m)};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  n = std::min(n, kMaxCtas);
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
-template <int NT>
-cudaError_t launch_group(const GemmArgs* const* gs, const int* splits, int n, int C,
-                         cudaStream_t stream) {
-  using C_ = Cfg<NT>;
-  GemmBatch batch;
-  std::memset(&batch, 0, sizeof(batch));
-  batch.n = n;
-  int ctas = 0;
-  for (int i = 0; i < n; ++i) {
-    const GemmArgs& g = *gs[i];
-    GemmProblem& P = batch.p[i];
-    const int S = splits[i];
-    if (!make_packed_map(&P.tw, g.wq, g.N, g.K, kBM) || !make_packed_map(&P.tx, g.xq, g.M, g.K, NT))
-      return cudaErrorInvalidValue;
-    if (g.y != nullptr && !make_output_map(&P.ty, g.y, g.M, g.N, g.ldy, kBM / S, NT))
-      return cudaErrorInvalidValue;
-    P.s_x = g.s_x;
-    P.s_w = g.w_scale;
-    P.bias = g.bias;
-    P.y = static_cast<__nv_bfloat16*>(g.y);
-    P.acc = g.acc;
-    P.M = g.M;
-    P.N = g.N;
-    P.K = g.K;
-    P.ldy = g.ldy;
-    P.tiles_n = (g.N + kBM - 1) / kBM;
-    P.tiles = P.tiles_n * ((g.M + NT - 1) / NT);
-    P.S = S;
-    batch.tile_start[i] = ctas;
-    ctas += (P.tiles * S + C - 1) / C * C;     // whole clusters
+// A tile's cost in K stages, plus a fixed share for its epilogue and ramp.
+constexpr int kTileOverhead = 2;
+
+// Deals the launch's tiles to at most sm_count() CTAs, longest first, each to
+// the CTA with the least work so far (ties: the lowest index), and writes the
+// per-CTA lists.  Returns the number of CTAs.
+int schedule(Batch& b) {
+  const int T = b.tile_start[b.n];
+  const int G = std::min(sm_count(), T);
+  std::vector<int> ids(T), cost(T);
+  for (int p = 0; p < b.n; ++p)
+    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t) cost[t] = b.p[p].nks + kTileOverhead;
+  for (int t = 0; t < T; ++t) ids[t] = t;
+  std::stable_sort(ids.begin(), ids.end(), [&](int x, int y) { return cost[x] > cost[y]; });
+  using Load = std::pair<long long, int>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < G; ++c) heap.push({0, c});
+  std::vector<std::vector<int>> lists(G);
+  for (int t : ids) {
+    Load l = heap.top();
+    heap.pop();
+    lists[l.second].push_back(t);
+    l.first += cost[t];
+    heap.push(l);
   }
-  batch.tile_start[n] = ctas;
-  auto kern = w4a4_gemm_kernel<NT>;
+  int k = 0;
+  for (int c = 0; c < G; ++c) {
+    b.cta_begin[c] = static_cast<uint16_t>(k);
+    for (int t : lists[c]) b.order[k++] = static_cast<uint16_t>(t);
+  }
+  b.cta_begin[G] = static_cast<uint16_t>(k);
+  return G;
+}
+
+template <int NT, bool kImage>
+cudaError_t launch_batch(Batch& batch, cudaStream_t stream) {
+  using C = Cfg<NT, kImage>;
+  const int G = schedule(batch);
+  if (G == 0) return cudaSuccess;
+  auto kern = w4a4_gemm_kernel<NT, kImage>;
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = once_per_device(attr_done, [&]() {
-    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes);
-    if (r == cudaSuccess)
-      r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    return r;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.gridDim = dim3(G, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C_::kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  int na = 0;
-  if (pdl_enabled()) {
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-  }
-  if (C > 1) {
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = C;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = na;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, kern, batch, device_error_word());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-int token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
-
-// Split-K factors of a launch (1 or the launch's cluster size C per problem).
-// Requested: the same factor everywhere.  Automatic: one factor for all,
-// raised while the launch has fewer CTAs than SMs.
-template <int NT>
-int choose_splits(const GemmArgs* const* gs, int n, int split_k, int* splits) {
-  if (!Cfg<NT>::kCanSplit) {
-    for (int i = 0; i < n; ++i) splits[i] = 1;
-    return 1;
+// Fills problem slot `P` for the tiles of `g` from t0 on.
+template <int NT, bool kImage>
+bool fill_problem(Problem& P, const GemmArgs& g, int t0) {
+  using C = Cfg<NT, kImage>;
+  std::memset(&P, 0, sizeof(P));
+  if (!encode(&P.tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K / 2, g.N, g.K / 2, kAPack, kBM,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return false;
+  if (kImage) {
+    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq8, g.K, g.M, g.K, kKS, NT,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+      return false;
+  } else {
+    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K / 2, g.M, g.K / 2, kAPack, NT,
+                CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+      return false;
   }
-  if (split_k > 0) {
-    for (int i = 0; i < n; ++i) splits[i] = split_k;
-    return split_k;
-  }
-  int min_nkt = 1 << 30, max_nkt = 0;
-  for (int i = 0; i < n; ++i) {
-    const int nkt = (gs[i]->K + kKP - 1) / kKP;
-    min_nkt = std::min(min_nkt, nkt);
-    max_nkt = std::max(max_nkt, nkt);
-  }
-  for (int i = 0; i < n; ++i) splits[i] = 1;
-  if (NT <= 64 && max_nkt > 2 * min_nkt) {
-    // Weight-streaming launches (few tokens): linears more than twice as deep
-    // in K as the shallowest of the launch are split over a cluster of C
-    // CTAs, so that no CTA walks more than about twice the K tiles of the
-    // shallowest; the others stay whole.  (The split costs no extra shared
-    // memory: partial sums land in the stage memory of the owner once the
-    // cluster is done with its stages.)  With many tokens the launch already
-    // has several waves of CTAs and splitting measured slower.
-    int C = 1;
-    while (C < 8 && max_nkt > 2 * min_nkt * C) C *= 2;
-    for (int i = 0; i < n; ++i) {
-      const int nkt = (gs[i]->K + kKP - 1) / kKP;
-      if (nkt > 2 * min_nkt && C <= nkt) splits[i] = C;
-    }
-    return C;
-  }
-  // similar depths: one factor for all, raised while the launch has fewer
-  // CTAs than SMs
-  int C = 1;
-  auto total = [&]() {
-    int t = 0;
-    for (int i = 0; i < n; ++i)
-      t += ((gs[i]->N + kBM - 1) / kBM) * ((gs[i]->M + NT - 1) / NT) * splits[i];
-    return t;
-  };
-  while (C < 8 && total() < 148 && 2 * C <= min_nkt) {
-    C *= 2;
-    for (int i = 0; i < n; ++i) splits[i] = C;
-  }
-  return C;
+  if (g.y != nullptr &&
+      !encode(&P.ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M,
+              static_cast<uint64_t>(g.ldy) * 2, kBM, C::kCh, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE))
+    return false;
+  P.s_x = g.s_x;
+  P.s_w = g.w_scale;
+  P.bias = g.bias;
+  P.y = static_cast<__nv_bfloat16*>(g.y);
+  P.acc = g.y == nullptr ? g.acc : nullptr;
+  P.M = g.M;
+  P.N = g.N;
+  P.K = g.K;
+  P.ldy = g.ldy;
+  P.tiles_n = (g.N + kBM - 1) / kBM;
+  P.nks = (g.K + kKS - 1) / kKS;     // a ragged last stage reads zeros past K
+  P.tile_base = t0;
+  return true;
 }
 
-template <int NT>
-cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cudaStream_t stream) {
-  // (Giving the deepest linears of a batch a launch of their own, with their
-  // own split-K factor, balances the K walk per CTA but measured slower on
-  // the DiT shapes: each extra launch costs more than the imbalance.)
-  for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
-    const int m = std::min(kMaxBatch, n - i0);
-    int splits[kMaxBatch];
-    const int C = choose_splits<NT>(gs + i0, m, split_k, splits);
-    // CTAs are dispatched in index order: the split (deepest) linears first,
-    // so that a partial second wave holds only short CTAs
-    const GemmArgs* order[kMaxBatch];
-    int osplit[kMaxBatch];
-    int k = 0;
-    for (int pass = 0; pass < 2; ++pass)
-      for (int i = 0; i < m; ++i)
-        if ((splits[i] > 1) == (pass == 0)) {
-          order[k] = gs[i0 + i];
-          osplit[k++] = splits[i];
-        }
-    cudaError_t e = launch_group<NT>(order, osplit, m, C, stream);
+// All problems of one (token tile, activation form) group, in launches of at
+// most kMaxBatch problems and kMaxTiles tiles (a problem with more tiles is
+// cut into tile ranges).
+template <int NT, bool kImage>
+cudaError_t launch_group(const std::vector<const GemmArgs*>& gs, cudaStream_t stream) {
+  Batch batch;
+  std::memset(&batch, 0, sizeof(batch));
+  int tiles = 0;
+  auto flush = [&]() -> cudaError_t {
+    if (batch.n == 0) return cudaSuccess;
+    batch.tile_start[batch.n] = tiles;
+    cudaError_t e = launch_batch<NT, kImage>(batch, stream);
+    std::memset(&batch, 0, sizeof(batch));
+    tiles = 0;
+    return e;
+  };
+  for (const GemmArgs* g : gs) {
+    const int total = ((g->N + kBM - 1) / kBM) * ((g->M + NT - 1) / NT);
+    for (int t0 = 0; t0 < total;) {
+      if (batch.n == kMaxBatch || tiles == kMaxTiles) {
+        cudaError_t e = flush();
+        if (e != cudaSuccess) return e;
+      }
+      const int take = std::min(total - t0, kMaxTiles - tiles);
+      if (!fill_problem<NT, kImage>(batch.p[batch.n], *g, t0)) return cudaErrorInvalidValue;
+      batch.tile_start[batch.n] = tiles;
+      ++batch.n;
+      tiles += take;
+      t0 += take;
+    }
+  }
+  return flush();
+}
+
+int token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+template <bool kImage>
+cudaError_t launch_form(const std::vector<const GemmArgs*>& v, cudaStream_t stream) {
+  static const int kTiles[4] = {16, 32, 64, 128};
+  for (int t : kTiles) {
+    std::vector<const GemmArgs*> grp;
+    for (const GemmArgs* g : v)
+      if (token_tile(g->M) == t) grp.push_back(g);
+    if (grp.empty()) continue;
+    cudaError_t e;
+    switch (t) {
+      case 16: e = launch_group<16, kImage>(grp, stream); break;
+      case 32: e = launch_group<32, kImage>(grp, stream); break;
+      case 64: e = launch_group<64, kImage>(grp, stream); break;
+      default: e = launch_group<128, kImage>(grp, stream); break;
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -626,46 +658,19 @@ cudaError_t launch_nt_batches(const GemmArgs* const* gs, int n, int split_k, cud
 bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
                    uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
                    CUtensorMapSwizzle swizzle) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {pitch};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode(map, dt, ptr, inner, outer, pitch, box_inner, box_outer, swizzle,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-int gemm_choose_split(int M, int N, int K) {
-  const int nt = token_tile(M);
-  if (nt == 256) return 1;
-  const int tiles = ((N + kBM - 1) / kBM) * ((M + nt - 1) / nt);
-  const int nkt = (K + kKP - 1) / kKP;
-  int S = 1;
-  while (S < 8 && tiles * S < 148 && 2 * S <= nkt) S *= 2;
-  return S;
-}
-
-cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream) {
-  // group by token tile (a template parameter of the kernel)
-  static const int kTiles[5] = {16, 32, 64, 128, 256};
-  for (int t : kTiles) {
-    std::vector<const GemmArgs*> grp;
-    for (int i = 0; i < n; ++i)
-      if (gs[i].M > 0 && token_tile(gs[i].M) == t) grp.push_back(&gs[i]);
-    if (grp.empty()) continue;
-    cudaError_t e;
-    switch (t) {
-      case 16: e = launch_nt_batches<16>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
-      case 32: e = launch_nt_batches<32>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
-      case 64: e = launch_nt_batches<64>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
-      case 128: e = launch_nt_batches<128>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
-      default: e = launch_nt_batches<256>(grp.data(), static_cast<int>(grp.size()), split_k, stream); break;
-    }
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int /*split_k*/,
+                                   cudaStream_t stream) {
+  // linears whose activations come as the int8 image, and the packed rest
+  std::vector<const GemmArgs*> img, pk;
+  for (int i = 0; i < n; ++i)
+    if (gs[i].M > 0) (gs[i].xq8 != nullptr ? img : pk).push_back(&gs[i]);
+  cudaError_t e = launch_form<true>(img, stream);
+  if (e == cudaSuccess) e = launch_form<false>(pk, stream);
+  return e;
 }
 
 cudaError_t launch_w4a4_gemm(const GemmArgs& g, cudaStream_t stream) {

@@ -84,7 +84,7 @@ qvla_status check_linear(const qvla_packed_linear* L, bool need_weights) {
   qvla_status st = check_shape(L->N, L->K, L->block);
   if (st != QVLA_OK) return st;
   // rot == NULL: Hadamard-only linear (R_SVD = I), which has no tensor-core image
-  if (!L->perm || (!L->rot && L->rot_tc)) return QVLA_ERR_ARG;
+  if (!L->perm) return QVLA_ERR_ARG;
   if (need_weights && (!L->wq || !L->w_scale)) return QVLA_ERR_ARG;
   if (!aligned16(L->perm) || (L->rot && !aligned16(L->rot))) return QVLA_ERR_ALIGN;
   if (L->rot_tc && !aligned16(L->rot_tc)) return QVLA_ERR_ALIGN;
@@ -394,7 +394,7 @@ static qvla_status pack_impl(const float* W, int N, int K, int block, const int3
                                          cudaMemcpyHostToDevice, stream) != cudaSuccess))
     return QVLA_ERR_CUDA;
 
-  if (!hadamard_only && rot_tc_out && (block == 64 || block == 128)) {
+  if (rot_tc_out && (block == 64 || block == 128)) {
     if (!aligned16(rot_tc_out)) return QVLA_ERR_ALIGN;
     if (launch_rot_tc_image(rsvd_dev, K, block, rot_tc_out, stream) != cudaSuccess)
       return QVLA_ERR_CUDA;
@@ -512,17 +512,18 @@ qvla_status qvla_pack_weights_gptq(const float* W, int N, int K, int block, cons
 
 qvla_status qvla_pack_weights_w8(const float* W, int N, int K, int block, const int32_t* perm_in,
                                  const double* rsvd_in, int32_t* perm_out, float* rot_out,
-                                 uint8_t* wq_out, float* w_scale_out, void* workspace,
-                                 size_t ws_bytes, cudaStream_t stream) {
-  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, 8, perm_out, rot_out, nullptr,
+                                 uint16_t* rot_tc_out, uint8_t* wq_out, float* w_scale_out,
+                                 void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return pack_impl(W, N, K, block, perm_in, rsvd_in, false, 8, perm_out, rot_out, rot_tc_out,
                    wq_out, w_scale_out, workspace, ws_bytes, stream);
 }
 
 qvla_status qvla_pack_weights_hadamard(const float* W, int N, int K, int block,
-                                       const int32_t* perm_in, int32_t* perm_out, uint8_t* wq_out,
+                                       const int32_t* perm_in, int32_t* perm_out,
+                                       uint16_t* rot_tc_out, uint8_t* wq_out,
                                        float* w_scale_out, void* workspace, size_t ws_bytes,
                                        cudaStream_t stream) {
-  return pack_impl(W, N, K, block, perm_in, nullptr, true, 4, perm_out, nullptr, nullptr,
+  return pack_impl(W, N, K, block, perm_in, nullptr, true, 4, perm_out, nullptr, rot_tc_out,
                    wq_out, w_scale_out, workspace, ws_bytes, stream);
 }
 
@@ -656,6 +657,8 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
     if (st != QVLA_OK) return st;
     v[i].ws = p.workspace;
     v[i].ws_bytes = p.ws_bytes;
+    if (p.M > 0 && p.xq8 && !aligned16(p.xq8)) return QVLA_ERR_ALIGN;
+    v[i].xq8 = p.M > 0 ? p.xq8 : nullptr;
   }
   // the problems run concurrently: their scratch ranges must be disjoint
   for (int i = 0; i < n; ++i)
@@ -844,6 +847,8 @@ qvla_status qvla_w4a4_gemm_batched(const qvla_linear_problem* probs, int n, int 
     if (p.M > 0 && !p.y) return QVLA_ERR_ARG;
     qvla_status st = prepare_gemm(p.xq, p.s_x, p.M, p.L, p.y, p.ldy, nullptr, split_k, &v[i]);
     if (st != QVLA_OK) return st;
+    if (p.M > 0 && p.xq8 && !aligned16(p.xq8)) return QVLA_ERR_ALIGN;
+    v[i].xq8 = p.M > 0 ? p.xq8 : nullptr;
   }
   if (n == 0) return QVLA_OK;
   qvla_status st = check_sm100();

@@ -53,6 +53,7 @@ struct ActArgs {
   float* xr_out;          // rotate-only mode when non-null and xq == nullptr
   void* ws;               // optional scratch for the permuted copy of x
   size_t ws_bytes;
+  int8_t* xq8;            // optional int8 image of the codes (GEMM operand order)
 };
 cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream);
 // independent linears in as few launches as possible (grouped by kernel config)
@@ -99,6 +100,7 @@ cudaError_t launch_rotate_weights(const float* W, int N, int K, int block, const
 // ---- GEMM (gemm_w4a4.cu)
 struct GemmArgs {
   const uint8_t* xq;
+  const int8_t* xq8;      // int8 image of the codes, or nullptr (unpack xq)
   const float* s_x;
   int M, N, K;
   const uint8_t* wq;
@@ -118,7 +120,6 @@ bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, ui
                    CUtensorMapSwizzle swizzle);
 // independent linears in as few launches as possible (grouped by token tile)
 cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaStream_t stream);
-int gemm_choose_split(int M, int N, int K);
 // W8A8 variant (gemm_w8a8.cu): int8 codes [M][K] and [N][K] straight into the
 // tensor cores (xq and wq hold one int8 code per byte; split_k is ignored)
 cudaError_t launch_w8a8_gemm(const GemmArgs& g, cudaStream_t stream);

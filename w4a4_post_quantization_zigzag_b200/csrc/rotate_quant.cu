@@ -245,6 +245,7 @@ struct ActProblem {
   const float* table;
   const int32_t* step_dev;
   uint8_t* xq;
+  int8_t* xq8;                // int8 image of the codes (tensor-core route), or null
   float* s_x;
   float* xr_out;
   int M, ldx, K, T, Lcount, step_host, layer;
@@ -884,9 +885,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(r[c]);
           uint32_t wv[4];
           quant_pack<32>(f, s, rs, -8, 7, wv);
-          if (valid)
+          if (valid) {
             *reinterpret_cast<uint4*>(P.xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS + c0) / 2) =
                 make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            if (P.xq8 != nullptr) {
+              // the GEMM's int8 image of these 32 codes: 16*q, even codes
+              // first, then odd codes
+              uint4* d8 = reinterpret_cast<uint4*>(P.xq8 + static_cast<size_t>(m0 + t) * K + B * BS + c0);
+              d8[0] = make_uint4((wv[0] << 4) & 0xF0F0F0F0u, (wv[1] << 4) & 0xF0F0F0F0u,
+                                 (wv[2] << 4) & 0xF0F0F0F0u, (wv[3] << 4) & 0xF0F0F0F0u);
+              d8[1] = make_uint4(wv[0] & 0xF0F0F0F0u, wv[1] & 0xF0F0F0F0u, wv[2] & 0xF0F0F0F0u,
+                                 wv[3] & 0xF0F0F0F0u);
+            }
+          }
         }
       }
       tc_fence_before();
@@ -913,9 +924,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Permuted copy of bf16 rows: out[m][j] = x[m][perm[j]].  One CTA per row:
-// the row is staged in shared memory with 16-byte loads and written back in
-// permuted order with 16-byte stores (coalesced both ways).
+// Permuted copy of bf16 rows: out[m][j] = x[m][perm[j]].  One CTA per run of
+// `rpc` rows of one problem: the rows are staged in shared memory with 16-byte
+// loads (all of them in flight at once), then every thread takes 8 output
+// positions, loads their 8 permutation entries once, and writes those
+// positions of every staged row with 16-byte stores (coalesced both ways).
 struct PermJob {
   const __nv_bfloat16* x;
   const int32_t* perm;
@@ -924,38 +937,106 @@ struct PermJob {
 };
 struct PermBatch {
   int n;
-  int row_start[kMaxBatch + 1];
+  int rpc;                          // rows per CTA
+  int cta_start[kMaxBatch + 1];
   PermJob j[kMaxBatch];
 };
 
 __global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermBatch batch) {
   extern __shared__ __align__(16) uint8_t smem[];
   int ji = 0;
-  while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.row_start[ji + 1]) ++ji;
+  while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[ji + 1]) ++ji;
   const PermJob& J = batch.j[ji];
-  const int row = static_cast<int>(blockIdx.x) - batch.row_start[ji];
-  const int K = J.K;
-  unsigned short* srow = reinterpret_cast<unsigned short*>(smem);
+  const int r0 = (static_cast<int>(blockIdx.x) - batch.cta_start[ji]) * batch.rpc;
+  const int nr = min(batch.rpc, J.M - r0);
+  const int K = J.K, kc = K / 8;                  // 16-byte chunks per row
+  unsigned short* s = reinterpret_cast<unsigned short*>(smem);
   pdl_wait();
   pdl_launch_dependents();
-  const uint4* src = reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(row) * J.ldx);
-  for (int i = threadIdx.x; i < K / 8; i += 256) reinterpret_cast<uint4*>(srow)[i] = __ldg(src + i);
+  for (int e = threadIdx.x; e < nr * kc; e += 256) {
+    const int r = e / kc, c = e - r * kc;
+    reinterpret_cast<uint4*>(s + static_cast<size_t>(r) * K)[c] =
+        __ldg(reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(r0 + r) * J.ldx) + c);
+  }
   cta_sync();
-  uint4* dst = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(row) * K);
-  for (int i = threadIdx.x; i < K / 8; i += 256) {
+  for (int i = threadIdx.x; i < kc; i += 256) {
     const int4 p0 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
     const int4 p1 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
-    const int p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    uint32_t w[4];
+    int p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int a = p[2 * q], b = p[2 * q + 1];
-      const uint32_t lo = srow[static_cast<unsigned>(a) < static_cast<unsigned>(K) ? a : 0];
-      const uint32_t hi = srow[static_cast<unsigned>(b) < static_cast<unsigned>(K) ? b : 0];
-      w[q] = lo | (hi << 16);
+    for (int q = 0; q < 8; ++q) p[q] = static_cast<unsigned>(p[q]) < static_cast<unsigned>(K) ? p[q] : 0;
+    for (int r = 0; r < nr; ++r) {
+      const unsigned short* sr = s + static_cast<size_t>(r) * K;
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        w[q] = static_cast<uint32_t>(sr[p[2 * q]]) | (static_cast<uint32_t>(sr[p[2 * q + 1]]) << 16);
+      reinterpret_cast<uint4*>(J.out + static_cast<size_t>(r0 + r) * K)[i] =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
-    dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
   }
+}
+
+// The GEMM's int8 image of packed codes, for the routes that write only the
+// packed form: every 16 packed bytes (32 codes) become 32 image bytes, 16*q
+// of the even codes, then of the odd codes.
+struct ExpandJob {
+  const uint8_t* xq;
+  int8_t* xq8;
+};
+struct ExpandBatch {
+  int n;
+  long long start[kMaxBatch + 1];   // prefix sums of 16-byte packed chunks
+  ExpandJob j[kMaxBatch];
+};
+
+__global__ void __launch_bounds__(256) expand_codes_kernel(const __grid_constant__ ExpandBatch b) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const long long total = b.start[b.n];
+  for (long long u = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; u < total;
+       u += static_cast<long long>(gridDim.x) * blockDim.x) {
+    int ji = 0;
+    while (ji + 1 < b.n && u >= b.start[ji + 1]) ++ji;
+    const long long local = u - b.start[ji];
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(b.j[ji].xq) + local);
+    uint4* d = reinterpret_cast<uint4*>(b.j[ji].xq8) + 2 * local;
+    d[0] = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u, (w.z << 4) & 0xF0F0F0F0u,
+                      (w.w << 4) & 0xF0F0F0F0u);
+    d[1] = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
+  }
+}
+
+cudaError_t launch_expand(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
+  std::vector<const ActArgs*> w;
+  for (const ActArgs* a : v)
+    if (a->xq8 != nullptr && a->xq != nullptr && a->M > 0) w.push_back(a);
+  for (size_t i0 = 0; i0 < w.size(); i0 += kMaxBatch) {
+    const int n = static_cast<int>(std::min<size_t>(kMaxBatch, w.size() - i0));
+    ExpandBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.n = n;
+    long long chunks = 0;
+    for (int i = 0; i < n; ++i) {
+      b.j[i].xq = w[i0 + i]->xq;
+      b.j[i].xq8 = w[i0 + i]->xq8;
+      b.start[i] = chunks;
+      chunks += static_cast<long long>(w[i0 + i]->M) * (w[i0 + i]->K / 32);
+    }
+    b.start[n] = chunks;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>((chunks + 255) / 256, 148 * 8)), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, expand_codes_kernel, b);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
 }
 
 // Quantise fp32 rows (already rotated): one CTA per row.
@@ -1286,13 +1367,25 @@ bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
 }
 
 // Permuted copies x_perm = x[:, perm] of the problems that have scratch.
+constexpr int kPermSmemCap = 96 * 1024;
 cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
     const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
     PermBatch b;
     std::memset(&b, 0, sizeof(b));
     b.n = n;
-    int rows = 0, kmax = 0;
+    long long rows = 0;
+    int kmax = 0;
+    for (int i = 0; i < n; ++i) {
+      rows += v[i0 + i]->M;
+      kmax = std::max(kmax, v[i0 + i]->K);
+    }
+    // about two CTAs per SM, as many rows per CTA as that takes (each CTA
+    // reuses its permutation slice for all of them), within the staging cap
+    int rpc = static_cast<int>(std::min<long long>(16, (rows + 295) / 296));
+    rpc = std::max(1, std::min(rpc, kPermSmemCap / (2 * kmax)));
+    b.rpc = rpc;
+    int ctas = 0;
     for (int i = 0; i < n; ++i) {
       const ActArgs& a = *v[i0 + i];
       b.j[i].x = static_cast<const __nv_bfloat16*>(a.x);
@@ -1301,23 +1394,23 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
       b.j[i].ldx = a.ldx;
       b.j[i].M = a.M;
       b.j[i].K = a.K;
-      b.row_start[i] = rows;
-      rows += a.M;
-      kmax = std::max(kmax, a.K);
+      b.cta_start[i] = ctas;
+      ctas += (a.M + rpc - 1) / rpc;
     }
-    b.row_start[n] = rows;
+    b.cta_start[n] = ctas;
     static std::atomic<unsigned long long> attr_done{0};
     {
       cudaError_t e = once_per_device(attr_done, []() {
         return cudaFuncSetAttribute(permute_rows_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, QVLA_MAX_K * 2);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    std::max(kPermSmemCap, QVLA_MAX_K * 2));
       });
       if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(rows, 1, 1);
+    cfg.gridDim = dim3(ctas, 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(kmax) * 2;
+    cfg.dynamicSmemBytes = static_cast<size_t>(rpc) * kmax * 2;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1348,6 +1441,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     P.table = a.table;
     P.step_dev = a.step_dev;
     P.xq = a.xq;
+    P.xq8 = a.xq8;
     P.s_x = a.s_x;
     P.xr_out = a.xr_out;
     P.M = a.M;
@@ -1376,6 +1470,11 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
       cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
       if (r == cudaSuccess)
         r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      // the grid is sized for tc_ctas_per_sm() CTAs per SM: ask for the
+      // shared-memory carveout that holds them
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
       return r;
     });
     if (e != cudaSuccess) return e;
@@ -1503,6 +1602,12 @@ cudaError_t launch_rotate_quant_batch(const ActArgs* as, int n, cudaStream_t str
   cudaError_t e = launch_tc_subset(bf, stream);     // leaves the rest in bf
   if (e == cudaSuccess && !bf.empty()) e = launch_dtype<__nv_bfloat16>(bf, stream);
   if (e == cudaSuccess && !f32.empty()) e = launch_dtype<float>(f32, stream);
+  // the int8 images the CUDA-core routes did not write
+  if (e == cudaSuccess) {
+    std::vector<const ActArgs*> rest(bf);
+    rest.insert(rest.end(), f32.begin(), f32.end());
+    e = launch_expand(rest, stream);
+  }
   return e;
 }
 

@@ -222,17 +222,23 @@ def backbone_prefill(seed: int = 2, M: int = 1024, d: int = 2048, f: int = 16384
 
 
 def dit_denoise_loop(seed: int = 3, layers: int = 16, tokens: int = 16, batch: int = 32,
-                     d: int = 1536, f: int = 6144, steps: int = 8, block: int = 64) -> Workload:
+                     d: int = 1536, f: int = 6144, steps: int = 8, block: int = 64,
+                     fuse_qkv: bool = False) -> Workload:
     """Full DiT denoise loop, small-M regime: 16 layers x (q,k,v,o d->d; up d->f;
     down f->d), 16 action tokens x batch 32, 8 denoising steps, per-step scale
     table [8][96]; weights ~ N(0, 0.02) with a 1-30x log-uniform spread of
-    column norms; block 64."""
+    column norms; block 64.
+
+    fuse_qkv: q, k and v, which read the same normalised input, become one
+    linear d -> 3d (concatenated weights, one permutation and rotation, one
+    activation pass); 4 linears per layer and a table [8][64]."""
     M = tokens * batch
     lins = []
     li = 0
+    shapes = ((("qkv", d, 3 * d), ("o", d, d), ("up", d, f), ("down", f, d)) if fuse_qkv else
+              (("q", d, d), ("k", d, d), ("v", d, d), ("o", d, d), ("up", d, f), ("down", f, d)))
     for layer in range(layers):
-        for nm, K, N in (("q", d, d), ("k", d, d), ("v", d, d), ("o", d, d),
-                         ("up", d, f), ("down", f, d)):
+        for nm, K, N in shapes:
             s = seed * 1000000 + li * 10
             lins.append(Linear(f"l{layer}.{nm}", M=M, K=K, N=N, block=block, x_seed=s,
                                w_seed=s + 1, b_seed=s + 2, layer=li,
@@ -240,7 +246,8 @@ def dit_denoise_loop(seed: int = 3, layers: int = 16, tokens: int = 16, batch: i
             li += 1
     sig = step_sigmas(steps)
     tab = scale_table(seed * 1000000 + 99, steps, len(lins), sig)
-    return Workload(f"dit_denoise_loop_M{M}_d{d}_f{f}_L{layers}_T{steps}_b{block}", lins,
+    tag = "_qkv_fused" if fuse_qkv else ""
+    return Workload(f"dit_denoise_loop_M{M}_d{d}_f{f}_L{layers}_T{steps}_b{block}{tag}", lins,
                     mode="table", steps=steps, table=tab, sigmas=sig)
 
 

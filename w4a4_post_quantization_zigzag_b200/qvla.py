@@ -86,7 +86,7 @@ class qvla_linear_problem(ctypes.Structure):
                 ("T", c_int32), ("Lcount", c_int32), ("step_dev", c_void_p),
                 ("step_host", c_int32), ("layer", c_int32), ("xq", c_void_p), ("s_x", c_void_p),
                 ("y", c_void_p), ("ldy", c_int32), ("workspace", c_void_p),
-                ("ws_bytes", c_size_t)]
+                ("ws_bytes", c_size_t), ("xq8", c_void_p)]
 
 
 _P = POINTER(qvla_packed_linear)
@@ -103,9 +103,11 @@ _sig = {
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                   c_void_p]),
     "qvla_pack_weights_hadamard": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
-                                           c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                           c_void_p]),
     "qvla_pack_weights_w8": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
-                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                     c_void_p]),
     "qvla_gptq_hessian_host": (c_int, [c_void_p, c_int, c_int, c_void_p]),
     "qvla_gptq_quantize_host": (c_int, [c_void_p, c_int, c_int, c_void_p, ctypes.c_double,
                                         c_void_p, c_void_p, c_void_p]),
@@ -257,12 +259,15 @@ def qvla_pack_weights(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] 
 
 
 def qvla_pack_weights_hadamard(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
-                               perm_in: Optional[np.ndarray] = None, stream=None) -> PackedLinear:
-    """Hadamard-only pack (R_SVD = I): the packed linear has rot = rot_tc = None."""
+                               perm_in: Optional[np.ndarray] = None, image: bool = True,
+                               stream=None) -> PackedLinear:
+    """Hadamard-only pack (R_SVD = I): rot = None; with `image` (blocks 64 /
+    128) the tensor-core image of R_B = H_b, else rot_tc = None."""
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
     N, K = W.shape
-    wq_b, _, _, ws_b = qvla_packed_sizes(N, K, block)
+    wq_b, _, tc_b, ws_b = qvla_packed_sizes(N, K, block)
     dev = W.device
+    rot_tc = torch.empty(tc_b // 2, dtype=torch.int16, device=dev) if (tc_b and image) else None
     perm = torch.empty(K, dtype=torch.int32, device=dev)
     wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
     s_w = torch.empty(N, dtype=torch.float32, device=dev)
@@ -272,13 +277,14 @@ def qvla_pack_weights_hadamard(W: torch.Tensor, block: int, bias: Optional[torch
         perm_in = np.ascontiguousarray(perm_in, dtype=np.int32)
         assert perm_in.shape == (K,)
         p_in = perm_in.ctypes.data_as(c_void_p)
-    _check(_lib.qvla_pack_weights_hadamard(_ptr(W), N, K, block, p_in, _ptr(perm), _ptr(wq),
-                                           _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
+    _check(_lib.qvla_pack_weights_hadamard(_ptr(W), N, K, block, p_in, _ptr(perm),
+                                           _ptr(rot_tc), _ptr(wq), _ptr(s_w), _ptr(ws), ws_b,
+                                           _stream(stream)),
            "qvla_pack_weights_hadamard")
     if bias is not None:
         assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
         bias = bias.contiguous()
-    return PackedLinear(N, K, block, perm, None, wq, s_w, bias, rot_tc=None)
+    return PackedLinear(N, K, block, perm, None, wq, s_w, bias, rot_tc=rot_tc)
 
 
 def _host_f64(a, shape):
@@ -358,12 +364,15 @@ def qvla_pack_weights_gptq(W: torch.Tensor, block: int, x_cal: Optional[torch.Te
 
 def qvla_pack_weights_w8(W: torch.Tensor, block: int, bias: Optional[torch.Tensor] = None,
                          perm_in: Optional[np.ndarray] = None,
-                         rsvd_in: Optional[np.ndarray] = None, stream=None) -> PackedLinear:
-    """W8A8 variant: the same P and R, int8 weight codes wq [N, K]."""
+                         rsvd_in: Optional[np.ndarray] = None, image: bool = True,
+                         stream=None) -> PackedLinear:
+    """W8A8 variant: the same P and R (and, with `image`, the tensor-core image
+    of R_B for blocks 64 / 128), int8 weight codes wq [N, K]."""
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
     N, K = W.shape
-    _, rot_b, _, ws_b = qvla_packed_sizes(N, K, block)
+    _, rot_b, tc_b, ws_b = qvla_packed_sizes(N, K, block)
     dev = W.device
+    rot_tc = torch.empty(tc_b // 2, dtype=torch.int16, device=dev) if (tc_b and image) else None
     perm = torch.empty(K, dtype=torch.int32, device=dev)
     rot = torch.empty(rot_b // 4, dtype=torch.float32, device=dev)
     wq = torch.empty(N, K, dtype=torch.int8, device=dev)
@@ -379,12 +388,14 @@ def qvla_pack_weights_w8(W: torch.Tensor, block: int, bias: Optional[torch.Tenso
         assert rsvd_in.shape == (K // block, block, block)
         r_in = rsvd_in.ctypes.data_as(c_void_p)
     _check(_lib.qvla_pack_weights_w8(_ptr(W), N, K, block, p_in, r_in, _ptr(perm), _ptr(rot),
-                                     _ptr(wq), _ptr(s_w), _ptr(ws), ws_b, _stream(stream)),
+                                     _ptr(rot_tc), _ptr(wq), _ptr(s_w), _ptr(ws), ws_b,
+                                     _stream(stream)),
            "qvla_pack_weights_w8")
     if bias is not None:
         assert bias.is_cuda and bias.dtype == torch.float32 and bias.shape == (N,)
         bias = bias.contiguous()
-    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias)
+    return PackedLinear(N, K, block, perm, rot.view(K // block, block, block), wq, s_w, bias,
+                        rot_tc=rot_tc)
 
 
 def qvla_rotate_quant_a8_workspace_bytes(M: int, K: int) -> int:
@@ -594,13 +605,28 @@ class LinearProblem:
                  mode: int = QVLA_SCALE_DYNAMIC, table: Optional[torch.Tensor] = None,
                  step=None, layer: int = 0, xq: Optional[torch.Tensor] = None,
                  s_x: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-                 workspace: Optional[torch.Tensor] = None):
+                 workspace: Optional[torch.Tensor] = None, xq8=None):
+        """xq8: the int8 image of the codes that the batched rotate-quantise
+        writes and the batched GEMM reads (a device int8 [M, K] tensor, or
+        True to allocate one); None leaves the GEMM to unpack xq."""
         M = x.shape[0] if x is not None else xq.shape[0]
         dev = (x if x is not None else xq).device
+        if x is not None:
+            _expect_rows(x, L.K)
         self.L, self.x, self.table, self.step = L, x, table, step
         self.xq = xq if xq is not None else torch.empty(M, L.K // 2, dtype=torch.uint8, device=dev)
         self.s_x = s_x if s_x is not None else torch.empty(M, dtype=torch.float32, device=dev)
         self.y = y if y is not None else torch.empty(M, L.N, dtype=torch.bfloat16, device=dev)
+        if xq8 is True:
+            xq8 = torch.empty(M, L.K, dtype=torch.int8, device=dev)
+        self.xq8 = xq8
+        _expect(self.xq, torch.uint8, (M, L.K // 2), dev, "xq")
+        _expect(self.s_x, torch.float32, (M,), dev, "s_x")
+        if xq8 is not None:
+            _expect(xq8, torch.int8, (M, L.K), dev, "xq8")
+        if self.y.dim() != 2 or tuple(self.y.shape) != (M, L.N) or self.y.stride(1) != 1 \
+                or self.y.dtype != torch.bfloat16:
+            raise ValueError(f"y: expected bf16 [{M}, {L.N}] rows with unit stride")
         T, Lc = (table.shape if table is not None else (0, 0))
         sd, sh = _step_args(step)
         self.c = qvla_linear_problem(
@@ -611,7 +637,8 @@ class LinearProblem:
             sd.value if sd is not None else None, sh, layer, self.xq.data_ptr(),
             self.s_x.data_ptr(), self.y.data_ptr(), self.y.stride(0),
             workspace.data_ptr() if workspace is not None else None,
-            workspace.numel() * workspace.element_size() if workspace is not None else 0)
+            workspace.numel() * workspace.element_size() if workspace is not None else 0,
+            xq8.data_ptr() if xq8 is not None else None)
         self.workspace = workspace
 
 
