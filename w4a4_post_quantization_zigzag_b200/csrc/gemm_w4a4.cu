@@ -16,21 +16,26 @@
 // product is unchanged.
 //
 // One persistent CTA per SM, warp-specialised (320 threads):
-//   warp 0      TMA producer: per pipeline stage (128 of K) a 128-row box of
-//               packed weights and an NT-token box of activation codes go into
-//               a ring of shared-memory stages;
+//   warp 0      TMA producer: per pipeline stage (256 of K) a 128-row box of
+//               packed weights and the NT-token activation box(es) go into a
+//               ring of shared-memory stages;
 //   warp 1      MMA issuer: tcgen05.mma with A (weights) read from tensor
-//               memory and B (activations) from shared memory; int32
-//               accumulators in tensor memory, two buffers when they fit;
+//               memory and B (activations) from shared memory, eight K = 32
+//               MMAs and one commit per stage; int32 accumulators in tensor
+//               memory, two buffers when they fit;
 //   warps 2-5   unpack: each thread owns one weight row (one tensor-memory
-//               lane), reads the row's 64 packed bytes of the stage and stores
-//               its 128 int8 values into a ring of tensor-memory A stages
-//               (tcgen05.st), so the weights never make a second trip through
-//               shared memory; with nibble-packed activations these warps also
-//               unpack the B tile into a 128-byte-swizzled shared-memory tile;
+//               lane), reads the row's 128 packed bytes of the stage and
+//               stores its 256 int8 values into the stage's tensor-memory A
+//               slot (tcgen05.st), so the weights never make a second trip
+//               through shared memory; with nibble-packed activations these
+//               warps also unpack the B tile into 128-byte-swizzled shared
+//               memory;
 //   warps 6-9   epilogue: tcgen05.ld of the accumulator (one output channel per
 //               thread), dequantise, add the bias, round to bf16, stage
 //               32-token chunks in shared memory, TMA tensor stores.
+// Shared-memory stage s and tensor-memory A slot s form one ring: the unpack
+// warps' arrival says both that the stage's bytes were read and that its A is
+// ready, and one MMA commit frees both.
 // The activation operand is either the int8 image of the codes written by the
 // rotate-quantise step (16*q, the same order inside each 32-code group; a TMA
 // box lands directly in the MMA layout) or the nibble-packed codes.
@@ -58,10 +63,9 @@ namespace qvla {
 namespace {
 
 constexpr int kBM = 128;                  // weight rows per tile (UMMA M, tensor-memory lanes)
-constexpr int kKS = 128;                  // K per pipeline stage
-constexpr int kAPack = kKS / 2;           // packed weight bytes per row per stage
+constexpr int kKS = 256;                  // K per pipeline stage
+constexpr int kAPack = kKS / 2;           // packed weight bytes per row per stage (one 128B-swizzled box)
 constexpr int kACols = kKS / 4;           // tensor-memory columns of one unpacked A stage
-constexpr int kSA = 8;                    // A stages in tensor memory
 constexpr int kThreads = 320;
 constexpr int kOutSlots = 4;              // output staging ring (32-token chunks)
 constexpr int kTmemCols = 512;
@@ -76,25 +80,31 @@ struct Cfg {
   static constexpr int kAccCols = NT < 32 ? 32 : NT;
   static constexpr int kACol0 = kAcc * kAccCols;                 // first A-stage column
   static constexpr int kABytes = kBM * kAPack;                   // packed weight box
-  static constexpr int kBBytes = NT * (kImage ? kKS : kAPack);   // activation box
-  static constexpr int kUBytes = kImage ? 0 : NT * kKS;          // unpacked activations
+  // activations: the image as two 128-byte boxes (K halves) of NT rows, or
+  // one 128-byte box of packed codes plus their unpacked two halves
+  static constexpr int kBBytes = kImage ? 2 * NT * 128 : NT * 128;
+  static constexpr int kUBytes = kImage ? 0 : 2 * NT * 128;
   static constexpr int kStage = kABytes + kBBytes + kUBytes;
   static constexpr int kCh = NT < 32 ? NT : 32;                  // tokens per output chunk
   static constexpr int kOutBytes = kOutSlots * kCh * kBM * 2;
-  static constexpr int kRing = (200 * 1024 - kOutBytes) / kStage;
-  static constexpr int kS = kRing > 8 ? 8 : kRing;
+  static constexpr int kRing = (208 * 1024 - kOutBytes) / kStage;
+  static constexpr int kTmemStages = (kTmemCols - kACol0) / kACols;
+  static constexpr int kS0 = kRing < kTmemStages ? kRing : kTmemStages;
+  // one ring: smem stage s and tensor-memory A stage s go together
+  static constexpr int kS = kS0 > 8 ? 8 : kS0;
   // at least 116 KB, so that two CTAs never share an SM (each takes all of
   // tensor memory)
   static constexpr int kNeed = kS * kStage + kOutBytes + 1024;
   static constexpr int kSmem = kNeed < 116 * 1024 ? 116 * 1024 : kNeed;
-  static_assert(kACol0 + kSA * kACols <= kTmemCols, "tensor memory");
+  static_assert(kACol0 + kS * kACols <= kTmemCols, "tensor memory");
   static_assert(kStage % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "alignment");
   static_assert(kS >= 2, "pipeline depth");
 };
 
 struct Barriers {
-  uint64_t full[8], empty[8];              // shared-memory stages
-  uint64_t a_full[kSA], a_empty[kSA];      // tensor-memory A stages
+  uint64_t full[8];                        // TMA: packed weights and activations landed
+  uint64_t unp_done[8];                    // the four unpack warps are done with the stage
+  uint64_t mma_done[8];                    // the MMAs reading the stage have completed
   uint64_t acc_full[2], acc_empty[2];      // accumulators
   uint64_t drain;
   uint32_t tmem;
@@ -103,9 +113,9 @@ struct Barriers {
 // One linear of a launch.  Its tiles are numbered n-tile fastest (tiles that
 // share an activation box are neighbours), from tile_base on.
 struct Problem {
-  CUtensorMap tw;                 // packed weights [N][K/2]: box 64 B x 128 rows, 64B swizzle
-  CUtensorMap tx;                 // activations: int8 image [M][K] (box 128 x NT, 128B
-                                  // swizzle) or packed [M][K/2] (box 64 x NT, 64B swizzle)
+  CUtensorMap tw;                 // packed weights [N][K/2]: box 128 B x 128 rows, 128B swizzle
+  CUtensorMap tx;                 // activations: int8 image [M][K] or packed [M][K/2], box
+                                  // 128 B x NT rows, 128B swizzle
   CUtensorMap ty;                 // bf16 output [M][ldy]: box 128 channels x kCh tokens
   const float* s_x;
   const float* s_w;
@@ -114,7 +124,7 @@ struct Problem {
   int32_t* acc;                   // int32 [M][N] accumulators instead of y (or null)
   int M, N, K, ldy;
   int tiles_n;                    // ceil(N / 128)
-  int nks;                        // K stages: ceil(K / 128)
+  int nks;                        // K stages: ceil(K / 256)
   int tile_base;                  // first tile of this problem in the launch
 };
 struct Batch {
@@ -153,18 +163,32 @@ QVLA_DEVICE void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[NT < 32 ? NT : 32])
   }
 }
 
+// 16 packed bytes (32 codes) -> 8 words of 16*q int8: the even codes of the
+// four words, then the odd codes.
+QVLA_DEVICE void unpack32(const uint4 v, uint32_t* o) {
+  o[0] = (v.x << 4) & 0xF0F0F0F0u;
+  o[1] = (v.y << 4) & 0xF0F0F0F0u;
+  o[2] = (v.z << 4) & 0xF0F0F0F0u;
+  o[3] = (v.w << 4) & 0xF0F0F0F0u;
+  o[4] = v.x & 0xF0F0F0F0u;
+  o[5] = v.y & 0xF0F0F0F0u;
+  o[6] = v.z & 0xF0F0F0F0u;
+  o[7] = v.w & 0xF0F0F0F0u;
+}
+
 template <int NT, bool kImage>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a4_gemm_kernel(const __grid_constant__ Batch batch, unsigned int* err) {
   using C = Cfg<NT, kImage>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
+  __shared__ float sx_s[NT];                     // s_x of the epilogue's current tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t_begin = batch.cta_begin[blockIdx.x];
   const int t_end = batch.cta_begin[blockIdx.x + 1];
 
-  // 1024-byte aligned stage memory (swizzled TMA destinations)
+  // 1024-byte aligned stage memory (128B-swizzled TMA destinations)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* const base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint8_t* const stages = base;
@@ -173,11 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < C::kS; ++s) {
       mbar_init(&bars.full[s], 1);
-      mbar_init(&bars.empty[s], 5);          // four unpack warps + the MMA commit
-    }
-    for (int a = 0; a < kSA; ++a) {
-      mbar_init(&bars.a_full[a], 4);
-      mbar_init(&bars.a_empty[a], 1);
+      mbar_init(&bars.unp_done[s], 4);
+      mbar_init(&bars.mma_done[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
@@ -204,7 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       constexpr uint32_t kTx = C::kABytes + C::kBBytes;
-      constexpr int kBX = kImage ? kKS : kAPack;          // activation box x step
       // Weights do not depend on the previous kernel in the stream: the first
       // ring's worth of weight boxes are requested before waiting for it
       // (programmatic dependent launch), the activation boxes after.
@@ -237,13 +257,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = stages + s * C::kStage;
           if (g >= pre) {
             if (g >= C::kS) {
-              ok = mbar_wait(&bars.empty[s], ((g / C::kS) - 1) & 1, err);
+              // the unpack warps have read the stage and the MMAs are done with it
+              const uint32_t ph = ((g / C::kS) - 1) & 1;
+              ok = mbar_wait(&bars.unp_done[s], ph, err) && mbar_wait(&bars.mma_done[s], ph, err);
               if (!ok) break;
             }
             mbar_arrive_expect_tx(&bars.full[s], kTx);
             tma_load_2d(st, &P.tw, &bars.full[s], ks * kAPack, tr.n0);
           }
-          tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kBX, tr.m0);
+          if constexpr (kImage) {
+            tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kKS, tr.m0);
+            tma_load_2d(st + C::kABytes + NT * 128, &P.tx, &bars.full[s], ks * kKS + 128, tr.m0);
+          } else {
+            tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kAPack, tr.m0);
+          }
         }
       }
       // never leave with copies in flight: the last load of every stage has landed
@@ -264,26 +291,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bars.acc_empty[b], (use - 1) & 1, err);
           if (!ok) break;
         }
-        tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(b * C::kAccCols);
         for (int ks = 0; ks < nks; ++ks, ++g) {
-          const int s = g % C::kS, a = g % kSA;
-          ok = mbar_wait(&bars.a_full[a], (g / kSA) & 1, err);
-          if (ok && kImage) ok = mbar_wait(&bars.full[s], (g / C::kS) & 1, err);
+          const int s = g % C::kS;
+          // the stage's A is in tensor memory (and, when the unpack warps got
+          // the stage, its TMA bytes, activations included, had landed)
+          ok = mbar_wait(&bars.unp_done[s], (g / C::kS) & 1, err);
           if (!ok) break;
           tc_fence_after();
           const uint32_t bs =
               smem_u32(stages + s * C::kStage + C::kABytes + (kImage ? 0 : C::kBBytes));
-          const uint32_t at = tmem + static_cast<uint32_t>(C::kACol0 + a * kACols);
+          const uint32_t at = tmem + static_cast<uint32_t>(C::kACol0 + s * kACols);
 #pragma unroll
           for (int kk = 0; kk < kKS / 32; ++kk) {
-            // 32 codes of K: A columns [8kk, 8kk+8) of the stage, B bytes
-            // [32kk, 32kk+32) of every 128-byte row
-            const uint64_t bd = smem_desc_kmajor_sw128(bs + 32 * kk);
+            // 32 codes of K: A columns [8kk, 8kk+8) of the stage; B half kk/4,
+            // bytes [32(kk%4), +32) of each 128-byte row
+            const uint64_t bd = smem_desc_kmajor_sw128(bs + (kk >> 2) * (NT * 128) + 32 * (kk & 3));
             umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&bars.a_empty[a]);
-          umma_commit(&bars.empty[s]);
+          umma_commit(&bars.mma_done[s]);
         }
         if (!ok) break;
         umma_commit(&bars.acc_full[b]);
@@ -297,75 +323,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;                // weight row of the tile
     const int wt = tid - 64;                       // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    constexpr int kBItems = (NT * 4 + 127) / 128;  // packed activation chunks per thread
+    constexpr int kBItems = (NT * 8 + 127) / 128;  // packed activation chunks per thread
     bool ok = true;
     int g = 0;
     for (int i = t_begin; i < t_end && ok; ++i) {
       const int nks = batch.p[decode<NT>(batch, batch.order[i]).p].nks;
       for (int ks = 0; ks < nks; ++ks, ++g) {
-        const int s = g % C::kS, a = g % kSA;
+        const int s = g % C::kS;
         // warp-uniform outcome: the tensor-memory stores below are warp-wide
         ok = __all_sync(kFull, mbar_wait(&bars.full[s], (g / C::kS) & 1, err));
         if (!ok) break;
         const uint32_t st = smem_u32(stages + s * C::kStage);
-        // the row's 64 packed bytes; 64-byte swizzle: 16-byte chunk c of row r
-        // sits at chunk c ^ ((r >> 1) & 3)
-        uint4 w[4];
+        // the row's 128 packed bytes; 128-byte swizzle: 16-byte chunk c of row
+        // r sits at chunk c ^ (r & 7)
+        uint4 w[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) w[c] = lds128(st + row * kAPack + ((c ^ ((row >> 1) & 3)) << 4));
+        for (int c = 0; c < 8; ++c) w[c] = lds128(st + row * kAPack + ((c ^ (row & 7)) << 4));
+        // the previous use of this stage (tensor-memory A, unpacked activations)
+        // is over once its MMAs have completed
+        if (g >= C::kS) {
+          ok = __all_sync(kFull, mbar_wait(&bars.mma_done[s], ((g / C::kS) - 1) & 1, err));
+          if (!ok) break;
+        }
+        tc_fence_after();
         if constexpr (!kImage) {
           // activation chunk e: code row br = e % NT, 32-code group c = e / NT
-          // (consecutive threads take consecutive rows: conflict-free)
+          // (consecutive threads take consecutive rows: conflict-free); group
+          // c goes to K half c / 4 as 16-byte chunks 2(c%4) (even codes) and
+          // 2(c%4)+1 (odd codes) of a 128-byte swizzled row
           const uint32_t bp = st + C::kABytes, bu = st + C::kABytes + C::kBBytes;
 #pragma unroll
           for (int k = 0; k < kBItems; ++k) {
             const int e = wt + k * 128;
-            if (e < NT * 4) {
+            if (e < NT * 8) {
               const int br = e % NT, c = e / NT;
-              const uint4 v = lds128(bp + br * kAPack + ((c ^ ((br >> 1) & 3)) << 4));
-              uint4 ev, od;
-              ev.x = (v.x << 4) & 0xF0F0F0F0u;
-              ev.y = (v.y << 4) & 0xF0F0F0F0u;
-              ev.z = (v.z << 4) & 0xF0F0F0F0u;
-              ev.w = (v.w << 4) & 0xF0F0F0F0u;
-              od.x = v.x & 0xF0F0F0F0u;
-              od.y = v.y & 0xF0F0F0F0u;
-              od.z = v.z & 0xF0F0F0F0u;
-              od.w = v.w & 0xF0F0F0F0u;
-              // 128-byte swizzled K-major row: chunk 2c even codes, 2c+1 odd codes
-              sts128(bu + br * kKS + (((2 * c) ^ (br & 7)) << 4), ev);
-              sts128(bu + br * kKS + (((2 * c + 1) ^ (br & 7)) << 4), od);
+              const uint4 v = lds128(bp + br * 128 + ((c ^ (br & 7)) << 4));
+              uint32_t o[8];
+              unpack32(v, o);
+              const uint32_t rowp = bu + (c >> 2) * (NT * 128) + br * 128;
+              const int cl = c & 3;
+              sts128(rowp + (((2 * cl) ^ (br & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+              sts128(rowp + (((2 * cl + 1) ^ (br & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
             }
           }
         }
-        if (g >= kSA) {
-          ok = __all_sync(kFull, mbar_wait(&bars.a_empty[a], ((g / kSA) - 1) & 1, err));
-          if (!ok) break;
-        }
-        tc_fence_after();
-        // 32 columns: for packed chunk c, columns [8c, 8c+4) the even codes of
-        // its four words, [8c+4, 8c+8) the odd codes
-        uint32_t av[32];
+        // 64 columns: packed chunk c -> columns [8c, 8c+8)
+        const uint32_t ta = tmem + lane_base + static_cast<uint32_t>(C::kACol0 + s * kACols);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          av[8 * c + 0] = (w[c].x << 4) & 0xF0F0F0F0u;
-          av[8 * c + 1] = (w[c].y << 4) & 0xF0F0F0F0u;
-          av[8 * c + 2] = (w[c].z << 4) & 0xF0F0F0F0u;
-          av[8 * c + 3] = (w[c].w << 4) & 0xF0F0F0F0u;
-          av[8 * c + 4] = w[c].x & 0xF0F0F0F0u;
-          av[8 * c + 5] = w[c].y & 0xF0F0F0F0u;
-          av[8 * c + 6] = w[c].z & 0xF0F0F0F0u;
-          av[8 * c + 7] = w[c].w & 0xF0F0F0F0u;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t av[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) unpack32(w[4 * h + c], av + 8 * c);
+          tmem_st32(ta + 32 * h, av);
         }
-        tmem_st32(tmem + lane_base + static_cast<uint32_t>(C::kACol0 + a * kACols), av);
         tmem_st_wait();
         if constexpr (!kImage) fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars.a_full[a]);
-          mbar_arrive(&bars.empty[s]);
-        }
+        if (lane == 0) mbar_arrive(&bars.unp_done[s]);
       }
     }
   } else {
@@ -381,7 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tr = decode<NT>(batch, batch.order[i]);
       const Problem& P = batch.p[tr.p];
       const int b = tc % C::kAcc, use = tc / C::kAcc;
-      // one outcome for all four epilogue warps (they share named barriers)
+      // the tile's token scales, staged while its MMAs run (the previous
+      // tile's readers all passed the barrier that closed its last chunk)
+      if (P.acc == nullptr)
+        for (int j = et; j < NT; j += 128) sx_s[j] = tr.m0 + j < P.M ? __ldg(P.s_x + tr.m0 + j) : 0.f;
+      // one outcome for all four epilogue warps (they share named barriers);
+      // also publishes sx_s
       ok = named_barrier_all(2, 128, mbar_wait(&bars.acc_full[b], use & 1, err));
       if (!ok) break;
       tc_fence_after();
@@ -418,10 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier(1, 128);
 #pragma unroll
         for (int j = 0; j < C::kCh; ++j) {
-          const int m = tr.m0 + c0 + j;
-          const float sx = m < P.M ? __ldg(P.s_x + m) : 0.f;
           const int32_t a = static_cast<int32_t>(r[j]) >> 8;
-          ot[j * kBM + row] = __float2bfloat16_rn(fmaf(sx * sw, static_cast<float>(a), bn));
+          ot[j * kBM + row] = __float2bfloat16_rn(fmaf(sx_s[c0 + j] * sw, static_cast<float>(a), bn));
         }
         fence_proxy_async_smem();
         named_barrier(1, 128);
@@ -438,6 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (et == 0) bulk_commit();                // one group per chunk, maybe empty
         ++chunk;
       }
+      // sx_s is rewritten for the next tile only after every thread is done
+      // with this one
+      named_barrier(1, 128);
     }
     if (et == 0) bulk_wait0();
     pdl_launch_dependents();
@@ -500,7 +521,7 @@ int sm_count() {
   return n;
 }
 
-// A tile's cost in K stages, plus a fixed share for its epilogue and ramp.
+// A tile's cost in 128-wide K steps, plus a fixed share for its epilogue.
 constexpr int kTileOverhead = 2;
 
 // Deals the launch's tiles to at most sm_count() CTAs, longest first, each to
@@ -511,7 +532,8 @@ int schedule(Batch& b) {
   const int G = std::min(sm_count(), T);
   std::vector<int> ids(T), cost(T);
   for (int p = 0; p < b.n; ++p)
-    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t) cost[t] = b.p[p].nks + kTileOverhead;
+    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t)
+      cost[t] = (b.p[p].K + 127) / 128 + kTileOverhead;
   for (int t = 0; t < T; ++t) ids[t] = t;
   std::stable_sort(ids.begin(), ids.end(), [&](int x, int y) { return cost[x] > cost[y]; });
   using Load = std::pair<long long, int>;
@@ -566,15 +588,15 @@ bool fill_problem(Problem& P, const GemmArgs& g, int t0) {
   using C = Cfg<NT, kImage>;
   std::memset(&P, 0, sizeof(P));
   if (!encode(&P.tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, g.K / 2, g.N, g.K / 2, kAPack, kBM,
-              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return false;
   if (kImage) {
-    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq8, g.K, g.M, g.K, kKS, NT,
+    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq8, g.K, g.M, g.K, 128, NT,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
       return false;
   } else {
-    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K / 2, g.M, g.K / 2, kAPack, NT,
-                CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    if (!encode(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, g.K / 2, g.M, g.K / 2, 128, NT,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
       return false;
   }
   if (g.y != nullptr &&
