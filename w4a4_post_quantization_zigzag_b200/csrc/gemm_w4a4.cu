@@ -396,8 +396,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tr = decode<NT>(batch, batch.order[i]);
       const Problem& P = batch.p[tr.p];
       const int b = tc % C::kAcc, use = tc / C::kAcc;
-      // the tile's token scales, staged while its MMAs run (the previous
-      // tile's readers all passed the barrier that closed its last chunk)
+      // the tile's token scales, output-channel scale and bias, loaded while
+      // its MMAs run (the previous tile's readers of sx_s all passed the
+      // barrier that closed its last chunk)
+      const int n = tr.n0 + row;
+      const bool nv = n < P.N;
+      const float sw = (P.acc == nullptr && nv) ? __ldg(P.s_w + n) : 0.f;
+      const float bn = (P.bias != nullptr && nv) ? __ldg(P.bias + n) : 0.f;
       if (P.acc == nullptr)
         for (int j = et; j < NT; j += 128) sx_s[j] = tr.m0 + j < P.M ? __ldg(P.s_x + tr.m0 + j) : 0.f;
       // one outcome for all four epilogue warps (they share named barriers);
@@ -405,10 +410,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = named_barrier_all(2, 128, mbar_wait(&bars.acc_full[b], use & 1, err));
       if (!ok) break;
       tc_fence_after();
-      const int n = tr.n0 + row;
-      const bool nv = n < P.N;
-      const float sw = (P.acc == nullptr && nv) ? __ldg(P.s_w + n) : 0.f;
-      const float bn = (P.bias != nullptr && nv) ? __ldg(P.bias + n) : 0.f;
       const bool tma = tr.n0 + kBM <= P.N || (P.N & 7) == 0;
       const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(b * C::kAccCols);
 #pragma unroll 1

@@ -653,8 +653,10 @@ QVLA_DEVICE void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint6
       : "memory");
 }
 
+// Block 64 runs two CTAs per SM (the grid is sized for that): the register
+// budget must let two 320-thread CTAs share the register file.
 template <int BS, int MODE, bool kTmaA>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
     rotq_tc_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
   using C = TcCfg<BS>;
   extern __shared__ uint8_t smem_raw[];
@@ -951,18 +953,44 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant
   const int nr = min(batch.rpc, J.M - r0);
   const int K = J.K, kc = K / 8;                  // 16-byte chunks per row
   unsigned short* s = reinterpret_cast<unsigned short*>(smem);
+  // the permutation does not depend on the previous kernel: its first slice
+  // is read before waiting for it, in flight together with the rows
+  const int i0 = threadIdx.x;
+  int4 pa = make_int4(0, 0, 0, 0), pb = make_int4(0, 0, 0, 0);
+  if (i0 < kc) {
+    pa = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i0);
+    pb = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i0 + 1);
+  }
   pdl_wait();
   pdl_launch_dependents();
-  for (int e = threadIdx.x; e < nr * kc; e += 256) {
-    const int r = e / kc, c = e - r * kc;
-    reinterpret_cast<uint4*>(s + static_cast<size_t>(r) * K)[c] =
-        __ldg(reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(r0 + r) * J.ldx) + c);
+  // rows into shared memory: each round puts up to 8 loads per thread in
+  // flight before storing any of them
+  for (int e0 = 0; e0 < nr * kc; e0 += 8 * 256) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * 256 + threadIdx.x;
+      if (e < nr * kc) {
+        const int r = e / kc, c = e - r * kc;
+        v[u] = __ldg(reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(r0 + r) * J.ldx) + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * 256 + threadIdx.x;
+      if (e < nr * kc) {
+        const int r = e / kc, c = e - r * kc;
+        reinterpret_cast<uint4*>(s + static_cast<size_t>(r) * K)[c] = v[u];
+      }
+    }
   }
   cta_sync();
   for (int i = threadIdx.x; i < kc; i += 256) {
-    const int4 p0 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
-    const int4 p1 = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
-    int p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    if (i != i0) {
+      pa = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
+      pb = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
+    }
+    int p[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
     for (int q = 0; q < 8; ++q) p[q] = static_cast<unsigned>(p[q]) < static_cast<unsigned>(K) ? p[q] : 0;
     for (int r = 0; r < nr; ++r) {
