@@ -128,14 +128,24 @@ QVLA_DEVICE int quant_code_fast(float v, float s, float rs, int qmin, int qmax) 
   return static_cast<int>(r);
 }
 
-// Codes of N consecutive values, packed two per byte (value 2k in the low
-// nibble of byte k) into N/8 32-bit words: the same codes as quant_code, as
-// straight-line code (so the independent elements overlap) with the rare
-// near-half-integer elements redone by exact division afterwards.  The code's
-// 4-bit two's complement is read from the mantissa of code + 2^23 + 16.
+// 4-bit codes of N consecutive values, packed two per byte (value 2k in the
+// low nibble of byte k) into N/8 32-bit words: the same codes as
+// quant_code(v, s, -8, 7), as straight-line code (so the independent elements
+// overlap) with the rare near-half-integer elements redone by exact division
+// afterwards.  Three identities keep it short:
+//   * clamping the quotient before rounding gives the same code as clamping
+//     the rounded quotient (the bounds are integers and rint is monotonic),
+//     and a clamped quotient is an integer, never near a half-integer;
+//   * |q - rint(q)| is exact and at most 1/2, so "within 2^-18 of a
+//     half-integer" is |q - rint(q)| > 1/2 - 2^-18, tracked as one running max;
+//   * four codes c_j in [-8, 7] go into one float as
+//     2^23 + sum_j (c_j + 8) 16^j, every partial sum an integer in
+//     [2^23, 2^24), so its low 16 mantissa bits are the four offset nibbles;
+//     XOR 8 turns an offset nibble c + 8 into the 4-bit two's complement of c.
+constexpr float kNearHalf = 0.499996185302734375f;   // 1/2 - 2^-18
+
 template <int N>
-QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float rs, int qmin, int qmax,
-                            uint32_t (&w)[N / 8]) {
+QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float rs, uint32_t (&w)[N / 8]) {
   static_assert(N % 8 == 0 && N <= 32, "8..32 values");
   float c[N];
   if (s == 0.f) {
@@ -143,28 +153,34 @@ QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float rs, int qmin, in
     for (int i = 0; i < N; ++i) c[i] = 0.f;
   } else if (rs == 0.f) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) c[i] = exact_rint_quotient(v[i], s);
+    for (int i = 0; i < N; ++i) c[i] = fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f);
   } else {
-    uint32_t near = 0u;
+    float dmax = 0.f;
 #pragma unroll
     for (int i = 0; i < N; ++i) {
-      const float q = v[i] * rs;
+      const float q = fminf(fmaxf(v[i] * rs, -8.f), 7.f);
       c[i] = rintf(q);
-      near |= (fabsf(fabsf(q - c[i]) - 0.5f) < 3.814697265625e-06f ? 1u : 0u) << i;
+      dmax = fmaxf(dmax, fabsf(q - c[i]));
     }
-    if (near) {
+    if (dmax > kNearHalf) {
 #pragma unroll
       for (int i = 0; i < N; ++i)
-        if ((near >> i) & 1u) c[i] = exact_rint_quotient(v[i], s);
+        if (fabsf(fminf(fmaxf(v[i] * rs, -8.f), 7.f) - c[i]) > kNearHalf)
+          c[i] = fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f);
     }
   }
 #pragma unroll
-  for (int k = 0; k < N / 8; ++k) w[k] = 0u;
+  for (int k = 0; k < N / 8; ++k) {
+    float h[2];
 #pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const float cl = fminf(fmaxf(c[i], static_cast<float>(qmin)), static_cast<float>(qmax));
-    const uint32_t nib = __float_as_uint(cl + 8388624.0f) & 15u;      // 2^23 + 16
-    w[i >> 3] |= nib << (4 * (i & 7));
+    for (int g = 0; g < 2; ++g) {
+      const float* cg = c + 8 * k + 4 * g;
+      float a = cg[0] + 8423560.0f;                  // 2^23 + 8 * (1 + 16 + 256 + 4096)
+      a = fmaf(cg[1], 16.f, a);
+      a = fmaf(cg[2], 256.f, a);
+      h[g] = fmaf(cg[3], 4096.f, a);
+    }
+    w[k] = __byte_perm(__float_as_uint(h[0]), __float_as_uint(h[1]), 0x5410) ^ 0x88888888u;
   }
 }
 
@@ -251,6 +267,7 @@ struct ActProblem {
   int M, ldx, K, T, Lcount, step_host, layer;
   int gx;                     // token tiles
   int bpc;                    // rotation blocks per CTA
+  int a_rows;                 // rows of the permuted-x TMA box (tokens, <= 128)
 };
 struct ActBatch {
   int n;
@@ -464,7 +481,7 @@ __global__ void __launch_bounds__(kThreads)
         const float4 b = *reinterpret_cast<const float4*>(keep + t * kpitch + k + 4);
         const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         uint32_t w[1];
-        quant_pack<8>(f, s, rs, -8, 7, w);
+        quant_pack<8>(f, s, rs, w);
         *reinterpret_cast<uint32_t*>(dst + k / 2) = w[0];
       }
     }
@@ -616,10 +633,14 @@ __global__ void __launch_bounds__(kCThreads)
 // memory).  bf16 activations are exact in bf16; R_B is carried as three bf16
 // parts (hi + mid + lo, pack time), so the product has ~fp32 accuracy.
 // Per CTA: a tile of 128 tokens (the UMMA M dimension) and a run of blocks.
-//   warp 0      bulk-copies the R_B parts (pre-swizzled images) into a ring
+// With the permuted copy of x (the usual route):
+//   warp 0      loads the A tiles by TMA and bulk-copies the R_B parts
+//               (pre-swizzled images) into a ring
 //   warp 1      issues the MMAs (3 parts x b/16 K-steps per block)
-//   warps 2-5   gather x[m, perm[B*b + i]] into a 128B-swizzled A tile
-//   warps 6-9   read the accumulator (one token per thread) and quantise
+//   warps 2-9   read the accumulator and quantise: one token per thread,
+//               warps 2-5 the first half of the block's columns, 6-9 the rest
+// Without it, warps 2-5 gather x[m, perm[B*b + i]] into the A tile instead
+// and warps 6-9 take every column.
 // DYNAMIC mode runs the blocks twice: pass 0 takes each token's max |x'|
 // (reduced over the cluster that shares the row), pass 1 quantises.
 // ===========================================================================
@@ -634,16 +655,18 @@ template <int BS>
 struct TcCfg {
   static constexpr int kAStage = kTM * BS * 2;          // bf16 A tile
   static constexpr int kRStage = BS * BS * 2;           // one bf16 part of R_B^T
-  static constexpr int kAS = 2;
+  static constexpr int kAS = BS == 64 ? 3 : 2;          // A tiles in flight
   static constexpr int kRS = BS == 64 ? 6 : 4;
   static constexpr int kTmemCols = 2 * BS;              // double-buffered fp32 accumulator
   static constexpr int kSmem = kAS * kAStage + kRS * kRStage + 1024;
 };
 
 struct TcBars {
-  uint64_t full_a[2], empty_a[2], full_r[6], empty_r[6], acc_full[2], acc_empty[2];
+  uint64_t full_a[3], empty_a[3], full_r[6], empty_r[6], acc_full[2], acc_empty[2];
   uint32_t tmem;
 };
+static_assert(TcCfg<64>::kAS <= 3 && TcCfg<128>::kAS <= 3 && TcCfg<64>::kRS <= 6 &&
+                  TcCfg<128>::kRS <= 6, "ring barriers");
 
 QVLA_DEVICE void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -659,6 +682,11 @@ template <int BS, int MODE, bool kTmaA>
 __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
     rotq_tc_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
   using C = TcCfg<BS>;
+  // epilogue warps: 6-9, or 2-9 in two column halves when the A tiles come
+  // by TMA and the gather warps are free
+  constexpr int kEpiWarps = kTmaA ? 8 : 4;
+  constexpr int kFirstEpi = 10 - kEpiWarps;
+  constexpr int kHalves = kEpiWarps / 4;
   extern __shared__ uint8_t smem_raw[];
   __shared__ TcBars bars;
   __shared__ unsigned int amax_s[kTM];
@@ -687,11 +715,13 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
   uint8_t* const rstage = base + C::kAS * C::kAStage;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kAS; ++i) {
       mbar_init(&bars.full_a[i], kTmaA ? 1 : 128);
       mbar_init(&bars.empty_a[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.acc_full[i], 1);
-      mbar_init(&bars.acc_empty[i], 128);
+      mbar_init(&bars.acc_empty[i], 32 * kEpiWarps);
     }
     for (int i = 0; i < C::kRS; ++i) {
       mbar_init(&bars.full_r[i], 1);
@@ -699,6 +729,7 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
     }
     fence_mbar_init();
   }
+  if (tid < kTM) amax_s[tid] = 0u;
   if (warp == 1) {
     __syncwarp();                  // tcgen05 alloc/ld/dealloc are warp-wide
     tmem_alloc(&bars.tmem, C::kTmemCols);
@@ -708,13 +739,57 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
   cta_sync();
   tc_fence_after();
   const uint32_t tmem = bars.tmem;
-  const bool epi = warp >= 6;
+  const bool epi = warp >= kFirstEpi;
   // cluster barrier phase 1 ("row maxima published"): threads that are not in
   // the epilogue arrive once their pass-0 work is issued, so the epilogue's
   // wait never depends on work that waits for the epilogue
   bool arrived1 = false;
 
-  if (warp == 0) {
+  if (warp == 0 && kTmaA) {
+    // ------------------------------------- A tiles (permuted x) and R_B parts
+    if (lane == 0) {
+      auto issue_r = [&](int u) -> bool {
+        const int rr = u % C::kRS, B = B0 + (u / 3) % nbc;
+        if (!mbar_wait(&bars.empty_r[rr], ((u / C::kRS) & 1) ^ 1u, err)) return false;
+        mbar_arrive_expect_tx(&bars.full_r[rr], C::kRStage);
+        bulk_copy_g2s(rstage + rr * C::kRStage,
+                      P.rot_tc + (static_cast<size_t>(B) * 3 + u % 3) * BS * BS, C::kRStage,
+                      &bars.full_r[rr]);
+        return true;
+      };
+      const int U = 3 * W;
+      int ur = 0, issued = 0;
+      bool ok = true;
+      // the parts that fit the ring go out before the wait for the permuted copy
+      while (ok && ur < min(U, C::kRS)) ok = issue_r(ur++) ;
+      pdl_wait();
+      for (int w = 0; ok && w < W; ++w) {
+        const int B = B0 + w % nbc, as = w % C::kAS;
+        if (!mbar_wait(&bars.empty_a[as], ((w / C::kAS) & 1) ^ 1u, err)) break;
+        // a box of a_rows tokens (fewer than 128 for a short batch: the
+        // MMA's rows past them hold stale values, and so do only its result
+        // rows past them, which nothing reads)
+        mbar_arrive_expect_tx(&bars.full_a[as], (BS / 64) * 128 * P.a_rows);
+#pragma unroll
+        for (int kc = 0; kc < BS / 64; ++kc)
+          tma_load_2d(astage + as * C::kAStage + kc * (kTM * 128), &P.txp, &bars.full_a[as],
+                      B * BS + kc * 64, m0);
+        ++issued;
+        if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
+          cluster_arrive_relaxed();
+          arrived1 = true;
+        }
+        // the parts of the next block: they wait only for the MMAs of blocks
+        // whose A tiles are already out
+        while (ok && ur < min(U, 3 * (w + 2))) ok = issue_r(ur++);
+      }
+      // never leave with copies in flight
+      for (int u = max(0, ur - C::kRS); u < ur; ++u)
+        mbar_wait(&bars.full_r[u % C::kRS], (u / C::kRS) & 1, err);
+      for (int w = max(0, issued - C::kAS); w < issued; ++w)
+        mbar_wait(&bars.full_a[w % C::kAS], (w / C::kAS) & 1, err);
+    }
+  } else if (warp == 0) {
     // ---------------------------------------------------------- R_B parts
     if (lane == 0) {
       for (int w = 0; w < W; ++w) {
@@ -743,8 +818,8 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
       constexpr uint32_t idesc = idesc_bf16_f32(kTM, BS);
       const uint32_t a_base = smem_u32(astage), r_base = smem_u32(rstage);
       for (int w = 0; w < W; ++w) {
-        const int as = w & 1, ab = w & 1;
-        if (!mbar_wait(&bars.full_a[as], (w >> 1) & 1, err)) break;
+        const int as = w % C::kAS, ab = w & 1;
+        if (!mbar_wait(&bars.full_a[as], (w / C::kAS) & 1, err)) break;
         if (!mbar_wait(&bars.acc_empty[ab], ((w >> 1) & 1) ^ 1u, err)) break;
         tc_fence_after();
         for (int sp = 0; sp < 3; ++sp) {
@@ -768,36 +843,14 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
         }
       }
     }
-  } else if (!epi && kTmaA) {
-    // ------------------------------------------- A tiles by TMA (permuted x)
-    if (tid == 64) {
-      pdl_wait();
-      int issued = 0;
-      for (int w = 0; w < W; ++w) {
-        const int B = B0 + w % nbc, as = w & 1;
-        if (!mbar_wait(&bars.empty_a[as], ((w >> 1) & 1) ^ 1u, err)) break;
-        mbar_arrive_expect_tx(&bars.full_a[as], C::kAStage);
-#pragma unroll
-        for (int kc = 0; kc < BS / 64; ++kc)
-          tma_load_2d(astage + as * C::kAStage + kc * (kTM * 128), &P.txp, &bars.full_a[as],
-                      B * BS + kc * 64, m0);
-        ++issued;
-        if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
-          cluster_arrive_relaxed();
-          arrived1 = true;
-        }
-      }
-      for (int w = issued - 2 < 0 ? 0 : issued - 2; w < issued; ++w)
-        mbar_wait(&bars.full_a[w & 1], (w >> 1) & 1, err);
-    }
   } else if (!epi) {
-    // ------------------------------------------------------------- gather
+    // ----------------------------------------------- gather (no TMA route)
     const int t = tid - 64;                    // token row of the tile
     pdl_wait();
     const bool valid = t < ntok;
     const __nv_bfloat16* xrow = x + static_cast<size_t>(m0 + (valid ? t : 0)) * ldx;
     for (int w = 0; w < W; ++w) {
-      const int B = B0 + w % nbc, as = w & 1;
+      const int B = B0 + w % nbc, as = w % C::kAS;
       const int32_t* pB = P.perm + static_cast<size_t>(B) * BS;
       uint32_t v[BS / 2];
 #pragma unroll
@@ -810,7 +863,7 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
         }
         v[i / 2] = lo | (hi << 16);
       }
-      if (!mbar_wait(&bars.empty_a[as], ((w >> 1) & 1) ^ 1u, err)) break;
+      if (!mbar_wait(&bars.empty_a[as], ((w / C::kAS) & 1) ^ 1u, err)) break;
       uint8_t* at = astage + as * C::kAStage;
 #pragma unroll
       for (int c8 = 0; c8 < BS / 8; ++c8) {
@@ -829,6 +882,8 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
     // ----------------------------------------------------------- epilogue
     const int q4 = warp & 3;
     const int t = q4 * 32 + lane;              // token row = TMEM lane
+    constexpr int kCols = BS / kHalves;        // accumulator columns of this thread
+    const int cbeg = ((warp - kFirstEpi) >> 2) * kCols;
     const bool valid = t < ntok;
     pdl_wait();
     pdl_launch_dependents();
@@ -836,11 +891,16 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
     if (MODE == kTable) s = table_scale(P.table, P.T, P.Lcount, P.step_dev, P.step_host, P.layer, err);
     float amax = 0.f;
     bool reduced = false;
-    // row maximum over every CTA of the cluster that shares these tokens
-    // (once per thread, also when this CTA holds no block or gave up early)
+    // row maximum over both column halves and every CTA of the cluster that
+    // shares these tokens (once per thread, also when this CTA holds no block
+    // or gave up early); maxima of non-negative floats order as their bits
     auto reduce_rows = [&]() {
+      if (kHalves > 1 || cs > 1) atomicMax(&amax_s[t], __float_as_uint(amax));
+      if (kHalves > 1 && cs == 1) {
+        named_barrier(1, 32 * kEpiWarps);
+        amax = __uint_as_float(amax_s[t]);
+      }
       if (cs > 1) {
-        amax_s[t] = __float_as_uint(amax);
         asm volatile("barrier.cluster.arrive.release;" ::: "memory");
         asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
         unsigned int mx = 0u;
@@ -866,7 +926,7 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
       tc_fence_after();
       const float rs = quant_recip(s);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BS; c0 += 32) {
+      for (int c0 = cbeg; c0 < cbeg + kCols; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * BS + c0, r);
         tmem_ld_wait();
@@ -882,11 +942,18 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(__uint_as_float(r[c])));
         } else {
-          float f[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(r[c]);
+          // two halves of 16 codes: half the registers of one pass
           uint32_t wv[4];
-          quant_pack<32>(f, s, rs, -8, 7, wv);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float f[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) f[c] = __uint_as_float(r[16 * hh + c]);
+            uint32_t w2[2];
+            quant_pack<16>(f, s, rs, w2);
+            wv[2 * hh] = w2[0];
+            wv[2 * hh + 1] = w2[1];
+          }
           if (valid) {
             *reinterpret_cast<uint4*>(P.xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS + c0) / 2) =
                 make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -907,7 +974,7 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
       if (MODE == kDynamic && w == nbc - 1) reduce_rows();
     }
     if (MODE == kDynamic && !reduced) reduce_rows();
-    if (MODE != kRotateOnly && group == 0 && valid) P.s_x[m0 + t] = s;
+    if (MODE != kRotateOnly && group == 0 && valid && cbeg == 0) P.s_x[m0 + t] = s;
   }
 
   if (MODE == kDynamic && cs > 1) {
@@ -927,80 +994,105 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
 }
 
 // Permuted copy of bf16 rows: out[m][j] = x[m][perm[j]].  One CTA per run of
-// `rpc` rows of one problem: the rows are staged in shared memory with 16-byte
-// loads (all of them in flight at once), then every thread takes 8 output
-// positions, loads their 8 permutation entries once, and writes those
-// positions of every staged row with 16-byte stores (coalesced both ways).
+// `rpc` consecutive rows of one problem, as a pipeline over a ring of row
+// buffers in shared memory:
+//   warp 8      bulk-copies whole rows (16-byte aligned, K * 2 bytes) into
+//               the ring, one mbarrier per slot
+//   warps 0-7   per row, every thread takes its runs of 8 output positions,
+//               gathers them from the staged row and writes them with one
+//               16-byte store (coalesced); the permutation entries of its
+//               runs stay in registers for all rows
+// so the loads of later rows are in flight while earlier rows are scattered.
 struct PermJob {
   const __nv_bfloat16* x;
   const int32_t* perm;
   __nv_bfloat16* out;
   int ldx, M, K;
 };
+constexpr int kPermMaxStages = 8;
+constexpr int kPermWorkers = 256;
 struct PermBatch {
   int n;
   int rpc;                          // rows per CTA
+  int stages;                       // row buffers in the ring
+  int row_bytes;                    // bytes of one ring slot (largest K of the batch, x 2)
   int cta_start[kMaxBatch + 1];
   PermJob j[kMaxBatch];
 };
 
-__global__ void __launch_bounds__(256) permute_rows_kernel(const __grid_constant__ PermBatch batch) {
-  extern __shared__ __align__(16) uint8_t smem[];
+// kPC: runs of 8 positions per worker thread (K <= 2048 * kPC)
+template <int kPC>
+__global__ void __launch_bounds__(kPermWorkers + 32)
+    permute_rows_kernel(const __grid_constant__ PermBatch batch, unsigned int* err) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t full[kPermMaxStages], empty[kPermMaxStages];
   int ji = 0;
   while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[ji + 1]) ++ji;
   const PermJob& J = batch.j[ji];
   const int r0 = (static_cast<int>(blockIdx.x) - batch.cta_start[ji]) * batch.rpc;
   const int nr = min(batch.rpc, J.M - r0);
-  const int K = J.K, kc = K / 8;                  // 16-byte chunks per row
-  unsigned short* s = reinterpret_cast<unsigned short*>(smem);
-  // the permutation does not depend on the previous kernel: its first slice
-  // is read before waiting for it, in flight together with the rows
-  const int i0 = threadIdx.x;
-  int4 pa = make_int4(0, 0, 0, 0), pb = make_int4(0, 0, 0, 0);
-  if (i0 < kc) {
-    pa = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i0);
-    pb = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i0 + 1);
+  const int K = J.K, kc = K / 8, S = batch.stages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the permutation does not depend on the previous kernel: read before
+  // waiting for it
+  int p[kPC][8];
+#pragma unroll
+  for (int c = 0; c < kPC; ++c) {
+    const int i = tid + kPermWorkers * c;
+    int4 a = make_int4(0, 0, 0, 0), b = make_int4(0, 0, 0, 0);
+    if (tid < kPermWorkers && i < kc) {
+      a = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
+      b = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
+    }
+    const int q[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) p[c][u] = static_cast<unsigned>(q[u]) < static_cast<unsigned>(K) ? q[u] : 0;
   }
-  pdl_wait();
-  pdl_launch_dependents();
-  // rows into shared memory: each round puts up to 8 loads per thread in
-  // flight before storing any of them
-  for (int e0 = 0; e0 < nr * kc; e0 += 8 * 256) {
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = e0 + u * 256 + threadIdx.x;
-      if (e < nr * kc) {
-        const int r = e / kc, c = e - r * kc;
-        v[u] = __ldg(reinterpret_cast<const uint4*>(J.x + static_cast<size_t>(r0 + r) * J.ldx) + c);
-      }
+  if (tid == 0) {
+    for (int st = 0; st < S; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kPermWorkers);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = e0 + u * 256 + threadIdx.x;
-      if (e < nr * kc) {
-        const int r = e / kc, c = e - r * kc;
-        reinterpret_cast<uint4*>(s + static_cast<size_t>(r) * K)[c] = v[u];
-      }
-    }
+    fence_mbar_init();
   }
   cta_sync();
-  for (int i = threadIdx.x; i < kc; i += 256) {
-    if (i != i0) {
-      pa = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
-      pb = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i + 1);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (warp == kPermWorkers / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int r = 0; r < nr; ++r) {
+        const int st = r % S;
+        if (!mbar_wait(&empty[st], ((r / S) & 1) ^ 1u, err)) break;
+        mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(K) * 2u);
+        bulk_copy_g2s(smem + static_cast<size_t>(st) * batch.row_bytes,
+                      J.x + static_cast<size_t>(r0 + r) * J.ldx, static_cast<uint32_t>(K) * 2u, &full[st]);
+        ++issued;
+      }
+      // never leave with copies in flight
+      for (int r = max(0, issued - S); r < issued; ++r) mbar_wait(&full[r % S], (r / S) & 1, err);
     }
-    int p[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-#pragma unroll
-    for (int q = 0; q < 8; ++q) p[q] = static_cast<unsigned>(p[q]) < static_cast<unsigned>(K) ? p[q] : 0;
+  } else {
+    // ------------------------------------------------------------- workers
     for (int r = 0; r < nr; ++r) {
-      const unsigned short* sr = s + static_cast<size_t>(r) * K;
-      uint32_t w[4];
+      const int st = r % S;
+      if (!mbar_wait(&full[st], (r / S) & 1, err)) break;
+      const unsigned short* sr =
+          reinterpret_cast<const unsigned short*>(smem + static_cast<size_t>(st) * batch.row_bytes);
+      uint4* orow = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(r0 + r) * K);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        w[q] = static_cast<uint32_t>(sr[p[2 * q]]) | (static_cast<uint32_t>(sr[p[2 * q + 1]]) << 16);
-      reinterpret_cast<uint4*>(J.out + static_cast<size_t>(r0 + r) * K)[i] =
-          make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c = 0; c < kPC; ++c) {
+        const int i = tid + kPermWorkers * c;
+        if (i < kc) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            w[q] = static_cast<uint32_t>(sr[p[c][2 * q]]) | (static_cast<uint32_t>(sr[p[c][2 * q + 1]]) << 16);
+          orow[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      mbar_arrive(&empty[st]);
     }
   }
 }
@@ -1269,16 +1361,17 @@ bool rsvd_path_forced() {
   return p && std::strcmp(p, "fma") == 0;
 }
 
-// Composite-path launches: every (token tile, block) pair of the batch gets a
+// Composite-path launches: every (token tile, block) pair of a launch gets a
 // CTA while they fit eight per SM; beyond that each CTA walks several blocks.
 template <typename Tin, int MODE>
 cudaError_t launch_comp(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
-  long long pairs = 0;
-  for (const ActArgs* a : v) pairs += static_cast<long long>((a->M + kCTT - 1) / kCTT) * (a->K / kCBS);
   const long long slots = 8LL * 148;
-  const int bpc = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
   for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
     const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+    long long pairs = 0;
+    for (int i = 0; i < n; ++i)
+      pairs += static_cast<long long>((v[i0 + i]->M + kCTT - 1) / kCTT) * (v[i0 + i]->K / kCBS);
+    const int bpc = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
     ActBatch batch;
     std::memset(&batch, 0, sizeof(batch));
     batch.n = n;
@@ -1373,8 +1466,10 @@ int tc_cluster(int M, int K) {
   return cs;
 }
 
-// One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
-// mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
+// Rows of the permuted-x box: the batch's token count rounded up to 16, at
+// most one 128-token tile.
+int xperm_box_rows(int M) { return std::min(kTM, (M + 15) / 16 * 16); }
+
 bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
   static const EncodeTiledFnR enc = []() -> EncodeTiledFnR {
     void* p = nullptr;
@@ -1387,7 +1482,7 @@ bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
   if (!enc) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTM)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(xperm_box_rows(M))};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1395,7 +1490,30 @@ bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
 }
 
 // Permuted copies x_perm = x[:, perm] of the problems that have scratch.
-constexpr int kPermSmemCap = 96 * 1024;
+// The ring holds about 48 KB of rows (2 to 8 of them); the rows of a launch
+// are spread over about three CTAs per SM.
+constexpr int kPermRingBytes = 48 * 1024;
+template <int kPC>
+cudaError_t launch_permute_kernel(const PermBatch& b, int ctas, cudaStream_t stream) {
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, []() {
+    return cudaFuncSetAttribute(permute_rows_kernel<kPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                2 * QVLA_MAX_K * 2);
+  });
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.blockDim = dim3(kPermWorkers + 32, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(b.stages) * b.row_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, permute_rows_kernel<kPC>, b, device_error_word());
+}
+
 cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
     const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
@@ -1408,11 +1526,9 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
       rows += v[i0 + i]->M;
       kmax = std::max(kmax, v[i0 + i]->K);
     }
-    // about two CTAs per SM, as many rows per CTA as that takes (each CTA
-    // reuses its permutation slice for all of them), within the staging cap
-    int rpc = static_cast<int>(std::min<long long>(16, (rows + 295) / 296));
-    rpc = std::max(1, std::min(rpc, kPermSmemCap / (2 * kmax)));
-    b.rpc = rpc;
+    b.row_bytes = kmax * 2;
+    b.stages = std::max(2, std::min(kPermMaxStages, kPermRingBytes / b.row_bytes));
+    b.rpc = static_cast<int>(std::max<long long>(1, (rows + 3 * 148 - 1) / (3 * 148)));
     int ctas = 0;
     for (int i = 0; i < n; ++i) {
       const ActArgs& a = *v[i0 + i];
@@ -1423,34 +1539,20 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
       b.j[i].M = a.M;
       b.j[i].K = a.K;
       b.cta_start[i] = ctas;
-      ctas += (a.M + rpc - 1) / rpc;
+      ctas += (a.M + b.rpc - 1) / b.rpc;
     }
     b.cta_start[n] = ctas;
-    static std::atomic<unsigned long long> attr_done{0};
-    {
-      cudaError_t e = once_per_device(attr_done, []() {
-        return cudaFuncSetAttribute(permute_rows_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    std::max(kPermSmemCap, QVLA_MAX_K * 2));
-      });
-      if (e != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ctas, 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(rpc) * kmax * 2;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, permute_rows_kernel, b);
+    const int runs = (kmax / 8 + kPermWorkers - 1) / kPermWorkers;   // runs of 8 per thread
+    cudaError_t e = runs <= 1   ? launch_permute_kernel<1>(b, ctas, stream)
+                    : runs <= 4 ? launch_permute_kernel<4>(b, ctas, stream)
+                                : launch_permute_kernel<16>(b, ctas, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
 
+// One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
+// mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
 template <int BS, int MODE, bool kTmaA>
 cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cudaStream_t stream) {
   using C = TcCfg<BS>;
@@ -1481,6 +1583,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     P.layer = a.layer;
     const int nb = a.K / BS;
     P.gx = (a.M + kTM - 1) / kTM;
+    P.a_rows = xperm_box_rows(a.M);
     batch.cta_start[i] = ctas;
     if (MODE == kDynamic) {
       P.bpc = (nb + cs - 1) / cs;
@@ -1549,13 +1652,14 @@ cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t st
     }
     return cudaSuccess;
   }
-  // blocks per CTA: spread the batch's (token tile, block) pairs over one wave
-  long long pairs = 0;
-  for (const ActArgs* a : v) pairs += static_cast<long long>((a->M + kTM - 1) / kTM) * (a->K / BS);
+  // blocks per CTA: spread each launch's (token tile, block) pairs over one wave
   const long long slots = 148LL * tc_ctas_per_sm<BS>();
-  const int G = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
   for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
     const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+    long long pairs = 0;
+    for (int i = 0; i < n; ++i)
+      pairs += static_cast<long long>((v[i0 + i]->M + kTM - 1) / kTM) * (v[i0 + i]->K / BS);
+    const int G = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
     cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, G, 1, stream);
     if (e != cudaSuccess) return e;
   }
