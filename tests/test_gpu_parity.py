@@ -274,6 +274,9 @@ GEMM_CASES = [
     (64, 384, 1024, 4), (64, 200, 512, 2), (100, 256, 2048, 8), (128, 512, 768, 1),
     (200, 384, 1024, 1), (256, 256, 512, 0), (300, 1000, 1056, 1), (520, 256, 2048, 0),
     (33, 640, 4096, 16), (120, 512, 1024, 2), (260, 384, 1024, 4),
+    # small token tiles with long K: the tiles are split over K between the
+    # two CTAs of a cluster (odd stage counts, a ragged last stage)
+    (16, 256, 2048, 0), (30, 384, 1056, 0), (40, 512, 1056, 0), (64, 128, 8192, 0),
 ]
 
 

@@ -87,18 +87,25 @@ struct Cfg {
   static constexpr int kStage = kABytes + kBBytes + kUBytes;
   static constexpr int kCh = NT < 32 ? NT : 32;                  // tokens per output chunk
   static constexpr int kOutBytes = kOutSlots * kCh * kBM * 2;
-  static constexpr int kRing = (208 * 1024 - kOutBytes) / kStage;
+  // small token tiles may split the K of a long tile over the two CTAs of a
+  // cluster: the second CTA's int32 partial lands in the first one's
+  // receive buffer, [token / 4][weight row][4 tokens]
+  static constexpr bool kSplit = NT <= 64;
+  static constexpr int kRecvBytes = kSplit ? kBM * NT * 4 : 0;
+  static constexpr int kBudget = 226 * 1024;                     // dynamic shared memory
+  static constexpr int kRing = (kBudget - 1024 - kOutBytes - kRecvBytes) / kStage;
   static constexpr int kTmemStages = (kTmemCols - kACol0) / kACols;
   static constexpr int kS0 = kRing < kTmemStages ? kRing : kTmemStages;
   // one ring: smem stage s and tensor-memory A stage s go together
   static constexpr int kS = kS0 > 8 ? 8 : kS0;
   // at least 116 KB, so that two CTAs never share an SM (each takes all of
   // tensor memory)
-  static constexpr int kNeed = kS * kStage + kOutBytes + 1024;
+  static constexpr int kNeed = kS * kStage + kOutBytes + kRecvBytes + 1024;
   static constexpr int kSmem = kNeed < 116 * 1024 ? 116 * 1024 : kNeed;
   static_assert(kACol0 + kS * kACols <= kTmemCols, "tensor memory");
   static_assert(kStage % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "alignment");
   static_assert(kS >= 2, "pipeline depth");
+  static_assert(kNeed <= kBudget, "shared memory");
 };
 
 struct Barriers {
@@ -107,6 +114,7 @@ struct Barriers {
   uint64_t mma_done[8];                    // the MMAs reading the stage have completed
   uint64_t acc_full[2], acc_empty[2];      // accumulators
   uint64_t drain;
+  uint64_t recv_full;                      // the cluster partner's partial has landed
   uint32_t tmem;
 };
 
@@ -129,9 +137,14 @@ struct Problem {
 };
 struct Batch {
   int n;
+  int split;                      // launched in clusters of two CTAs
   int tile_start[kMaxBatch + 1];  // launch tile ids of each problem
   uint16_t cta_begin[kMaxCtas + 1];
-  uint16_t order[kMaxTiles];      // launch tile ids, CTA by CTA
+  uint16_t order[kMaxTiles + kMaxCtas];   // launch tile ids, CTA by CTA (a split tile twice)
+  // with `split`, the role of each CTA's first tile: 0 the whole tile, 1 its
+  // first K half and the epilogue (cluster rank 0), 2 its second K half,
+  // sent to rank 0 (cluster rank 1)
+  int8_t role[kMaxCtas];
   Problem p[kMaxBatch];
 };
 
@@ -182,17 +195,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<NT, kImage>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
-  __shared__ float sx_s[NT];                     // s_x of the epilogue's current tile
+  __shared__ __align__(16) float sx_s[NT];       // s_x of the epilogue's current tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t_begin = batch.cta_begin[blockIdx.x];
   const int t_end = batch.cta_begin[blockIdx.x + 1];
+  // K stages [k0, k1) of the CTA's i-th tile: all of them, or one half when
+  // the tile is split over the cluster pair
+  const int role = (C::kSplit && batch.split) ? batch.role[blockIdx.x] : 0;
+  auto krange = [&](int i, int nks, int& k0, int& k1) {
+    k0 = 0;
+    k1 = nks;
+    if (role != 0 && i == t_begin) {
+      if (role == 1) k1 = nks / 2;
+      else k0 = nks / 2;
+    }
+  };
 
   // 1024-byte aligned stage memory (128B-swizzled TMA destinations)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* const base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint8_t* const stages = base;
   __nv_bfloat16* const outs = reinterpret_cast<__nv_bfloat16*>(base + C::kS * C::kStage);
+  uint8_t* const recv = base + C::kS * C::kStage + C::kOutBytes;
 
   if (tid == 0) {
     for (int s = 0; s < C::kS; ++s) {
@@ -205,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.acc_empty[b], 4);
     }
     mbar_init(&bars.drain, 1);
+    mbar_init(&bars.recv_full, 1);
     fence_mbar_init();
     for (int p = 0; p < batch.n; ++p) {
       tma_prefetch_desc(&batch.p[p].tw);
@@ -218,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   cta_sync();
+  // the partner's barriers are initialised before anything reaches them
+  if (batch.split) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bars.tmem;
 
@@ -230,15 +258,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (programmatic dependent launch), the activation boxes after.
       int pre = 0;
       {
-        int i = t_begin, ks = 0;
+        int i = t_begin, ks = -1;
         while (pre < C::kS && i < t_end) {
           const Tile tr = decode<NT>(batch, batch.order[i]);
           const Problem& P = batch.p[tr.p];
+          int k0, k1;
+          krange(i, P.nks, k0, k1);
+          if (ks < 0) ks = k0;
           mbar_arrive_expect_tx(&bars.full[pre], kTx);
           tma_load_2d(stages + pre * C::kStage, &P.tw, &bars.full[pre], ks * kAPack, tr.n0);
           ++pre;
-          if (++ks == P.nks) {
-            ks = 0;
+          if (++ks == k1) {
+            ks = -1;
             ++i;
           }
         }
@@ -249,10 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = t_begin; i < t_end && ok; ++i) {
         const Tile tr = decode<NT>(batch, batch.order[i]);
         const Problem& P = batch.p[tr.p];
+        int k0, k1;
+        krange(i, P.nks, k0, k1);
         // the tile's weight boxes past the ring depth go to L2 now, so HBM
         // streaming is not limited by the ring
-        for (int ks = C::kS; ks < P.nks; ++ks) tma_prefetch_l2_2d(&P.tw, ks * kAPack, tr.n0);
-        for (int ks = 0; ks < P.nks; ++ks, ++g) {
+        for (int ks = k0 + C::kS; ks < k1; ++ks) tma_prefetch_l2_2d(&P.tw, ks * kAPack, tr.n0);
+        for (int ks = k0; ks < k1; ++ks, ++g) {
           const int s = g % C::kS;
           uint8_t* st = stages + s * C::kStage;
           if (g >= pre) {
@@ -285,14 +318,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0, tc = 0;
       for (int i = t_begin; i < t_end && ok; ++i, ++tc) {
         const Tile tr = decode<NT>(batch, batch.order[i]);
-        const int nks = batch.p[tr.p].nks;
+        int k0, k1;
+        krange(i, batch.p[tr.p].nks, k0, k1);
         const int b = tc % C::kAcc, use = tc / C::kAcc;
         if (use >= 1) {
           ok = mbar_wait(&bars.acc_empty[b], (use - 1) & 1, err);
           if (!ok) break;
         }
         const uint32_t d = tmem + static_cast<uint32_t>(b * C::kAccCols);
-        for (int ks = 0; ks < nks; ++ks, ++g) {
+        for (int ks = k0; ks < k1; ++ks, ++g) {
           const int s = g % C::kS;
           // the stage's A is in tensor memory (and, when the unpack warps got
           // the stage, its TMA bytes, activations included, had landed)
@@ -307,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 32 codes of K: A columns [8kk, 8kk+8) of the stage; B half kk/4,
             // bytes [32(kk%4), +32) of each 128-byte row
             const uint64_t bd = smem_desc_kmajor_sw128(bs + (kk >> 2) * (NT * 128) + 32 * (kk & 3));
-            umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks > k0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars.mma_done[s]);
         }
@@ -327,8 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int g = 0;
     for (int i = t_begin; i < t_end && ok; ++i) {
-      const int nks = batch.p[decode<NT>(batch, batch.order[i]).p].nks;
-      for (int ks = 0; ks < nks; ++ks, ++g) {
+      int k0, k1;
+      krange(i, batch.p[decode<NT>(batch, batch.order[i]).p].nks, k0, k1);
+      for (int ks = k0; ks < k1; ++ks, ++g) {
         const int s = g % C::kS;
         // warp-uniform outcome: the tensor-memory stores below are warp-wide
         ok = __all_sync(kFull, mbar_wait(&bars.full[s], (g / C::kS) & 1, err));
@@ -412,11 +447,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool tma = tr.n0 + kBM <= P.N || (P.N & 7) == 0;
       const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(b * C::kAccCols);
+      const bool first = i == t_begin;
+      if (role == 2 && first) {
+        // second K half of a split tile: the int32 partial goes to the
+        // receive buffer of cluster rank 0; once all four warps have stored
+        // theirs (the barrier orders them before the release), one thread
+        // arrives on rank 0's barrier, releasing at cluster scope
+        const uint32_t rv = map_shared_rank(smem_u32(recv), 0u);
+#pragma unroll 1
+        for (int c0 = 0; c0 < NT; c0 += C::kCh) {
+          uint32_t r[C::kCh];
+          tmem_ld_chunk<NT>(tacc + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < C::kCh; j += 4)
+            st_shared_cluster_v4(rv + static_cast<uint32_t>((((c0 + j) >> 2) * kBM + row) * 16),
+                                 make_int4(static_cast<int>(r[j]), static_cast<int>(r[j + 1]),
+                                           static_cast<int>(r[j + 2]), static_cast<int>(r[j + 3])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.acc_empty[b]);
+        named_barrier(1, 128);
+        if (et == 0) mbar_arrive_remote_release(map_shared_rank(smem_u32(&bars.recv_full), 0u));
+        continue;
+      }
+      if (role == 1 && first) {
+        // first K half: the partner's partial must have landed
+        ok = named_barrier_all(2, 128, mbar_wait_cluster(&bars.recv_full, 0, err));
+        if (!ok) break;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < NT; c0 += C::kCh) {
         uint32_t r[C::kCh];
         tmem_ld_chunk<NT>(tacc + c0, r);
         tmem_ld_wait();
+        if (role == 1 && first) {
+          // plus the partner's partial (the other K half; 256 * acc stays
+          // within int32 for K <= QVLA_MAX_K)
+#pragma unroll
+          for (int j = 0; j < C::kCh; j += 4) {
+            const uint4 v = lds128(smem_u32(recv) + static_cast<uint32_t>((((c0 + j) >> 2) * kBM + row) * 16));
+            r[j] += v.x;
+            r[j + 1] += v.y;
+            r[j + 2] += v.z;
+            r[j + 3] += v.w;
+          }
+        }
         if (c0 + C::kCh >= NT) {
           // the accumulator may be reused once every warp has read it
           tc_fence_before();
@@ -437,10 +514,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the store that last read this slot has finished reading it
         if (et == 0) bulk_wait_read<kOutSlots - 1>();
         named_barrier(1, 128);
+        // the chunk's token scales as 16-byte shared loads (one per four
+        // tokens, broadcast to the warp)
+        float sxc[C::kCh];
+#pragma unroll
+        for (int j = 0; j < C::kCh; j += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(sx_s + c0 + j);
+          sxc[j] = v4.x;
+          sxc[j + 1] = v4.y;
+          sxc[j + 2] = v4.z;
+          sxc[j + 3] = v4.w;
+        }
 #pragma unroll
         for (int j = 0; j < C::kCh; ++j) {
           const int32_t a = static_cast<int32_t>(r[j]) >> 8;
-          ot[j * kBM + row] = __float2bfloat16_rn(fmaf(sx_s[c0 + j] * sw, static_cast<float>(a), bn));
+          ot[j * kBM + row] = __float2bfloat16_rn(fmaf(sxc[j] * sw, static_cast<float>(a), bn));
         }
         fence_proxy_async_smem();
         named_barrier(1, 128);
@@ -466,6 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   cta_sync();
+  // neither CTA of a pair leaves while the other may still reach its
+  // shared memory
+  if (batch.split) cluster_sync();
   if (warp == 1) {
     __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
@@ -525,59 +616,158 @@ int sm_count() {
 // A tile's cost in 128-wide K steps, plus a fixed share for its epilogue.
 constexpr int kTileOverhead = 2;
 
-// Deals the launch's tiles to at most sm_count() CTAs, longest first, each to
-// the CTA with the least work so far (ties: the lowest index), and writes the
-// per-CTA lists.  Returns the number of CTAs.
-int schedule(Batch& b) {
-  const int T = b.tile_start[b.n];
-  const int G = std::min(sm_count(), T);
-  std::vector<int> ids(T), cost(T);
-  for (int p = 0; p < b.n; ++p)
-    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t)
-      cost[t] = (b.p[p].K + 127) / 128 + kTileOverhead;
-  for (int t = 0; t < T; ++t) ids[t] = t;
-  std::stable_sort(ids.begin(), ids.end(), [&](int x, int y) { return cost[x] > cost[y]; });
+// Longest-first list scheduling: each tile of `ids` (sorted by decreasing
+// cost) to the CTA with the least work so far (ties: the lowest index),
+// appended to that CTA's list.  Returns the largest load.
+long long lpt(const std::vector<int>& ids, const std::vector<int>& cost,
+              std::vector<long long>& load, std::vector<std::vector<int>>& lists) {
   using Load = std::pair<long long, int>;
   std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-  for (int c = 0; c < G; ++c) heap.push({0, c});
-  std::vector<std::vector<int>> lists(G);
+  for (int c = 0; c < static_cast<int>(load.size()); ++c) heap.push({load[c], c});
   for (int t : ids) {
     Load l = heap.top();
     heap.pop();
     lists[l.second].push_back(t);
     l.first += cost[t];
+    load[l.second] = l.first;
     heap.push(l);
   }
+  long long mx = 0;
+  for (long long v : load) mx = std::max(mx, v);
+  return mx;
+}
+
+// Deals the launch's tiles to the CTAs and writes the per-CTA lists; returns
+// the number of CTAs.  With `pairs` > 0 (small token tiles, clusters of two
+// available) the tiles much longer than the average load may be split over
+// K between the two CTAs of a cluster: each half is the first tile of its
+// CTA, rank 0 takes the first K half and the epilogue.  The split schedule is
+// used when it shortens the longest list by more than a twentieth.
+int schedule(Batch& b, int pairs) {
+  const int T = b.tile_start[b.n];
+  std::vector<int> ids(T), cost(T), units(T), nks(T);
+  for (int p = 0; p < b.n; ++p)
+    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t) {
+      units[t] = (b.p[p].K + 127) / 128;
+      nks[t] = b.p[p].nks;
+      cost[t] = units[t] + kTileOverhead;
+    }
+  for (int t = 0; t < T; ++t) ids[t] = t;
+  std::stable_sort(ids.begin(), ids.end(), [&](int x, int y) { return cost[x] > cost[y]; });
+
+  const int G1 = std::min(sm_count(), T);
+  std::vector<long long> load1(G1, 0);
+  std::vector<std::vector<int>> lists1(G1);
+  const long long span1 = G1 > 0 ? lpt(ids, cost, load1, lists1) : 0;
+
+  b.split = 0;
+  std::vector<std::vector<int>> lists = lists1;
+  std::vector<int8_t> role;
+  if (pairs > 0 && T > 0) {
+    const int G2 = 2 * pairs;
+    long long total = 0;
+    for (int t = 0; t < T; ++t) total += cost[t];
+    std::vector<int> split, rest;
+    for (int t : ids) {
+      const bool long_tile = nks[t] >= 2 && 5 * cost[t] > 6 * (total / G2) &&
+                             static_cast<int>(split.size()) < pairs;
+      (long_tile ? split : rest).push_back(t);
+    }
+    if (!split.empty()) {
+      std::vector<long long> load2(G2, 0);
+      std::vector<std::vector<int>> lists2(G2);
+      std::vector<int8_t> role2(G2, 0);
+      for (size_t k = 0; k < split.size(); ++k) {
+        const int t = split[k], h = 2 * (nks[t] / 2);       // 128-wide units of the first half
+        lists2[2 * k].push_back(t);
+        lists2[2 * k + 1].push_back(t);
+        role2[2 * k] = 1;
+        role2[2 * k + 1] = 2;
+        load2[2 * k] = h + kTileOverhead + 1;
+        load2[2 * k + 1] = (units[t] - h) + 1;
+      }
+      const long long span2 = lpt(rest, cost, load2, lists2);
+      if (20 * span2 < 19 * span1) {
+        b.split = 1;
+        lists.swap(lists2);
+        role.swap(role2);
+      }
+    }
+  }
+  const int G = static_cast<int>(lists.size());
   int k = 0;
   for (int c = 0; c < G; ++c) {
     b.cta_begin[c] = static_cast<uint16_t>(k);
+    b.role[c] = b.split ? role[c] : 0;
     for (int t : lists[c]) b.order[k++] = static_cast<uint16_t>(t);
   }
   b.cta_begin[G] = static_cast<uint16_t>(k);
   return G;
 }
 
+// Clusters of two CTAs of this kernel the device holds at once (one CTA per
+// SM), cached per device; 0 when that cannot be had.
+template <int NT, bool kImage>
+int cluster_pairs() {
+  using C = Cfg<NT, kImage>;
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int c = cache[dev].load(std::memory_order_relaxed);
+  if (c != 0) return c > 0 ? c : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * kMaxCtas, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel<NT, kImage>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  n = std::min(n, kMaxCtas / 2);
+  cache[dev].store(n > 0 ? n : -1, std::memory_order_relaxed);
+  return n;
+}
+
 template <int NT, bool kImage>
 cudaError_t launch_batch(Batch& batch, cudaStream_t stream) {
   using C = Cfg<NT, kImage>;
-  const int G = schedule(batch);
-  if (G == 0) return cudaSuccess;
   auto kern = w4a4_gemm_kernel<NT, kImage>;
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = once_per_device(attr_done, [&]() {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
   if (e != cudaSuccess) return e;
+  const int G = schedule(batch, C::kSplit ? cluster_pairs<NT, kImage>() : 0);
+  if (G == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (batch.split) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, batch, device_error_word());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -413,6 +413,33 @@ QVLA_DEVICE void st_shared_cluster_v4(uint32_t addr, int4 v) {
                : "memory");
 }
 
+// Arrival on an mbarrier of another CTA of the cluster (`addr` from mapa),
+// releasing this thread's earlier writes at cluster scope.
+QVLA_DEVICE void mbar_arrive_remote_release(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+// As mbar_wait, acquiring at cluster scope: after it returns, the writes that
+// other CTAs of the cluster released into the phase are visible.
+QVLA_DEVICE bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                   uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      report(err, QVLA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 QVLA_DEVICE void st_shared_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }

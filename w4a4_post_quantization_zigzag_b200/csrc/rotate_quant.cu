@@ -1008,12 +1008,12 @@ struct PermJob {
   const int32_t* perm;
   __nv_bfloat16* out;
   int ldx, M, K;
+  int rpc;                          // rows per CTA
 };
 constexpr int kPermMaxStages = 8;
 constexpr int kPermWorkers = 256;
 struct PermBatch {
   int n;
-  int rpc;                          // rows per CTA
   int stages;                       // row buffers in the ring
   int row_bytes;                    // bytes of one ring slot (largest K of the batch, x 2)
   int cta_start[kMaxBatch + 1];
@@ -1029,8 +1029,8 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
   int ji = 0;
   while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.cta_start[ji + 1]) ++ji;
   const PermJob& J = batch.j[ji];
-  const int r0 = (static_cast<int>(blockIdx.x) - batch.cta_start[ji]) * batch.rpc;
-  const int nr = min(batch.rpc, J.M - r0);
+  const int r0 = (static_cast<int>(blockIdx.x) - batch.cta_start[ji]) * J.rpc;
+  const int nr = min(J.rpc, J.M - r0);
   const int K = J.K, kc = K / 8, S = batch.stages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the permutation does not depend on the previous kernel: read before
@@ -1490,8 +1490,9 @@ bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
 }
 
 // Permuted copies x_perm = x[:, perm] of the problems that have scratch.
-// The ring holds about 48 KB of rows (2 to 8 of them); the rows of a launch
-// are spread over about three CTAs per SM.
+// The ring holds about 48 KB of rows (2 to 8 of them); the elements of a
+// launch are spread evenly over about three CTAs per SM (fewer rows per CTA
+// where the rows are longer).
 constexpr int kPermRingBytes = 48 * 1024;
 template <int kPC>
 cudaError_t launch_permute_kernel(const PermBatch& b, int ctas, cudaStream_t stream) {
@@ -1520,15 +1521,15 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
     PermBatch b;
     std::memset(&b, 0, sizeof(b));
     b.n = n;
-    long long rows = 0;
+    long long elems = 0;
     int kmax = 0;
     for (int i = 0; i < n; ++i) {
-      rows += v[i0 + i]->M;
+      elems += static_cast<long long>(v[i0 + i]->M) * v[i0 + i]->K;
       kmax = std::max(kmax, v[i0 + i]->K);
     }
     b.row_bytes = kmax * 2;
     b.stages = std::max(2, std::min(kPermMaxStages, kPermRingBytes / b.row_bytes));
-    b.rpc = static_cast<int>(std::max<long long>(1, (rows + 3 * 148 - 1) / (3 * 148)));
+    const long long per_cta = (elems + 3 * 148 - 1) / (3 * 148);
     int ctas = 0;
     for (int i = 0; i < n; ++i) {
       const ActArgs& a = *v[i0 + i];
@@ -1538,8 +1539,9 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
       b.j[i].ldx = a.ldx;
       b.j[i].M = a.M;
       b.j[i].K = a.K;
+      b.j[i].rpc = static_cast<int>(std::max<long long>(1, (per_cta + a.K - 1) / a.K));
       b.cta_start[i] = ctas;
-      ctas += (a.M + b.rpc - 1) / b.rpc;
+      ctas += (a.M + b.j[i].rpc - 1) / b.j[i].rpc;
     }
     b.cta_start[n] = ctas;
     const int runs = (kmax / 8 + kPermWorkers - 1) / kPermWorkers;   // runs of 8 per thread
