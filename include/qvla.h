@@ -388,12 +388,16 @@ qvla_status qvla_quant_act_f32(const float* xr, int M, int K, qvla_scale_mode mo
  * accumulate 256*acc exactly (|256*acc| <= 256*64*K < 2^31 for
  * K <= QVLA_MAX_K) and the epilogue shifts it back.
  * One persistent CTA per SM walks a list of 128-channel x (16..128)-token
- * tiles that the host deals out longest first; no workspace.
+ * tiles that the host deals out longest first; no workspace.  For token
+ * tiles of at most 64, a tile much longer than the average list may be split
+ * over K between the two CTAs of a cluster, the second sending its int32
+ * partial through distributed shared memory (the sum is exact either way).
  * xq device [M][K/2]; s_x device [M]; y device bf16 [M][ldy].
  * split_k: 0, 1, 2, 4, 8 or 16, at most ceil(K / 256); accepted for source
  * compatibility and otherwise ignored (the tile schedule balances the work;
  * results do not depend on it).
- * N may be any positive size; ragged M, N and K tails are zero-filled.      */
+ * N may be any positive size up to 2^22 and M up to 2^20 (QVLA_ERR_CUDA
+ * beyond); ragged M, N and K tails are zero-filled.                          */
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,
                            const qvla_packed_linear* L, void* y, int ldy, int split_k,
                            cudaStream_t stream);

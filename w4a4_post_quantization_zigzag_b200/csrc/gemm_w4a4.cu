@@ -140,7 +140,9 @@ struct Batch {
   int split;                      // launched in clusters of two CTAs
   int tile_start[kMaxBatch + 1];  // launch tile ids of each problem
   uint16_t cta_begin[kMaxCtas + 1];
-  uint16_t order[kMaxTiles + kMaxCtas];   // launch tile ids, CTA by CTA (a split tile twice)
+  // the tiles, CTA by CTA (a split tile twice), each packed as
+  // problem | n-tile << 4 | m-tile << 19
+  uint32_t order[kMaxTiles + kMaxCtas];
   // with `split`, the role of each CTA's first tile: 0 the whole tile, 1 its
   // first K half and the epilogue (cluster rank 0), 2 its second K half,
   // sent to rank 0 (cluster rank 1)
@@ -153,13 +155,11 @@ struct Tile {
 };
 
 template <int NT>
-QVLA_DEVICE Tile decode(const Batch& b, int t) {
-  int p = 0;
-  while (p + 1 < b.n && t >= b.tile_start[p + 1]) ++p;
-  const int local = t - b.tile_start[p] + b.p[p].tile_base;
-  const int tn = b.p[p].tiles_n;
-  return Tile{p, (local % tn) * kBM, (local / tn) * NT};
+QVLA_DEVICE Tile decode(uint32_t w) {
+  return Tile{static_cast<int>(w & 15u), static_cast<int>((w >> 4) & 0x7FFFu) * kBM,
+              static_cast<int>(w >> 19) * NT};
 }
+constexpr int kListCache = 64;            // list entries a CTA keeps in shared memory
 
 // Wait until at most N bulk groups of this thread still read shared memory.
 template <int N>
@@ -196,10 +196,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
   __shared__ __align__(16) float sx_s[NT];       // s_x of the epilogue's current tile
+  // the head of the CTA's tile list and the problems' stage counts, read from
+  // the kernel parameters once by one warp (every role walks the list)
+  __shared__ uint32_t list_s[kListCache];
+  __shared__ uint8_t nks_s[kMaxBatch];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t_begin = batch.cta_begin[blockIdx.x];
   const int t_end = batch.cta_begin[blockIdx.x + 1];
+  auto tile_at = [&](int i) -> Tile {
+    const int j = i - t_begin;
+    return decode<NT>(j < kListCache ? list_s[j] : batch.order[i]);
+  };
   // K stages [k0, k1) of the CTA's i-th tile: all of them, or one half when
   // the tile is split over the cluster pair
   const int role = (C::kSplit && batch.split) ? batch.role[blockIdx.x] : 0;
@@ -219,6 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __nv_bfloat16* const outs = reinterpret_cast<__nv_bfloat16*>(base + C::kS * C::kStage);
   uint8_t* const recv = base + C::kS * C::kStage + C::kOutBytes;
 
+  constexpr uint32_t kTx = C::kABytes + C::kBBytes;
+  int pre = 0;                                   // stages the producer issued during setup
   if (tid == 0) {
     for (int s = 0; s < C::kS; ++s) {
       mbar_init(&bars.full[s], 1);
@@ -236,52 +246,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&batch.p[p].tw);
       tma_prefetch_desc(&batch.p[p].tx);
     }
+    // The producer's ramp, while the other warps set up: the first ring's
+    // worth of weight boxes (they do not depend on the previous kernel in the
+    // stream), then, once that kernel is done (programmatic dependent
+    // launch), the same stages' activation boxes.
+    for (int pass = 0; pass < 2; ++pass) {
+      int i = t_begin, ks = -1, n = 0;
+      while (n < C::kS && i < t_end) {
+        const Tile tr = decode<NT>(batch.order[i]);
+        const Problem& P = batch.p[tr.p];
+        int k0, k1;
+        krange(i, P.nks, k0, k1);
+        if (ks < 0) ks = k0;
+        uint8_t* st = stages + n * C::kStage;
+        if (pass == 0) {
+          mbar_arrive_expect_tx(&bars.full[n], kTx);
+          tma_load_2d(st, &P.tw, &bars.full[n], ks * kAPack, tr.n0);
+        } else if constexpr (kImage) {
+          tma_load_2d(st + C::kABytes, &P.tx, &bars.full[n], ks * kKS, tr.m0);
+          tma_load_2d(st + C::kABytes + NT * 128, &P.tx, &bars.full[n], ks * kKS + 128, tr.m0);
+        } else {
+          tma_load_2d(st + C::kABytes, &P.tx, &bars.full[n], ks * kAPack, tr.m0);
+        }
+        ++n;
+        if (++ks == k1) {
+          ks = -1;
+          ++i;
+        }
+      }
+      pre = n;
+      if (pass == 0) pdl_wait();
+    }
   }
   if (warp == 1) {
     __syncwarp();                  // tcgen05 alloc/ld/st/dealloc are warp-wide
     tmem_alloc(&bars.tmem, kTmemCols);
     tmem_relinquish();
   }
+  if (warp == 2) {
+    for (int j = lane; j < kListCache && t_begin + j < t_end; j += 32) list_s[j] = batch.order[t_begin + j];
+    if (lane < batch.n) nks_s[lane] = static_cast<uint8_t>(batch.p[lane].nks);
+  }
   tc_fence_before();
   cta_sync();
-  // the partner's barriers are initialised before anything reaches them
-  if (batch.split) cluster_sync();
+  // cluster barrier phase 1 ("barriers initialised"): every thread arrives
+  // now; a thread waits for it only before its first access to the
+  // partner's shared memory, or at the end
+  if (batch.split) cluster_arrive_release();
+  bool cluster_waited = false;
   tc_fence_after();
   const uint32_t tmem = bars.tmem;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      constexpr uint32_t kTx = C::kABytes + C::kBBytes;
-      // Weights do not depend on the previous kernel in the stream: the first
-      // ring's worth of weight boxes are requested before waiting for it
-      // (programmatic dependent launch), the activation boxes after.
-      int pre = 0;
-      {
-        int i = t_begin, ks = -1;
-        while (pre < C::kS && i < t_end) {
-          const Tile tr = decode<NT>(batch, batch.order[i]);
-          const Problem& P = batch.p[tr.p];
-          int k0, k1;
-          krange(i, P.nks, k0, k1);
-          if (ks < 0) ks = k0;
-          mbar_arrive_expect_tx(&bars.full[pre], kTx);
-          tma_load_2d(stages + pre * C::kStage, &P.tw, &bars.full[pre], ks * kAPack, tr.n0);
-          ++pre;
-          if (++ks == k1) {
-            ks = -1;
-            ++i;
-          }
-        }
-      }
-      pdl_wait();
+      // past the stages issued during setup
       bool ok = true;
       int g = 0;
       for (int i = t_begin; i < t_end && ok; ++i) {
-        const Tile tr = decode<NT>(batch, batch.order[i]);
+        const Tile tr = tile_at(i);
         const Problem& P = batch.p[tr.p];
         int k0, k1;
-        krange(i, P.nks, k0, k1);
+        krange(i, nks_s[tr.p], k0, k1);
         // the tile's weight boxes past the ring depth go to L2 now, so HBM
         // streaming is not limited by the ring
         for (int ks = k0 + C::kS; ks < k1; ++ks) tma_prefetch_l2_2d(&P.tw, ks * kAPack, tr.n0);
@@ -297,12 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mbar_arrive_expect_tx(&bars.full[s], kTx);
             tma_load_2d(st, &P.tw, &bars.full[s], ks * kAPack, tr.n0);
-          }
-          if constexpr (kImage) {
-            tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kKS, tr.m0);
-            tma_load_2d(st + C::kABytes + NT * 128, &P.tx, &bars.full[s], ks * kKS + 128, tr.m0);
-          } else {
-            tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kAPack, tr.m0);
+            if constexpr (kImage) {
+              tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kKS, tr.m0);
+              tma_load_2d(st + C::kABytes + NT * 128, &P.tx, &bars.full[s], ks * kKS + 128, tr.m0);
+            } else {
+              tma_load_2d(st + C::kABytes, &P.tx, &bars.full[s], ks * kAPack, tr.m0);
+            }
           }
         }
       }
@@ -317,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int g = 0, tc = 0;
       for (int i = t_begin; i < t_end && ok; ++i, ++tc) {
-        const Tile tr = decode<NT>(batch, batch.order[i]);
+        const Tile tr = tile_at(i);
         int k0, k1;
-        krange(i, batch.p[tr.p].nks, k0, k1);
+        krange(i, nks_s[tr.p], k0, k1);
         const int b = tc % C::kAcc, use = tc / C::kAcc;
         if (use >= 1) {
           ok = mbar_wait(&bars.acc_empty[b], (use - 1) & 1, err);
@@ -362,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     for (int i = t_begin; i < t_end && ok; ++i) {
       int k0, k1;
-      krange(i, batch.p[decode<NT>(batch, batch.order[i]).p].nks, k0, k1);
+      krange(i, nks_s[tile_at(i).p], k0, k1);
       for (int ks = k0; ks < k1; ++ks, ++g) {
         const int s = g % C::kS;
         // warp-uniform outcome: the tensor-memory stores below are warp-wide
@@ -428,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int tc = 0, chunk = 0;
     for (int i = t_begin; i < t_end && ok; ++i, ++tc) {
-      const Tile tr = decode<NT>(batch, batch.order[i]);
+      const Tile tr = tile_at(i);
       const Problem& P = batch.p[tr.p];
       const int b = tc % C::kAcc, use = tc / C::kAcc;
       // the tile's token scales, output-channel scale and bias, loaded while
@@ -454,6 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // theirs (the barrier orders them before the release), one thread
         // arrives on rank 0's barrier, releasing at cluster scope
         const uint32_t rv = map_shared_rank(smem_u32(recv), 0u);
+        cluster_wait();
+        cluster_waited = true;
 #pragma unroll 1
         for (int c0 = 0; c0 < NT; c0 += C::kCh) {
           uint32_t r[C::kCh];
@@ -554,9 +582,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   cta_sync();
-  // neither CTA of a pair leaves while the other may still reach its
-  // shared memory
-  if (batch.split) cluster_sync();
+  // phase 2: neither CTA of a pair leaves while the other may still reach
+  // its shared memory
+  if (batch.split) {
+    if (!cluster_waited) cluster_wait();
+    cluster_sync();
+  }
   if (warp == 1) {
     __syncwarp();                  // lane 0 comes from the MMA loop
     tc_fence_after();
@@ -694,12 +725,20 @@ int schedule(Batch& b, int pairs) {
       }
     }
   }
+  // launch tile id -> problem | n-tile << 4 | m-tile << 19
+  std::vector<uint32_t> packed(T);
+  for (int p = 0; p < b.n; ++p)
+    for (int t = b.tile_start[p]; t < b.tile_start[p + 1]; ++t) {
+      const int local = t - b.tile_start[p] + b.p[p].tile_base;
+      packed[t] = static_cast<uint32_t>(p) | static_cast<uint32_t>(local % b.p[p].tiles_n) << 4 |
+                  static_cast<uint32_t>(local / b.p[p].tiles_n) << 19;
+    }
   const int G = static_cast<int>(lists.size());
   int k = 0;
   for (int c = 0; c < G; ++c) {
     b.cta_begin[c] = static_cast<uint16_t>(k);
     b.role[c] = b.split ? role[c] : 0;
-    for (int t : lists[c]) b.order[k++] = static_cast<uint16_t>(t);
+    for (int t : lists[c]) b.order[k++] = packed[t];
   }
   b.cta_begin[G] = static_cast<uint16_t>(k);
   return G;
@@ -827,6 +866,9 @@ cudaError_t launch_group(const std::vector<const GemmArgs*>& gs, cudaStream_t st
     return e;
   };
   for (const GemmArgs* g : gs) {
+    // the packed tile coordinates hold 2^15 weight tiles and 2^13 token tiles
+    if ((g->N + kBM - 1) / kBM > (1 << 15) || (g->M + NT - 1) / NT > (1 << 13))
+      return cudaErrorInvalidValue;
     const int total = ((g->N + kBM - 1) / kBM) * ((g->M + NT - 1) / NT);
     for (int t0 = 0; t0 < total;) {
       if (batch.n == kMaxBatch || tiles == kMaxTiles) {

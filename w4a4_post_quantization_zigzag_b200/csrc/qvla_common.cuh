@@ -375,6 +375,10 @@ QVLA_DEVICE void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
 }
 
+QVLA_DEVICE void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
 QVLA_DEVICE void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
 
 QVLA_DEVICE void cluster_sync() {

@@ -648,15 +648,18 @@ using EncodeTiledFnR = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-constexpr int kTcThreads = 320;
 constexpr int kTM = 128;
 
-template <int BS>
+// kLat: the latency configuration for launches whose (token tile, block)
+// pairs fit three CTAs per SM: six warps, one block per CTA, rings of two A
+// tiles and one R_B, 57 KB of shared memory (block 64).
+template <int BS, bool kLat = false>
 struct TcCfg {
+  static constexpr int kThreads = kLat ? 192 : 320;
   static constexpr int kAStage = kTM * BS * 2;          // bf16 A tile
   static constexpr int kRStage = BS * BS * 2;           // one bf16 part of R_B^T
-  static constexpr int kAS = BS == 64 ? 3 : 2;          // A tiles in flight
-  static constexpr int kRS = BS == 64 ? 6 : 4;
+  static constexpr int kAS = kLat ? 2 : BS == 64 ? 3 : 2;   // A tiles in flight
+  static constexpr int kRS = kLat ? 3 : BS == 64 ? 6 : 4;
   static constexpr int kTmemCols = 2 * BS;              // double-buffered fp32 accumulator
   static constexpr int kSmem = kAS * kAStage + kRS * kRStage + 1024;
 };
@@ -666,7 +669,7 @@ struct TcBars {
   uint32_t tmem;
 };
 static_assert(TcCfg<64>::kAS <= 3 && TcCfg<128>::kAS <= 3 && TcCfg<64>::kRS <= 6 &&
-                  TcCfg<128>::kRS <= 6, "ring barriers");
+                  TcCfg<128>::kRS <= 6 && TcCfg<64, true>::kRS >= 3, "ring barriers");
 
 QVLA_DEVICE void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -676,16 +679,19 @@ QVLA_DEVICE void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint6
       : "memory");
 }
 
-// Block 64 runs two CTAs per SM (the grid is sized for that): the register
-// budget must let two 320-thread CTAs share the register file.
-template <int BS, int MODE, bool kTmaA>
-__global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
+// Block 64 runs two CTAs per SM (three in the latency configuration; the
+// grid is sized for that): the register budget must let them share the
+// register file.
+template <int BS, int MODE, bool kTmaA, bool kLat>
+__global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64 ? 2 : 1)
     rotq_tc_kernel(const __grid_constant__ ActBatch batch, unsigned int* err) {
-  using C = TcCfg<BS>;
+  using C = TcCfg<BS, kLat>;
   // epilogue warps: 6-9, or 2-9 in two column halves when the A tiles come
-  // by TMA and the gather warps are free
-  constexpr int kEpiWarps = kTmaA ? 8 : 4;
-  constexpr int kFirstEpi = 10 - kEpiWarps;
+  // by TMA and the gather warps are free; 2-5 in the latency configuration
+  constexpr int kWarps = C::kThreads / 32;
+  constexpr int kEpiWarps = (kTmaA && !kLat) ? 8 : 4;
+  constexpr int kFirstEpi = kWarps - kEpiWarps;
+  static_assert(!kLat || kTmaA, "the latency configuration loads A by TMA");
   constexpr int kHalves = kEpiWarps / 4;
   extern __shared__ uint8_t smem_raw[];
   __shared__ TcBars bars;
@@ -821,11 +827,23 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
         const int as = w % C::kAS, ab = w & 1;
         if (!mbar_wait(&bars.full_a[as], (w / C::kAS) & 1, err)) break;
         if (!mbar_wait(&bars.acc_empty[ab], ((w >> 1) & 1) ^ 1u, err)) break;
-        tc_fence_after();
-        for (int sp = 0; sp < 3; ++sp) {
-          const int u = 3 * w + sp, rr = u % C::kRS;
-          if (!mbar_wait(&bars.full_r[rr], (u / C::kRS) & 1, err)) break;
-          tc_fence_after();
+        // when the ring holds whole blocks, the block's three R_B parts are
+        // all waited for before the first MMA (a wait issued right behind
+        // MMAs costs far more than one ahead); otherwise part by part, so
+        // that the MMAs of the first parts free ring slots for the next
+        constexpr bool kWhole = C::kRS % 3 == 0;
+        bool okr = true;
+        for (int sp = 0; kWhole && sp < 3 && okr; ++sp)
+          okr = mbar_wait(&bars.full_r[(3 * w + sp) % C::kRS], ((3 * w + sp) / C::kRS) & 1, err);
+        if (!okr) break;
+        if (kWhole) tc_fence_after();
+        for (int sp = 0; sp < 3 && okr; ++sp) {
+          const int rr = (3 * w + sp) % C::kRS;
+          if (!kWhole) {
+            okr = mbar_wait(&bars.full_r[rr], ((3 * w + sp) / C::kRS) & 1, err);
+            if (!okr) break;
+            tc_fence_after();
+          }
 #pragma unroll
           for (int k = 0; k < BS / 16; ++k) {
             const int kc = k >> 2, kk = k & 3;
@@ -833,8 +851,11 @@ __global__ void __launch_bounds__(kTcThreads, BS == 64 ? 2 : 1)
             const uint64_t bd = smem_desc_kmajor_sw128(r_base + rr * C::kRStage + kc * (BS * 128) + kk * 32);
             umma_bf16(tmem + ab * BS, ad, bd, idesc, (sp | k) != 0 ? 1u : 0u);
           }
-          umma_commit(&bars.empty_r[rr]);
+          if (!kWhole) umma_commit(&bars.empty_r[rr]);
         }
+        if (!okr) break;
+        if (kWhole)
+          for (int sp = 0; sp < 3; ++sp) umma_commit(&bars.empty_r[(3 * w + sp) % C::kRS]);
         umma_commit(&bars.empty_a[as]);
         umma_commit(&bars.acc_full[ab]);
         if (MODE == kDynamic && cs > 1 && w == nbc - 1) {
@@ -1454,8 +1475,10 @@ cudaError_t launch_mode(const std::vector<const ActArgs*>& v, cudaStream_t strea
 }
 
 // ---------------------------------------------------------------- TC host
-template <int BS>
-int tc_ctas_per_sm() { return TcCfg<BS>::kSmem <= 110 * 1024 ? 2 : 1; }
+template <int BS, bool kLat = false>
+int tc_ctas_per_sm() {
+  return kLat ? 3 : TcCfg<BS>::kSmem <= 110 * 1024 ? 2 : 1;
+}
 
 template <int BS>
 int tc_cluster(int M, int K) {
@@ -1555,9 +1578,9 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
 
 // One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
 // mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
-template <int BS, int MODE, bool kTmaA>
+template <int BS, int MODE, bool kTmaA, bool kLat = false>
 cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cudaStream_t stream) {
-  using C = TcCfg<BS>;
+  using C = TcCfg<BS, kLat>;
   ActBatch batch;
   std::memset(&batch, 0, sizeof(batch));
   batch.n = n;
@@ -1596,7 +1619,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     }
   }
   batch.cta_start[n] = ctas;
-  auto kern = rotq_tc_kernel<BS, MODE, kTmaA>;
+  auto kern = rotq_tc_kernel<BS, MODE, kTmaA, kLat>;
   static std::atomic<unsigned long long> attr_done{0};
   {
     cudaError_t e = once_per_device(attr_done, [&]() {
@@ -1614,7 +1637,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);
-  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -1654,15 +1677,25 @@ cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t st
     }
     return cudaSuccess;
   }
-  // blocks per CTA: spread each launch's (token tile, block) pairs over one wave
+  // blocks per CTA: spread each launch's (token tile, block) pairs over one
+  // wave; a launch whose pairs fit one wave of the latency configuration
+  // takes that (one block per CTA)
   const long long slots = 148LL * tc_ctas_per_sm<BS>();
   for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
     const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
     long long pairs = 0;
     for (int i = 0; i < n; ++i)
       pairs += static_cast<long long>((v[i0 + i]->M + kTM - 1) / kTM) * (v[i0 + i]->K / BS);
+    cudaError_t e;
+    if constexpr (BS == 64 && MODE == kTable && kTmaA) {
+      if (pairs <= 148LL * tc_ctas_per_sm<BS, true>()) {
+        e = launch_tc_group<BS, MODE, kTmaA, true>(v.data() + i0, n, 1, 1, stream);
+        if (e != cudaSuccess) return e;
+        continue;
+      }
+    }
     const int G = static_cast<int>(std::max<long long>(1, (pairs + slots - 1) / slots));
-    cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, G, 1, stream);
+    e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, G, 1, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
