@@ -409,15 +409,23 @@ class DeviceStep:
                        for i, (lin, L) in enumerate(zip(wl.linears, self.packs)) if not self.w8[i]]
                       for t in range(T)]
         self.idx8 = [i for i in range(len(wl.linears)) if self.w8[i]]
+        # the W8A8 linears as batched problems: xq8 holds their 8-bit codes
+        # (the packed-code field is unused for them: one shared dummy each)
+        dummy = {i: torch.empty(wl.linears[i].M, wl.linears[i].K // 2, dtype=torch.uint8,
+                                device=dev) for i in self.idx8}
+        self.probs8 = [[Q.LinearProblem(self.packs[i], self.xs[t][i], xq=dummy[i], s_x=self.sx[i],
+                                        y=self.ys[i], workspace=self.wss[i], xq8=self.xq[i])
+                        for i in self.idx8] for t in range(T)]
 
     def w8_linears(self, t, phase):
-        Q = self.Q
-        for i in self.idx8:
-            if phase == 0:
-                Q.qvla_rotate_quant_act_a8(self.xs[t][i], self.packs[i], xq8=self.xq[i],
-                                           s_x=self.sx[i], workspace=self.wss[i])
-            else:
-                Q.qvla_w8a8_gemm(self.xq[i], self.sx[i], self.packs[i], y=self.ys[i])
+        """The W8A8 linears of the step: one batched 8-bit activation pass,
+        then one batched W8A8 GEMM."""
+        if not self.idx8:
+            return
+        if phase == 0:
+            self.Q.qvla_rotate_quant_act_a8_batched(self.probs8[t])
+        else:
+            self.Q.qvla_w8a8_gemm_batched(self.probs8[t])
 
     def step_batched(self, t, rec=None):
         Q = self.Q

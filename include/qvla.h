@@ -460,6 +460,26 @@ qvla_status qvla_rotate_quant_act_batched(const qvla_linear_problem* probs, int 
 qvla_status qvla_w4a4_gemm_batched(const qvla_linear_problem* probs, int n, int split_k,
                                    cudaStream_t stream);
 
+/* The W8A8 linears of a step, batched the same way (the variant the pages keep
+ * at 8 bits for the attention-output and FFN-down projections).  For these
+ * two entry points each problem's xq8 holds the 8-bit codes themselves
+ * (device int8 [M][K], one code per byte: q, not 16 * q), L is a pack from
+ * qvla_pack_weights_w8(), and xq is not used.
+ * qvla_rotate_quant_act_a8_batched: qvla_rotate_quant_act_a8() for every
+ * problem (reads x, writes xq8 and s_x); each problem's workspace /
+ * ws_bytes is its scratch as in qvla_rotate_quant_act_a8() (at least
+ * M * K * 4 bytes, else QVLA_ERR_WORKSPACE; M * K * 6 for the tensor-core
+ * route), 16-byte aligned, and no two workspaces may overlap (QVLA_ERR_ARG).
+ * mode, table and step fields are ignored (8-bit activations take the
+ * per-token dynamic scale).  Two launches for all problems (the rotations,
+ * then the row quantisation), plus the permuted copy on the tensor-core route.
+ * qvla_w8a8_gemm_batched: qvla_w8a8_gemm() for every problem (reads xq8,
+ * s_x, writes y), one launch per token tile for up to 16 linears.
+ * Results are identical to the single-linear calls.  Asynchronous.         */
+qvla_status qvla_rotate_quant_act_a8_batched(const qvla_linear_problem* probs, int n,
+                                             cudaStream_t stream);
+qvla_status qvla_w8a8_gemm_batched(const qvla_linear_problem* probs, int n, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

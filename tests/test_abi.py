@@ -153,6 +153,33 @@ def test_variant_entry_points_reject_bad_arguments():
     assert lib.qvla_w8a8_gemm_s32(None, 0, ctypes.byref(L), None, None) == q.QVLA_OK
 
 
+def test_batched_w8a8_entry_points_reject_bad_arguments():
+    """The batched W8A8 entry points check every problem on the host: scratch
+    below M * K * 4 bytes, overlapping scratch, missing outputs."""
+    q = _lib_mod()
+    lib = q._lib
+    L = q.qvla_packed_linear(128, 256, 64, 16, 16, None, 16, 16, None)
+
+    def prob(M, ws, ws_bytes, xq8=16, y=16):
+        return q.qvla_linear_problem(ctypes.pointer(L), 16, q.QVLA_DTYPE_BF16, M, 256, 0, None, 0,
+                                     0, None, 0, 0, 16, 16, y, 128, ws, ws_bytes, xq8)
+
+    def call(fn, *ps):
+        arr = (q.qvla_linear_problem * len(ps))(*ps)
+        return fn(arr, len(ps), None)
+
+    a8 = lib.qvla_rotate_quant_act_a8_batched
+    g8 = lib.qvla_w8a8_gemm_batched
+    assert a8(None, 1, None) == q.QVLA_ERR_ARG and g8(None, -1, None) == q.QVLA_ERR_ARG
+    assert a8(None, 0, None) == q.QVLA_OK and g8(None, 0, None) == q.QVLA_OK
+    assert call(a8, prob(4, 1 << 20, 4 * 256 * 4 - 1)) == q.QVLA_ERR_WORKSPACE
+    assert call(a8, prob(4, None, 0)) == q.QVLA_ERR_WORKSPACE
+    assert call(a8, prob(4, 1 << 20, 4 * 256 * 4, xq8=None)) == q.QVLA_ERR_ARG
+    assert call(a8, prob(4, 1 << 20, 1 << 16), prob(4, (1 << 20) + 4096, 1 << 16)) == q.QVLA_ERR_ARG
+    assert call(g8, prob(4, None, 0, y=None)) == q.QVLA_ERR_ARG
+    assert call(a8, prob(0, None, 0)) == q.QVLA_OK
+
+
 def test_selftest_wait_limit_is_checked_on_the_host():
     """Out-of-range wait limits are rejected before anything is launched."""
     q = _lib_mod()

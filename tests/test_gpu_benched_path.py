@@ -84,3 +84,38 @@ def test_dit_denoise_loop_layer_graph_replay_every_step(q):
     wl = bench.make_workload("dit_denoise_loop")
     wl.linears = wl.linears[:6]                 # q, k, v, o, up, down of layer 0
     _replay_and_check(q, wl, 4, 12)
+
+
+def test_mixed_precision_step_batched_equals_per_linear(q):
+    """The benchmark's mixed-precision step (down projections at W8A8, through
+    the batched 8-bit entry points) gives the same outputs, scales and codes as
+    one call per linear, replayed from a graph."""
+    wl = bench.make_workload("dit_mlp_stack")
+    dev = torch.device("cuda")
+    ds = bench.DeviceStep(wl, q, dev, precision="mix")
+    assert ds.idx8 and all(wl.linears[i].name.endswith("down") for i in ds.idx8)
+    stream = torch.cuda.Stream()
+    t = 3
+    with torch.cuda.stream(stream):
+        ds.step_per_linear(t)
+    torch.cuda.synchronize()
+    ref = [(x.clone(), s.clone(), y.clone()) for x, s, y in zip(ds.xq, ds.sx, ds.ys)]
+    for v in ds.ys:
+        v.zero_()
+    with torch.cuda.stream(stream):
+        ds.step_batched(t)                      # set-up calls outside capture
+    torch.cuda.synchronize()
+    for v in ds.ys:
+        v.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        ds.step_batched(t)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    assert q.qvla_read_error_word(clear=True) == 0
+    for i, (xq, s, y) in enumerate(ref):
+        assert torch.equal(ds.xq[i], xq), wl.linears[i].name
+        assert torch.equal(ds.sx[i], s), wl.linears[i].name
+        assert torch.equal(ds.ys[i], y), wl.linears[i].name
+    del g, ds

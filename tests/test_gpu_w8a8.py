@@ -139,3 +139,32 @@ def test_w8a8_linear_end_to_end(q, M, K, N, b):
     y_ref = O.dequantize(O.int_gemm(qx, ref.qw), out["s_x"], ref.s_w, ref.bias)
     check_y(y.float().cpu().numpy(), y_ref)
     assert q.qvla_read_error_word(clear=True) == 0
+
+
+def test_batched_w8a8_matches_single_calls(q):
+    """qvla_rotate_quant_act_a8_batched + qvla_w8a8_gemm_batched over linears of
+    different token tiles, widths, blocks and input types (both workspace
+    sizes) give exactly the single-linear results."""
+    shapes = [(50, 1024, 384, 64, "bf16", True), (50, 4096, 256, 64, "bf16", False),
+              (16, 512, 200, 32, "f32", True), (130, 1024, 256, 128, "bf16", True),
+              (7, 256, 136, 64, "f32", False)]
+    probs, singles = [], []
+    for i, (M, K, N, b, dt, full_ws) in enumerate(shapes):
+        W = I.weights(9700 + i, N, K, n_outlier_rows=2)
+        ref = O.pack_linear(W, b, bits=8)
+        L = q.qvla_pack_weights_w8(cu(W), b, perm_in=ref.perm.astype(np.int32), rsvd_in=ref.rsvd,
+                                   bias=cu(I.bias(9750 + i, N)))
+        x = I.activations(9800 + i, M, K, std=1.1, n_outlier_cols=3, dtype=dt)
+        xd = cu(x) if dt == "f32" else cu(x).to(torch.bfloat16)
+        nbytes = q.qvla_rotate_quant_a8_workspace_bytes(M, K) if full_ws else M * K * 4
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        probs.append(q.LinearProblem(L, xd, workspace=ws, xq8=True))
+        xq8, s_x = q.qvla_rotate_quant_act_a8(xd, L, workspace=ws.clone())
+        singles.append((xq8, s_x, q.qvla_w8a8_gemm(xq8, s_x, L)))
+    q.qvla_rotate_quant_act_a8_batched(probs)
+    q.qvla_w8a8_gemm_batched(probs)
+    torch.cuda.synchronize()
+    for p, (xq8, s_x, y) in zip(probs, singles):
+        assert torch.equal(p.xq8, xq8) and torch.equal(p.s_x, s_x)
+        assert torch.equal(p.y, y)
+    assert q.qvla_read_error_word(clear=True) == 0

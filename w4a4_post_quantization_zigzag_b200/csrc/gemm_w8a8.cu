@@ -13,14 +13,18 @@
 // K = 32 per instruction) into a tensor-memory accumulator, warps 2-5 read it
 // back with tcgen05.ld and apply the epilogue (bf16 tile in shared memory,
 // one TMA tensor store; plain stores for a tile cut by N with N % 8 != 0).
-// One 128 x NT output tile per CTA, no split-K.
+// One 128 x NT output tile per CTA, no split-K; one launch takes the tiles of
+// up to 16 linears that share the token tile (a CTA finds its linear by the
+// prefix sums of their tile counts).
 //
 // All waits are bounded (2 s) and flag QVLA_DEVERR_TIMEOUT instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
+#include <vector>
 
 #include "qvla_common.cuh"
 #include "qvla_internal.h"
@@ -55,10 +59,16 @@ struct W8Problem {
   int32_t* acc;                     // int32 [M][N] output instead of y (tests)
   int M, N, K, ldy, tiles_n;
 };
+constexpr int kW8MaxBatch = 16;
+struct W8Batch {
+  int n;
+  int tile_start[kW8MaxBatch + 1];  // first CTA of each linear
+  W8Problem p[kW8MaxBatch];
+};
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    w8a8_gemm_kernel(const __grid_constant__ W8Problem P, unsigned int* err) {
+    w8a8_gemm_kernel(const __grid_constant__ W8Batch batch, unsigned int* err) {
   using C = W8Cfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full[8], empty[8], acc_full;
@@ -66,8 +76,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float sx_s[NT];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = (blockIdx.x % P.tiles_n) * kBM;
-  const int m0 = (blockIdx.x / P.tiles_n) * NT;
+  int pi = 0;
+  while (pi + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.tile_start[pi + 1]) ++pi;
+  const W8Problem& P = batch.p[pi];
+  const int local = static_cast<int>(blockIdx.x) - batch.tile_start[pi];
+  const int n0 = (local % P.tiles_n) * kBM;
+  const int m0 = (local / P.tiles_n) * NT;
   const int nks = (P.K + kKS - 1) / kKS;
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* const base = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -192,20 +206,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int NT>
-cudaError_t launch_nt(const GemmArgs& g, cudaStream_t stream) {
-  using C = W8Cfg<NT>;
-  W8Problem P;
+bool fill_w8(W8Problem& P, const GemmArgs& g) {
   std::memset(&P, 0, sizeof(P));
   const uint64_t K = static_cast<uint64_t>(g.K);
   if (!encode_map_2d(&P.tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.wq, K, g.N, K, kKS, kBM,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_map_2d(&P.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.xq, K, g.M, K, kKS, NT,
                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+    return false;
   if (g.y != nullptr &&
       !encode_map_2d(&P.ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M,
                      static_cast<uint64_t>(g.ldy) * 2, kBM, NT, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+    return false;
   P.s_x = g.s_x;
   P.s_w = g.w_scale;
   P.bias = g.bias;
@@ -216,26 +228,67 @@ cudaError_t launch_nt(const GemmArgs& g, cudaStream_t stream) {
   P.K = g.K;
   P.ldy = g.ldy;
   P.tiles_n = (g.N + kBM - 1) / kBM;
-  const int tiles = P.tiles_n * ((g.M + NT - 1) / NT);
+  return true;
+}
+
+// The linears of one token tile, in launches of at most kW8MaxBatch.
+template <int NT>
+cudaError_t launch_nt(const std::vector<const GemmArgs*>& gs, cudaStream_t stream) {
+  using C = W8Cfg<NT>;
   auto kern = w8a8_gemm_kernel<NT>;
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = once_per_device(attr_done, [&]() {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
   if (e != cudaSuccess) return e;
-  kern<<<tiles, kThreads, C::kSmem, stream>>>(P, device_error_word());
-  return cudaGetLastError();
+  for (size_t i0 = 0; i0 < gs.size(); i0 += kW8MaxBatch) {
+    const int n = static_cast<int>(std::min<size_t>(kW8MaxBatch, gs.size() - i0));
+    W8Batch batch;
+    std::memset(&batch, 0, sizeof(batch));
+    batch.n = n;
+    long long tiles = 0;
+    for (int i = 0; i < n; ++i) {
+      const GemmArgs& g = *gs[i0 + i];
+      if (!fill_w8<NT>(batch.p[i], g)) return cudaErrorInvalidValue;
+      batch.tile_start[i] = static_cast<int>(tiles);
+      tiles += static_cast<long long>(batch.p[i].tiles_n) * ((g.M + NT - 1) / NT);
+    }
+    if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    batch.tile_start[n] = static_cast<int>(tiles);
+    if (tiles == 0) continue;
+    kern<<<static_cast<unsigned>(tiles), kThreads, C::kSmem, stream>>>(batch, device_error_word());
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
+
+int w8_token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 }  // namespace
 
+cudaError_t launch_w8a8_gemm_batch(const GemmArgs* gs, int n, cudaStream_t stream) {
+  static const int kTiles[5] = {16, 32, 64, 128, 256};
+  for (int t : kTiles) {
+    std::vector<const GemmArgs*> grp;
+    for (int i = 0; i < n; ++i)
+      if (gs[i].M > 0 && w8_token_tile(gs[i].M) == t) grp.push_back(&gs[i]);
+    if (grp.empty()) continue;
+    cudaError_t e;
+    switch (t) {
+      case 16: e = launch_nt<16>(grp, stream); break;
+      case 32: e = launch_nt<32>(grp, stream); break;
+      case 64: e = launch_nt<64>(grp, stream); break;
+      case 128: e = launch_nt<128>(grp, stream); break;
+      default: e = launch_nt<256>(grp, stream); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_w8a8_gemm(const GemmArgs& g, cudaStream_t stream) {
-  if (g.M <= 0) return cudaSuccess;
-  if (g.M <= 16) return launch_nt<16>(g, stream);
-  if (g.M <= 32) return launch_nt<32>(g, stream);
-  if (g.M <= 64) return launch_nt<64>(g, stream);
-  if (g.M <= 128) return launch_nt<128>(g, stream);
-  return launch_nt<256>(g, stream);
+  return launch_w8a8_gemm_batch(&g, 1, stream);
 }
 
 }  // namespace qvla

@@ -710,6 +710,72 @@ qvla_status qvla_rotate_quant_act_a8(const void* x, qvla_dtype xdt, int M, int l
   return cuda_status(launch_quant_rows(q, stream));
 }
 
+qvla_status qvla_rotate_quant_act_a8_batched(const qvla_linear_problem* probs, int n,
+                                             cudaStream_t stream) {
+  if (n < 0 || (n > 0 && !probs)) return QVLA_ERR_ARG;
+  std::vector<ActArgs> acts;
+  std::vector<QuantArgs> quants;
+  std::vector<std::pair<uintptr_t, size_t>> ranges;
+  for (int i = 0; i < n; ++i) {
+    const qvla_linear_problem& p = probs[i];
+    qvla_status st = check_linear(p.L, false);
+    if (st != QVLA_OK) return st;
+    if (p.M < 0) return QVLA_ERR_SHAPE;
+    if (p.xdt != QVLA_DTYPE_F32 && p.xdt != QVLA_DTYPE_BF16) return QVLA_ERR_ARG;
+    if (p.M == 0) continue;
+    const int K = p.L->K;
+    if (!p.x || !p.xq8 || !p.s_x) return QVLA_ERR_ARG;
+    if (p.ldx < K) return QVLA_ERR_SHAPE;
+    const size_t esz = p.xdt == QVLA_DTYPE_F32 ? 4 : 2;
+    if (!aligned16(p.x) || (p.ldx * esz) % 16 || !aligned16(p.xq8) || !aligned16(p.s_x) ||
+        !aligned16(p.workspace))
+      return QVLA_ERR_ALIGN;
+    const size_t xr_bytes = static_cast<size_t>(p.M) * K * 4, perm_bytes = static_cast<size_t>(p.M) * K * 2;
+    if (!p.workspace || p.ws_bytes < xr_bytes) return QVLA_ERR_WORKSPACE;
+    ranges.push_back({reinterpret_cast<uintptr_t>(p.workspace), p.ws_bytes});
+    // the rotation into the workspace (fp32 rows; the permuted copy of x
+    // after them when there is room), then the 8-bit quantisation of the rows
+    ActArgs a = {};
+    a.x = p.x;
+    a.xdt = static_cast<qvla_dtype>(p.xdt);
+    a.M = p.M;
+    a.ldx = p.ldx;
+    a.K = K;
+    a.block = p.L->block;
+    a.perm = p.L->perm;
+    a.rot = p.L->rot;
+    a.rot_tc = (p.L->rot_tc && (p.L->block == 64 || p.L->block == 128)) ? p.L->rot_tc : nullptr;
+    a.dynamic = 1;
+    a.xr_out = static_cast<float*>(p.workspace);
+    if (p.ws_bytes >= xr_bytes + perm_bytes) {
+      a.ws = static_cast<uint8_t*>(p.workspace) + xr_bytes;
+      a.ws_bytes = perm_bytes;
+    }
+    acts.push_back(a);
+    QuantArgs q = {};
+    q.xr = a.xr_out;
+    q.rows = p.M;
+    q.K = K;
+    q.qmin = -128;
+    q.qmax = 127;
+    q.dynamic = 1;
+    q.bits = 8;
+    q.q_out = reinterpret_cast<uint8_t*>(p.xq8);
+    q.s_out = p.s_x;
+    quants.push_back(q);
+  }
+  // the problems run concurrently: their workspaces must be disjoint
+  for (size_t i = 0; i < ranges.size(); ++i)
+    for (size_t j = i + 1; j < ranges.size(); ++j)
+      if (ranges[i].first < ranges[j].first + ranges[j].second &&
+          ranges[j].first < ranges[i].first + ranges[i].second)
+        return QVLA_ERR_ARG;
+  if (acts.empty()) return QVLA_OK;
+  cudaError_t e = launch_rotate_quant_batch(acts.data(), static_cast<int>(acts.size()), stream);
+  if (e == cudaSuccess) e = launch_quant_rows_batch(quants.data(), static_cast<int>(quants.size()), stream);
+  return cuda_status(e);
+}
+
 qvla_status qvla_rotate_act_f32(const void* x, qvla_dtype xdt, int M, int ldx,
                                 const qvla_packed_linear* L, float* xr_out, cudaStream_t stream) {
   return rotate_act_impl(x, xdt, M, ldx, L, xr_out, nullptr, 0, stream);
@@ -876,6 +942,22 @@ qvla_status qvla_w8a8_gemm(const int8_t* xq8, const float* s_x, int M,
 qvla_status qvla_w8a8_gemm_s32(const int8_t* xq8, int M, const qvla_packed_linear* L,
                                int32_t* acc, cudaStream_t stream) {
   return w8a8_common(xq8, nullptr, M, L, nullptr, 0, acc, stream);
+}
+
+qvla_status qvla_w8a8_gemm_batched(const qvla_linear_problem* probs, int n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && !probs)) return QVLA_ERR_ARG;
+  std::vector<GemmArgs> v(n);
+  for (int i = 0; i < n; ++i) {
+    const qvla_linear_problem& p = probs[i];
+    if (p.M > 0 && !p.y) return QVLA_ERR_ARG;
+    qvla_status st = prepare_gemm(reinterpret_cast<const uint8_t*>(p.xq8), p.s_x, p.M, p.L, p.y,
+                                  p.ldy, nullptr, 0, &v[i]);
+    if (st != QVLA_OK) return st;
+  }
+  if (n == 0) return QVLA_OK;
+  qvla_status st = check_sm100();
+  if (st != QVLA_OK) return st;
+  return cuda_status(launch_w8a8_gemm_batch(v.data(), n, stream));
 }
 
 qvla_status qvla_w4a4_gemm(const uint8_t* xq, const float* s_x, int M,

@@ -74,6 +74,8 @@ struct QuantArgs {
   int bits;                // 4 (default when 0) or 8
 };
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream);
+// independent row sets in as few launches as possible (one CTA per row)
+cudaError_t launch_quant_rows_batch(const QuantArgs* as, int n, cudaStream_t stream);
 
 // ---- GPTQ rounding on the host (gptq_host.cu)
 // H = X'^T X' (fp64, K x K) of T rotated calibration rows xr [T][K].
@@ -123,5 +125,7 @@ cudaError_t launch_w4a4_gemm_batch(const GemmArgs* gs, int n, int split_k, cudaS
 // W8A8 variant (gemm_w8a8.cu): int8 codes [M][K] and [N][K] straight into the
 // tensor cores (xq and wq hold one int8 code per byte; split_k is ignored)
 cudaError_t launch_w8a8_gemm(const GemmArgs& g, cudaStream_t stream);
+// independent W8A8 linears, grouped by token tile, up to 16 per launch
+cudaError_t launch_w8a8_gemm_batch(const GemmArgs* gs, int n, cudaStream_t stream);
 
 }  // namespace qvla

@@ -1180,18 +1180,36 @@ cudaError_t launch_expand(const std::vector<const ActArgs*>& v, cudaStream_t str
   return cudaGetLastError();
 }
 
-// Quantise fp32 rows (already rotated): one CTA per row.
+// Quantise fp32 rows (already rotated): one CTA per row, the rows of up to
+// kMaxBatch independent sets in one launch.
+struct QuantJob {
+  const float* xr;
+  const float* table;
+  const int32_t* step_dev;
+  uint8_t* q_out;
+  float* s_out;
+  int K, qmin, qmax, dynamic, T, Lcount, step_host, layer, bits;
+};
+struct QuantBatch {
+  int n;
+  int row_start[kMaxBatch + 1];   // first CTA of each set
+  QuantJob j[kMaxBatch];
+};
+
 __global__ void __launch_bounds__(kThreads)
-    quant_rows_kernel(const float* __restrict__ xr, int K, int qmin, int qmax, int dynamic,
-                      const float* __restrict__ table, int T, int Lcount,
-                      const int32_t* __restrict__ step_dev, int step_host, int layer,
-                      uint8_t* __restrict__ q_out, float* __restrict__ s_out, int bits,
-                      unsigned int* err) {
+    quant_rows_kernel(const __grid_constant__ QuantBatch batch, unsigned int* err) {
   __shared__ float red[kWarps];
   __shared__ float s_sh;
-  const int row = blockIdx.x, tid = threadIdx.x;
+  int ji = 0;
+  while (ji + 1 < batch.n && static_cast<int>(blockIdx.x) >= batch.row_start[ji + 1]) ++ji;
+  const QuantJob& J = batch.j[ji];
+  const float* __restrict__ xr = J.xr;
+  uint8_t* __restrict__ q_out = J.q_out;
+  float* __restrict__ s_out = J.s_out;
+  const int K = J.K, qmin = J.qmin, qmax = J.qmax, bits = J.bits;
+  const int row = static_cast<int>(blockIdx.x) - batch.row_start[ji], tid = threadIdx.x;
   const float* src = xr + static_cast<size_t>(row) * K;
-  if (dynamic) {
+  if (J.dynamic) {
     float mx = 0.f;
     for (int k = tid; k < K; k += kThreads) mx = fmaxf(mx, fabsf(src[k]));
 #pragma unroll
@@ -1204,7 +1222,7 @@ __global__ void __launch_bounds__(kThreads)
       s_sh = __fdiv_rn(m, static_cast<float>(qmax));
     }
   } else if (tid == 0) {
-    s_sh = table_scale(table, T, Lcount, step_dev, step_host, layer, err);
+    s_sh = table_scale(J.table, J.T, J.Lcount, J.step_dev, J.step_host, J.layer, err);
   }
   cta_sync();
   const float s = s_sh;
@@ -1782,12 +1800,32 @@ cudaError_t launch_rotate_quant(const ActArgs& a, cudaStream_t stream) {
   return launch_rotate_quant_batch(&a, 1, stream);
 }
 
+cudaError_t launch_quant_rows_batch(const QuantArgs* as, int n, cudaStream_t stream) {
+  for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+    const int m = std::min(kMaxBatch, n - i0);
+    QuantBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.n = m;
+    long long rows = 0;
+    for (int i = 0; i < m; ++i) {
+      const QuantArgs& a = as[i0 + i];
+      b.j[i] = QuantJob{a.xr, a.table, a.step_dev, a.q_out, a.s_out, a.K, a.qmin, a.qmax,
+                        a.dynamic, a.T, a.Lcount, a.step_host, a.layer, a.bits == 8 ? 8 : 4};
+      b.row_start[i] = static_cast<int>(rows);
+      rows += std::max(0, a.rows);
+    }
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    b.row_start[m] = static_cast<int>(rows);
+    if (rows == 0) continue;
+    quant_rows_kernel<<<static_cast<unsigned>(rows), kThreads, 0, stream>>>(b, device_error_word());
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_quant_rows(const QuantArgs& a, cudaStream_t stream) {
-  quant_rows_kernel<<<a.rows, kThreads, 0, stream>>>(a.xr, a.K, a.qmin, a.qmax, a.dynamic,
-                                                     a.table, a.T, a.Lcount, a.step_dev,
-                                                     a.step_host, a.layer, a.q_out, a.s_out,
-                                                     a.bits == 8 ? 8 : 4, device_error_word());
-  return cudaGetLastError();
+  return launch_quant_rows_batch(&a, 1, stream);
 }
 
 }  // namespace qvla

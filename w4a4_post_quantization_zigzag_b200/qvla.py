@@ -68,7 +68,8 @@ EXPORTED = (
     "qvla_pack_weights_hadamard", "qvla_pack_weights_w8", "qvla_rotate_quant_act_a8",
     "qvla_rotate_quant_a8_workspace_bytes", "qvla_w8a8_gemm", "qvla_w8a8_gemm_s32",
     "qvla_gptq_quantize_host", "qvla_pack_weights_gptq", "qvla_gptq_hessian_host",
-    "qvla_selftest_wait_timeout", "qvla_source_hash",
+    "qvla_selftest_wait_timeout", "qvla_source_hash", "qvla_rotate_quant_act_a8_batched",
+    "qvla_w8a8_gemm_batched",
 )
 
 QVLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -138,6 +139,8 @@ _sig = {
     "qvla_w4a4_gemm_s32": (c_int, [c_void_p, c_int, _P, c_void_p, c_int, c_void_p]),
     "qvla_rotate_quant_act_batched": (c_int, [_PP, c_int, c_void_p]),
     "qvla_w4a4_gemm_batched": (c_int, [_PP, c_int, c_int, c_void_p]),
+    "qvla_rotate_quant_act_a8_batched": (c_int, [_PP, c_int, c_void_p]),
+    "qvla_w8a8_gemm_batched": (c_int, [_PP, c_int, c_void_p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -657,3 +660,19 @@ def qvla_w4a4_gemm_batched(problems, split_k: int = 0, stream=None):
     arr = _problem_array(problems)
     _check(_lib.qvla_w4a4_gemm_batched(arr, len(problems), split_k, _stream(stream)),
            "qvla_w4a4_gemm_batched")
+
+
+def qvla_rotate_quant_act_a8_batched(problems, stream=None):
+    """8-bit activation codes of W8A8 linears: each problem's xq8 (int8
+    [M, K]) receives the codes themselves and s_x the per-token scales; each
+    problem needs a workspace (qvla_rotate_quant_a8_workspace_bytes)."""
+    arr = _problem_array(problems)
+    _check(_lib.qvla_rotate_quant_act_a8_batched(arr, len(problems), _stream(stream)),
+           "qvla_rotate_quant_act_a8_batched")
+
+
+def qvla_w8a8_gemm_batched(problems, stream=None):
+    """W8A8 GEMMs of the problems (xq8 holds 8-bit codes, L a W8 pack)."""
+    arr = _problem_array(problems)
+    _check(_lib.qvla_w8a8_gemm_batched(arr, len(problems), _stream(stream)),
+           "qvla_w8a8_gemm_batched")
