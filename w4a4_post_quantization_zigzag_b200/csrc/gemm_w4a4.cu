@@ -66,7 +66,7 @@ constexpr int kBM = 128;                  // weight rows per tile (UMMA M, tenso
 constexpr int kKS = 256;                  // K per pipeline stage
 constexpr int kAPack = kKS / 2;           // packed weight bytes per row per stage (one 128B-swizzled box)
 constexpr int kACols = kKS / 4;           // tensor-memory columns of one unpacked A stage
-constexpr int kThreads = 320;
+constexpr int kBaseThreads = 320;
 constexpr int kOutSlots = 4;              // output staging ring (32-token chunks)
 constexpr int kTmemCols = 512;
 constexpr int kMaxBatch = 16;
@@ -78,7 +78,12 @@ template <int NT, bool kImage>
 struct Cfg {
   static constexpr int kAcc = NT >= 256 ? 1 : 2;                  // accumulator buffers
   static constexpr int kAccCols = NT < 32 ? 32 : NT;
-  static constexpr int kACol0 = kAcc * kAccCols;                 // first A-stage column
+  // MMA issuers: with small token tiles a second thread issues every other
+  // stage of a tile into its own accumulator (the epilogue adds the two), so
+  // that the tensor pipe runs one issuer's MMAs while the other waits
+  static constexpr int kIss = NT <= 64 ? 2 : 1;
+  static constexpr int kThreads = kBaseThreads + 32 * (kIss - 1);  // warp 10: second issuer
+  static constexpr int kACol0 = kAcc * kIss * kAccCols;          // first A-stage column
   static constexpr int kABytes = kBM * kAPack;                   // packed weight box
   // activations: the image as two 128-byte boxes (K halves) of NT rows, or
   // one 128-byte box of packed codes plus their unpacked two halves
@@ -190,7 +195,7 @@ QVLA_DEVICE void unpack32(const uint4 v, uint32_t* o) {
 }
 
 template <int NT, bool kImage>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<NT, kImage>::kThreads, 1)
     w4a4_gemm_kernel(const __grid_constant__ Batch batch, unsigned int* err) {
   using C = Cfg<NT, kImage>;
   extern __shared__ uint8_t smem_raw[];
@@ -236,10 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.mma_done[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.acc_full[b], 1);
+      mbar_init(&bars.acc_full[b], C::kIss);
       mbar_init(&bars.acc_empty[b], 4);
     }
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.drain, C::kIss);
     mbar_init(&bars.recv_full, 1);
     fence_mbar_init();
     for (int p = 0; p < batch.n; ++p) {
@@ -336,9 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = g - C::kS < 0 ? 0 : g - C::kS; j < g; ++j)
         mbar_wait(&bars.full[j % C::kS], (j / C::kS) & 1, err);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || (C::kIss == 2 && warp == kBaseThreads / 32)) {
+    // ------------------------------------------------------------- MMA issuers
+    // issuer j takes the stages ks of each tile with (ks - k0) % kIss == j,
+    // into accumulator column block (b * kIss + j)
     if (lane == 0) {
+      const int j = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc = idesc_i8(kBM, NT);
       bool ok = true;
       int g = 0, tc = 0;
@@ -351,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bars.acc_empty[b], (use - 1) & 1, err);
           if (!ok) break;
         }
-        const uint32_t d = tmem + static_cast<uint32_t>(b * C::kAccCols);
+        const uint32_t d = tmem + static_cast<uint32_t>((b * C::kIss + j) * C::kAccCols);
         for (int ks = k0; ks < k1; ++ks, ++g) {
+          if ((ks - k0) % C::kIss != j) continue;         // the other issuer's stage
           const int s = g % C::kS;
           // the stage's A is in tensor memory (and, when the unpack warps got
           // the stage, its TMA bytes, activations included, had landed)
@@ -367,11 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 32 codes of K: A columns [8kk, 8kk+8) of the stage; B half kk/4,
             // bytes [32(kk%4), +32) of each 128-byte row
             const uint64_t bd = smem_desc_kmajor_sw128(bs + (kk >> 2) * (NT * 128) + 32 * (kk & 3));
-            umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks > k0 || kk > 0) ? 1u : 0u);
+            umma_i8_tmem_a(d, at + 8 * kk, bd, idesc, (ks >= k0 + C::kIss || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars.mma_done[s]);
         }
         if (!ok) break;
+        // (an issuer without a stage in this tile still arrives: its
+        // accumulator is then not read)
         umma_commit(&bars.acc_full[b]);
       }
       umma_commit(&bars.drain);
@@ -472,8 +483,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool tma = tr.n0 + kBM <= P.N || (P.N & 7) == 0;
-      const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(b * C::kAccCols);
+      const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(b * C::kIss * C::kAccCols);
       const bool first = i == t_begin;
+      // the second issuer's accumulator holds stages when the tile has two or more
+      int k0, k1;
+      krange(i, nks_s[tr.p], k0, k1);
+      const bool two = C::kIss == 2 && k1 - k0 >= 2;
+      auto load_acc = [&](int c0, uint32_t (&r)[C::kCh]) {
+        tmem_ld_chunk<NT>(tacc + c0, r);
+        tmem_ld_wait();
+        if (two) {
+          uint32_t r2[C::kCh];
+          tmem_ld_chunk<NT>(tacc + C::kAccCols + c0, r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < C::kCh; ++q) r[q] += r2[q];
+        }
+      };
       if (role == 2 && first) {
         // second K half of a split tile: the int32 partial goes to the
         // receive buffer of cluster rank 0; once all four warps have stored
@@ -485,8 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c0 = 0; c0 < NT; c0 += C::kCh) {
           uint32_t r[C::kCh];
-          tmem_ld_chunk<NT>(tacc + c0, r);
-          tmem_ld_wait();
+          load_acc(c0, r);
 #pragma unroll
           for (int j = 0; j < C::kCh; j += 4)
             st_shared_cluster_v4(rv + static_cast<uint32_t>((((c0 + j) >> 2) * kBM + row) * 16),
@@ -508,8 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < NT; c0 += C::kCh) {
         uint32_t r[C::kCh];
-        tmem_ld_chunk<NT>(tacc + c0, r);
-        tmem_ld_wait();
+        load_acc(c0, r);
         if (role == 1 && first) {
           // plus the partner's partial (the other K half; 256 * acc stays
           // within int32 for K <= QVLA_MAX_K)
@@ -756,7 +780,7 @@ int cluster_pairs() {
   if (c != 0) return c > 0 ? c : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * kMaxCtas, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -788,7 +812,7 @@ cudaError_t launch_batch(Batch& batch, cudaStream_t stream) {
   if (G == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
