@@ -1030,13 +1030,12 @@ struct PermJob {
   __nv_bfloat16* out;
   int ldx, M, K;
   int rpc;                          // rows per CTA
+  int stages;                       // row slots of K * 2 bytes in the ring
 };
-constexpr int kPermMaxStages = 8;
+constexpr int kPermMaxStages = 32;
 constexpr int kPermWorkers = 256;
 struct PermBatch {
   int n;
-  int stages;                       // row buffers in the ring
-  int row_bytes;                    // bytes of one ring slot (largest K of the batch, x 2)
   int cta_start[kMaxBatch + 1];
   PermJob j[kMaxBatch];
 };
@@ -1052,7 +1051,8 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
   const PermJob& J = batch.j[ji];
   const int r0 = (static_cast<int>(blockIdx.x) - batch.cta_start[ji]) * J.rpc;
   const int nr = min(J.rpc, J.M - r0);
-  const int K = J.K, kc = K / 8, S = batch.stages;
+  const int K = J.K, kc = K / 8, S = J.stages;
+  const int row_bytes = K * 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the permutation does not depend on the previous kernel: read before
   // waiting for it
@@ -1087,7 +1087,7 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
         const int st = r % S;
         if (!mbar_wait(&empty[st], ((r / S) & 1) ^ 1u, err)) break;
         mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(K) * 2u);
-        bulk_copy_g2s(smem + static_cast<size_t>(st) * batch.row_bytes,
+        bulk_copy_g2s(smem + static_cast<size_t>(st) * row_bytes,
                       J.x + static_cast<size_t>(r0 + r) * J.ldx, static_cast<uint32_t>(K) * 2u, &full[st]);
         ++issued;
       }
@@ -1100,7 +1100,7 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
       const int st = r % S;
       if (!mbar_wait(&full[st], (r / S) & 1, err)) break;
       const unsigned short* sr =
-          reinterpret_cast<const unsigned short*>(smem + static_cast<size_t>(st) * batch.row_bytes);
+          reinterpret_cast<const unsigned short*>(smem + static_cast<size_t>(st) * row_bytes);
       uint4* orow = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(r0 + r) * K);
 #pragma unroll
       for (int c = 0; c < kPC; ++c) {
@@ -1531,22 +1531,64 @@ bool make_xperm_map(CUtensorMap* map, void* ptr, int M, int K) {
 }
 
 // Permuted copies x_perm = x[:, perm] of the problems that have scratch.
-// The ring holds about 48 KB of rows (2 to 8 of them); the elements of a
-// launch are spread evenly over about three CTAs per SM (fewer rows per CTA
-// where the rows are longer).
-constexpr int kPermRingBytes = 48 * 1024;
+// Each CTA's ring is about 48 KB (128 KB for the longest rows, whose variant
+// holds the permutation of 16 runs per thread in registers and so runs one
+// CTA per SM), cut into as many slots as it holds of the CTA's own rows (2 to
+// 32); the elements of a launch are spread evenly over the CTAs (fewer rows
+// per CTA where the rows are longer).
 template <int kPC>
-cudaError_t launch_permute_kernel(const PermBatch& b, int ctas, cudaStream_t stream) {
+int permute_ring_bytes() { return kPC >= 16 ? 128 * 1024 : 48 * 1024; }
+
+// CTAs per SM the register file allows (shared memory is counted by the caller).
+template <int kPC>
+int permute_reg_occupancy() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  int c = cache[dev].load(std::memory_order_relaxed);
+  if (c > 0) return c;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, permute_rows_kernel<kPC>, kPermWorkers + 32, 0) !=
+          cudaSuccess || c <= 0) {
+    cudaGetLastError();
+    c = 1;
+  }
+  cache[dev].store(c, std::memory_order_relaxed);
+  return c;
+}
+
+template <int kPC>
+cudaError_t launch_permute_kernel(PermBatch& b, const ActArgs* const* as, int kmax,
+                                  cudaStream_t stream) {
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = once_per_device(attr_done, []() {
     return cudaFuncSetAttribute(permute_rows_kernel<kPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 2 * QVLA_MAX_K * 2);
   });
   if (e != cudaSuccess) return e;
+  // one ring of shared memory per CTA, as many row slots as it holds for the
+  // CTA's own rows (so short rows keep more of them in flight)
+  const int smem = std::max(permute_ring_bytes<kPC>(), 2 * kmax * 2);
+  for (int i = 0; i < b.n; ++i) b.j[i].stages = std::min(kPermMaxStages, smem / (as[i]->K * 2));
+  // the elements spread over one wave of resident CTAs; the longest rows
+  // (one CTA per SM) take three CTAs per SM in waves, measured faster than
+  // one long CTA per SM
+  const int occ = kPC >= 16 ? 3
+                            : std::max(1, std::min(permute_reg_occupancy<kPC>(), 227 * 1024 / (smem + 2048)));
+  long long elems = 0;
+  for (int i = 0; i < b.n; ++i) elems += static_cast<long long>(as[i]->M) * as[i]->K;
+  const long long slots = 148LL * occ;
+  const long long per_cta = (elems + slots - 1) / slots;
+  int ctas = 0;
+  for (int i = 0; i < b.n; ++i) {
+    b.j[i].rpc = static_cast<int>(std::max<long long>(1, (per_cta + as[i]->K - 1) / as[i]->K));
+    b.cta_start[i] = ctas;
+    ctas += (as[i]->M + b.j[i].rpc - 1) / b.j[i].rpc;
+  }
+  b.cta_start[b.n] = ctas;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, 1, 1);
   cfg.blockDim = dim3(kPermWorkers + 32, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(b.stages) * b.row_bytes;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1562,33 +1604,22 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
     PermBatch b;
     std::memset(&b, 0, sizeof(b));
     b.n = n;
-    long long elems = 0;
     int kmax = 0;
     for (int i = 0; i < n; ++i) {
-      elems += static_cast<long long>(v[i0 + i]->M) * v[i0 + i]->K;
-      kmax = std::max(kmax, v[i0 + i]->K);
-    }
-    b.row_bytes = kmax * 2;
-    b.stages = std::max(2, std::min(kPermMaxStages, kPermRingBytes / b.row_bytes));
-    const long long per_cta = (elems + 3 * 148 - 1) / (3 * 148);
-    int ctas = 0;
-    for (int i = 0; i < n; ++i) {
       const ActArgs& a = *v[i0 + i];
+      kmax = std::max(kmax, a.K);
       b.j[i].x = static_cast<const __nv_bfloat16*>(a.x);
       b.j[i].perm = a.perm;
       b.j[i].out = static_cast<__nv_bfloat16*>(a.ws);
       b.j[i].ldx = a.ldx;
       b.j[i].M = a.M;
       b.j[i].K = a.K;
-      b.j[i].rpc = static_cast<int>(std::max<long long>(1, (per_cta + a.K - 1) / a.K));
-      b.cta_start[i] = ctas;
-      ctas += (a.M + b.j[i].rpc - 1) / b.j[i].rpc;
     }
-    b.cta_start[n] = ctas;
     const int runs = (kmax / 8 + kPermWorkers - 1) / kPermWorkers;   // runs of 8 per thread
-    cudaError_t e = runs <= 1   ? launch_permute_kernel<1>(b, ctas, stream)
-                    : runs <= 4 ? launch_permute_kernel<4>(b, ctas, stream)
-                                : launch_permute_kernel<16>(b, ctas, stream);
+    const ActArgs* const* as = v.data() + i0;
+    cudaError_t e = runs <= 1   ? launch_permute_kernel<1>(b, as, kmax, stream)
+                    : runs <= 4 ? launch_permute_kernel<4>(b, as, kmax, stream)
+                                : launch_permute_kernel<16>(b, as, kmax, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
