@@ -1714,13 +1714,21 @@ template <int BS, int MODE, bool kTmaA>
 cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   if (v.empty()) return cudaSuccess;
   if (MODE == kDynamic) {
+    // the cluster size each linear would take alone; a launch of several
+    // halves it until all its clusters fit one wave (clusters of one CTA per
+    // SM are only co-resident a GPC's worth at a time)
+    const long long slots = 148LL * tc_ctas_per_sm<BS>();
     for (int cs = 1; cs <= 16; cs *= 2) {
       std::vector<const ActArgs*> g;
       for (const ActArgs* a : v)
         if (tc_cluster<BS>(a->M, a->K) == cs) g.push_back(a);
       for (size_t i0 = 0; i0 < g.size(); i0 += kMaxBatch) {
         const int n = static_cast<int>(std::min<size_t>(kMaxBatch, g.size() - i0));
-        cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(g.data() + i0, n, 1, cs, stream);
+        long long tiles = 0;
+        for (int i = 0; i < n; ++i) tiles += (g[i0 + i]->M + kTM - 1) / kTM;
+        int c = cs;
+        while (c > 1 && tiles * c > slots) c /= 2;
+        cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(g.data() + i0, n, 1, c, stream);
         if (e != cudaSuccess) return e;
       }
     }
