@@ -330,11 +330,18 @@ qvla_status qvla_rotate_quant_act(const void* x, qvla_dtype xdt, int M, int ldx,
                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Scratch that lets qvla_rotate_quant_act take its fastest route
- * (tensor-core rotation fed by TMA from a permuted copy of x): M * K * 2 bytes
- * when that route applies (bf16 input, block 64 or 128, M > 0), else 0.
- * Without it (workspace NULL or too small) the call still works, gathering
- * the permuted inputs directly.  The scratch is only used while the call's
- * kernels run; reusing it for another call on the same stream is safe.     */
+ * (tensor-core rotation fed by TMA from a permuted copy of x):
+ * M * K * 2 + M * (K / block) * 4 bytes when that route applies (bf16 input,
+ * block 64 or 128, M > 0), else 0.  The first M * K * 2 bytes hold the
+ * permuted copy; the rest, in DYNAMIC mode, the row maxima of each CTA when
+ * the two passes (maximum, then quantisation) run as two launches, which
+ * spreads the blocks of wide and narrow linears evenly over the SMs.  With
+ * only M * K * 2 bytes the DYNAMIC passes run in one launch, the maximum
+ * reduced over a thread-block cluster; without scratch (workspace NULL or
+ * smaller) the call still works, gathering the permuted inputs directly.
+ * All routes give the same codes and scales.  The scratch is only used
+ * while the call's kernels run; reusing it for another call on the same
+ * stream is safe.                                                          */
 qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtype xdt,
                                               size_t* bytes);
 

@@ -95,8 +95,8 @@ def test_argument_errors_before_any_cuda_call():
     assert lib.qvla_rotate_quant_act(None, 1, 0, 256, ctypes.byref(Lok), 0, None, 0, 0, None, 0,
                                      0, None, None, None, 0, None) == q.QVLA_OK
     # scratch size query: the tensor-core route (bf16, block 64 / 128) uses it
-    assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 128) == 1024 * 2048 * 2
-    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64) == 50 * 2048 * 2
+    assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 128) == 1024 * 2048 * 2 + 1024 * 16 * 4
+    assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64) == 50 * 2048 * 2 + 50 * 32 * 4
     assert q.qvla_rotate_quant_workspace_bytes(50, 2048, 64, torch.float32) == 0
     assert q.qvla_rotate_quant_workspace_bytes(0, 2048, 64) == 0
     assert q.qvla_rotate_quant_workspace_bytes(1024, 2048, 256) == 0

@@ -43,7 +43,7 @@ def test_c_program_against_the_header(exe):
     assert d["status"][0].startswith("ok") or "OK" in d["status"][0].upper()
     assert d["sizes"] == ["0", str(256 * 1024 // 2), str(4 * 1024 * 64), str(6 * 1024 * 64)]
     assert d["badshape"] == ["2"]                                   # QVLA_ERR_SHAPE
-    assert d["rqws"] == ["0", str(50 * 2048 * 2)]
+    assert d["rqws"] == ["0", str(50 * 2048 * 2 + 50 * (2048 // 64) * 4)]
     assert d["a8ws"] == ["0", str(50 * 1024 * 6)]
     assert d["nulllinear"] == ["1"]                                 # QVLA_ERR_ARG
     assert d["gptqshape"] == ["2"]

@@ -586,7 +586,9 @@ qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtyp
   if (!bytes) return QVLA_ERR_ARG;
   if (M < 0 || K <= 0 || K > QVLA_MAX_K || !valid_block(block) || K % block) return QVLA_ERR_SHAPE;
   const bool tc = xdt == QVLA_DTYPE_BF16 && (block == 64 || block == 128) && M > 0;
-  *bytes = tc ? static_cast<size_t>(M) * K * 2 : 0;
+  // the permuted copy of x, then (DYNAMIC) the row maxima of up to K / block
+  // CTAs per token
+  *bytes = tc ? static_cast<size_t>(M) * K * 2 + static_cast<size_t>(M) * (K / block) * 4 : 0;
   return QVLA_OK;
 }
 

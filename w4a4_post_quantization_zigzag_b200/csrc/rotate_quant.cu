@@ -268,9 +268,18 @@ struct ActProblem {
   int gx;                     // token tiles
   int bpc;                    // rotation blocks per CTA
   int a_rows;                 // rows of the permuted-x TMA box (tokens, <= 128)
+  // DYNAMIC as two launches (ActBatch::phase 1 and 2): the row maxima of
+  // every CTA's blocks, [ngroups][M] as fp32 bits
+  unsigned int* amax;
+  int ngroups;
 };
 struct ActBatch {
   int n;
+  // DYNAMIC only.  0: both passes in one launch, the row maximum reduced over
+  // a cluster along the blocks (grid y);  1: the maximum pass alone, each
+  // CTA's row maxima to ActProblem::amax;  2: the quantising pass alone,
+  // the scale from the maxima phase 1 wrote.  Phases 1 and 2 take no cluster.
+  int phase;
   int cta_start[kMaxBatch + 1];
   ActProblem p[kMaxBatch];
 };
@@ -704,15 +713,16 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
   const int M = P.M, ldx = P.ldx, K = P.K;
   const int local = static_cast<int>(blockIdx.x) - batch.cta_start[pi];
   const int tile = local % P.gx;
-  const int group = MODE == kDynamic ? static_cast<int>(blockIdx.y) : local / P.gx;
+  const int phase = MODE == kDynamic ? batch.phase : 0;
+  const int group = MODE == kDynamic && phase == 0 ? static_cast<int>(blockIdx.y) : local / P.gx;
   const int m0 = tile * kTM;
   const int ntok = min(kTM, M - m0);
   const int nb = K / BS;
   const int B0 = group * P.bpc;
   const int nbc = max(0, min(P.bpc, nb - B0));
-  const int passes = MODE == kDynamic ? 2 : 1;
+  const int passes = MODE == kDynamic && phase == 0 ? 2 : 1;
   const int W = passes * nbc;                  // work items: (pass, block)
-  const int cs = MODE == kDynamic ? static_cast<int>(gridDim.y) : 1;
+  const int cs = MODE == kDynamic && phase == 0 ? static_cast<int>(gridDim.y) : 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -937,11 +947,25 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
         cluster_arrive_relaxed();          // phase 2: done reading peers
         amax = __uint_as_float(mx);
       }
+      if (phase == 1 && valid && cbeg == 0)
+        P.amax[static_cast<size_t>(group) * M + m0 + t] = __float_as_uint(amax);
       s = __fdiv_rn(amax, 7.0f);
       reduced = true;
     };
+    if (MODE == kDynamic && phase == 2) {
+      // the row maximum over the maxima of every CTA of the first launch that
+      // held these tokens (written before it completed, which pdl_wait above
+      // waited for)
+      unsigned int mx = 0u;
+      if (valid)
+        for (int g = 0; g < P.ngroups; ++g)
+          mx = max(mx, __ldcg(P.amax + static_cast<size_t>(g) * M + m0 + t));
+      amax = __uint_as_float(mx);
+      s = __fdiv_rn(amax, 7.0f);
+      reduced = true;
+    }
     for (int w = 0; w < W; ++w) {
-      const int ab = w & 1, pass = w / nbc, B = B0 + w % nbc;
+      const int ab = w & 1, pass = phase == 0 ? w / nbc : phase - 1, B = B0 + w % nbc;
       // one outcome per warp, and a converged warp for the warp-wide loads
       if (!__all_sync(0xffffffffu, mbar_wait(&bars.acc_full[ab], (w >> 1) & 1, err))) break;
       tc_fence_after();
@@ -992,10 +1016,10 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
       }
       tc_fence_before();
       mbar_arrive(&bars.acc_empty[ab]);
-      if (MODE == kDynamic && w == nbc - 1) reduce_rows();
+      if (MODE == kDynamic && phase < 2 && w == nbc - 1) reduce_rows();
     }
     if (MODE == kDynamic && !reduced) reduce_rows();
-    if (MODE != kRotateOnly && group == 0 && valid && cbeg == 0) P.s_x[m0 + t] = s;
+    if (MODE != kRotateOnly && phase != 1 && group == 0 && valid && cbeg == 0) P.s_x[m0 + t] = s;
   }
 
   if (MODE == kDynamic && cs > 1) {
@@ -1626,13 +1650,16 @@ cudaError_t launch_permute(const std::vector<const ActArgs*>& v, cudaStream_t st
 }
 
 // One launch of up to kMaxBatch problems sharing (BS, MODE) and, in DYNAMIC
-// mode, the cluster size `cs`; TABLE / rotate-only take `G` blocks per CTA.
+// mode, the cluster size `cs`; TABLE / rotate-only and the two DYNAMIC
+// phases (`phase` 1, 2: see ActBatch) take `G` blocks per CTA.
 template <int BS, int MODE, bool kTmaA, bool kLat = false>
-cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cudaStream_t stream) {
+cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cudaStream_t stream,
+                            int phase = 0) {
   using C = TcCfg<BS, kLat>;
   ActBatch batch;
   std::memset(&batch, 0, sizeof(batch));
   batch.n = n;
+  batch.phase = phase;
   int ctas = 0;
   for (int i = 0; i < n; ++i) {
     const ActArgs& a = *as[i];
@@ -1659,12 +1686,18 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     P.gx = (a.M + kTM - 1) / kTM;
     P.a_rows = xperm_box_rows(a.M);
     batch.cta_start[i] = ctas;
-    if (MODE == kDynamic) {
+    if (MODE == kDynamic && phase == 0) {
       P.bpc = (nb + cs - 1) / cs;
       ctas += P.gx;
     } else {
       P.bpc = std::min(G, nb);
       ctas += P.gx * ((nb + P.bpc - 1) / P.bpc);
+      if (MODE == kDynamic) {
+        // the maxima follow the permuted copy in the scratch
+        P.amax = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(a.ws) +
+                                                 static_cast<size_t>(a.M) * a.K * 2);
+        P.ngroups = (nb + P.bpc - 1) / P.bpc;
+      }
     }
   }
   batch.cta_start[n] = ctas;
@@ -1685,7 +1718,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ctas, MODE == kDynamic ? cs : 1, 1);
+  cfg.gridDim = dim3(ctas, MODE == kDynamic && phase == 0 ? cs : 1, 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
@@ -1696,7 +1729,7 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
-  if (MODE == kDynamic && cs > 1) {
+  if (MODE == kDynamic && phase == 0 && cs > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = 1;
     attr[na].val.clusterDim.y = cs;
@@ -1710,14 +1743,93 @@ cudaError_t launch_tc_group(const ActArgs* const* as, int n, int G, int cs, cuda
   return cudaGetLastError();
 }
 
+// DYNAMIC launch costs, in passes of one CTA over one rotation block (a
+// launch adds one): the one-launch route with a cluster along the blocks,
+// and the two-launch route (maxima, then quantisation) with `G` blocks per
+// CTA and no cluster.  Both assume the CTAs that fit one wave run together.
+template <int BS>
+long long cluster_route_cost(const std::vector<const ActArgs*>& v, long long slots) {
+  long long cost = 0;
+  for (int cs = 1; cs <= 16; cs *= 2) {
+    std::vector<const ActArgs*> g;
+    for (const ActArgs* a : v)
+      if (tc_cluster<BS>(a->M, a->K) == cs) g.push_back(a);
+    for (size_t i0 = 0; i0 < g.size(); i0 += kMaxBatch) {
+      const size_t n = std::min<size_t>(kMaxBatch, g.size() - i0);
+      long long tiles = 0, per = 0;
+      for (size_t i = 0; i < n; ++i) tiles += (g[i0 + i]->M + kTM - 1) / kTM;
+      int c = cs;
+      while (c > 1 && tiles * c > slots) c /= 2;
+      for (size_t i = 0; i < n; ++i) per = std::max<long long>(per, (g[i0 + i]->K / BS + c - 1) / c);
+      cost += 2 * per * ((tiles * c + slots - 1) / slots) + 1;
+    }
+  }
+  return cost;
+}
+
+template <int BS>
+int split_route_blocks(const ActArgs* const* as, int n, long long slots, long long* cost) {
+  int nbmax = 1;
+  for (int i = 0; i < n; ++i) nbmax = std::max(nbmax, as[i]->K / BS);
+  long long best = -1;
+  int bestG = 1;
+  for (int G = 1; G <= nbmax; ++G) {
+    long long ctas = 0;
+    for (int i = 0; i < n; ++i) {
+      const int nb = as[i]->K / BS, g = std::min(G, nb);
+      ctas += static_cast<long long>((as[i]->M + kTM - 1) / kTM) * ((nb + g - 1) / g);
+    }
+    const long long c = (ctas + slots - 1) / slots * G;
+    if (best < 0 || c <= best) {           // ties: fewer, longer CTAs
+      best = c;
+      bestG = G;
+    }
+  }
+  *cost = 2 * (best + 1);
+  return bestG;
+}
+
+// scratch for the two-launch DYNAMIC route: the permuted copy, then the row
+// maxima of up to K / BS CTAs per token
+template <int BS>
+bool has_amax_scratch(const ActArgs* a) {
+  return a->ws_bytes >= static_cast<size_t>(a->M) * a->K * 2 + static_cast<size_t>(a->M) * (a->K / BS) * 4;
+}
+
 template <int BS, int MODE, bool kTmaA>
 cudaError_t launch_tc_mode(const std::vector<const ActArgs*>& v, cudaStream_t stream) {
   if (v.empty()) return cudaSuccess;
   if (MODE == kDynamic) {
+    const long long slots = 148LL * tc_ctas_per_sm<BS>();
+    if (kTmaA) {
+      // two launches per batch when every problem has room for the maxima and
+      // that is shorter: the blocks of wide and narrow linears then spread
+      // evenly over the SMs, where one cluster size per launch cannot
+      bool room = true;
+      for (const ActArgs* a : v) room = room && has_amax_scratch<BS>(a);
+      if (room) {
+        long long split = 0;
+        std::vector<int> Gs;
+        for (size_t i0 = 0; i0 < v.size(); i0 += kMaxBatch) {
+          const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+          long long c = 0;
+          Gs.push_back(split_route_blocks<BS>(v.data() + i0, n, slots, &c));
+          split += c;
+        }
+        if (split < cluster_route_cost<BS>(v, slots)) {
+          for (size_t i0 = 0, k = 0; i0 < v.size(); i0 += kMaxBatch, ++k) {
+            const int n = static_cast<int>(std::min<size_t>(kMaxBatch, v.size() - i0));
+            cudaError_t e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, Gs[k], 1, stream, 1);
+            if (e == cudaSuccess) e = launch_tc_group<BS, MODE, kTmaA>(v.data() + i0, n, Gs[k], 1, stream, 2);
+            if (e != cudaSuccess) return e;
+          }
+          return cudaSuccess;
+        }
+      }
+    }
     // the cluster size each linear would take alone; a launch of several
     // halves it until all its clusters fit one wave (clusters of one CTA per
     // SM are only co-resident a GPC's worth at a time)
-    const long long slots = 148LL * tc_ctas_per_sm<BS>();
     for (int cs = 1; cs <= 16; cs *= 2) {
       std::vector<const ActArgs*> g;
       for (const ActArgs* a : v)
