@@ -355,8 +355,10 @@ qvla_status qvla_rotate_quant_workspace_bytes(int M, int K, int block, qvla_dtyp
  * lives in a fixed array inside the library, QVLA_NOALLOC_SCRATCH_BYTES bytes
  * per device, kept for as long as the library is loaded.  Arguments and
  * results are those of qvla_rotate_quant_act.
- *  - A call whose scratch need exceeds QVLA_NOALLOC_SCRATCH_BYTES returns
- *    QVLA_ERR_WORKSPACE and does nothing.
+ *  - A call whose permuted copy (M * K * 2 bytes, when the tensor-core
+ *    route applies) exceeds QVLA_NOALLOC_SCRATCH_BYTES returns
+ *    QVLA_ERR_WORKSPACE and does nothing.  The DYNAMIC row maxima that
+ *    follow it in a full workspace are used only when they fit as well.
  *  - The first call on a device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
  *  - Every call on a device shares the one array: calls that may run at the

@@ -82,6 +82,26 @@ def test_noalloc_runs_the_permuted_copy_route(q):
     assert q.qvla_read_error_word(clear=True) == 0
 
 
+def test_noalloc_at_the_array_size_keeps_the_one_launch_route(q):
+    """A permuted copy that fills the array exactly (1024 x 8192 bf16 = 16 MiB)
+    leaves no room for the row maxima of the two-launch dynamic route: the call
+    still runs, on the cluster route, and gives the bits of the allocating
+    entry point (which has room and takes the two-launch route)."""
+    M, K, b = 1024, 8192, 128
+    assert M * K * 2 == q.QVLA_NOALLOC_SCRATCH_BYTES
+    assert q.qvla_rotate_quant_workspace_bytes(M, K, b) > q.QVLA_NOALLOC_SCRATCH_BYTES
+    L = _packed(q, 128, K, b, 9400)
+    x = torch.from_numpy(I.activations(9401, M, K, n_outlier_cols=5)).cuda().to(torch.bfloat16)
+    ws = torch.empty(q.qvla_rotate_quant_workspace_bytes(M, K, b), dtype=torch.uint8, device="cuda")
+    ref_q, ref_s = q.qvla_rotate_quant_act(x, L, q.QVLA_SCALE_DYNAMIC, workspace=ws)
+    xq = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    q.qvla_rotate_quant_act_noalloc(x, L, xq, sx, q.QVLA_SCALE_DYNAMIC)
+    torch.cuda.synchronize()
+    assert torch.equal(xq, ref_q) and torch.equal(sx, ref_s)
+    assert q.qvla_read_error_word(clear=True) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_array(q):
     M, K, b = 1024, 16384, 128                # needs 32 MiB of scratch
     assert q.qvla_rotate_quant_workspace_bytes(M, K, b) > q.QVLA_NOALLOC_SCRATCH_BYTES

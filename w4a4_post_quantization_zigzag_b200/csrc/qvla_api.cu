@@ -637,7 +637,10 @@ qvla_status qvla_rotate_quant_act_noalloc(const void* x, qvla_dtype xdt, int M, 
   size_t need = 0;
   if ((st = qvla_rotate_quant_workspace_bytes(M, L->K, L->block, xdt, &need)) != QVLA_OK)
     return st;
-  if (need > QVLA_NOALLOC_SCRATCH_BYTES) return QVLA_ERR_WORKSPACE;
+  // the permuted copy must fit; the row maxima of the two-launch DYNAMIC
+  // route are used only if they fit as well (the route checks the size)
+  if (need > 0 && static_cast<size_t>(M) * L->K * 2 > QVLA_NOALLOC_SCRATCH_BYTES)
+    return QVLA_ERR_WORKSPACE;
   if (need > 0) {
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != QVLA_OK) return st;

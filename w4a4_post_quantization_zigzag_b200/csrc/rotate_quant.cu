@@ -1043,11 +1043,15 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
 // buffers in shared memory:
 //   warp 8      bulk-copies whole rows (16-byte aligned, K * 2 bytes) into
 //               the ring, one mbarrier per slot
-//   warps 0-7   per row, every thread takes its runs of 8 output positions,
-//               gathers them from the staged row and writes them with one
-//               16-byte store (coalesced); the permutation entries of its
-//               runs stay in registers for all rows
-// so the loads of later rows are in flight while earlier rows are scattered.
+//   warps 0-7   in groups of `gw` warps, each group one row at a time (rows
+//               g, g + groups, ...): every thread takes its runs of 8 output
+//               positions, gathers them from the staged row and writes them
+//               with one 16-byte store (coalesced); the permutation entries
+//               of its runs stay in registers for all rows
+// so the loads of later rows are in flight while earlier rows are scattered,
+// and short rows are scattered several at a time.  Slot st always serves
+// group st % groups (the slot count is a multiple of the group count), so a
+// group never waits on a slot phase that another group has yet to consume.
 struct PermJob {
   const __nv_bfloat16* x;
   const int32_t* perm;
@@ -1055,6 +1059,7 @@ struct PermJob {
   int ldx, M, K;
   int rpc;                          // rows per CTA
   int stages;                       // row slots of K * 2 bytes in the ring
+  int gw;                           // warps per row group: 1, 2, 4 or 8
 };
 constexpr int kPermMaxStages = 32;
 constexpr int kPermWorkers = 256;
@@ -1078,12 +1083,14 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
   const int K = J.K, kc = K / 8, S = J.stages;
   const int row_bytes = K * 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gthr = 32 * J.gw, ng = kPermWorkers / gthr;   // threads per group, groups
+  const int grp = tid / gthr, gt = tid - grp * gthr;      // this worker's group, index in it
   // the permutation does not depend on the previous kernel: read before
   // waiting for it
   int p[kPC][8];
 #pragma unroll
   for (int c = 0; c < kPC; ++c) {
-    const int i = tid + kPermWorkers * c;
+    const int i = gt + gthr * c;
     int4 a = make_int4(0, 0, 0, 0), b = make_int4(0, 0, 0, 0);
     if (tid < kPermWorkers && i < kc) {
       a = __ldg(reinterpret_cast<const int4*>(J.perm) + 2 * i);
@@ -1096,7 +1103,7 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
   if (tid == 0) {
     for (int st = 0; st < S; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], kPermWorkers);
+      mbar_init(&empty[st], gthr);
     }
     fence_mbar_init();
   }
@@ -1120,7 +1127,7 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
     }
   } else {
     // ------------------------------------------------------------- workers
-    for (int r = 0; r < nr; ++r) {
+    for (int r = grp; r < nr; r += ng) {
       const int st = r % S;
       if (!mbar_wait(&full[st], (r / S) & 1, err)) break;
       const unsigned short* sr =
@@ -1128,7 +1135,7 @@ __global__ void __launch_bounds__(kPermWorkers + 32)
       uint4* orow = reinterpret_cast<uint4*>(J.out + static_cast<size_t>(r0 + r) * K);
 #pragma unroll
       for (int c = 0; c < kPC; ++c) {
-        const int i = tid + kPermWorkers * c;
+        const int i = gt + gthr * c;
         if (i < kc) {
           uint32_t w[4];
 #pragma unroll
@@ -1258,8 +1265,8 @@ __global__ void __launch_bounds__(kThreads)
     if (tid == 0) s_out[row] = s;
     return;
   }
-  const float rs = quant_recip(s);
   uint8_t* dst = q_out + static_cast<size_t>(row) * (K / 2);
+  const float rs = quant_recip(s);
   for (int j = tid; j < K / 2; j += kThreads) {
     const int q0 = quant_code_fast(src[2 * j], s, rs, qmin, qmax);
     const int q1 = quant_code_fast(src[2 * j + 1], s, rs, qmin, qmax);
@@ -1592,7 +1599,16 @@ cudaError_t launch_permute_kernel(PermBatch& b, const ActArgs* const* as, int km
   // one ring of shared memory per CTA, as many row slots as it holds for the
   // CTA's own rows (so short rows keep more of them in flight)
   const int smem = std::max(permute_ring_bytes<kPC>(), 2 * kmax * 2);
-  for (int i = 0; i < b.n; ++i) b.j[i].stages = std::min(kPermMaxStages, smem / (as[i]->K * 2));
+  for (int i = 0; i < b.n; ++i) {
+    // rows scattered at a time: groups of the fewest warps whose threads hold
+    // the row's runs of 8 (kPC each), while the ring keeps two slots per group
+    const int K = as[i]->K, slots = std::min(kPermMaxStages, smem / (K * 2));
+    int gw = 1;
+    while (gw < kPermWorkers / 32 && (K / 8 > 32 * gw * kPC || slots < 2 * (kPermWorkers / 32 / gw))) gw *= 2;
+    const int ng = kPermWorkers / 32 / gw;
+    b.j[i].gw = gw;
+    b.j[i].stages = slots / ng * ng;               // a multiple of the group count
+  }
   // the elements spread over one wave of resident CTAs; the longest rows
   // (one CTA per SM) take three CTAs per SM in waves, measured faster than
   // one long CTA per SM
