@@ -63,6 +63,67 @@ def test_act_quant_from_fp32_is_bit_exact(q, M, K):
     no_device_error(q)
 
 
+def _near_boundary_row(rng, s, K, hs, amax=None):
+    """K fp32 values whose quotients by s sit on and within a few ulps of the
+    half-integers hs (where rint flips), plus integers, zeros, subnormals and,
+    without amax, saturating values; amax (dynamic mode) caps |v| and is
+    placed once so that it is the row maximum."""
+    s = np.float32(s)
+    vals = []
+    for h in hs:
+        v = np.float32(np.float64(h) * np.float64(s))
+        for k in range(-4, 5):
+            w = v
+            step = np.float32(np.inf) if k > 0 else np.float32(-np.inf)
+            for _ in range(abs(k)):
+                w = np.nextafter(w, step)
+            vals.append(w)
+    vals += [np.float32(0), np.float32(-0.0), np.float32(1e-40), np.float32(-1e-40)]
+    vals += [np.float32(n) * s for n in range(-7, 8)]
+    if amax is None:
+        vals += [np.float32(x) * s for x in (7.49, 7.5, 7.51, -8.49, -8.5, -8.51, 9, -9, 40, -40)]
+        vals += [np.float32(3e38), np.float32(-3e38)]
+    v = np.array(vals, np.float32)
+    if amax is not None:
+        v = v[np.abs(v) <= np.float32(amax)]
+    out = rng.uniform(-1, 1, K).astype(np.float32) * (np.float32(amax) if amax is not None else s * 6)
+    pos = rng.permutation(K)
+    n = min(len(v), K - 1)
+    out[pos[:n]] = v[:n]
+    if amax is not None:
+        out[pos[n]] = np.float32(amax)
+    return out
+
+
+@pytest.mark.parametrize("K", [1024, 256])
+def test_act_quant_near_rounding_boundaries_is_bit_exact(q, K):
+    """The epilogue quantiser (fused clamp by a saturating FMA, paired FMAs,
+    exact division only near a half-integer) against clamp(rint(fp32(v / s)))
+    on quotients within a few ulps of every half-integer, in both modes."""
+    rng = np.random.default_rng(77 + K)
+    # dynamic: s = fp32(amax / 7) per row, a power of two and irregular ones
+    amaxes = [7.0, 7.7, 1.0e-3 * 3.3, 5.0e4 + 0.3, 0.1, 123.456]
+    rows = []
+    for a in amaxes:
+        s = np.float32(a) / np.float32(7)
+        rows.append(_near_boundary_row(rng, s, K, np.arange(-6.5, 7.0, 1.0), amax=a))
+    xr = np.stack(rows)
+    qx_ref, s_ref = O.quantize_acts_dynamic_fp32(xr)
+    xq, sx = q.qvla_quant_act_f32(cu(xr), q.QVLA_SCALE_DYNAMIC)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), O.pack_nibbles(qx_ref))
+    # table: one irregular scale, quotients from -9.5 to 8.5 (saturation both ends)
+    tab = np.full((2, 3), 0.01234567, np.float32)
+    tab[1, 2] = np.float32(0.0123456789)
+    st = O.table_scale(tab, 1, 2)
+    xt = np.stack([_near_boundary_row(rng, st, K, np.arange(-9.5, 9.0, 1.0)) for _ in range(3)])
+    qt_ref, _ = O.quantize_acts_table_fp32(xt, st)
+    xq_t, s_t = q.qvla_quant_act_f32(cu(xt), q.QVLA_SCALE_TABLE, table=cu(tab), step=1, layer=2)
+    assert (s_t.cpu().numpy() == st).all()
+    assert np.array_equal(xq_t.cpu().numpy(), O.pack_nibbles(qt_ref))
+    no_device_error(q)
+
+
 def test_quant_near_rounding_boundaries_is_bit_exact(q):
     """Values at, and one or two ulp around, every half-integer multiple of the
     scale: the codes must equal clamp(rint(fp32(v / s))) exactly (ties to even),

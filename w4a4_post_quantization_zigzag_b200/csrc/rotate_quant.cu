@@ -128,60 +128,114 @@ QVLA_DEVICE int quant_code_fast(float v, float s, float rs, int qmin, int qmax) 
   return static_cast<int>(r);
 }
 
+// Two fp32 lanes in one 64-bit register, for the paired FMA (sm_100).
+QVLA_DEVICE uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+QVLA_DEVICE void f2split(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+QVLA_DEVICE uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+QVLA_DEVICE float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+QVLA_DEVICE float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 4-bit codes of N consecutive values, packed two per byte (value 2k in the
 // low nibble of byte k) into N/8 32-bit words: the same codes as
-// quant_code(v, s, -8, 7), as straight-line code (so the independent elements
-// overlap) with the rare near-half-integer elements redone by exact division
-// afterwards.  Three identities keep it short:
-//   * clamping the quotient before rounding gives the same code as clamping
-//     the rounded quotient (the bounds are integers and rint is monotonic),
-//     and a clamped quotient is an integer, never near a half-integer;
-//   * |q - rint(q)| is exact and at most 1/2, so "within 2^-18 of a
-//     half-integer" is |q - rint(q)| > 1/2 - 2^-18, tracked as one running max;
-//   * four codes c_j in [-8, 7] go into one float as
-//     2^23 + sum_j (c_j + 8) 16^j, every partial sum an integer in
-//     [2^23, 2^24), so its low 16 mantissa bits are the four offset nibbles;
-//     XOR 8 turns an offset nibble c + 8 into the 4-bit two's complement of c.
+// quant_code(v, s, -8, 7) = clamp(rint(fp32(v / s)), -8, 7), as straight-line
+// FMA-pipe code (so the independent elements overlap) with the rare elements
+// near a rounding boundary redone by the IEEE division afterwards.  With
+// a = fp32(1 / fp32(15 s)) (quant_recip15) and c8 = fp32(8 / 15):
+//   * x = sat(fma(v, a, c8)) is (v/s + 8) / 15 clamped to [0, 1]: the
+//     saturation is the clamp to [-8, 7] (clamping before rounding gives the
+//     code of clamping after it: integer bounds, monotone rounding; NaN
+//     saturates to 0, code -8, as the clamp of NaN gives);
+//   * e = fp32(15 x + 1.5 * 2^23) - 1.5 * 2^23 is the offset code c + 8 =
+//     rint(15 x) in [0, 15] (one rounding of the exact product, in a binade
+//     of unit spacing: ties to even, as rint);
+//   * |15 x - (fp32(v / s) + 8)| <= 2^-18.8 (2^-23 relative error in a, two
+//     2^-25 roundings in x, 2^-22 in the IEEE quotient), so unless
+//     d = 15 x - e (formed by one FMA) lies within 2^-18 of +-1/2 both round
+//     to the same integer; near +-1/2 (about 1 element in 10^5) the exact
+//     division decides;
+//   * four offset codes go into one float as 2^23 + sum_j e_j 16^j, every
+//     partial sum an integer in [2^23, 2^24), so its low 16 mantissa bits are
+//     the four nibbles; XOR 8 turns an offset nibble into the 4-bit two's
+//     complement of c.
+// Values 8k + j and 8k + 4 + j share one paired FMA (the two packed floats of
+// a word are built side by side).
 constexpr float kNearHalf = 0.499996185302734375f;   // 1/2 - 2^-18
+constexpr float kRound = 12582912.0f;                // 1.5 * 2^23
+constexpr float kC8 = 0.533333361148834228515625f;   // fp32(8 / 15)
 
 template <int N>
-QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float rs, uint32_t (&w)[N / 8]) {
+QVLA_DEVICE void quant_pack(const float (&v)[N], float s, float a15, uint32_t (&w)[N / 8]) {
   static_assert(N % 8 == 0 && N <= 32, "8..32 values");
-  float c[N];
+  float ne[N];                                       // -(c + 8)
   if (s == 0.f) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) c[i] = 0.f;
-  } else if (rs == 0.f) {
+    for (int i = 0; i < N; ++i) ne[i] = -8.f;
+  } else if (a15 == 0.f) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) c[i] = fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f);
+    for (int i = 0; i < N; ++i) ne[i] = -(fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f) + 8.f);
   } else {
+    const uint64_t k15 = f2(15.f, 15.f), kR = f2(kRound, kRound), kM1 = f2(-1.f, -1.f);
     float dmax = 0.f;
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const float q = fminf(fmaxf(v[i] * rs, -8.f), 7.f);
-      c[i] = rintf(q);
-      dmax = fmaxf(dmax, fabsf(q - c[i]));
+    for (int k = 0; k < N / 8; ++k) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i0 = 8 * k + j, i1 = i0 + 4;
+        const uint64_t x = f2(fma_sat(v[i0], a15, kC8), fma_sat(v[i1], a15, kC8));
+        const uint64_t m = ffma2(x, k15, kR);         // 1.5 * 2^23 + e
+        const uint64_t n = ffma2(m, kM1, kR);         // -e, exact
+        float d0, d1;
+        f2split(ffma2(x, k15, n), d0, d1);            // 15 x - e, exact
+        dmax = max3(dmax, fabsf(d0), fabsf(d1));
+        f2split(n, ne[i0], ne[i1]);
+      }
     }
     if (dmax > kNearHalf) {
 #pragma unroll
       for (int i = 0; i < N; ++i)
-        if (fabsf(fminf(fmaxf(v[i] * rs, -8.f), 7.f) - c[i]) > kNearHalf)
-          c[i] = fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f);
+        if (fabsf(fmaf(fma_sat(v[i], a15, kC8), 15.f, ne[i])) > kNearHalf)
+          ne[i] = -(fminf(fmaxf(exact_rint_quotient(v[i], s), -8.f), 7.f) + 8.f);
     }
   }
+  const uint64_t k23 = f2(8388608.0f, 8388608.0f);    // 2^23
 #pragma unroll
   for (int k = 0; k < N / 8; ++k) {
-    float h[2];
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const float* cg = c + 8 * k + 4 * g;
-      float a = cg[0] + 8423560.0f;                  // 2^23 + 8 * (1 + 16 + 256 + 4096)
-      a = fmaf(cg[1], 16.f, a);
-      a = fmaf(cg[2], 256.f, a);
-      h[g] = fmaf(cg[3], 4096.f, a);
-    }
-    w[k] = __byte_perm(__float_as_uint(h[0]), __float_as_uint(h[1]), 0x5410) ^ 0x88888888u;
+    const float* n = ne + 8 * k;
+    uint64_t h = ffma2(f2(n[0], n[4]), f2(-1.f, -1.f), k23);
+    h = ffma2(f2(n[1], n[5]), f2(-16.f, -16.f), h);
+    h = ffma2(f2(n[2], n[6]), f2(-256.f, -256.f), h);
+    h = ffma2(f2(n[3], n[7]), f2(-4096.f, -4096.f), h);
+    float h0, h1;
+    f2split(h, h0, h1);
+    w[k] = __byte_perm(__float_as_uint(h0), __float_as_uint(h1), 0x5410) ^ 0x88888888u;
   }
+}
+
+// fp32(1 / fp32(15 s)) for quant_pack, or 0 to force the exact path: s == 0,
+// or 15 s or its reciprocal outside the normal range (the error bound of
+// quant_pack takes both roundings as relative).
+QVLA_DEVICE float quant_recip15(float s) {
+  const float t = fabsf(15.f * s);
+  if (!(t >= 1.17549435e-38f && t <= 4.2535296e37f)) return 0.f;   // [2^-126, 2^125]; NaN too
+  return __frcp_rn(15.f * s);
 }
 
 // fp32(1 / s) for quant_code_fast, or 0 to force the exact path (s == 0 or a
@@ -481,7 +535,7 @@ __global__ void __launch_bounds__(kThreads)
   const int nch = nbc * BS;                    // channels held by this CTA (multiple of 32)
   for (int t = warp; t < ntok; t += kWarps) {
     const float s = scale_s[t];
-    const float rs = quant_recip(s);
+    const float a15 = quant_recip15(s);
     uint8_t* dst = xq + static_cast<size_t>(m0 + t) * (K / 2) + (B0 * BS) / 2;
     for (int c0 = 0; c0 < nch; c0 += 256) {
       const int k = c0 + 8 * lane;            // 8 channels -> 4 bytes per lane
@@ -490,7 +544,7 @@ __global__ void __launch_bounds__(kThreads)
         const float4 b = *reinterpret_cast<const float4*>(keep + t * kpitch + k + 4);
         const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         uint32_t w[1];
-        quant_pack<8>(f, s, rs, w);
+        quant_pack<8>(f, s, a15, w);
         *reinterpret_cast<uint32_t*>(dst + k / 2) = w[0];
       }
     }
@@ -969,7 +1023,7 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
       // one outcome per warp, and a converged warp for the warp-wide loads
       if (!__all_sync(0xffffffffu, mbar_wait(&bars.acc_full[ab], (w >> 1) & 1, err))) break;
       tc_fence_after();
-      const float rs = quant_recip(s);
+      const float a15 = quant_recip15(s);
 #pragma unroll 1
       for (int c0 = cbeg; c0 < cbeg + kCols; c0 += 32) {
         uint32_t r[32];
@@ -995,7 +1049,7 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
 #pragma unroll
             for (int c = 0; c < 16; ++c) f[c] = __uint_as_float(r[16 * hh + c]);
             uint32_t w2[2];
-            quant_pack<16>(f, s, rs, w2);
+            quant_pack<16>(f, s, a15, w2);
             wv[2 * hh] = w2[0];
             wv[2 * hh + 1] = w2[1];
           }
@@ -1266,6 +1320,21 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
   uint8_t* dst = q_out + static_cast<size_t>(row) * (K / 2);
+  if (qmin == -8 && qmax == 7 && K % 8 == 0) {
+    // activations: the epilogue quantiser of the rotation kernels, 8 values
+    // (one 32-bit word of codes) per thread
+    const float a15 = quant_recip15(s);
+    for (int j = tid; j < K / 8; j += kThreads) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = src[8 * j + u];
+      uint32_t wd[1];
+      quant_pack<8>(f, s, a15, wd);
+      *reinterpret_cast<uint32_t*>(dst + 4 * j) = wd[0];
+    }
+    if (tid == 0) s_out[row] = s;
+    return;
+  }
   const float rs = quant_recip(s);
   for (int j = tid; j < K / 2; j += kThreads) {
     const int q0 = quant_code_fast(src[2 * j], s, rs, qmin, qmax);
