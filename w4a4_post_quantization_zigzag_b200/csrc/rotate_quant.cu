@@ -147,6 +147,12 @@ QVLA_DEVICE float fma_sat(float a, float b, float c) {
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// One 32-byte store (sm_100); the address must be 32-byte aligned.
+QVLA_DEVICE void st_global_v8(void* p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y),
+               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
 QVLA_DEVICE float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -1018,6 +1024,11 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
       s = __fdiv_rn(amax, 7.0f);
       reduced = true;
     }
+    // 32-byte aligned outputs take 32-byte stores (each row's offsets are
+    // multiples of 32 bytes: K is a multiple of 64)
+    const bool xq32 = (reinterpret_cast<uintptr_t>(P.xq) & 31u) == 0;
+    const bool xq8_32 = (reinterpret_cast<uintptr_t>(P.xq8) & 31u) == 0;
+    uint4 keep = make_uint4(0u, 0u, 0u, 0u);
     for (int w = 0; w < W; ++w) {
       const int ab = w & 1, pass = phase == 0 ? w / nbc : phase - 1, B = B0 + w % nbc;
       // one outcome per warp, and a converged warp for the warp-wide loads
@@ -1054,16 +1065,33 @@ __global__ void __launch_bounds__(TcCfg<BS, kLat>::kThreads, kLat ? 3 : BS == 64
             wv[2 * hh + 1] = w2[1];
           }
           if (valid) {
-            *reinterpret_cast<uint4*>(P.xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS + c0) / 2) =
-                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            // full 32-byte sectors where the buffers allow (one request per
+            // sector instead of two): the codes of two 32-column chunks go
+            // out together, the image of a chunk in one store
+            uint8_t* dq = P.xq + static_cast<size_t>(m0 + t) * (K / 2) + (B * BS + c0) / 2;
+            const uint4 cw = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            if (kCols % 64 == 0 && xq32) {
+              if (((c0 - cbeg) & 32) == 0)
+                keep = cw;                          // first chunk of a pair (32-byte aligned)
+              else
+                st_global_v8(dq - 16, keep, cw);
+            } else {
+              *reinterpret_cast<uint4*>(dq) = cw;
+            }
             if (P.xq8 != nullptr) {
               // the GEMM's int8 image of these 32 codes: 16*q, even codes
               // first, then odd codes
-              uint4* d8 = reinterpret_cast<uint4*>(P.xq8 + static_cast<size_t>(m0 + t) * K + B * BS + c0);
-              d8[0] = make_uint4((wv[0] << 4) & 0xF0F0F0F0u, (wv[1] << 4) & 0xF0F0F0F0u,
-                                 (wv[2] << 4) & 0xF0F0F0F0u, (wv[3] << 4) & 0xF0F0F0F0u);
-              d8[1] = make_uint4(wv[0] & 0xF0F0F0F0u, wv[1] & 0xF0F0F0F0u, wv[2] & 0xF0F0F0F0u,
-                                 wv[3] & 0xF0F0F0F0u);
+              int8_t* d8 = P.xq8 + static_cast<size_t>(m0 + t) * K + B * BS + c0;
+              const uint4 lo = make_uint4((wv[0] << 4) & 0xF0F0F0F0u, (wv[1] << 4) & 0xF0F0F0F0u,
+                                          (wv[2] << 4) & 0xF0F0F0F0u, (wv[3] << 4) & 0xF0F0F0F0u);
+              const uint4 hi = make_uint4(wv[0] & 0xF0F0F0F0u, wv[1] & 0xF0F0F0F0u, wv[2] & 0xF0F0F0F0u,
+                                          wv[3] & 0xF0F0F0F0u);
+              if (xq8_32) {
+                st_global_v8(d8, lo, hi);
+              } else {
+                reinterpret_cast<uint4*>(d8)[0] = lo;
+                reinterpret_cast<uint4*>(d8)[1] = hi;
+              }
             }
           }
         }
