@@ -266,7 +266,8 @@ def test_rotation_fp32_vs_fp64(q, path, M, K, b, dt):
     (8, 1024, 32, "bf16", "dynamic"), (8, 1024, 256, "bf16", "table"),
     (3, 16384, 128, "bf16", "dynamic"), (300, 2048, 64, "bf16", "dynamic"),
     (257, 1536, 64, "bf16", "table"), (200, 4096, 128, "bf16", "table"),
-    (1, 256, 64, "bf16", "table"), (33, 512, 64, "f32", "table"), (100, 1024, 64, "f32", "table")])
+    (1, 256, 64, "bf16", "table"), (33, 512, 64, "f32", "table"), (100, 1024, 64, "f32", "table"),
+    (600, 1024, 64, "bf16", "table")])
 @pytest.mark.parametrize("scratch", [False, True])
 def test_rotate_quant_end_to_end(q, path, scratch, M, K, b, dt, mode):
     """scratch=True gives the call its workspace, which routes large bf16 inputs

@@ -67,7 +67,7 @@ def test_a8_activation_codes(q, M, K, b, dt):
     assert q.qvla_read_error_word(clear=True) == 0
 
 
-@pytest.mark.parametrize("M,K,b", [(50, 4096, 64), (3, 1024, 128), (200, 2048, 64)])
+@pytest.mark.parametrize("M,K,b", [(50, 4096, 64), (3, 1024, 128), (200, 2048, 64), (520, 1024, 64)])
 def test_a8_routes_agree(q, M, K, b):
     """A workspace of M*K*6 bytes (room for the permuted copy) and the minimum
     M*K*4 give identical codes and scales."""
